@@ -1,0 +1,258 @@
+"""Checks that pin the CPU oracle to things other than itself.
+
+Each ``pin_*`` function raises AssertionError when the oracle in use disagrees
+with an independent fact: an exhaustive brute force, a closed form, an
+invariant, or a special case that reduces to a library routine.  The pages
+print no worked example, so these are the oracle's only anchors; the planted-
+mistake test runs every pin against deliberately broken oracle builds to show
+that each plausible mistake is caught by at least one of them.
+"""
+
+from __future__ import annotations
+
+import itertools
+import math
+
+import numpy as np
+import torch
+
+import oracle
+from grouped_gemm_02_b200 import workload as wl
+
+
+def _bits(a: torch.Tensor) -> np.ndarray:
+    return wl.bf16_bits(a)
+
+
+def _f64(a: torch.Tensor) -> torch.Tensor:
+    return a.to(torch.float64)
+
+
+def _dense_swiglu(x64: torch.Tensor, W1: torch.Tensor, W3: torch.Tensor, W2: torch.Tensor) -> torch.Tensor:
+    """Dense SwiGLU FFN with library calls: silu(x W1^T) * (x W3^T), then W2."""
+    g = x64 @ _f64(W1).T
+    u = x64 @ _f64(W3).T
+    return (torch.nn.functional.silu(g) * u) @ _f64(W2).T
+
+
+# --------------------------------------------------------------------------- widening
+
+def pin_bf16_widening_exhaustive():
+    """All 65536 bf16 patterns through the logits step with Wg = 1, d = 1, no bias."""
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    x = pats.reshape(-1, 1)
+    one = np.array([[0x3F80]], dtype=np.uint16)          # bf16 1.0
+    L = oracle.router_logits(x, one, None)[:, 0]
+    ref = torch.from_numpy(pats.view(np.int16).copy()).view(torch.bfloat16).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(L), nan)
+    assert np.array_equal(L[~nan], ref[~nan])
+
+
+# --------------------------------------------------------------------------- logits
+
+def pin_router_logits_matmul():
+    s = wl.TINY.with_(T=9, d=40, E=6)
+    inp = wl.make_inputs(s, seed=3, weights=False)
+    L = oracle.router_logits(_bits(inp["x"]), _bits(inp["Wg"]), inp["bias"].numpy())
+    ref = (_f64(inp["x"]) @ _f64(inp["Wg"]).T + inp["bias"].to(torch.float64)).numpy()
+    assert np.allclose(L, ref, rtol=1e-12, atol=1e-12)
+    L0 = oracle.router_logits(_bits(inp["x"]), _bits(inp["Wg"]), None)
+    assert np.allclose(L0, (_f64(inp["x"]) @ _f64(inp["Wg"]).T).numpy(), rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- top-k
+
+def _rank_key(v: float, i: int):
+    return (1 if math.isnan(v) else 0, 0.0 if math.isnan(v) else -v, i)
+
+
+def pin_topk_bruteforce():
+    """For E <= 7 and every k: the chosen set is the only k-subset whose members all
+    rank ahead of every non-member; found by enumerating every subset."""
+    rng = np.random.default_rng(11)
+    for E in range(1, 8):
+        for trial in range(6):
+            L = rng.integers(-2, 3, size=(3, E)).astype(np.float32) * 0.5   # many ties
+            if trial == 5 and E > 2:
+                L[0, 1] = np.nan
+            for k in range(1, E + 1):
+                idx, w = oracle.topk(L, k)
+                for t in range(L.shape[0]):
+                    row = L[t]
+                    winners = []
+                    for S in itertools.combinations(range(E), k):
+                        rest = [j for j in range(E) if j not in S]
+                        if all(_rank_key(row[i], i) < _rank_key(row[j], j) for i in S for j in rest):
+                            winners.append(set(S))
+                    assert len(winners) == 1
+                    assert set(idx[t].tolist()) == winners[0]
+                    keys = [_rank_key(row[i], i) for i in idx[t]]
+                    assert all(keys[a] < keys[a + 1] for a in range(k - 1))
+
+
+def pin_topk_full_softmax():
+    """k = E: the gates are the full softmax (library routine), taken in chosen order."""
+    L = wl.random_logits(5, 9, seed=4).numpy()
+    idx, w = oracle.topk(L, 9)
+    ref = torch.softmax(torch.from_numpy(L).to(torch.float64), dim=1).numpy()
+    assert np.allclose(w, np.take_along_axis(ref, idx.astype(np.int64), axis=1), rtol=1e-13, atol=1e-15)
+
+
+def pin_gate_invariants():
+    L = wl.random_logits(40, 64, seed=5).numpy() * 3
+    for k in (1, 2, 8):
+        idx, w = oracle.topk(L, k)
+        assert np.allclose(w.sum(axis=1), 1.0, atol=1e-12)
+        assert np.all(np.diff(w, axis=1) <= 1e-15)
+        assert np.all(w > 0)
+        # the largest gate belongs to the largest logit of the token
+        assert np.array_equal(idx[:, 0], np.argmax(L, axis=1))
+
+
+# --------------------------------------------------------------------------- permutation
+
+def pin_permutation():
+    for seed, (T, E, k, alpha) in enumerate([(1, 1, 1, 1.0), (50, 8, 2, 1.0), (300, 64, 8, 0.1),
+                                             (7, 384, 8, 0.02), (0, 4, 2, 1.0)]):
+        idx = wl.random_routing(T, E, k, alpha, seed).numpy()
+        counts, offsets, perm, inv = oracle.permutation(idx, E)
+        flat = idx.ravel()
+        P = flat.size
+        assert np.array_equal(counts, np.bincount(flat, minlength=E))
+        assert counts.sum() == P and offsets[0] == 0 and offsets[-1] == P
+        assert np.all(np.diff(offsets) == counts)
+        assert np.all(counts <= T)
+        assert np.array_equal(np.sort(perm), np.arange(P))
+        assert np.array_equal(inv[perm], np.arange(P))
+        # library stable sort of the expert ids is the same permutation
+        assert np.array_equal(perm, np.argsort(flat, kind="stable"))
+        for e in range(E):
+            seg = perm[offsets[e]:offsets[e + 1]]
+            assert np.all(flat[seg] == e)
+            assert np.all(np.diff(seg) > 0)
+
+
+# --------------------------------------------------------------------------- expert FFN
+
+def _small_layer(E=5, k=2, T=11, d=24, f=16, seed=7, fs=0):
+    s = wl.LayerShape("pin", T=T, d=d, f=f, E=E, k=k, alpha=1.0, f_shared=fs)
+    return s, wl.make_inputs(s, seed=seed)
+
+
+def pin_ffn_expert_major_bruteforce():
+    """Expert-major evaluation of every expert on every token, masked by the routing
+    (y = sum_e mask[t,e] w[t,e] FFN_e(x_t)), with library matmuls."""
+    s, inp = _small_layer(fs=12)
+    idx = wl.random_routing(s.T, s.E, s.k, 1.0, 1).numpy()
+    w = wl.random_gates(s.T, s.k, 1).numpy().astype(np.float64)
+    shared = {n: _bits(inp[n]) for n in ("Ws1", "Ws3", "Ws2")}
+    y = oracle.moe_ffn(_bits(inp["x"]), _bits(inp["W1"]), _bits(inp["W3"]), _bits(inp["W2"]),
+                       idx, w, shared=shared)
+    x64 = _f64(inp["x"])
+    ref = torch.zeros(s.T, s.d, dtype=torch.float64)
+    for e in range(s.E):
+        gate = torch.zeros(s.T, dtype=torch.float64)
+        for t in range(s.T):
+            for j in range(s.k):
+                if idx[t, j] == e:
+                    gate[t] += w[t, j]
+        ref += gate[:, None] * _dense_swiglu(x64, inp["W1"][e], inp["W3"][e], inp["W2"][e])
+    ref += _dense_swiglu(x64, inp["Ws1"], inp["Ws3"], inp["Ws2"])
+    assert np.allclose(y, ref.numpy(), rtol=1e-11, atol=1e-12)
+
+
+def pin_ffn_identical_experts():
+    """Identical experts and gates summing to 1 give the dense SwiGLU FFN."""
+    s, inp = _small_layer(E=6, k=3, seed=8)
+    W1 = inp["W1"][2:3].expand(s.E, -1, -1).contiguous()
+    W3 = inp["W3"][4:5].expand(s.E, -1, -1).contiguous()
+    W2 = inp["W2"][0:1].expand(s.E, -1, -1).contiguous()
+    L = oracle.router_logits(_bits(inp["x"]), _bits(inp["Wg"]), inp["bias"].numpy()).astype(np.float32)
+    idx, w = oracle.topk(L, s.k)
+    y = oracle.moe_ffn(_bits(inp["x"]), _bits(W1), _bits(W3), _bits(W2), idx, w)
+    ref = _dense_swiglu(_f64(inp["x"]), W1[0], W3[0], W2[0]).numpy()
+    assert np.allclose(y, ref, rtol=1e-11, atol=1e-12)
+
+
+def pin_ffn_single_expert_dense():
+    """E = 1, k = 1: the layer is one dense SwiGLU FFN with gate 1."""
+    s, inp = _small_layer(E=1, k=1, seed=9)
+    idx = np.zeros((s.T, 1), dtype=np.int32)
+    w = np.ones((s.T, 1))
+    y = oracle.moe_ffn(_bits(inp["x"]), _bits(inp["W1"]), _bits(inp["W3"]), _bits(inp["W2"]), idx, w)
+    ref = _dense_swiglu(_f64(inp["x"]), inp["W1"][0], inp["W3"][0], inp["W2"][0]).numpy()
+    assert np.allclose(y, ref, rtol=1e-11, atol=1e-12)
+
+
+def pin_ffn_unrouted_expert_is_inert():
+    """Changing the weights of an expert no token is routed to changes nothing; a
+    missing (None) expert that no token uses is accepted."""
+    s, inp = _small_layer(E=4, k=1, seed=10)
+    idx = (np.arange(s.T) % 3).astype(np.int32).reshape(-1, 1)        # expert 3 unused
+    w = np.ones((s.T, 1))
+    args = lambda W1: (_bits(inp["x"]), _bits(W1), _bits(inp["W3"]), _bits(inp["W2"]), idx, w)
+    y0 = oracle.moe_ffn(*args(inp["W1"]))
+    W1b = inp["W1"].clone()
+    W1b[3] = W1b[3] * 3 + 1
+    y1 = oracle.moe_ffn(*args(W1b))
+    assert np.array_equal(y0, y1)
+    per = [_bits(inp["W1"][e]) if e < 3 else None for e in range(4)]
+    y2 = oracle.moe_ffn(_bits(inp["x"]), per, [_bits(inp["W3"][e]) for e in range(4)],
+                        [_bits(inp["W2"][e]) for e in range(4)], idx, w)
+    assert np.array_equal(y0, y2)
+
+
+def pin_ffn_token_subset_and_threads():
+    """A token subset returns the same rows; the thread count does not change a bit."""
+    s, inp = _small_layer(E=5, k=2, T=13, seed=12)
+    idx = wl.random_routing(s.T, s.E, s.k, 1.0, 2).numpy()
+    w = wl.random_gates(s.T, s.k, 2).numpy().astype(np.float64)
+    a = (_bits(inp["x"]), _bits(inp["W1"]), _bits(inp["W3"]), _bits(inp["W2"]), idx, w)
+    y1 = oracle.moe_ffn(*a, nthreads=1)
+    y4 = oracle.moe_ffn(*a, nthreads=4)
+    assert np.array_equal(y1, y4)
+    sub = np.array([12, 0, 5], dtype=np.int64)
+    ys = oracle.moe_ffn(*a, tokens=sub, nthreads=2)
+    assert np.array_equal(ys, y1[sub])
+    assert oracle.moe_ffn(*a, tokens=np.zeros(0, dtype=np.int64)).shape == (0, s.d)
+
+
+def pin_hand_worked_layer():
+    """A layer small enough to work by hand (tests/golden/hand_worked_layer.json)."""
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "hand_worked_layer.json")
+    g = json.load(open(path))
+    bf = lambda a: torch.tensor(a, dtype=torch.float32).to(torch.bfloat16)
+    x, Wg = bf(g["x"]), bf(g["Wg"])
+    W1, W3, W2 = bf(g["W1"]), bf(g["W3"]), bf(g["W2"])
+    sh = {n: _bits(bf(g[n])) for n in ("Ws1", "Ws3", "Ws2")}
+    for n in ("x", "Wg", "W1", "W3", "W2", "Ws1", "Ws3", "Ws2"):      # all exact in bf16
+        assert torch.equal(bf(g[n]).to(torch.float64), torch.tensor(g[n], dtype=torch.float64))
+    res = oracle.moe_layer(_bits(x), _bits(Wg), np.array(g["bias"], dtype=np.float32),
+                           _bits(W1), _bits(W3), _bits(W2), k=g["k"])
+    assert res["idx"].tolist() == g["expected_idx"]
+    # closed form of the worked example (derivation in the fixture)
+    silu = lambda z: z / (1.0 + math.exp(-z))
+    g1 = 1.0 / (1.0 + math.exp(-0.5))                  # softmax over logits (2, 1.5)
+    g2 = 1.0 - g1
+    h1 = silu(1.0) * 2.0                              # expert 1: g = 1, u = 2
+    h2 = silu(-2.0) * 3.0                             # expert 2: g = -2, u = 3
+    y = [g1 * h1 * 1.0 + g2 * h2 * 2.0, g1 * h1 * -1.0 + g2 * h2 * 0.5]
+    assert np.allclose(res["w"][0], [g1, g2], rtol=1e-15)
+    assert np.allclose(res["out"][0], y, rtol=1e-14, atol=0)
+    # the same token with the shared expert: g = 3, u = -1, W2s = (1, 2), gate 1
+    hs = silu(3.0) * -1.0
+    out_s = oracle.moe_ffn(_bits(x), _bits(W1), _bits(W3), _bits(W2), res["idx"], res["w"], shared=sh)
+    assert np.allclose(out_s[0], [y[0] + hs * 1.0, y[1] + hs * 2.0], rtol=1e-14, atol=0)
+
+
+def pin_empty_batch():
+    s, inp = _small_layer(T=0, E=3, k=2, seed=13)
+    res = oracle.moe_layer(_bits(inp["x"]), _bits(inp["Wg"]), inp["bias"].numpy(), _bits(inp["W1"]),
+                           _bits(inp["W3"]), _bits(inp["W2"]), k=2)
+    assert res["out"].shape == (0, s.d) and res["counts"].sum() == 0 and res["offsets"][-1] == 0
+
+
+ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

@@ -1,0 +1,65 @@
+"""Plant plausible mistakes in copies of the oracle and check that a pin catches each.
+
+Every mutant is a textual edit of moe_oracle.c compiled into a temporary
+library on the CPU; the real oracle is never modified.  A mutant that passes
+every pin would mean the pins cannot tell that mistake from the definition.
+"""
+
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+from tests import oracle_pins as P
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "moe_oracle.c")
+
+MUTANTS = {
+    "gate_and_up_swapped": ("h[r] = g / (1.0 + exp(-g)) * u;", "h[r] = u / (1.0 + exp(-u)) * g;"),
+    "silu_sign": ("h[r] = g / (1.0 + exp(-g)) * u;", "h[r] = g / (1.0 + exp(g)) * u;"),
+    "silu_dropped": ("h[r] = g / (1.0 + exp(-g)) * u;", "h[r] = g * u;"),
+    "down_proj_transposed": ("z += bf16_value(W2[c * f + r]) * h[r];", "z += bf16_value(W2[r * d + c]) * h[r];"),
+    "gate_weight_dropped": ("y[c] += gate * z;", "y[c] += z;"),
+    "bias_dropped": ("s += (double)bias[e];", "s += 0.0;"),
+    "widening_shift": ("uint32_t u = (uint32_t)bits << 16;", "uint32_t u = (uint32_t)bits << 15;"),
+    "tie_to_higher_index": ("return ia < ib;", "return ia > ib;"),
+    "nan_ranks_first": ("return bn;          /* the non-NaN one ranks first */", "return an;"),
+    "gates_unnormalised": ("w[t * k + j] = exp((double)row[idx[t * k + j]] - top) / z;",
+                           "w[t * k + j] = exp((double)row[idx[t * k + j]] - top);"),
+    "permutation_unstable": ("for (int64_t q = 0; q < P; q++) {      /* ascending q keeps each segment stable */",
+                             "for (int64_t q = P - 1; q >= 0; q--) {"),
+    "shared_expert_dropped": ("if (J->fs > 0)\n            expert_ffn_add", "if (0)\n            expert_ffn_add"),
+    "x_row_stride": ("const uint16_t *xt = J->x + t * J->d;", "const uint16_t *xt = J->x + t;"),
+}
+
+
+@pytest.fixture(scope="module")
+def tmpdir_mod():
+    with tempfile.TemporaryDirectory() as d:
+        yield d
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmpdir_mod):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    path_c = os.path.join(tmpdir_mod, f"{name}.c")
+    path_so = os.path.join(tmpdir_mod, f"lib_{name}.so")
+    open(path_c, "w").write(src.replace(old, new))
+    subprocess.run(["gcc", "-O2", "-std=c11", "-D_GNU_SOURCE", "-fPIC", "-shared", "-o", path_so, path_c,
+                    "-lm", "-lpthread"], check=True)
+    prev = oracle.use(oracle.load(path_so))
+    caught = []
+    try:
+        for pin in P.ALL_PINS:
+            try:
+                pin()
+            except (AssertionError, oracle.OracleError) as e:
+                caught.append(pin.__name__)
+                break
+    finally:
+        oracle.use(prev)
+    assert caught, f"no pin caught the planted mistake {name}"
