@@ -1,0 +1,110 @@
+// common.cuh -- types shared by the host entry points and the kernels:
+// device error bits, workspace layout, and the tile plan the scheduler reads.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace moe {
+
+using bf16 = __nv_bfloat16;
+
+// Sticky device error bits, OR-ed into the first word of the workspace.
+enum : uint32_t {
+    DEVERR_EXPERT_RANGE = 1u,   // a top-k expert id outside [0, E): that pair is dropped
+    DEVERR_TIMEOUT = 2u,        // a bounded wait inside a kernel gave up
+    DEVERR_NAN_LOGIT = 4u,      // a router logit was NaN (ranked below every number)
+};
+
+constexpr int kMaxExperts = 512;
+constexpr int kMaxTopK = 8;
+constexpr int kMaxGroups = kMaxExperts + 1;   // routed experts + the shared expert
+constexpr int kHistChunk = 4096;              // pairs per CTA in the multi-CTA histogram
+constexpr int kTileRows = 256;                // most tokens one tile carries (MMA N <= 256)
+
+// The tile plan, written by the plan step from the live histogram and read by
+// every role of the grouped GEMM.  A "block" is one expert (or the shared
+// expert) with at least one token; blocks are ordered by token count, largest
+// first, so the heaviest tiles are handed out first.  A block's n tokens are
+// cut into `units` equal chunks of `chunk` rows (a multiple of 16, <= 256);
+// each unit times each M-tile of the weights is one tile.
+struct PlanHeader {
+    int32_t n_blocks;
+    int32_t tiles1;     // tiles of the gate/up GEMM (M-tile = 64 rows of W1 and 64 of W3)
+    int32_t tiles2;     // tiles of the down GEMM (M-tile = 128 rows of W2)
+    int32_t n_max;      // widest tile (tokens) in this launch
+    int32_t pairs;      // routed pairs with a valid expert id (== offsets[E])
+    int32_t pad[3];
+};
+
+struct PlanArrays {
+    // Each array has kMaxGroups (+1 for prefixes) entries.
+    int32_t* group;     // expert id; E means the shared expert
+    int32_t* row0;      // first row of the block in the B operand
+    int32_t* rows;      // tokens in the block
+    int32_t* chunk;     // rows per unit
+    int32_t* units;
+    int32_t* tb1;       // tile prefix, gate/up GEMM  [n_blocks + 1]
+    int32_t* tb2;       // tile prefix, down GEMM     [n_blocks + 1]
+};
+
+constexpr size_t kPlanInts = 8 + 5 * kMaxGroups + 2 * (kMaxGroups + 1);
+
+__host__ __device__ inline PlanArrays plan_arrays(int32_t* base)
+{
+    PlanArrays a;
+    int32_t* p = base + 8;
+    a.group = p; p += kMaxGroups;
+    a.row0 = p; p += kMaxGroups;
+    a.rows = p; p += kMaxGroups;
+    a.chunk = p; p += kMaxGroups;
+    a.units = p; p += kMaxGroups;
+    a.tb1 = p; p += kMaxGroups + 1;
+    a.tb2 = p;
+    return a;
+}
+
+__host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace layout.  The control part (error word, plan, histogram scratch)
+// is all that moe_permute and moe_grouped_gemm need; moe_layer_forward also
+// keeps every intermediate of the layer in the workspace.
+struct WsLayout {
+    size_t err;            // uint32 sticky error word
+    size_t plan;           // int32[kPlanInts]
+    size_t block_counts;   // int32[hist_blocks * E]
+    size_t ctrl_end;
+    // layer intermediates
+    size_t logits, topk_idx, topk_w, counts, offsets, perm, inv_perm, xp, h, y_p, hs, ys;
+    size_t total;
+};
+
+__host__ __device__ inline int hist_blocks(int64_t P) { return (int)((P + kHistChunk - 1) / kHistChunk); }
+
+__host__ inline WsLayout ws_layout(int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, int64_t fs)
+{
+    WsLayout L{};
+    const int64_t P = T * k;
+    size_t o = 0;
+    L.err = o; o += 256;
+    L.plan = o; o = align_up(o + kPlanInts * 4, 256);
+    L.block_counts = o; o = align_up(o + (size_t)(hist_blocks(P) > 0 ? hist_blocks(P) : 1) * E * 4, 256);
+    L.ctrl_end = o;
+    L.logits = o; o = align_up(o + (size_t)T * E * 4, 256);
+    L.topk_idx = o; o = align_up(o + (size_t)P * 4, 256);
+    L.topk_w = o; o = align_up(o + (size_t)P * 4, 256);
+    L.counts = o; o = align_up(o + (size_t)E * 4, 256);
+    L.offsets = o; o = align_up(o + (size_t)(E + 1) * 4, 256);
+    L.perm = o; o = align_up(o + (size_t)P * 4, 256);
+    L.inv_perm = o; o = align_up(o + (size_t)P * 4, 256);
+    L.xp = o; o = align_up(o + (size_t)P * d * 2, 1024);
+    L.h = o; o = align_up(o + (size_t)P * f * 2, 1024);
+    L.y_p = o; o = align_up(o + (size_t)P * d * 2, 1024);
+    L.hs = o; o = align_up(o + (size_t)(fs > 0 ? T : 0) * fs * 2, 1024);
+    L.ys = o; o = align_up(o + (size_t)(fs > 0 ? T : 0) * d * 2, 1024);
+    L.total = o;
+    return L;
+}
+
+}  // namespace moe

@@ -1,0 +1,444 @@
+// moe_capi.cu -- the C ABI declared in include/moe.h: host-side argument
+// checks, workspace layout, TMA tensor maps and kernel launches.  No entry
+// point allocates, frees or synchronises (moe_get_device_error excepted).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "common.cuh"
+#include "grouped_gemm.cuh"
+#include "permute.cuh"
+#include "ptx.cuh"
+#include "route.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool ready = false;
+    bool supported = false;
+    int sm_count = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Per-device one-time set-up: architecture check, SM count, kernel attributes.
+int device_setup(DeviceState** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState& st = g_dev[dev];
+    if (!st.ready) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        st.supported = (major == 10 && minor == 0);
+        st.sm_count = sms;
+        if (st.supported) {
+            if (cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kGemmSmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kGemmSmemBytes) != cudaSuccess)
+                return MOE_ERR_CUDA;
+            if (!g_encode) {
+                cudaDriverEntryPointQueryResult q;
+                void* fn = nullptr;
+                if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+                        cudaSuccess ||
+                    q != cudaDriverEntryPointSuccess || !fn)
+                    return MOE_ERR_CUDA;
+                g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+            }
+        }
+        st.ready = true;
+    }
+    if (!st.supported) return MOE_ERR_DEVICE;
+    *out = &st;
+    return MOE_OK;
+}
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Common size checks.
+int check_sizes(int64_t T, int64_t d, int64_t E, int64_t k)
+{
+    if (T < 0 || d <= 0 || E < 1 || E > kMaxExperts || k < 1 || k > kMaxTopK || k > E) return MOE_ERR_ARG;
+    if (T * k >= (int64_t(1) << 31) || T >= (int64_t(1) << 31)) return MOE_ERR_ARG;
+    if (d % 64 != 0) return MOE_ERR_ALIGN;
+    return MOE_OK;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, inner] matrix; box = [64, box_rows],
+// 128-byte swizzle, zero fill outside the matrix.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows)
+{
+    if (rows == 0) rows = 1;   // a map needs one row; such a map is never read
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- step launchers
+int run_route(const bf16* x, const bf16* Wg, const float* bias, int T, int d, int E, int k, float* logits,
+              int32_t* idx, float* w, uint32_t* err, cudaStream_t st)
+{
+    const int max_tok_per_launch = 65535 * kRouterTokens;
+    for (int t0 = 0; t0 < T; t0 += max_tok_per_launch) {
+        const int nt = std::min(T - t0, max_tok_per_launch);
+        dim3 grid((E + kRouterWarps - 1) / kRouterWarps, (nt + kRouterTokens - 1) / kRouterTokens);
+        router_logits_kernel<<<grid, 256, 0, st>>>(x + (size_t)t0 * d, Wg, bias, nt, d, E, logits + (size_t)t0 * E);
+    }
+    topk_softmax_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, idx, w, err);
+    return launch_status();
+}
+
+int run_permute(const int32_t* idx, const bf16* x, int T, int d, int E, int k, int32_t* counts, int32_t* offsets,
+                int32_t* perm, int32_t* inv_perm, bf16* xp, uint32_t* err, int32_t* block_counts, int32_t* plan,
+                int f, int shared_rows, int fs, int sms, cudaStream_t st)
+{
+    const int64_t P = (int64_t)T * k;
+    const int nb = hist_blocks(P);
+    hist_kernel<<<nb, 512, 0, st>>>(idx, P, E, block_counts, err);
+    scan_kernel<<<1, 1024, 0, st>>>(block_counts, nb, E, counts, offsets, plan, f, d, shared_rows, fs);
+    scatter_kernel<<<nb, 256, 0, st>>>(idx, P, E, block_counts, perm, inv_perm);
+    const int64_t warps = P;
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, (int64_t)sms * 16));
+    gather_rows_kernel<<<blocks, 256, 0, st>>>(x, perm, offsets, E, k, d, xp);
+    return launch_status();
+}
+
+struct GemmOperands {
+    const bf16 *xp, *x, *W1, *W3, *W2, *Ws1, *Ws3, *Ws2;
+    const int32_t* perm;
+    const float* gate_w;
+    bf16 *h, *y_p, *hs, *ys;
+    int T, P, d, f, fs, E;
+};
+
+int run_gemms(const GemmOperands& o, const int32_t* plan, uint32_t* err, int sms, cudaStream_t st)
+{
+    CUtensorMap a0, a1, b, a0s, a1s, bs;
+    const uint64_t E = (uint64_t)o.E;
+    // gate/up GEMM: A = W1/W3 rows (16-row boxes), B = xp rows; shared: Ws1/Ws3 and x
+    if (!make_map(&a0, o.W1, o.d, E * o.f, 16) || !make_map(&a1, o.W3, o.d, E * o.f, 16) ||
+        !make_map(&b, o.xp, o.d, (uint64_t)o.P, 16))
+        return MOE_ERR_CUDA;
+    if (o.fs > 0) {
+        if (!make_map(&a0s, o.Ws1, o.d, o.fs, 16) || !make_map(&a1s, o.Ws3, o.d, o.fs, 16) ||
+            !make_map(&bs, o.x, o.d, (uint64_t)o.T, 16))
+            return MOE_ERR_CUDA;
+    } else {
+        a0s = a0;
+        a1s = a1;
+        bs = b;
+    }
+    GemmArgs g1{};
+    g1.plan = plan;
+    g1.E = o.E;
+    g1.M = o.f;
+    g1.M_shared = o.fs;
+    g1.K = o.d;
+    g1.K_shared = o.d;
+    g1.out = o.h;
+    g1.ld_out = o.f;
+    g1.out_shared = o.hs;
+    g1.ld_out_shared = o.fs;
+    g1.perm = o.perm;
+    g1.gate_w = o.gate_w;
+    g1.err = err;
+    grouped_gemm_kernel<true><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(a0, a1, b, a0s, a1s, bs, g1);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+
+    // down GEMM: A = W2 rows (128-row boxes), B = h rows; shared: Ws2 and hs
+    if (!make_map(&a0, o.W2, o.f, E * o.d, 128) || !make_map(&b, o.h, o.f, (uint64_t)o.P, 16)) return MOE_ERR_CUDA;
+    a1 = a0;
+    if (o.fs > 0) {
+        if (!make_map(&a0s, o.Ws2, o.fs, o.d, 128) || !make_map(&bs, o.hs, o.fs, (uint64_t)o.T, 16))
+            return MOE_ERR_CUDA;
+        a1s = a0s;
+    } else {
+        a0s = a0;
+        a1s = a0;
+        bs = b;
+    }
+    GemmArgs g2 = g1;
+    g2.M = o.d;
+    g2.M_shared = o.d;
+    g2.K = o.f;
+    g2.K_shared = o.fs;
+    g2.out = o.y_p;
+    g2.ld_out = o.d;
+    g2.out_shared = o.ys;
+    g2.ld_out_shared = o.d;
+    grouped_gemm_kernel<false><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(a0, a1, b, a0s, a1s, bs, g2);
+    return launch_status();
+}
+
+int run_combine(const bf16* y_p, const int32_t* inv_perm, const bf16* ys, int T, int k, int d, bf16* out,
+                cudaStream_t st)
+{
+    combine_kernel<<<T, 128, 0, st>>>(y_p, inv_perm, ys, T, k, d, out);
+    return launch_status();
+}
+
+template <class T>
+T* at(void* ws, size_t off)
+{
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_workspace_size(int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, int64_t f_shared, size_t* bytes)
+{
+    if (!bytes || T < 0 || d < 0 || f < 0 || E < 1 || E > kMaxExperts || k < 1 || k > kMaxTopK || f_shared < 0)
+        return MOE_ERR_ARG;
+    *bytes = ws_layout(T, d, f, E, k, f_shared).total;
+    return MOE_OK;
+}
+
+int moe_workspace_init(void* ws, size_t ws_bytes, int64_t T, int64_t E, int64_t k, void* stream)
+{
+    if (!ws || T < 0 || E < 1 || E > kMaxExperts || k < 1 || k > kMaxTopK) return MOE_ERR_ARG;
+    const WsLayout L = ws_layout(T, 0, 0, E, k, 0);
+    if (ws_bytes < L.ctrl_end) return MOE_ERR_WS;
+    return cudaMemsetAsync(ws, 0, L.ctrl_end, as_stream(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_route(const moe_bf16* x, const moe_bf16* Wg, const float* bias, int64_t T, int64_t d, int64_t E, int64_t k,
+              float* logits, int32_t* topk_idx, float* topk_w, void* ws, void* stream)
+{
+    int rc = check_sizes(T, d, E, k);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!x || !Wg || !logits || !topk_idx || !topk_w) return MOE_ERR_ARG;
+    if (!al16(x) || !al16(Wg)) return MOE_ERR_ALIGN;
+    DeviceState* dev;
+    if ((rc = device_setup(&dev))) return rc;
+    if (!ws) return MOE_ERR_ARG;
+    uint32_t* err = at<uint32_t>(ws, 0);
+    return run_route(reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(Wg), bias, (int)T, (int)d,
+                     (int)E, (int)k, logits, topk_idx, topk_w, err, as_stream(stream));
+}
+
+int moe_topk(const float* logits, int64_t T, int64_t E, int64_t k, int32_t* topk_idx, float* topk_w, void* ws,
+             void* stream)
+{
+    int rc = check_sizes(T, 64, E, k);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!logits || !topk_idx || !topk_w || !ws) return MOE_ERR_ARG;
+    DeviceState* dev;
+    if ((rc = device_setup(&dev))) return rc;
+    topk_softmax_kernel<<<(unsigned)((T + 7) / 8), 256, 0, as_stream(stream)>>>(logits, (int)T, (int)E, (int)k,
+                                                                                 topk_idx, topk_w, at<uint32_t>(ws, 0));
+    return launch_status();
+}
+
+int moe_permute(const int32_t* topk_idx, const moe_bf16* x, int64_t T, int64_t d, int64_t E, int64_t k,
+                int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm, moe_bf16* xp, void* ws,
+                size_t ws_bytes, void* stream)
+{
+    int rc = check_sizes(T, d, E, k);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!topk_idx || !x || !counts || !offsets || !perm || !inv_perm || !xp || !ws) return MOE_ERR_ARG;
+    if (!al16(x) || !al16(xp) || !al16(ws)) return MOE_ERR_ALIGN;
+    const WsLayout L = ws_layout(T, d, 0, E, k, 0);
+    if (ws_bytes < L.ctrl_end) return MOE_ERR_WS;
+    DeviceState* dev;
+    if ((rc = device_setup(&dev))) return rc;
+    return run_permute(topk_idx, reinterpret_cast<const bf16*>(x), (int)T, (int)d, (int)E, (int)k, counts, offsets,
+                       perm, inv_perm, reinterpret_cast<bf16*>(xp), at<uint32_t>(ws, L.err),
+                       at<int32_t>(ws, L.block_counts), nullptr, 0, 0, 0, dev->sm_count, as_stream(stream));
+}
+
+int moe_grouped_gemm(const moe_bf16* xp, const int32_t* counts, const int32_t* offsets, const int32_t* perm,
+                     const float* topk_w, const moe_bf16* W1, const moe_bf16* W3, const moe_bf16* W2, int64_t T,
+                     int64_t d, int64_t f, int64_t E, int64_t k, moe_bf16* h, moe_bf16* y_p, void* ws,
+                     size_t ws_bytes, void* stream)
+{
+    int rc = check_sizes(T, d, E, k);
+    if (rc) return rc;
+    if (f <= 0) return MOE_ERR_ARG;
+    if (f % 64 != 0) return MOE_ERR_ALIGN;
+    if (T == 0) return MOE_OK;
+    if (!xp || !counts || !offsets || !perm || !topk_w || !W1 || !W3 || !W2 || !h || !y_p || !ws) return MOE_ERR_ARG;
+    if (!al16(xp) || !al16(W1) || !al16(W3) || !al16(W2) || !al16(h) || !al16(y_p) || !al16(ws)) return MOE_ERR_ALIGN;
+    const WsLayout L = ws_layout(T, d, f, E, k, 0);
+    if (ws_bytes < L.ctrl_end) return MOE_ERR_WS;
+    DeviceState* dev;
+    if ((rc = device_setup(&dev))) return rc;
+    cudaStream_t st = as_stream(stream);
+    int32_t* plan = at<int32_t>(ws, L.plan);
+    plan_kernel<<<1, 1024, 0, st>>>(counts, offsets, (int)E, plan, (int)f, (int)d, 0, 0);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    GemmOperands o{};
+    o.xp = reinterpret_cast<const bf16*>(xp);
+    o.x = o.xp;
+    o.W1 = reinterpret_cast<const bf16*>(W1);
+    o.W3 = reinterpret_cast<const bf16*>(W3);
+    o.W2 = reinterpret_cast<const bf16*>(W2);
+    o.perm = perm;
+    o.gate_w = topk_w;
+    o.h = reinterpret_cast<bf16*>(h);
+    o.y_p = reinterpret_cast<bf16*>(y_p);
+    o.T = (int)T;
+    o.P = (int)(T * k);
+    o.d = (int)d;
+    o.f = (int)f;
+    o.fs = 0;
+    o.E = (int)E;
+    return run_gemms(o, plan, at<uint32_t>(ws, L.err), dev->sm_count, st);
+}
+
+int moe_combine(const moe_bf16* y_p, const int32_t* inv_perm, const moe_bf16* shared_out, int64_t T, int64_t k,
+                int64_t d, moe_bf16* out, void* stream)
+{
+    if (T < 0 || k < 1 || k > kMaxTopK || d <= 0 || T * k >= (int64_t(1) << 31)) return MOE_ERR_ARG;
+    if (d % 64 != 0) return MOE_ERR_ALIGN;
+    if (T == 0) return MOE_OK;
+    if (!y_p || !inv_perm || !out) return MOE_ERR_ARG;
+    if (!al16(y_p) || !al16(out) || (shared_out && !al16(shared_out))) return MOE_ERR_ALIGN;
+    DeviceState* dev;
+    int rc;
+    if ((rc = device_setup(&dev))) return rc;
+    return run_combine(reinterpret_cast<const bf16*>(y_p), inv_perm, reinterpret_cast<const bf16*>(shared_out),
+                       (int)T, (int)k, (int)d, reinterpret_cast<bf16*>(out), as_stream(stream));
+}
+
+int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const moe_bf16* W1,
+                      const moe_bf16* W3, const moe_bf16* W2, const moe_bf16* Ws1, const moe_bf16* Ws3,
+                      const moe_bf16* Ws2, int64_t f_shared, int64_t T, int64_t d, int64_t f, int64_t E, int64_t k,
+                      moe_bf16* out, void* ws, size_t ws_bytes, void* stream)
+{
+    int rc = check_sizes(T, d, E, k);
+    if (rc) return rc;
+    if (f <= 0 || f_shared < 0) return MOE_ERR_ARG;
+    if (f % 64 != 0 || f_shared % 64 != 0) return MOE_ERR_ALIGN;
+    if (T == 0) return MOE_OK;
+    if (!x || !Wg || !W1 || !W3 || !W2 || !out || !ws) return MOE_ERR_ARG;
+    if (f_shared > 0 && (!Ws1 || !Ws3 || !Ws2)) return MOE_ERR_ARG;
+    if (!al16(x) || !al16(Wg) || !al16(W1) || !al16(W3) || !al16(W2) || !al16(out) || !al16(ws)) return MOE_ERR_ALIGN;
+    if (f_shared > 0 && (!al16(Ws1) || !al16(Ws3) || !al16(Ws2))) return MOE_ERR_ALIGN;
+    const WsLayout L = ws_layout(T, d, f, E, k, f_shared);
+    if (ws_bytes < L.total) return MOE_ERR_WS;
+    DeviceState* dev;
+    if ((rc = device_setup(&dev))) return rc;
+    cudaStream_t st = as_stream(stream);
+    uint32_t* err = at<uint32_t>(ws, L.err);
+    int32_t* plan = at<int32_t>(ws, L.plan);
+    float* logits = at<float>(ws, L.logits);
+    int32_t* idx = at<int32_t>(ws, L.topk_idx);
+    float* w = at<float>(ws, L.topk_w);
+    int32_t* counts = at<int32_t>(ws, L.counts);
+    int32_t* offsets = at<int32_t>(ws, L.offsets);
+    int32_t* perm = at<int32_t>(ws, L.perm);
+    int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
+    bf16* xp = at<bf16>(ws, L.xp);
+    bf16* h = at<bf16>(ws, L.h);
+    bf16* y_p = at<bf16>(ws, L.y_p);
+    bf16* hs = f_shared > 0 ? at<bf16>(ws, L.hs) : nullptr;
+    bf16* ys = f_shared > 0 ? at<bf16>(ws, L.ys) : nullptr;
+    const bf16* xb = reinterpret_cast<const bf16*>(x);
+
+    if ((rc = run_route(xb, reinterpret_cast<const bf16*>(Wg), bias, (int)T, (int)d, (int)E, (int)k, logits, idx, w,
+                        err, st)))
+        return rc;
+    if ((rc = run_permute(idx, xb, (int)T, (int)d, (int)E, (int)k, counts, offsets, perm, inv_perm, xp, err,
+                          at<int32_t>(ws, L.block_counts), plan, (int)f, f_shared > 0 ? (int)T : 0, (int)f_shared,
+                          dev->sm_count, st)))
+        return rc;
+    GemmOperands o{};
+    o.xp = xp;
+    o.x = xb;
+    o.W1 = reinterpret_cast<const bf16*>(W1);
+    o.W3 = reinterpret_cast<const bf16*>(W3);
+    o.W2 = reinterpret_cast<const bf16*>(W2);
+    o.Ws1 = reinterpret_cast<const bf16*>(Ws1);
+    o.Ws3 = reinterpret_cast<const bf16*>(Ws3);
+    o.Ws2 = reinterpret_cast<const bf16*>(Ws2);
+    o.perm = perm;
+    o.gate_w = w;
+    o.h = h;
+    o.y_p = y_p;
+    o.hs = hs;
+    o.ys = ys;
+    o.T = (int)T;
+    o.P = (int)(T * k);
+    o.d = (int)d;
+    o.f = (int)f;
+    o.fs = (int)f_shared;
+    o.E = (int)E;
+    if ((rc = run_gemms(o, plan, err, dev->sm_count, st))) return rc;
+    return run_combine(y_p, inv_perm, ys, (int)T, (int)k, (int)d, reinterpret_cast<bf16*>(out), st);
+}
+
+int moe_workspace_tensor(void* ws, int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, int64_t f_shared, int which,
+                         void** ptr)
+{
+    if (!ws || !ptr || T < 0 || d < 0 || f < 0 || E < 1 || E > kMaxExperts || k < 1 || k > kMaxTopK || f_shared < 0)
+        return MOE_ERR_ARG;
+    const WsLayout L = ws_layout(T, d, f, E, k, f_shared);
+    const size_t offs[12] = {L.logits, L.topk_idx, L.topk_w, L.counts, L.offsets, L.perm,
+                             L.inv_perm, L.xp, L.h, L.y_p, L.hs, L.ys};
+    if (which < 0 || which >= 12) return MOE_ERR_ARG;
+    *ptr = static_cast<uint8_t*>(ws) + offs[which];
+    return MOE_OK;
+}
+
+int moe_get_device_error(const void* ws, uint32_t* code, void* stream)
+{
+    if (!ws || !code) return MOE_ERR_ARG;
+    cudaStream_t st = as_stream(stream);
+    if (cudaMemcpyAsync(code, ws, sizeof(uint32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
+    return cudaStreamSynchronize(st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_clear_device_error(void* ws, void* stream)
+{
+    if (!ws) return MOE_ERR_ARG;
+    return cudaMemsetAsync(ws, 0, sizeof(uint32_t), as_stream(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+const char* moe_status_string(int status)
+{
+    switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_ARG: return "invalid argument";
+    case MOE_ERR_ALIGN: return "size or pointer alignment";
+    case MOE_ERR_WS: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA launch or runtime error";
+    case MOE_ERR_DEVICE: return "device is not sm_100 (B200)";
+    default: return "unknown status";
+    }
+}
+
+}  // extern "C"

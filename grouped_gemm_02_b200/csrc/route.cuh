@@ -1,0 +1,145 @@
+// route.cuh -- router logits (S1) and warp-per-token top-k with softmax gates (S2).
+//
+// Router: L[t,e] = sum_c x[t,c] * Wg[e,c] + b[e], fp32 accumulation in a fixed
+// order (each lane sums its 8-element slices in ascending order, then a fixed
+// butterfly over the warp).  Top-k: the k largest fp32 logits of a token in
+// descending order, ties to the lower expert index, NaN below every number;
+// gates are the softmax over the k chosen logits (Decoding the Skew, abstract:
+// the routing distribution decided at run time drives the expert GEMMs).
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kRouterTokens = 8;     // tokens per warp in the router kernel
+constexpr int kRouterWarps = 8;      // experts per CTA (one per warp)
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&o)[8])
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        o[2 * i] = __uint_as_float(w[i] << 16);
+        o[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+// grid (ceil(E / 8), ceil(T / 8)), block 256: warp w of CTA (bx, by) computes
+// expert bx*8+w for tokens by*8 .. by*8+7.  Requires d % 8 == 0.
+__global__ void __launch_bounds__(256) router_logits_kernel(const bf16* __restrict__ x, const bf16* __restrict__ Wg,
+                                                            const float* __restrict__ bias, int T, int d, int E,
+                                                            float* __restrict__ L)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * kRouterWarps + warp;
+    const int t0 = blockIdx.y * kRouterTokens;
+    if (e >= E) return;
+    const int nt = min(kRouterTokens, T - t0);
+    float acc[kRouterTokens];
+#pragma unroll
+    for (int i = 0; i < kRouterTokens; i++) acc[i] = 0.f;
+    const uint4* wrow = reinterpret_cast<const uint4*>(Wg + (size_t)e * d);
+    const int nvec = d / 8;
+    for (int v = lane; v < nvec; v += 32) {
+        float wv[8];
+        bf16x8_to_f32(__ldg(wrow + v), wv);
+#pragma unroll
+        for (int i = 0; i < kRouterTokens; i++) {
+            if (i < nt) {
+                float xv[8];
+                bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + i) * d) + v), xv);
+#pragma unroll
+                for (int j = 0; j < 8; j++) acc[i] = fmaf(xv[j], wv[j], acc[i]);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < kRouterTokens; i++) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    }
+    if (lane == 0) {
+        const float b = bias ? bias[e] : 0.f;
+        for (int i = 0; i < nt; i++) L[(size_t)(t0 + i) * E + e] = acc[i] + b;
+    }
+}
+
+// Order-preserving key: larger logit -> larger key; -0 and +0 equal; NaN lowest (0).
+__device__ __forceinline__ uint32_t logit_key(float v)
+{
+    if (v != v) return 0u;
+    if (v == 0.f) v = 0.f;
+    const uint32_t u = __float_as_uint(v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// One warp per token; E <= 512 (16 logits per lane), k <= 8.
+__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ L, int T, int E, int k,
+                                                           int32_t* __restrict__ topk_idx,
+                                                           float* __restrict__ topk_w, uint32_t* __restrict__ err)
+{
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (warp >= T) return;
+    const float* row = L + (size_t)warp * E;
+    constexpr int kPer = kMaxExperts / 32;
+    // Packed candidate: key in the high word, (0xFFFF - expert) in the low word, so
+    // the maximum packed value is the largest logit with the lowest index.
+    uint64_t cand[kPer];
+    bool nan_seen = false;
+#pragma unroll
+    for (int i = 0; i < kPer; i++) {
+        const int e = lane + 32 * i;
+        if (e < E) {
+            const float v = row[e];
+            nan_seen |= (v != v);
+            cand[i] = ((uint64_t)logit_key(v) << 32) | (uint64_t)(0xFFFFu - (uint32_t)e);
+        } else {
+            cand[i] = 0;   // below every real candidate (real ones have a nonzero low word or key)
+        }
+    }
+    if (__any_sync(0xffffffffu, nan_seen) && lane == 0) atomicOr(err, DEVERR_NAN_LOGIT);
+    int chosen[kMaxTopK];
+    float vals[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; j++) {
+        if (j < k) {
+            uint64_t best = 0;
+#pragma unroll
+            for (int i = 0; i < kPer; i++) best = cand[i] > best ? cand[i] : best;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
+                best = other > best ? other : best;
+            }
+            const int e = (int)(0xFFFFu - (uint32_t)(best & 0xFFFFu));
+            chosen[j] = e;
+            vals[j] = row[e];
+#pragma unroll
+            for (int i = 0; i < kPer; i++)
+                if (lane + 32 * i == e) cand[i] = 0;   // taken
+        }
+    }
+    if (lane == 0) {
+        // softmax over the chosen logits, shifted by the largest (vals[0])
+        float ex[kMaxTopK];
+        float z = 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; j++) {
+            if (j < k) {
+                ex[j] = expf(vals[j] - vals[0]);
+                z += ex[j];
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; j++) {
+            if (j < k) {
+                topk_idx[(size_t)warp * k + j] = chosen[j];
+                topk_w[(size_t)warp * k + j] = ex[j] / z;
+            }
+        }
+    }
+}
+
+}  // namespace moe

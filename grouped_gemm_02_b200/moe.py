@@ -1,0 +1,235 @@
+"""Python binding of the C ABI in include/moe.h (argument marshalling only).
+
+Every function here takes torch tensors that already live on the current CUDA
+device, checks their dtype/shape/contiguity, and passes raw pointers to the
+entry point of the same name in libmoe_b200.so.  All arithmetic runs in the
+library's kernels; there is no fallback: if the library is missing or the
+device is not a B200, the call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+MOE_OK = 0
+STATUS = {0: "ok", -1: "invalid argument", -2: "size or pointer alignment", -3: "workspace too small",
+          -4: "CUDA launch or runtime error", -5: "device is not sm_100 (B200)"}
+DEVERR_EXPERT_RANGE, DEVERR_TIMEOUT, DEVERR_NAN_LOGIT = 1, 2, 4
+
+_lib: Optional[C.CDLL] = None
+
+EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_topk", "moe_permute",
+           "moe_grouped_gemm", "moe_combine", "moe_layer_forward", "moe_workspace_tensor",
+           "moe_get_device_error", "moe_clear_device_error", "moe_status_string")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {status} ({STATUS.get(status, 'unknown')})")
+        self.status = status
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def lib() -> C.CDLL:
+    """Load libmoe_b200.so (it must have been built: grouped_gemm_02_b200/build.py)."""
+    global _lib
+    if _lib is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"CUDA library {path} is missing; build it with grouped_gemm_02_b200/build.py")
+        L = C.CDLL(path)
+        i64, vp, sz = C.c_int64, C.c_void_p, C.c_size_t
+        sig = {
+            "moe_workspace_size": [i64, i64, i64, i64, i64, i64, C.POINTER(sz)],
+            "moe_workspace_init": [vp, sz, i64, i64, i64, vp],
+            "moe_route": [vp, vp, vp, i64, i64, i64, i64, vp, vp, vp, vp, vp],
+            "moe_topk": [vp, i64, i64, i64, vp, vp, vp, vp],
+            "moe_permute": [vp, vp, i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_grouped_gemm": [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, vp, vp, sz, vp],
+            "moe_combine": [vp, vp, vp, i64, i64, i64, vp, vp],
+            "moe_layer_forward": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, vp, vp, sz, vp],
+            "moe_workspace_tensor": [vp, i64, i64, i64, i64, i64, i64, C.c_int, C.POINTER(vp)],
+            "moe_get_device_error": [vp, C.POINTER(C.c_uint32), vp],
+            "moe_clear_device_error": [vp, vp],
+            "moe_status_string": [C.c_int],
+        }
+        for name, args in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = C.c_char_p if name == "moe_status_string" else C.c_int
+        _lib = L
+    return _lib
+
+
+def _call(name: str, *args) -> None:
+    rc = getattr(lib(), name)(*args)
+    if rc != MOE_OK:
+        raise MoEError(name, rc)
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    assert t.is_cuda and t.is_contiguous(), "tensors must be contiguous CUDA tensors"
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> C.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return C.c_void_p(s.cuda_stream)
+
+
+def _bf16(t: torch.Tensor, shape=None) -> torch.Tensor:
+    assert t.dtype == torch.bfloat16, f"expected bf16, got {t.dtype}"
+    if shape is not None:
+        assert tuple(t.shape) == tuple(shape), f"expected shape {shape}, got {tuple(t.shape)}"
+    return t
+
+
+# ---------------------------------------------------------------- workspace
+
+def moe_workspace_size(T: int, d: int, f: int, E: int, k: int, f_shared: int = 0) -> int:
+    n = C.c_size_t(0)
+    _call("moe_workspace_size", T, d, f, E, k, f_shared, C.byref(n))
+    return int(n.value)
+
+
+def moe_workspace_init(ws: torch.Tensor, T: int, E: int, k: int, stream=None) -> None:
+    _call("moe_workspace_init", _p(ws), ws.numel(), T, E, k, _stream(stream))
+
+
+def new_workspace(T: int, d: int, f: int, E: int, k: int, f_shared: int = 0, device=None, stream=None) -> torch.Tensor:
+    """A layer-sized workspace (a torch uint8 tensor owned by the caller), initialised."""
+    n = moe_workspace_size(T, d, f, E, k, f_shared)
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device or torch.device("cuda"))
+    moe_workspace_init(ws, T, E, k, stream)
+    return ws
+
+
+def moe_workspace_tensor(ws: torch.Tensor, T: int, d: int, f: int, E: int, k: int, f_shared: int, which: int) -> int:
+    out = C.c_void_p(0)
+    _call("moe_workspace_tensor", _p(ws), T, d, f, E, k, f_shared, which, C.byref(out))
+    return int(out.value or 0)
+
+
+def moe_get_device_error(ws: torch.Tensor, stream=None) -> int:
+    code = C.c_uint32(0)
+    _call("moe_get_device_error", _p(ws), C.byref(code), _stream(stream))
+    return int(code.value)
+
+
+def moe_clear_device_error(ws: torch.Tensor, stream=None) -> None:
+    _call("moe_clear_device_error", _p(ws), _stream(stream))
+
+
+def moe_status_string(status: int) -> str:
+    return lib().moe_status_string(status).decode()
+
+
+# ---------------------------------------------------------------- steps
+
+def moe_route(x: torch.Tensor, Wg: torch.Tensor, bias: Optional[torch.Tensor], k: int, ws: torch.Tensor,
+              logits=None, topk_idx=None, topk_w=None, stream=None):
+    T, d = x.shape
+    E = Wg.shape[0]
+    _bf16(x), _bf16(Wg, (E, d))
+    if bias is not None:
+        assert bias.dtype == torch.float32 and bias.shape == (E,)
+    dev = x.device
+    logits = torch.empty(T, E, dtype=torch.float32, device=dev) if logits is None else logits
+    topk_idx = torch.empty(T, k, dtype=torch.int32, device=dev) if topk_idx is None else topk_idx
+    topk_w = torch.empty(T, k, dtype=torch.float32, device=dev) if topk_w is None else topk_w
+    _call("moe_route", _p(x), _p(Wg), _p(bias), T, d, E, k, _p(logits), _p(topk_idx), _p(topk_w), _p(ws),
+          _stream(stream))
+    return logits, topk_idx, topk_w
+
+
+def moe_topk(logits: torch.Tensor, k: int, ws: torch.Tensor, topk_idx=None, topk_w=None, stream=None):
+    T, E = logits.shape
+    assert logits.dtype == torch.float32
+    topk_idx = torch.empty(T, k, dtype=torch.int32, device=logits.device) if topk_idx is None else topk_idx
+    topk_w = torch.empty(T, k, dtype=torch.float32, device=logits.device) if topk_w is None else topk_w
+    _call("moe_topk", _p(logits), T, E, k, _p(topk_idx), _p(topk_w), _p(ws), _stream(stream))
+    return topk_idx, topk_w
+
+
+def moe_permute(topk_idx: torch.Tensor, x: torch.Tensor, E: int, ws: torch.Tensor, stream=None):
+    T, k = topk_idx.shape
+    d = x.shape[1]
+    assert topk_idx.dtype == torch.int32
+    _bf16(x, (T, d))
+    dev = x.device
+    P = T * k
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(max(P, 1), dtype=torch.int32, device=dev)[:P]
+    inv = torch.empty(max(P, 1), dtype=torch.int32, device=dev)[:P]
+    xp = torch.zeros(P, d, dtype=torch.bfloat16, device=dev)
+    _call("moe_permute", _p(topk_idx), _p(x), T, d, E, k, _p(counts), _p(offsets), _p(perm), _p(inv), _p(xp),
+          _p(ws), ws.numel(), _stream(stream))
+    return counts, offsets, perm, inv, xp
+
+
+def moe_grouped_gemm(xp, counts, offsets, perm, topk_w, W1, W3, W2, T: int, k: int, ws: torch.Tensor,
+                     h=None, y_p=None, stream=None):
+    E, f, d = W1.shape
+    _bf16(W1), _bf16(W3, (E, f, d)), _bf16(W2, (E, d, f)), _bf16(xp, (T * k, d))
+    dev = xp.device
+    h = torch.zeros(T * k, f, dtype=torch.bfloat16, device=dev) if h is None else h
+    y_p = torch.zeros(T * k, d, dtype=torch.bfloat16, device=dev) if y_p is None else y_p
+    _call("moe_grouped_gemm", _p(xp), _p(counts), _p(offsets), _p(perm), _p(topk_w.reshape(-1)), _p(W1), _p(W3),
+          _p(W2), T, d, f, E, k, _p(h), _p(y_p), _p(ws), ws.numel(), _stream(stream))
+    return h, y_p
+
+
+def moe_combine(y_p, inv_perm, T: int, k: int, shared_out=None, out=None, stream=None):
+    d = y_p.shape[1]
+    out = torch.empty(T, d, dtype=torch.bfloat16, device=y_p.device) if out is None else out
+    _call("moe_combine", _p(y_p), _p(inv_perm), _p(shared_out), T, k, d, _p(out), _stream(stream))
+    return out
+
+
+def moe_layer_forward(x, Wg, bias, W1, W3, W2, k: int, ws: torch.Tensor, Ws1=None, Ws3=None, Ws2=None,
+                      out=None, stream=None):
+    T, d = x.shape
+    E, f, _ = W1.shape
+    fs = 0 if Ws1 is None else Ws1.shape[0]
+    _bf16(x), _bf16(Wg, (E, d)), _bf16(W1, (E, f, d)), _bf16(W3, (E, f, d)), _bf16(W2, (E, d, f))
+    out = torch.empty(T, d, dtype=torch.bfloat16, device=x.device) if out is None else out
+    _call("moe_layer_forward", _p(x), _p(Wg), _p(bias), _p(W1), _p(W3), _p(W2), _p(Ws1), _p(Ws3), _p(Ws2), fs,
+          T, d, f, E, k, _p(out), _p(ws), ws.numel(), _stream(stream))
+    return out
+
+
+WS_TENSORS = ("logits", "topk_idx", "topk_w", "counts", "offsets", "perm", "inv_perm", "xp", "h", "y_p", "hs", "ys")
+
+
+def workspace_views(ws: torch.Tensor, T: int, d: int, f: int, E: int, k: int, f_shared: int = 0):
+    """Torch views of the layer intermediates that moe_layer_forward leaves in ``ws``."""
+    P = T * k
+    shapes = {"logits": ((T, E), torch.float32), "topk_idx": ((T, k), torch.int32), "topk_w": ((T, k), torch.float32),
+              "counts": ((E,), torch.int32), "offsets": ((E + 1,), torch.int32), "perm": ((P,), torch.int32),
+              "inv_perm": ((P,), torch.int32), "xp": ((P, d), torch.bfloat16), "h": ((P, f), torch.bfloat16),
+              "y_p": ((P, d), torch.bfloat16), "hs": ((T if f_shared else 0, f_shared), torch.bfloat16),
+              "ys": ((T if f_shared else 0, d), torch.bfloat16)}
+    base = ws.data_ptr()
+    views = {}
+    for i, name in enumerate(WS_TENSORS):
+        ptr = moe_workspace_tensor(ws, T, d, f, E, k, f_shared, i)
+        shape, dt = shapes[name]
+        n = 1
+        for s in shape:
+            n *= s
+        off = ptr - base
+        nbytes = n * torch.tensor([], dtype=dt).element_size()
+        views[name] = ws[off:off + nbytes].view(dt).view(shape)
+    return views

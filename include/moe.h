@@ -1,0 +1,163 @@
+/*
+ * moe.h -- C ABI of the B200 fused Mixture-of-Experts layer forward.
+ *
+ * The layer (Decoding the Skew: Distribution-Aware MoE Inference with Adaptive
+ * Kernel Dispatch, abstract; GC-MoE: Overlapping Expert-Parallel Token Dispatch
+ * with FP8/FP4 Grouped GEMM via CUDA Green Contexts, abstract):
+ *
+ *   L      = x Wg^T + b                         router logits            (moe_route)
+ *   idx, w = top-k of L, softmax over the k     gating                   (moe_route / moe_topk)
+ *   counts, offsets, perm, inv_perm, xp         histogram, scan, stable  (moe_permute)
+ *                                               permute and row gather
+ *   h   = silu(xp W1[e]^T) * (xp W3[e]^T)       grouped expert GEMMs     (moe_grouped_gemm)
+ *   y_p = w[perm] * (h W2[e]^T)
+ *   out = sum_j y_p[inv_perm[t*k+j]] (+ shared) deterministic combine    (moe_combine)
+ *
+ * and moe_layer_forward, which runs all of it with every intermediate in a
+ * caller-owned workspace.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers are DEVICE pointers unless stated otherwise.  bf16 tensors are
+ *   passed as raw 16-bit patterns (moe_bf16).  Every tensor is dense and
+ *   row-major (nn.Linear storage): x [T,d], Wg [E,d], W1/W3 [E,f,d],
+ *   W2 [E,d,f], Ws1/Ws3 [f_shared,d], Ws2 [d,f_shared], out [T,d].
+ * - Pair q = t*k + j is token t's j-th choice (j = 0 is the largest logit).
+ * - The caller owns every buffer.  No entry point allocates or frees memory,
+ *   and none synchronises the host, except moe_get_device_error.
+ * - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *   stream) on the current device, in call order.
+ * - Limits: 1 <= E <= 512, 1 <= k <= min(8, E), T >= 0, T*k < 2^31;
+ *   d and f (and f_shared) are multiples of 64; every pointer is 16-byte
+ *   aligned.  T == 0 returns MOE_OK and enqueues nothing.
+ * - Return value: MOE_OK, or a negative status found on the host before any
+ *   work is enqueued (MOE_ERR_ARG, MOE_ERR_ALIGN, MOE_ERR_WS), or
+ *   MOE_ERR_CUDA when a launch fails.  Conditions only the device can see
+ *   (an expert id outside [0, E), a NaN logit, a kernel wait that timed out)
+ *   set bits in a sticky error word inside the workspace; read them with
+ *   moe_get_device_error.
+ * - Kernels: hand-written for sm_100a (B200).  A device of another
+ *   architecture gives MOE_ERR_DEVICE.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef uint16_t moe_bf16;
+
+#define MOE_OK 0
+#define MOE_ERR_ARG (-1)     /* null pointer, size out of range */
+#define MOE_ERR_ALIGN (-2)   /* d, f or f_shared not a multiple of 64, or a pointer not 16-byte aligned */
+#define MOE_ERR_WS (-3)      /* workspace smaller than moe_workspace_size reports */
+#define MOE_ERR_CUDA (-4)    /* a CUDA launch or attribute call failed */
+#define MOE_ERR_DEVICE (-5)  /* current device is not sm_100 */
+
+/* Device error bits (OR-ed, sticky until moe_clear_device_error). */
+#define MOE_DEVERR_EXPERT_RANGE 1u  /* an expert id outside [0, E): that pair was dropped */
+#define MOE_DEVERR_TIMEOUT 2u       /* a bounded wait inside a kernel gave up; outputs are invalid */
+#define MOE_DEVERR_NAN_LOGIT 4u     /* a router logit was NaN; it ranked below every number */
+
+/* Bytes of workspace moe_layer_forward needs for these sizes (f_shared = 0:
+ * no shared expert).  The control part of it (error word, tile plan,
+ * histogram scratch) is also what moe_permute and moe_grouped_gemm need; a
+ * layer-sized workspace serves every entry point.  Returns MOE_ERR_ARG on
+ * negative sizes. */
+MOE_API int moe_workspace_size(int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, int64_t f_shared, size_t *bytes);
+
+/* Zero the workspace's control part (error word, plan).  Call once on a new
+ * workspace before its first use; enqueued on `stream`. */
+MOE_API int moe_workspace_init(void *ws, size_t ws_bytes, int64_t T, int64_t E, int64_t k, void *stream);
+
+/* Router (Decoding the Skew, abstract: the runtime routing distribution).
+ * logits [T,E] fp32 = x Wg^T + bias (bias [E] fp32, may be NULL), summed in
+ * fp32 in a fixed order; then, per token, the k largest logits in descending
+ * order (ties: lower expert id; NaN ranks lowest) -> topk_idx [T,k] int32,
+ * and softmax over those k logits -> topk_w [T,k] fp32.  `ws` (required)
+ * supplies the device error word. */
+MOE_API int moe_route(const moe_bf16 *x, const moe_bf16 *Wg, const float *bias, int64_t T, int64_t d, int64_t E, int64_t k,
+              float *logits, int32_t *topk_idx, float *topk_w, void *ws, void *stream);
+
+/* The top-k/softmax step of moe_route alone, on caller-provided fp32 logits
+ * [T,E]; same ordering and gate definition.  `ws` (required) supplies the
+ * device error word. */
+MOE_API int moe_topk(const float *logits, int64_t T, int64_t E, int64_t k, int32_t *topk_idx, float *topk_w, void *ws,
+             void *stream);
+
+/* Histogram, exclusive scan, stable permutation and row gather (Decoding the
+ * Skew, abstract: the live per-expert histogram kept on the GPU; Weave,
+ * abstract: token dispatch).  counts [E] = pairs per expert; offsets [E+1] =
+ * exclusive scan (offsets[E] = valid pairs); pairs are ordered expert-major and,
+ * inside an expert, by ascending q: perm [T*k] (position -> q), inv_perm [T*k]
+ * (q -> position); xp [T*k, d] row pos = x row perm[pos]/k (rows past
+ * offsets[E] are left untouched).  A pair whose expert id is outside [0, E) is
+ * dropped (inv_perm = -1, device error bit).  Needs a workspace of at least
+ * moe_workspace_size(T,d,f,E,k,0) for any f (its control part). */
+MOE_API int moe_permute(const int32_t *topk_idx, const moe_bf16 *x, int64_t T, int64_t d, int64_t E, int64_t k,
+                int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv_perm, moe_bf16 *xp, void *ws,
+                size_t ws_bytes, void *stream);
+
+/* Grouped expert GEMMs (Decoding the Skew, abstract: sparse expert GEMMs
+ * whose shapes follow the live routing histogram; GC-MoE, abstract:
+ * operand-swapped tcgen05 MMA with a fused SwiGLU).  From counts [E] and
+ * offsets [E+1] on the device it builds the tile plan in `ws` (tile widths
+ * chosen per expert from its count, heaviest experts first) and then, for
+ * every expert e and row r in [offsets[e], offsets[e+1]):
+ *   h [r, :]  = bf16( silu(xp[r] W1[e]^T) * (xp[r] W3[e]^T) )   h   [T*k, f]
+ *   y_p[r, :] = bf16( topk_w[perm[r]] * (h[r] W2[e]^T) )        y_p [T*k, d]
+ * with fp32 accumulation (topk_w is read as [T*k], indexed by q).  Rows past
+ * offsets[E] are left untouched. */
+MOE_API int moe_grouped_gemm(const moe_bf16 *xp, const int32_t *counts, const int32_t *offsets, const int32_t *perm,
+                     const float *topk_w, const moe_bf16 *W1, const moe_bf16 *W3, const moe_bf16 *W2, int64_t T,
+                     int64_t d, int64_t f, int64_t E, int64_t k, moe_bf16 *h, moe_bf16 *y_p, void *ws,
+                     size_t ws_bytes, void *stream);
+
+/* Deterministic combine: out[t,:] = bf16( sum_{j<k} y_p[inv_perm[t*k+j], :]
+ * (+ shared_out[t,:]) ), summed in fp32 in ascending j, no atomics.
+ * inv_perm < 0 adds nothing.  shared_out [T,d] may be NULL. */
+MOE_API int moe_combine(const moe_bf16 *y_p, const int32_t *inv_perm, const moe_bf16 *shared_out, int64_t T, int64_t k,
+                int64_t d, moe_bf16 *out, void *stream);
+
+/* The whole layer: route -> permute -> grouped GEMMs -> combine, with the
+ * optional always-on shared expert (GC-MoE, abstract: optional shared experts)
+ * Ws1/Ws3 [f_shared,d], Ws2 [d,f_shared] (all NULL and f_shared = 0 for none)
+ * added with gate 1.  out [T,d].  Every intermediate lives in `ws`
+ * (moe_workspace_size bytes).  Bit-identical to calling the steps one by one
+ * on the same inputs. */
+MOE_API int moe_layer_forward(const moe_bf16 *x, const moe_bf16 *Wg, const float *bias, const moe_bf16 *W1,
+                      const moe_bf16 *W3, const moe_bf16 *W2, const moe_bf16 *Ws1, const moe_bf16 *Ws3,
+                      const moe_bf16 *Ws2, int64_t f_shared, int64_t T, int64_t d, int64_t f, int64_t E, int64_t k,
+                      moe_bf16 *out, void *ws, size_t ws_bytes, void *stream);
+
+/* Device pointers of the layer intermediates inside a layer workspace
+ * (which: 0 logits, 1 topk_idx, 2 topk_w, 3 counts, 4 offsets, 5 perm,
+ * 6 inv_perm, 7 xp, 8 h, 9 y_p, 10 hs, 11 ys).  Host-only arithmetic. */
+MOE_API int moe_workspace_tensor(void *ws, int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, int64_t f_shared,
+                         int which, void **ptr);
+
+/* Copies the sticky device error word to *code (host int).  Synchronises
+ * `stream`. */
+MOE_API int moe_get_device_error(const void *ws, uint32_t *code, void *stream);
+
+/* Clears the sticky device error word; enqueued on `stream`. */
+MOE_API int moe_clear_device_error(void *ws, void *stream);
+
+/* Human-readable name of a status code. */
+MOE_API const char *moe_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,94 @@
+"""The C-ABI library without a GPU: it loads, exports every declared entry
+point, sizes workspaces, and rejects bad arguments on the host before any
+CUDA call."""
+
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from grouped_gemm_02_b200 import build, moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return moe.lib()
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"MOE_API\s+(?:const\s+)?\w+\s*\*?\s*(moe_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_api():
+    names = declared_symbols()
+    assert set(moe.EXPORTS) == set(names), names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), f"{name} missing from {moe.library_path()}"
+    out = os.popen(f"nm -D --defined-only {moe.library_path()}").read()
+    exported = set(re.findall(r" T (moe_\w+)", out))
+    assert exported == set(declared_symbols())
+
+
+def test_status_strings(L):
+    assert moe.moe_status_string(0) == "ok"
+    assert "workspace" in moe.moe_status_string(-3)
+
+
+def test_workspace_size_monotone(L):
+    a = moe.moe_workspace_size(32, 2048, 1024, 64, 8)
+    b = moe.moe_workspace_size(64, 2048, 1024, 64, 8)
+    c = moe.moe_workspace_size(32, 2048, 1024, 64, 8, 2048)
+    assert 0 < a < b and a < c
+    assert a % 256 == 0
+    # the big intermediates are counted: xp, y_p [P,d] and h [P,f] in bf16
+    P = 32 * 8
+    assert a >= P * 2048 * 2 * 2 + P * 1024 * 2
+    with pytest.raises(moe.MoEError):
+        moe.moe_workspace_size(-1, 2048, 1024, 64, 8)
+    with pytest.raises(moe.MoEError):
+        moe.moe_workspace_size(1, 2048, 1024, 513, 8)
+
+
+FAKE = C.c_void_p(0x10000)   # never dereferenced: every call below fails its host checks first
+
+
+def _layer(L, **kw):
+    a = dict(x=FAKE, Wg=FAKE, bias=None, W1=FAKE, W3=FAKE, W2=FAKE, Ws1=None, Ws3=None, Ws2=None, fs=0,
+             T=4, d=128, f=128, E=4, k=2, out=FAKE, ws=FAKE, ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    return L.moe_layer_forward(a["x"], a["Wg"], a["bias"], a["W1"], a["W3"], a["W2"], a["Ws1"], a["Ws3"],
+                               a["Ws2"], a["fs"], a["T"], a["d"], a["f"], a["E"], a["k"], a["out"], a["ws"],
+                               a["ws_bytes"], a["stream"])
+
+
+def test_host_argument_checks(L):
+    assert _layer(L, x=None) == -1
+    assert _layer(L, k=5, E=4) == -1          # k > E
+    assert _layer(L, k=9, E=16) == -1         # k > 8
+    assert _layer(L, E=513) == -1
+    assert _layer(L, T=-1) == -1
+    assert _layer(L, d=100) == -2             # d not a multiple of 64
+    assert _layer(L, f=96) == -2
+    assert _layer(L, x=C.c_void_p(0x10008)) == -2   # misaligned pointer
+    assert _layer(L, ws_bytes=1024) == -3
+    assert _layer(L, fs=64) == -1             # shared expert without weights
+    assert _layer(L, T=0) == 0                # empty batch: nothing to do
+    assert L.moe_combine(None, FAKE, None, 4, 2, 128, FAKE, None) == -1
+    assert L.moe_topk(FAKE, 4, 8, 9, FAKE, FAKE, FAKE, None) == -1
+    assert L.moe_permute(FAKE, FAKE, 4, 128, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, None) == -3
+
+
+def test_product_path_refuses_missing_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(moe, "_lib", None)
+    monkeypatch.setattr(moe, "library_path", lambda: str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        moe.lib()
