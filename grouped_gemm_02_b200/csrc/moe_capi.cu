@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/moe.h"
@@ -32,6 +33,16 @@ struct DeviceState {
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::atomic<int64_t> g_launches{0};
+thread_local cudaEvent_t t_phase[6] = {};
+thread_local bool t_phase_armed = false;
+
+inline void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+inline void phase_mark(bool on, int i, cudaStream_t st)
+{
+    if (on) cudaEventRecord(t_phase[i], st);
+}
 
 // Per-device one-time set-up: architecture check, SM count, kernel attributes.
 int device_setup(DeviceState** out)
@@ -112,8 +123,10 @@ int run_route(const bf16* x, const bf16* Wg, const float* bias, int T, int d, in
         const int nt = std::min(T - t0, max_tok_per_launch);
         dim3 grid((E + kRouterWarps - 1) / kRouterWarps, (nt + kRouterTokens - 1) / kRouterTokens);
         router_logits_kernel<<<grid, 256, 0, st>>>(x + (size_t)t0 * d, Wg, bias, nt, d, E, logits + (size_t)t0 * E);
+        count_launches(1);
     }
     topk_softmax_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, idx, w, err);
+    count_launches(1);
     return launch_status();
 }
 
@@ -129,6 +142,7 @@ int run_permute(const int32_t* idx, const bf16* x, int T, int d, int E, int k, i
     const int64_t warps = P;
     const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, (int64_t)sms * 16));
     gather_rows_kernel<<<blocks, 256, 0, st>>>(x, perm, offsets, E, k, d, xp);
+    count_launches(4);
     return launch_status();
 }
 
@@ -140,7 +154,8 @@ struct GemmOperands {
     int T, P, d, f, fs, E;
 };
 
-int run_gemms(const GemmOperands& o, const int32_t* plan, uint32_t* err, int sms, cudaStream_t st)
+int run_gemms(const GemmOperands& o, const int32_t* plan, uint32_t* err, int sms, cudaStream_t st,
+              bool prof = false)
 {
     CUtensorMap a0, a1, b, a0s, a1s, bs;
     const uint64_t E = (uint64_t)o.E;
@@ -172,7 +187,9 @@ int run_gemms(const GemmOperands& o, const int32_t* plan, uint32_t* err, int sms
     g1.gate_w = o.gate_w;
     g1.err = err;
     grouped_gemm_kernel<true><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(a0, a1, b, a0s, a1s, bs, g1);
+    count_launches(1);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    phase_mark(prof, 3, st);
 
     // down GEMM: A = W2 rows (128-row boxes), B = h rows; shared: Ws2 and hs
     if (!make_map(&a0, o.W2, o.f, E * o.d, 128) || !make_map(&b, o.h, o.f, (uint64_t)o.P, 16)) return MOE_ERR_CUDA;
@@ -196,6 +213,7 @@ int run_gemms(const GemmOperands& o, const int32_t* plan, uint32_t* err, int sms
     g2.out_shared = o.ys;
     g2.ld_out_shared = o.d;
     grouped_gemm_kernel<false><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(a0, a1, b, a0s, a1s, bs, g2);
+    count_launches(1);
     return launch_status();
 }
 
@@ -203,6 +221,7 @@ int run_combine(const bf16* y_p, const int32_t* inv_perm, const bf16* ys, int T,
                 cudaStream_t st)
 {
     combine_kernel<<<T, 128, 0, st>>>(y_p, inv_perm, ys, T, k, d, out);
+    count_launches(1);
     return launch_status();
 }
 
@@ -259,6 +278,7 @@ int moe_topk(const float* logits, int64_t T, int64_t E, int64_t k, int32_t* topk
     if ((rc = device_setup(&dev))) return rc;
     topk_softmax_kernel<<<(unsigned)((T + 7) / 8), 256, 0, as_stream(stream)>>>(logits, (int)T, (int)E, (int)k,
                                                                                  topk_idx, topk_w, at<uint32_t>(ws, 0));
+    count_launches(1);
     return launch_status();
 }
 
@@ -299,6 +319,7 @@ int moe_grouped_gemm(const moe_bf16* xp, const int32_t* counts, const int32_t* o
     cudaStream_t st = as_stream(stream);
     int32_t* plan = at<int32_t>(ws, L.plan);
     plan_kernel<<<1, 1024, 0, st>>>(counts, offsets, (int)E, plan, (int)f, (int)d, 0, 0);
+    count_launches(1);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     GemmOperands o{};
     o.xp = reinterpret_cast<const bf16*>(xp);
@@ -369,9 +390,13 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     bf16* ys = f_shared > 0 ? at<bf16>(ws, L.ys) : nullptr;
     const bf16* xb = reinterpret_cast<const bf16*>(x);
 
+    const bool prof = t_phase_armed;   // the armed events serve this call only
+    t_phase_armed = false;
+    phase_mark(prof, 0, st);
     if ((rc = run_route(xb, reinterpret_cast<const bf16*>(Wg), bias, (int)T, (int)d, (int)E, (int)k, logits, idx, w,
                         err, st)))
         return rc;
+    phase_mark(prof, 1, st);
     if ((rc = run_permute(idx, xb, (int)T, (int)d, (int)E, (int)k, counts, offsets, perm, inv_perm, xp, err,
                           at<int32_t>(ws, L.block_counts), plan, (int)f, f_shared > 0 ? (int)T : 0, (int)f_shared,
                           dev->sm_count, st)))
@@ -397,9 +422,30 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     o.f = (int)f;
     o.fs = (int)f_shared;
     o.E = (int)E;
-    if ((rc = run_gemms(o, plan, err, dev->sm_count, st))) return rc;
-    return run_combine(y_p, inv_perm, ys, (int)T, (int)k, (int)d, reinterpret_cast<bf16*>(out), st);
+    phase_mark(prof, 2, st);
+    if ((rc = run_gemms(o, plan, err, dev->sm_count, st, prof))) return rc;
+    phase_mark(prof, 4, st);
+    rc = run_combine(y_p, inv_perm, ys, (int)T, (int)k, (int)d, reinterpret_cast<bf16*>(out), st);
+    phase_mark(prof, 5, st);
+    return rc;
 }
+
+int moe_record_phase_events(void* const* events, int n)
+{
+    if (n == 0) {
+        t_phase_armed = false;
+        return MOE_OK;
+    }
+    if (!events || n < 6) return MOE_ERR_ARG;
+    for (int i = 0; i < 6; i++) {
+        if (!events[i]) return MOE_ERR_ARG;
+        t_phase[i] = reinterpret_cast<cudaEvent_t>(events[i]);
+    }
+    t_phase_armed = true;
+    return MOE_OK;
+}
+
+int64_t moe_launch_counter(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int moe_workspace_tensor(void* ws, int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, int64_t f_shared, int which,
                          void** ptr)

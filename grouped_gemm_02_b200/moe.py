@@ -26,7 +26,8 @@ _lib: Optional[C.CDLL] = None
 
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_topk", "moe_permute",
            "moe_grouped_gemm", "moe_combine", "moe_layer_forward", "moe_workspace_tensor",
-           "moe_get_device_error", "moe_clear_device_error", "moe_status_string")
+           "moe_record_phase_events", "moe_launch_counter", "moe_get_device_error", "moe_clear_device_error",
+           "moe_status_string")
 
 
 class MoEError(RuntimeError):
@@ -61,11 +62,13 @@ def lib() -> C.CDLL:
             "moe_get_device_error": [vp, C.POINTER(C.c_uint32), vp],
             "moe_clear_device_error": [vp, vp],
             "moe_status_string": [C.c_int],
+            "moe_record_phase_events": [C.POINTER(vp), C.c_int],
+            "moe_launch_counter": [],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
             fn.argtypes = args
-            fn.restype = C.c_char_p if name == "moe_status_string" else C.c_int
+            fn.restype = {"moe_status_string": C.c_char_p, "moe_launch_counter": C.c_int64}.get(name, C.c_int)
         _lib = L
     return _lib
 
@@ -129,6 +132,25 @@ def moe_get_device_error(ws: torch.Tensor, stream=None) -> int:
 
 def moe_clear_device_error(ws: torch.Tensor, stream=None) -> None:
     _call("moe_clear_device_error", _p(ws), _stream(stream))
+
+
+def moe_record_phase_events(events) -> None:
+    """Arm per-phase timing of the next moe_layer_forward on this thread: six
+    torch.cuda.Event(enable_timing=True) recorded before the router, the
+    permutation, the gate/up GEMM, the down GEMM and the combine, and after it."""
+    if not events:
+        _call("moe_record_phase_events", None, 0)
+        return
+    for e in events:
+        if not e.cuda_event:        # torch creates the CUDA event lazily, on its first record
+            e.record()
+    arr = (C.c_void_p * len(events))(*[C.c_void_p(e.cuda_event) for e in events])
+    _call("moe_record_phase_events", arr, len(events))
+
+
+def moe_launch_counter() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(lib().moe_launch_counter())
 
 
 def moe_status_string(status: int) -> str:

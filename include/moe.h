@@ -140,6 +140,16 @@ MOE_API int moe_layer_forward(const moe_bf16 *x, const moe_bf16 *Wg, const float
                       const moe_bf16 *Ws2, int64_t f_shared, int64_t T, int64_t d, int64_t f, int64_t E, int64_t k,
                       moe_bf16 *out, void *ws, size_t ws_bytes, void *stream);
 
+/* Per-phase timing of the next moe_layer_forward call made on this host
+ * thread: `events` holds n >= 6 cudaEvent_t handles; that call records
+ * events[0..5] on its stream before the router, the permutation, the gate/up
+ * GEMM, the down GEMM and the combine, and after the combine.  The array is
+ * used once (the call after it records nothing).  n = 0 cancels. */
+MOE_API int moe_record_phase_events(void *const *events, int n);
+
+/* Number of kernels this library has launched in this process so far. */
+MOE_API int64_t moe_launch_counter(void);
+
 /* Device pointers of the layer intermediates inside a layer workspace
  * (which: 0 logits, 1 topk_idx, 2 topk_w, 3 counts, 4 offsets, 5 perm,
  * 6 inv_perm, 7 xp, 8 h, 9 y_p, 10 hs, 11 ys).  Host-only arithmetic. */

@@ -1,0 +1,111 @@
+"""Host-side logic of bench.py: rank environment, max-over-ranks timing across
+two gloo processes, algorithmic byte counts, the traffic record's source check,
+and clock-sample parsing."""
+
+import json
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+from grouped_gemm_02_b200 import workload as wl
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    r, lr, w = bench.dist_env()
+    got = bench.reduce_max(10.0 + 5.0 * rank, w)
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((r, lr, w, got))
+
+
+def test_reduce_max_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res == [(0, 0, 2, 15.0), (1, 1, 2, 15.0)]
+
+
+def test_dist_env_defaults(monkeypatch):
+    for v in ("RANK", "LOCAL_RANK", "WORLD_SIZE"):
+        monkeypatch.delenv(v, raising=False)
+    assert bench.dist_env() == (0, 0, 1)
+    assert bench.reduce_max(3.5, 1) == 3.5
+
+
+def test_algorithmic_counts():
+    s = wl.DECODE64
+    counts = np.zeros(s.E, dtype=np.int64)
+    counts[:4] = [100, 100, 50, 6]
+    a = bench.algorithmic(s, counts)
+    assert a["active"] == 4 and a["pairs"] == 256
+    assert a["w_act"] == 4 * 3 * s.d * s.f * 2
+    assert a["flops"] == 6.0 * 256 * s.d * s.f
+    assert a["g1_bytes"] == 4 * 2 * s.f * s.d * 2 + 256 * s.d * 2 + 256 * s.f * 2
+    sh = wl.DEEPSEEK_V3.with_(T=8)
+    c2 = np.zeros(sh.E, dtype=np.int64)
+    c2[0] = 64
+    b = bench.algorithmic(sh, c2)
+    assert b["w_act"] == (1 * 3 + 3) * sh.d * sh.f * 2          # f_shared == f here
+
+
+def test_traffic_record_tied_to_kernel_source(tmp_path, monkeypatch):
+    rec = {"workload": "w", "source_sha": bench.kernel_source_hash(), "dram_bytes_per_launch": 123}
+    p = tmp_path / "t.json"
+    p.write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(p))
+    assert bench.committed_traffic("w") == 123
+    assert bench.committed_traffic("other") is None
+    rec["source_sha"] = "0" * 16
+    p.write_text(json.dumps(rec))
+    assert bench.committed_traffic("w") is None
+
+
+def test_clock_sampler_parse(tmp_path):
+    cs = bench.ClockSampler.__new__(bench.ClockSampler)
+    cs.path = str(tmp_path / "c.csv")
+    lines = ["0, 1965, 1965, 700.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+             "0, 1800, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+             "0, 1700, 1965, 998.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active"]
+    open(cs.path, "w").write("\n".join(lines) + "\n")
+
+    class P:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    cs.proc = P()
+    r = cs.stop()
+    assert r["sm_mhz"] == 1800.0 and r["sm_max_mhz"] == 1965.0 and r["reasons"] == ["sw_power_cap"]
+
+
+def test_workload_label_and_parse():
+    class A:
+        workload, T, alpha = "deepseek_v3", 64, 0.05
+    s = bench.parse_workload(A)
+    assert s.T == 64 and s.alpha == 0.05 and s.f_shared == 2048
+    assert "shared_f=2048" in bench.workload_label(s)
