@@ -488,3 +488,68 @@ const char* moe_status_string(int status)
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- permutation without a workspace
+// Some callers cannot hand this library a workspace: they run inside a host
+// framework that owns every device allocation and forbids allocating in its
+// execute path, or in a latency-critical loop where cudaMalloc's implicit
+// device synchronisation is not acceptable.  moe_permute_noalloc serves them:
+// its only scratch (the per-CTA expert counters of the histogram and a device
+// error word) lives in the static device array below, which every GPU that
+// loads this library holds until the process exits.
+namespace {
+
+constexpr int kNoAllocCounters = 65536;   // 256 KiB of int32 per-CTA counters (hist_blocks(T*k) * E)
+
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocCounters + 64];
+
+struct NoAllocState {
+    bool ready = false;
+    int32_t* scratch = nullptr;   // device address of g_noalloc_scratch on this device
+};
+NoAllocState g_noalloc[kMaxDevices];
+
+// Device address of the static scratch on the current device, looked up once
+// per device.  In host code g_noalloc_scratch names a host-side stand-in, so
+// only this address may be handed to a kernel.
+int noalloc_scratch(int32_t** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    NoAllocState& st = g_noalloc[dev];
+    if (!st.ready) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+        st.scratch = static_cast<int32_t*>(p);
+        st.ready = true;
+    }
+    *out = st.scratch;
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" int moe_permute_noalloc(const int32_t* topk_idx, const moe_bf16* x, int64_t T, int64_t d, int64_t E,
+                                   int64_t k, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,
+                                   moe_bf16* xp, void* stream)
+{
+    int rc = check_sizes(T, d, E, k);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!topk_idx || !x || !counts || !offsets || !perm || !inv_perm || !xp) return MOE_ERR_ARG;
+    if (!al16(x) || !al16(xp)) return MOE_ERR_ALIGN;
+    if ((int64_t)hist_blocks(T * k) * E > kNoAllocCounters) return MOE_ERR_WS;
+    DeviceState* dev;
+    if ((rc = device_setup(&dev))) return rc;
+    int32_t* scratch = nullptr;
+    if ((rc = noalloc_scratch(&scratch))) return rc;
+    cudaStream_t st = as_stream(stream);
+    // The array keeps the previous call's contents: the error word must start at
+    // zero; the counters are fully rewritten by the histogram kernel.
+    uint32_t* err = reinterpret_cast<uint32_t*>(scratch + kNoAllocCounters);
+    if (cudaMemsetAsync(err, 0, sizeof(uint32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+    return run_permute(topk_idx, reinterpret_cast<const bf16*>(x), (int)T, (int)d, (int)E, (int)k, counts, offsets,
+                       perm, inv_perm, reinterpret_cast<bf16*>(xp), err, scratch, nullptr, 0, 0, 0, dev->sm_count,
+                       st);
+}

@@ -25,7 +25,7 @@ DEVERR_EXPERT_RANGE, DEVERR_TIMEOUT, DEVERR_NAN_LOGIT = 1, 2, 4
 _lib: Optional[C.CDLL] = None
 
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_topk", "moe_permute",
-           "moe_grouped_gemm", "moe_combine", "moe_layer_forward", "moe_workspace_tensor",
+           "moe_permute_noalloc", "moe_grouped_gemm", "moe_combine", "moe_layer_forward", "moe_workspace_tensor",
            "moe_record_phase_events", "moe_launch_counter", "moe_get_device_error", "moe_clear_device_error",
            "moe_status_string")
 

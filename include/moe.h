@@ -108,6 +108,27 @@ MOE_API int moe_permute(const int32_t *topk_idx, const moe_bf16 *x, int64_t T, i
                 int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv_perm, moe_bf16 *xp, void *ws,
                 size_t ws_bytes, void *stream);
 
+/* moe_permute without a workspace, for callers that cannot allocate device
+ * memory for one: code hosted by a framework that owns all device memory and
+ * forbids allocation in its execute path, or latency-critical loops that
+ * cannot afford cudaMalloc's implicit device synchronisation.  The pages have
+ * no counterpart to this entry point; it exists for such callers only.
+ * Same inputs, outputs and ordering as moe_permute.  Its scratch is a static
+ * device array of 256 KiB (65536 int32 histogram counters plus an error word)
+ * that each GPU loading this library keeps until the process exits; the
+ * entry point allocates and frees nothing.  Sizes with
+ * ceil(T*k / 4096) * E > 65536 are rejected with MOE_ERR_WS.  The first call
+ * on a device looks up the array's device address (cudaGetSymbolAddress) for
+ * that device; make that first call before any stream capture.  Every call
+ * shares the one array, so calls whose work overlaps on the GPU (other
+ * streams, other host threads) race and must be serialised by the caller.
+ * Out-of-range expert ids are dropped as in moe_permute; with no workspace
+ * there is no error word to read, so a dropped pair shows as
+ * offsets[E] < T*k. */
+MOE_API int moe_permute_noalloc(const int32_t *topk_idx, const moe_bf16 *x, int64_t T, int64_t d, int64_t E,
+                                int64_t k, int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv_perm,
+                                moe_bf16 *xp, void *stream);
+
 /* Grouped expert GEMMs (Decoding the Skew, abstract: sparse expert GEMMs
  * whose shapes follow the live routing histogram; GC-MoE, abstract:
  * operand-swapped tcgen05 MMA with a fused SwiGLU).  From counts [E] and
