@@ -67,6 +67,46 @@ __host__ __device__ inline PlanArrays plan_arrays(int32_t* base)
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// How the tensor-core router covers a [T, E] x d problem: tokens in `units`
+// chunks of `chunk` rows (<= 256, a multiple of 16), experts in `mt` tiles of
+// 128, and -- when units * mt tiles alone would leave most SMs idle -- the
+// d-loop split into `splits` ranges of `kb_per` 64-wide blocks, so that one
+// tile streams about kRouterTileBytes of Wg and x; the top-k step adds the
+// fp32 partial sums in a fixed order.  The split depends on the sizes only
+// (not on the device), so the workspace size and every result bit do too.
+constexpr int kRouterTargetCtas = 148;
+constexpr int64_t kRouterTileBytes = 256 * 1024;
+
+struct RouterSplit {
+    int units, chunk, mt, splits, kb_per, tiles;
+};
+
+__host__ __device__ inline RouterSplit router_split(int64_t T, int64_t d, int64_t E)
+{
+    RouterSplit r{};
+    if (T <= 0 || d <= 0 || E <= 0) return r;
+    const int nk = (int)((d + 63) / 64);
+    r.mt = (int)((E + 127) / 128);
+    r.units = (int)((T + 255) / 256);
+    const int per = (int)((T + r.units - 1) / r.units);
+    r.chunk = (per + 15) / 16 * 16;
+    const int base = r.mt * r.units;
+    r.kb_per = nk;
+    r.splits = 1;
+    if (base < kRouterTargetCtas) {
+        const int64_t rows = (E < 128 ? E : 128) + r.chunk;          // weight rows + token rows per tile
+        int64_t want = (rows * d * 2 + kRouterTileBytes - 1) / kRouterTileBytes;
+        const int64_t cap = kRouterTargetCtas / base;
+        if (want > cap) want = cap;
+        if (want > nk) want = nk;
+        if (want < 1) want = 1;
+        r.kb_per = (int)((nk + want - 1) / want);
+        r.splits = (nk + r.kb_per - 1) / r.kb_per;
+    }
+    r.tiles = base * r.splits;
+    return r;
+}
+
 // Workspace layout.  The control part (error word, plan, histogram scratch)
 // is all that moe_permute and moe_grouped_gemm need; moe_layer_forward also
 // keeps every intermediate of the layer in the workspace.
@@ -74,6 +114,7 @@ struct WsLayout {
     size_t err;            // uint32 sticky error word
     size_t plan;           // int32[kPlanInts]
     size_t block_counts;   // int32[hist_blocks * E]
+    size_t router_partials;  // fp32[splits, T, E] when the router splits K
     size_t ctrl_end;
     // layer intermediates
     size_t logits, topk_idx, topk_w, counts, offsets, perm, inv_perm, xp, h, y_p, hs, ys;
@@ -90,6 +131,8 @@ __host__ inline WsLayout ws_layout(int64_t T, int64_t d, int64_t f, int64_t E, i
     L.err = o; o += 256;
     L.plan = o; o = align_up(o + kPlanInts * 4, 256);
     L.block_counts = o; o = align_up(o + (size_t)(hist_blocks(P) > 0 ? hist_blocks(P) : 1) * E * 4, 256);
+    const RouterSplit rs = router_split(T, d, E);
+    L.router_partials = o; o = align_up(o + (rs.splits > 1 ? (size_t)rs.splits * T * E * 4 : 0), 256);
     L.ctrl_end = o;
     L.logits = o; o = align_up(o + (size_t)T * E * 4, 256);
     L.topk_idx = o; o = align_up(o + (size_t)P * 4, 256);

@@ -1,31 +1,47 @@
-// grouped_gemm.cuh -- persistent tcgen05/TMEM grouped expert GEMM fed by TMA (S5, S5', S6, S7).
+// grouped_gemm.cuh -- persistent tcgen05/TMEM grouped GEMM fed by TMA (S1 on
+// tensor cores, S5, S5', S6, S7).
 //
-// The two expert GEMMs of the layer (Decoding the Skew, abstract: "sparse
-// expert GEMMs whose shapes vary with the runtime routing distribution";
-// GC-MoE, abstract: operand-swapped tcgen05 MMA with a fused SwiGLU and
-// optional shared experts):
+// The expert GEMMs of the layer (Decoding the Skew, abstract: "sparse expert
+// GEMMs whose shapes vary with the runtime routing distribution"; GC-MoE,
+// abstract: operand-swapped tcgen05 MMA with a fused SwiGLU and optional
+// shared experts):
 //
-//   gate/up (GATED):  h[r, :]   = silu(xp[r] W1[e]^T) * (xp[r] W3[e]^T)   -> bf16
-//   down:             y_p[r, :] = w[perm[r]] * (h[r] W2[e]^T)             -> bf16
+//   MODE_GATED:  h[r, :]   = silu(xp[r] W1[e]^T) * (xp[r] W3[e]^T)   -> bf16
+//   MODE_DOWN:   y_p[r, :] = w[perm[r]] * (h[r] W2[e]^T)             -> bf16
 //
-// for every row r of expert e's segment.  The MMA is operand-swapped: the
-// weights fill the M = 128 slot and the expert's tokens the N slot (16..256,
-// chosen per expert from its live count by the plan), so a decode expert with
-// 3 tokens costs one 16-wide MMA column block while a hot expert gets 256-wide
-// tiles.  For the gate/up GEMM one A tile holds 64 rows of W1 and the same 64
-// rows of W3, interleaved 16 rows at a time (rows 32q..32q+15 = W1, 32q+16..
-// 32q+31 = W3 for f rows 16q..16q+15), so that in TMEM lane quadrant q the
-// lanes 0-15 hold the gate and lanes 16-31 the up projection of the same f
-// rows; one shuffle pairs them in the epilogue.
+// for every row r of expert e's segment, and the router as a dense GEMM:
+//
+//   MODE_ROUTER: L[t, e] = x[t] Wg[e]^T (+ b[e])                     -> fp32
+//
+// split over K into fp32 partial sums when the token count alone cannot
+// fill the SMs (the top-k kernel then adds the partials in a fixed order).
+//
+// The MMA is operand-swapped: the weights fill the M = 128 slot and the tokens
+// the N slot (16..256, chosen per expert from its live count by the plan), so
+// a decode expert with 3 tokens costs one 16-wide MMA column block while a hot
+// expert gets 256-wide tiles.  For the gate/up GEMM one A tile holds 64 rows
+// of W1 and the same 64 rows of W3, interleaved 16 rows at a time (rows
+// 32q..32q+15 = W1, 32q+16..32q+31 = W3 for f rows 16q..16q+15), so that in
+// TMEM lane quadrant q the lanes 0-15 hold the gate and lanes 16-31 the up
+// projection of the same f rows; one shuffle pairs them in the epilogue.
 //
 // Warp roles (192 threads, one CTA per SM, persistent over the tile list):
 //   warp 0     TMA producer (one elected lane) -> ring of smem stages
 //   warp 1     TMEM allocator + MMA issuer (one elected lane)
-//   warps 2-5  epilogue: tcgen05.ld -> SwiGLU or gate scale -> bf16 -> global
+//   warps 2-5  epilogue: tcgen05.ld -> SwiGLU / gate scale / bias -> global
 // Two TMEM accumulators of 256 columns let the epilogue of tile i overlap the
-// mainloop of tile i+1.  Every wait is bounded: on timeout the kernel sets
-// DEVERR_TIMEOUT, drains its own copies and MMAs (again bounded), frees TMEM
-// and returns.
+// mainloop of tile i+1.
+//
+// Programmatic dependent launch: the kernel is launched so that it may start
+// while the previous kernel on the stream finishes.  Weight tiles (A) do not
+// depend on that kernel, so the producer fills the first ring stages with them
+// before griddepcontrol.wait; token tiles (B) are loaded after it.  Every
+// kernel of the layer waits before it triggers its dependents, so data made
+// two or more kernels earlier (the tile plan, perm, gates) is complete when a
+// kernel starts.
+//
+// Every wait is bounded: on timeout the kernel sets DEVERR_TIMEOUT, drains its
+// own copies and MMAs (again bounded), frees TMEM and returns.
 #pragma once
 
 #include <cuda.h>
@@ -34,6 +50,10 @@
 #include "ptx.cuh"
 
 namespace moe {
+
+constexpr int MODE_DOWN = 0;
+constexpr int MODE_GATED = 1;
+constexpr int MODE_ROUTER = 2;
 
 constexpr int kGemmThreads = 192;
 constexpr int kBlockK = 64;                          // bf16 elements per 128-byte swizzle row
@@ -47,28 +67,60 @@ constexpr uint32_t kTmemCols = 512;                  // 2 accumulators x 256 col
 constexpr uint64_t kWaitTimeoutNs = 1000000000ull;   // 1 s
 
 struct GemmArgs {
-    const int32_t* plan;        // PlanHeader + PlanArrays (device)
+    const int32_t* plan;        // PlanHeader + PlanArrays (device); unused by MODE_ROUTER
+    int plan_ready;             // plan written >= 2 kernels earlier: readable before griddepcontrol.wait
     int E;                      // routed experts; group E is the shared expert
-    int M, M_shared;            // output rows per expert: f (gate/up) or d (down); shared: f_shared or d
-    int K, K_shared;            // reduction length: d (gate/up) or f / f_shared (down)
+    int M, M_shared;            // output rows per group: f (gate/up) or d (down) or E (router); shared: f_shared or d
+    int K, K_shared;            // reduction length: d (gate/up, router) or f / f_shared (down)
     bf16* out;                  // h [pairs, f] or y_p [pairs, d]
     int ld_out;
     bf16* out_shared;           // hs [T, f_shared] or ys [T, d]
     int ld_out_shared;
     const int32_t* perm;        // down GEMM: gate of row r is gate_w[perm[r]]
     const float* gate_w;
+    // MODE_ROUTER: tokens split into `units` chunks of `chunk` rows, `mt` tiles of
+    // 128 experts, K split into `splits` ranges of `kb_per` 64-wide blocks.
+    int T, units, chunk, mt, splits, kb_per;
+    float* out_f32;             // splits == 1: logits [T, E] (+ bias); else partials [splits, T, E]
+    const float* bias;          // may be null
     uint32_t* err;
 };
 
 struct Tile {
-    int group, m, row0, rows, n_mma, K;
+    int group, m, row0, rows, n_mma, K, kb0, kb1, split;
     bool shared;
 };
 
-__device__ __forceinline__ Tile decode_tile(const int32_t* plan, int nb, int t, bool gated, const GemmArgs& a)
+template <int MODE>
+__device__ __forceinline__ int total_tiles(const GemmArgs& a, const PlanHeader* hdr)
 {
-    const PlanArrays pa = plan_arrays(const_cast<int32_t*>(plan));
-    const int32_t* tb = gated ? pa.tb1 : pa.tb2;
+    if (MODE == MODE_ROUTER) return a.units * a.mt * a.splits;
+    return MODE == MODE_GATED ? hdr->tiles1 : hdr->tiles2;
+}
+
+template <int MODE>
+__device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a)
+{
+    Tile tl;
+    if (MODE == MODE_ROUTER) {
+        const int per_unit = a.mt * a.splits;
+        const int u = t / per_unit;
+        const int r = t - u * per_unit;
+        tl.m = r / a.splits;
+        tl.split = r - tl.m * a.splits;
+        tl.group = 0;
+        tl.shared = false;
+        tl.row0 = u * a.chunk;
+        tl.rows = min(a.chunk, a.T - tl.row0);
+        tl.n_mma = (tl.rows + 15) & ~15;
+        tl.K = a.K;
+        const int nk = (a.K + kBlockK - 1) / kBlockK;
+        tl.kb0 = tl.split * a.kb_per;
+        tl.kb1 = min(nk, tl.kb0 + a.kb_per);
+        return tl;
+    }
+    const PlanArrays pa = plan_arrays(const_cast<int32_t*>(a.plan));
+    const int32_t* tb = MODE == MODE_GATED ? pa.tb1 : pa.tb2;
     int lo = 0, hi = nb - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -78,7 +130,6 @@ __device__ __forceinline__ Tile decode_tile(const int32_t* plan, int nb, int t, 
     const int local = t - __ldg(tb + lo);
     const int units = __ldg(pa.units + lo);
     const int chunk = __ldg(pa.chunk + lo);
-    Tile tl;
     tl.group = __ldg(pa.group + lo);
     tl.shared = tl.group == a.E;
     tl.m = local / units;
@@ -88,6 +139,9 @@ __device__ __forceinline__ Tile decode_tile(const int32_t* plan, int nb, int t, 
     tl.row0 = __ldg(pa.row0 + lo) + start;
     tl.n_mma = (tl.rows + 15) & ~15;
     tl.K = tl.shared ? a.K_shared : a.K;
+    tl.kb0 = 0;
+    tl.kb1 = (tl.K + kBlockK - 1) / kBlockK;
+    tl.split = 0;
     return tl;
 }
 
@@ -123,7 +177,74 @@ __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, Smem
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
-template <bool GATED>
+// Walks this CTA's (tile, k-block) sequence in order; shared by the two
+// passes of the producer.
+struct KIter {
+    int t, kb;
+    Tile tl;
+};
+
+template <int MODE>
+__device__ __forceinline__ bool kiter_begin(KIter& it, int nb, int total, const GemmArgs& a)
+{
+    it.t = blockIdx.x;
+    while (it.t < total) {
+        it.tl = decode_tile<MODE>(nb, it.t, a);
+        if (it.tl.kb0 < it.tl.kb1) {
+            it.kb = it.tl.kb0;
+            return true;
+        }
+        it.t += gridDim.x;
+    }
+    return false;
+}
+
+template <int MODE>
+__device__ __forceinline__ bool kiter_next(KIter& it, int nb, int total, const GemmArgs& a)
+{
+    if (++it.kb < it.tl.kb1) return true;
+    for (it.t += gridDim.x; it.t < total; it.t += gridDim.x) {
+        it.tl = decode_tile<MODE>(nb, it.t, a);
+        if (it.tl.kb0 < it.tl.kb1) {
+            it.kb = it.tl.kb0;
+            return true;
+        }
+    }
+    return false;
+}
+
+template <int MODE>
+__device__ __forceinline__ void issue_a(const KIter& it, uint32_t a_dst, uint32_t full, const CUtensorMap* mA0,
+                                        const CUtensorMap* mA1, const CUtensorMap* mA0s, const CUtensorMap* mA1s,
+                                        const GemmArgs& a, uint64_t pol)
+{
+    const Tile& tl = it.tl;
+    const int kc = it.kb * kBlockK;
+    if (MODE == MODE_GATED) {
+        const CUtensorMap* a0 = tl.shared ? mA0s : mA0;
+        const CUtensorMap* a1 = tl.shared ? mA1s : mA1;
+        const int a_row = (tl.shared ? 0 : tl.group * a.M) + tl.m * 64;
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            ptx::tma_load_2d(a_dst + (32 * q) * 128, a0, full, kc, a_row + 16 * q, pol);
+            ptx::tma_load_2d(a_dst + (32 * q + 16) * 128, a1, full, kc, a_row + 16 * q, pol);
+        }
+    } else {
+        const CUtensorMap* a0 = tl.shared ? mA0s : mA0;
+        const int a_row = (MODE == MODE_ROUTER || tl.shared ? 0 : tl.group * a.M) + tl.m * 128;
+        ptx::tma_load_2d(a_dst, a0, full, kc, a_row, pol);
+    }
+}
+
+__device__ __forceinline__ void issue_b(const Tile& tl, int kb, uint32_t b_dst, uint32_t full, const CUtensorMap* b,
+                                        uint64_t pol)
+{
+    const int kc = kb * kBlockK;
+    for (int i = 0; i < tl.n_mma / 16; i++)
+        ptx::tma_load_2d(b_dst + i * 16 * kBRowBytes, b, full, kc, tl.row0 + 16 * i, pol);
+}
+
+template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mA1,
                         const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mA0s,
@@ -136,10 +257,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t ring = ptx::smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+    // The plan comes from an earlier kernel; when that kernel is the one right
+    // before this launch, wait for it before reading anything.
+    const bool waited_early = MODE != MODE_ROUTER && !args.plan_ready;
+    if (waited_early) ptx::grid_dep_wait();
+
     const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(args.plan);
-    const int nb = hdr->n_blocks;
-    const int total = GATED ? hdr->tiles1 : hdr->tiles2;
-    const int n_max = max(16, hdr->n_max);
+    const int nb = MODE == MODE_ROUTER ? 0 : hdr->n_blocks;
+    const int total = total_tiles<MODE>(args, hdr);
+    const int n_max = MODE == MODE_ROUTER ? max(16, (min(args.chunk, args.T) + 15) & ~15) : max(16, hdr->n_max);
     const uint32_t stage_bytes = kATileBytes + (uint32_t)n_max * kBRowBytes;
     const int stages = min(kMaxStages, (int)(kRingBytes / stage_bytes));
 
@@ -160,7 +286,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == 0 && lane == 0) {
         ptx::prefetch_tensormap(&mA0);
         ptx::prefetch_tensormap(&mB);
-        if (GATED) ptx::prefetch_tensormap(&mA1);
+        if (MODE == MODE_GATED) ptx::prefetch_tensormap(&mA1);
     }
     if (warp == 1) {
         ptx::tmem_alloc(ptx::smem_u32(&ctl->tmem_base), kTmemCols);
@@ -175,47 +301,52 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // ------------------------------------------------------------ TMA producer
         if (ptx::elect_one()) {
             const uint64_t pol = ptx::policy_evict_normal();
-            int s = 0;
-            uint32_t ph = 0;
             uint32_t armed = 0, armed_ph = 0;   // slots with a load issued, and its phase
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const Tile tl = decode_tile(args.plan, nb, t, GATED, args);
-                const CUtensorMap* a0 = tl.shared ? &mA0s : &mA0;
-                const CUtensorMap* a1 = tl.shared ? &mA1s : &mA1;
-                const CUtensorMap* b = tl.shared ? &mBs : &mB;
-                const int Mrows = tl.shared ? args.M_shared : args.M;
-                const int a_row = (tl.shared ? 0 : tl.group * Mrows) + tl.m * (GATED ? 64 : 128);
-                const uint32_t tx = kATileBytes + (uint32_t)tl.n_mma * kBRowBytes;
-                const int nk = (tl.K + kBlockK - 1) / kBlockK;
-                for (int kb = 0; kb < nk; kb++) {
+            // pass 1 (before the dependency wait): weight tiles into the free stages
+            int pre = 0;
+            if (!waited_early) {
+                KIter it;
+                bool more = kiter_begin<MODE>(it, nb, total, args);
+                while (more && pre < stages) {
+                    const uint32_t full = ptx::smem_u32(&ctl->full[pre]);
+                    ptx::mbar_arrive_expect_tx(full, kATileBytes + (uint32_t)it.tl.n_mma * kBRowBytes);
+                    armed |= 1u << pre;
+                    issue_a<MODE>(it, ring + (uint32_t)pre * stage_bytes, full, &mA0, &mA1, &mA0s, &mA1s, args, pol);
+                    ++pre;
+                    more = kiter_next<MODE>(it, nb, total, args);
+                }
+                ptx::grid_dep_wait();
+            }
+            ptx::grid_dep_launch();
+            // pass 2: the same sequence again; the first `pre` stages only need their token tiles
+            int s = 0, n = 0;
+            uint32_t ph = 0;
+            KIter it;
+            bool more = kiter_begin<MODE>(it, nb, total, args);
+            while (more) {
+                const uint32_t a_dst = ring + (uint32_t)s * stage_bytes;
+                const uint32_t full = ptx::smem_u32(&ctl->full[s]);
+                const CUtensorMap* b = it.tl.shared ? &mBs : &mB;
+                if (n < pre) {
+                    issue_b(it.tl, it.kb, a_dst + kATileBytes, full, b, pol);
+                } else {
                     if (!bounded_wait(ptx::smem_u32(&ctl->empty[s]), ph ^ 1u, ctl, args.err)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t full = ptx::smem_u32(&ctl->full[s]);
-                    ptx::mbar_arrive_expect_tx(full, tx);
+                    ptx::mbar_arrive_expect_tx(full, kATileBytes + (uint32_t)it.tl.n_mma * kBRowBytes);
                     armed |= 1u << s;
                     armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
-                    const uint32_t a_dst = ring + (uint32_t)s * stage_bytes;
-                    const uint32_t b_dst = a_dst + kATileBytes;
-                    const int kc = kb * kBlockK;
-                    if (GATED) {
-#pragma unroll
-                        for (int q = 0; q < 4; q++) {
-                            ptx::tma_load_2d(a_dst + (32 * q) * 128, a0, full, kc, a_row + 16 * q, pol);
-                            ptx::tma_load_2d(a_dst + (32 * q + 16) * 128, a1, full, kc, a_row + 16 * q, pol);
-                        }
-                    } else {
-                        ptx::tma_load_2d(a_dst, a0, full, kc, a_row, pol);
-                    }
-                    for (int i = 0; i < tl.n_mma / 16; i++)
-                        ptx::tma_load_2d(b_dst + i * 16 * kBRowBytes, b, full, kc, tl.row0 + 16 * i, pol);
-                    if (++s == stages) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
+                    issue_a<MODE>(it, a_dst, full, &mA0, &mA1, &mA0s, &mA1s, args, pol);
+                    issue_b(it.tl, it.kb, a_dst + kATileBytes, full, b, pol);
                 }
+                ++n;
+                if (++s == stages) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+                more = kiter_next<MODE>(it, nb, total, args);
             }
             if (!ok) {
                 // drain: wait (bounded) for every load this thread issued
@@ -238,7 +369,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t aph = 0;
             bool ok = true, issued = false;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const Tile tl = decode_tile(args.plan, nb, t, GATED, args);
+                const Tile tl = decode_tile<MODE>(nb, t, args);
+                if (tl.kb0 >= tl.kb1) continue;
                 if (!bounded_wait(ptx::smem_u32(&ctl->tempty[acc]), aph ^ 1u, ctl, args.err)) {
                     ok = false;
                     break;
@@ -246,8 +378,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 ptx::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)acc * 256u;
                 const uint32_t idesc = ptx::idesc_bf16_f32(128, (uint32_t)tl.n_mma);
-                const int nk = (tl.K + kBlockK - 1) / kBlockK;
-                for (int kb = 0; kb < nk; kb++) {
+                for (int kb = tl.kb0; kb < tl.kb1; kb++) {
                     if (!bounded_wait(ptx::smem_u32(&ctl->full[s]), ph, ctl, args.err)) {
                         ok = false;
                         break;
@@ -258,7 +389,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < kBlockK / 16; kk++) {
                         ptx::mma_bf16_ss(d_tmem, ptx::sw128_kmajor_desc(a_addr + kk * 32),
-                                         ptx::sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0);
+                                         ptx::sw128_kmajor_desc(b_addr + kk * 32), idesc,
+                                         (kb > tl.kb0 || kk > 0) ? 1u : 0u);
                     }
                     issued = true;
                     ptx::mma_commit(ptx::smem_u32(&ctl->empty[s]));
@@ -287,7 +419,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int acc = 0;
         uint32_t aph = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
-            const Tile tl = decode_tile(args.plan, nb, t, GATED, args);
+            const Tile tl = decode_tile<MODE>(nb, t, args);
+            if (tl.kb0 >= tl.kb1) continue;
             const bool ok = bounded_wait(ptx::smem_u32(&ctl->tfull[acc]), aph, ctl, args.err);
             if (!__all_sync(0xffffffffu, ok)) break;   // the whole warp leaves together
             ptx::tc_fence_after();
@@ -299,7 +432,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 uint32_t v[16];
                 ptx::tmem_ld16(taddr + (uint32_t)c0, v);
                 ptx::tmem_ld_wait();
-                if (GATED) {
+                if (MODE == MODE_GATED) {
                     // lanes 0-15: gate of f row 16*quad + lane; lanes 16-31: up of the same row
                     const int half = lane >> 4;
                     const int frow = tl.m * 64 + quad * 16 + (lane & 15);
@@ -313,17 +446,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         if (col < tl.rows && frow < Mrows)
                             out[(size_t)(tl.row0 + col) * ld + frow] = __float2bfloat16_rn(silu_f(g) * u);
                     }
-                } else {
+                } else if (MODE == MODE_DOWN) {
                     const int drow = tl.m * 128 + quad * 32 + lane;
                     const int my_col = c0 + (lane & 15);
                     float my_scale = 1.0f;
-                    if (!tl.shared && my_col < tl.rows) my_scale = __ldg(args.gate_w + __ldg(args.perm + tl.row0 + my_col));
+                    if (!tl.shared && my_col < tl.rows)
+                        my_scale = __ldg(args.gate_w + __ldg(args.perm + tl.row0 + my_col));
 #pragma unroll
                     for (int j = 0; j < 16; j++) {
                         const float sc = __shfl_sync(0xffffffffu, my_scale, j);
                         const int col = c0 + j;
                         if (col < tl.rows && drow < Mrows)
-                            out[(size_t)(tl.row0 + col) * ld + drow] = __float2bfloat16_rn(__uint_as_float(v[j]) * sc);
+                            out[(size_t)(tl.row0 + col) * ld + drow] =
+                                __float2bfloat16_rn(__uint_as_float(v[j]) * sc);
+                    }
+                } else {
+                    // router: lane = expert, column = token; fp32 logits or split-K partials
+                    const int e = tl.m * 128 + quad * 32 + lane;
+                    if (e < args.E) {
+                        const bool whole = args.splits == 1;
+                        const float b = (whole && args.bias) ? __ldg(args.bias + e) : 0.f;
+                        float* dst = args.out_f32 + (size_t)(whole ? 0 : tl.split) * args.T * args.E;
+#pragma unroll
+                        for (int j = 0; j < 16; j++) {
+                            const int col = c0 + j;
+                            if (col < tl.rows) dst[(size_t)(tl.row0 + col) * args.E + e] = __uint_as_float(v[j]) + b;
+                        }
                     }
                 }
             }

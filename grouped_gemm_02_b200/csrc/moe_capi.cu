@@ -1,15 +1,21 @@
 // moe_capi.cu -- the C ABI declared in include/moe.h: host-side argument
 // checks, workspace layout, TMA tensor maps and kernel launches.  No entry
 // point allocates, frees or synchronises (moe_get_device_error excepted).
+//
+// Every kernel is launched with programmatic stream serialisation: it may
+// start while the previous kernel on the stream drains, waits
+// (griddepcontrol.wait) before touching that kernel's outputs, and lets its
+// own successor start only after that wait.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
-#include <atomic>
 #include <mutex>
+#include <utility>
 
 #include "../../include/moe.h"
 #include "common.cuh"
@@ -37,11 +43,27 @@ std::atomic<int64_t> g_launches{0};
 thread_local cudaEvent_t t_phase[6] = {};
 thread_local bool t_phase_armed = false;
 
-inline void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
-
 inline void phase_mark(bool on, int i, cudaStream_t st)
 {
     if (on) cudaEventRecord(t_phase[i], st);
+}
+
+// Launch with programmatic stream serialisation (see the file comment).
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Per-device one-time set-up: architecture check, SM count, kernel attributes.
@@ -60,9 +82,11 @@ int device_setup(DeviceState** out)
         st.supported = (major == 10 && minor == 0);
         st.sm_count = sms;
         if (st.supported) {
-            if (cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            if (cudaFuncSetAttribute(grouped_gemm_kernel<MODE_GATED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kGemmSmemBytes) != cudaSuccess ||
-                cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                cudaFuncSetAttribute(grouped_gemm_kernel<MODE_DOWN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kGemmSmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(grouped_gemm_kernel<MODE_ROUTER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kGemmSmemBytes) != cudaSuccess)
                 return MOE_ERR_CUDA;
             if (!g_encode) {
@@ -86,10 +110,7 @@ inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) 
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
-int launch_status()
-{
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
-}
+inline int status_of(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 // Common size checks.
 int check_sizes(int64_t T, int64_t d, int64_t E, int64_t k)
@@ -114,36 +135,83 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// ---------------------------------------------------------------- step launchers
-int run_route(const bf16* x, const bf16* Wg, const float* bias, int T, int d, int E, int k, float* logits,
-              int32_t* idx, float* w, uint32_t* err, cudaStream_t st)
+template <class T>
+T* at(void* ws, size_t off)
 {
-    const int max_tok_per_launch = 65535 * kRouterTokens;
-    for (int t0 = 0; t0 < T; t0 += max_tok_per_launch) {
-        const int nt = std::min(T - t0, max_tok_per_launch);
-        dim3 grid((E + kRouterWarps - 1) / kRouterWarps, (nt + kRouterTokens - 1) / kRouterTokens);
-        router_logits_kernel<<<grid, 256, 0, st>>>(x + (size_t)t0 * d, Wg, bias, nt, d, E, logits + (size_t)t0 * E);
-        count_launches(1);
-    }
-    topk_softmax_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, idx, w, err);
-    count_launches(1);
-    return launch_status();
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
+// ---------------------------------------------------------------- step launchers
+// Router logits on the tensor cores (MODE_ROUTER), split over K when the
+// tokens alone cannot fill the SMs.  Leaves either the logits (+ bias) in
+// `logits` (splits == 1) or fp32 partials in `partials`; reports the split.
+int run_router_gemm(const bf16* x, const bf16* Wg, const float* bias, int T, int d, int E, float* logits,
+                    float* partials, uint32_t* err, int sms, cudaStream_t st, RouterSplit* out)
+{
+    const RouterSplit rs = router_split(T, d, E);
+    *out = rs;
+    CUtensorMap a, b;
+    if (!make_map(&a, Wg, d, E, 128) || !make_map(&b, x, d, T, 16)) return MOE_ERR_CUDA;
+    GemmArgs g{};
+    g.E = E;
+    g.M = E;
+    g.M_shared = E;
+    g.K = d;
+    g.K_shared = d;
+    g.T = T;
+    g.units = rs.units;
+    g.chunk = rs.chunk;
+    g.mt = rs.mt;
+    g.splits = rs.splits;
+    g.kb_per = rs.kb_per;
+    g.out_f32 = rs.splits > 1 ? partials : logits;
+    g.bias = bias;
+    g.err = err;
+    const int grid = std::min(sms, rs.tiles);
+    return status_of(launch(grouped_gemm_kernel<MODE_ROUTER>, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, st,
+                            a, a, b, a, a, b, g));
+}
+
+// Top-k over the router's output: the logits themselves, or the split-K
+// partials (then the sums, + bias, are also stored in `logits`).
+struct TopkSource {
+    const float* src;
+    size_t stride;
+    int splits;
+    const float* bias;
+    float* logits_out;
+};
+
+TopkSource topk_source(const RouterSplit& rs, float* logits, float* partials, const float* bias, int T, int E)
+{
+    if (rs.splits > 1) return {partials, (size_t)T * E, rs.splits, bias, logits};
+    return {logits, 0, 1, nullptr, nullptr};
+}
+
+int run_topk(const TopkSource& s, int T, int E, int k, int32_t* idx, float* w, uint32_t* err, cudaStream_t st)
+{
+    return status_of(launch(topk_softmax_kernel, dim3((T + 7) / 8), dim3(256), 0, st, s.src, s.stride, s.splits,
+                            s.bias, T, E, k, s.logits_out, idx, w, err));
+}
+
+// The general (multi-CTA) histogram / scan / scatter / gather.
 int run_permute(const int32_t* idx, const bf16* x, int T, int d, int E, int k, int32_t* counts, int32_t* offsets,
                 int32_t* perm, int32_t* inv_perm, bf16* xp, uint32_t* err, int32_t* block_counts, int32_t* plan,
                 int f, int shared_rows, int fs, int sms, cudaStream_t st)
 {
     const int64_t P = (int64_t)T * k;
     const int nb = hist_blocks(P);
-    hist_kernel<<<nb, 512, 0, st>>>(idx, P, E, block_counts, err);
-    scan_kernel<<<1, 1024, 0, st>>>(block_counts, nb, E, counts, offsets, plan, f, d, shared_rows, fs);
-    scatter_kernel<<<nb, 256, 0, st>>>(idx, P, E, block_counts, perm, inv_perm);
-    const int64_t warps = P;
-    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, (int64_t)sms * 16));
-    gather_rows_kernel<<<blocks, 256, 0, st>>>(x, perm, offsets, E, k, d, xp);
-    count_launches(4);
-    return launch_status();
+    cudaError_t e = launch(hist_kernel, dim3(nb), dim3(512), 0, st, idx, P, E, block_counts, err);
+    if (e == cudaSuccess)
+        e = launch(scan_kernel, dim3(1), dim3(1024), 0, st, block_counts, nb, E, counts, offsets, plan, f, d,
+                   shared_rows, fs);
+    if (e == cudaSuccess)
+        e = launch(scatter_kernel, dim3(nb), dim3(256), 0, st, idx, P, E, (const int32_t*)block_counts, perm,
+                   inv_perm);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)sms * 16));
+    return status_of(launch(gather_rows_kernel, dim3(blocks), dim3(256), 0, st, x, (const int32_t*)perm,
+                            (const int32_t*)offsets, E, k, d, xp));
 }
 
 struct GemmOperands {
@@ -154,7 +222,8 @@ struct GemmOperands {
     int T, P, d, f, fs, E;
 };
 
-int run_gemms(const GemmOperands& o, const int32_t* plan, uint32_t* err, int sms, cudaStream_t st,
+// plan_ready: the plan was written two or more launches before the gate/up GEMM.
+int run_gemms(const GemmOperands& o, const int32_t* plan, bool plan_ready, uint32_t* err, int sms, cudaStream_t st,
               bool prof = false)
 {
     CUtensorMap a0, a1, b, a0s, a1s, bs;
@@ -174,6 +243,7 @@ int run_gemms(const GemmOperands& o, const int32_t* plan, uint32_t* err, int sms
     }
     GemmArgs g1{};
     g1.plan = plan;
+    g1.plan_ready = plan_ready ? 1 : 0;
     g1.E = o.E;
     g1.M = o.f;
     g1.M_shared = o.fs;
@@ -186,9 +256,9 @@ int run_gemms(const GemmOperands& o, const int32_t* plan, uint32_t* err, int sms
     g1.perm = o.perm;
     g1.gate_w = o.gate_w;
     g1.err = err;
-    grouped_gemm_kernel<true><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(a0, a1, b, a0s, a1s, bs, g1);
-    count_launches(1);
-    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch(grouped_gemm_kernel<MODE_GATED>, dim3(sms), dim3(kGemmThreads), kGemmSmemBytes, st, a0, a1, b, a0s,
+               a1s, bs, g1) != cudaSuccess)
+        return MOE_ERR_CUDA;
     phase_mark(prof, 3, st);
 
     // down GEMM: A = W2 rows (128-row boxes), B = h rows; shared: Ws2 and hs
@@ -204,6 +274,7 @@ int run_gemms(const GemmOperands& o, const int32_t* plan, uint32_t* err, int sms
         bs = b;
     }
     GemmArgs g2 = g1;
+    g2.plan_ready = 1;   // written before the gate/up GEMM
     g2.M = o.d;
     g2.M_shared = o.d;
     g2.K = o.f;
@@ -212,23 +283,17 @@ int run_gemms(const GemmOperands& o, const int32_t* plan, uint32_t* err, int sms
     g2.ld_out = o.d;
     g2.out_shared = o.ys;
     g2.ld_out_shared = o.d;
-    grouped_gemm_kernel<false><<<sms, kGemmThreads, kGemmSmemBytes, st>>>(a0, a1, b, a0s, a1s, bs, g2);
-    count_launches(1);
-    return launch_status();
+    return status_of(launch(grouped_gemm_kernel<MODE_DOWN>, dim3(sms), dim3(kGemmThreads), kGemmSmemBytes, st, a0,
+                            a1, b, a0s, a1s, bs, g2));
 }
 
 int run_combine(const bf16* y_p, const int32_t* inv_perm, const bf16* ys, int T, int k, int d, bf16* out,
                 cudaStream_t st)
 {
-    combine_kernel<<<T, 128, 0, st>>>(y_p, inv_perm, ys, T, k, d, out);
-    count_launches(1);
-    return launch_status();
-}
-
-template <class T>
-T* at(void* ws, size_t off)
-{
-    return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+    constexpr int kThreads = 64;
+    const int nvec = d / 8;
+    const int gy = std::max(1, std::min((nvec + kThreads - 1) / kThreads, 65535));
+    return status_of(launch(combine_kernel, dim3(T, gy), dim3(kThreads), 0, st, y_p, inv_perm, ys, T, k, d, out));
 }
 
 }  // namespace
@@ -252,19 +317,26 @@ int moe_workspace_init(void* ws, size_t ws_bytes, int64_t T, int64_t E, int64_t 
 }
 
 int moe_route(const moe_bf16* x, const moe_bf16* Wg, const float* bias, int64_t T, int64_t d, int64_t E, int64_t k,
-              float* logits, int32_t* topk_idx, float* topk_w, void* ws, void* stream)
+              float* logits, int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream)
 {
     int rc = check_sizes(T, d, E, k);
     if (rc) return rc;
     if (T == 0) return MOE_OK;
-    if (!x || !Wg || !logits || !topk_idx || !topk_w) return MOE_ERR_ARG;
-    if (!al16(x) || !al16(Wg)) return MOE_ERR_ALIGN;
+    if (!x || !Wg || !logits || !topk_idx || !topk_w || !ws) return MOE_ERR_ARG;
+    if (!al16(x) || !al16(Wg) || !al16(ws)) return MOE_ERR_ALIGN;
+    const WsLayout L = ws_layout(T, d, 0, E, k, 0);
+    if (ws_bytes < L.ctrl_end) return MOE_ERR_WS;
     DeviceState* dev;
     if ((rc = device_setup(&dev))) return rc;
-    if (!ws) return MOE_ERR_ARG;
-    uint32_t* err = at<uint32_t>(ws, 0);
-    return run_route(reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(Wg), bias, (int)T, (int)d,
-                     (int)E, (int)k, logits, topk_idx, topk_w, err, as_stream(stream));
+    cudaStream_t st = as_stream(stream);
+    uint32_t* err = at<uint32_t>(ws, L.err);
+    float* partials = at<float>(ws, L.router_partials);
+    RouterSplit rs;
+    if ((rc = run_router_gemm(reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(Wg), bias, (int)T,
+                              (int)d, (int)E, logits, partials, err, dev->sm_count, st, &rs)))
+        return rc;
+    return run_topk(topk_source(rs, logits, partials, bias, (int)T, (int)E), (int)T, (int)E, (int)k, topk_idx, topk_w,
+                    err, st);
 }
 
 int moe_topk(const float* logits, int64_t T, int64_t E, int64_t k, int32_t* topk_idx, float* topk_w, void* ws,
@@ -276,10 +348,8 @@ int moe_topk(const float* logits, int64_t T, int64_t E, int64_t k, int32_t* topk
     if (!logits || !topk_idx || !topk_w || !ws) return MOE_ERR_ARG;
     DeviceState* dev;
     if ((rc = device_setup(&dev))) return rc;
-    topk_softmax_kernel<<<(unsigned)((T + 7) / 8), 256, 0, as_stream(stream)>>>(logits, (int)T, (int)E, (int)k,
-                                                                                 topk_idx, topk_w, at<uint32_t>(ws, 0));
-    count_launches(1);
-    return launch_status();
+    const TopkSource s{logits, 0, 1, nullptr, nullptr};
+    return run_topk(s, (int)T, (int)E, (int)k, topk_idx, topk_w, at<uint32_t>(ws, 0), as_stream(stream));
 }
 
 int moe_permute(const int32_t* topk_idx, const moe_bf16* x, int64_t T, int64_t d, int64_t E, int64_t k,
@@ -318,9 +388,9 @@ int moe_grouped_gemm(const moe_bf16* xp, const int32_t* counts, const int32_t* o
     if ((rc = device_setup(&dev))) return rc;
     cudaStream_t st = as_stream(stream);
     int32_t* plan = at<int32_t>(ws, L.plan);
-    plan_kernel<<<1, 1024, 0, st>>>(counts, offsets, (int)E, plan, (int)f, (int)d, 0, 0);
-    count_launches(1);
-    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch(plan_kernel, dim3(1), dim3(1024), 0, st, counts, offsets, (int)E, plan, (int)f, (int)d, 0, 0) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
     GemmOperands o{};
     o.xp = reinterpret_cast<const bf16*>(xp);
     o.x = o.xp;
@@ -337,7 +407,7 @@ int moe_grouped_gemm(const moe_bf16* xp, const int32_t* counts, const int32_t* o
     o.f = (int)f;
     o.fs = 0;
     o.E = (int)E;
-    return run_gemms(o, plan, at<uint32_t>(ws, L.err), dev->sm_count, st);
+    return run_gemms(o, plan, /*plan_ready=*/false, at<uint32_t>(ws, L.err), dev->sm_count, st);
 }
 
 int moe_combine(const moe_bf16* y_p, const int32_t* inv_perm, const moe_bf16* shared_out, int64_t T, int64_t k,
@@ -377,6 +447,7 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     uint32_t* err = at<uint32_t>(ws, L.err);
     int32_t* plan = at<int32_t>(ws, L.plan);
     float* logits = at<float>(ws, L.logits);
+    float* partials = at<float>(ws, L.router_partials);
     int32_t* idx = at<int32_t>(ws, L.topk_idx);
     float* w = at<float>(ws, L.topk_w);
     int32_t* counts = at<int32_t>(ws, L.counts);
@@ -389,18 +460,36 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     bf16* hs = f_shared > 0 ? at<bf16>(ws, L.hs) : nullptr;
     bf16* ys = f_shared > 0 ? at<bf16>(ws, L.ys) : nullptr;
     const bf16* xb = reinterpret_cast<const bf16*>(x);
+    const int iT = (int)T, id = (int)d, iE = (int)E, ik = (int)k, shared_rows = f_shared > 0 ? (int)T : 0;
 
     const bool prof = t_phase_armed;   // the armed events serve this call only
     t_phase_armed = false;
     phase_mark(prof, 0, st);
-    if ((rc = run_route(xb, reinterpret_cast<const bf16*>(Wg), bias, (int)T, (int)d, (int)E, (int)k, logits, idx, w,
-                        err, st)))
+    RouterSplit rs;
+    if ((rc = run_router_gemm(xb, reinterpret_cast<const bf16*>(Wg), bias, iT, id, iE, logits, partials, err,
+                              dev->sm_count, st, &rs)))
         return rc;
-    phase_mark(prof, 1, st);
-    if ((rc = run_permute(idx, xb, (int)T, (int)d, (int)E, (int)k, counts, offsets, perm, inv_perm, xp, err,
-                          at<int32_t>(ws, L.block_counts), plan, (int)f, f_shared > 0 ? (int)T : 0, (int)f_shared,
-                          dev->sm_count, st)))
-        return rc;
+    const TopkSource src = topk_source(rs, logits, partials, bias, iT, iE);
+    const int64_t P = T * k;
+    if (T <= kSmallTokens) {
+        // one CTA: top-k, histogram, scan, stable ranks and the tile plan
+        phase_mark(prof, 1, st);
+        if (launch(route_permute_small_kernel, dim3(1), dim3(1024), 0, st, src.src, src.stride, src.splits, src.bias,
+                   iT, iE, ik, src.logits_out, idx, w, counts, offsets, perm, inv_perm, plan, (int)f, id, shared_rows,
+                   (int)f_shared, err) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)dev->sm_count * 16));
+        if (launch(gather_rows_kernel, dim3(blocks), dim3(256), 0, st, xb, (const int32_t*)perm,
+                   (const int32_t*)offsets, iE, ik, id, xp) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    } else {
+        if ((rc = run_topk(src, iT, iE, ik, idx, w, err, st))) return rc;
+        phase_mark(prof, 1, st);
+        if ((rc = run_permute(idx, xb, iT, id, iE, ik, counts, offsets, perm, inv_perm, xp, err,
+                              at<int32_t>(ws, L.block_counts), plan, (int)f, shared_rows, (int)f_shared,
+                              dev->sm_count, st)))
+            return rc;
+    }
     GemmOperands o{};
     o.xp = xp;
     o.x = xb;
@@ -416,16 +505,17 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     o.y_p = y_p;
     o.hs = hs;
     o.ys = ys;
-    o.T = (int)T;
-    o.P = (int)(T * k);
-    o.d = (int)d;
+    o.T = iT;
+    o.P = (int)P;
+    o.d = id;
     o.f = (int)f;
     o.fs = (int)f_shared;
-    o.E = (int)E;
+    o.E = iE;
     phase_mark(prof, 2, st);
-    if ((rc = run_gemms(o, plan, err, dev->sm_count, st, prof))) return rc;
+    // the plan was written two or more launches before the gate/up GEMM (the gather is in between)
+    if ((rc = run_gemms(o, plan, /*plan_ready=*/true, err, dev->sm_count, st, prof))) return rc;
     phase_mark(prof, 4, st);
-    rc = run_combine(y_p, inv_perm, ys, (int)T, (int)k, (int)d, reinterpret_cast<bf16*>(out), st);
+    rc = run_combine(y_p, inv_perm, ys, iT, ik, id, reinterpret_cast<bf16*>(out), st);
     phase_mark(prof, 5, st);
     return rc;
 }

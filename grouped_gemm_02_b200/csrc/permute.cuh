@@ -15,6 +15,8 @@
 #pragma once
 
 #include "common.cuh"
+#include "ptx.cuh"
+#include "route.cuh"
 
 namespace moe {
 
@@ -24,6 +26,8 @@ namespace moe {
 __global__ void __launch_bounds__(512) hist_kernel(const int32_t* __restrict__ idx, int64_t P, int E,
                                                    int32_t* __restrict__ block_counts, uint32_t* __restrict__ err)
 {
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
     __shared__ int32_t cnt[kMaxExperts];
     for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
@@ -166,6 +170,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ block_
 {
     __shared__ int warp_sums[32];
     __shared__ int s_pairs;
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
     const int tid = threadIdx.x;
     int c = 0;
     if (tid < E)
@@ -197,10 +203,78 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
                                                     int f_shared)
 {
     __shared__ int warp_sums[32];
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
     const int tid = threadIdx.x;
     const int c = tid < E ? counts[tid] : 0;
     const int off = tid < E ? offsets[tid] : 0;
     build_plan(c, off, E, offsets[E], plan, f, d, shared_rows, f_shared, warp_sums);
+}
+
+// ---------------------------------------------------------------- small-T fused routing + permutation
+// One CTA of 1024 threads does S2-S4 (minus the row gather) and the tile plan
+// when T <= kSmallTokens (then T*k <= 1024 <= kSmallPairs): top-k per token (one warp per token, summing the
+// router's split-K partials), histogram, scan, stable ranks and the plan, so a
+// decode-sized layer pays one launch instead of five.
+constexpr int kSmallTokens = 128;
+constexpr int kSmallPairs = kSmallTokens * kMaxTopK;
+
+__global__ void __launch_bounds__(1024) route_permute_small_kernel(
+    const float* __restrict__ Lp, size_t split_stride, int splits, const float* __restrict__ bias, int T, int E, int k,
+    float* __restrict__ logits_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+    int32_t* __restrict__ inv_perm, int32_t* __restrict__ plan, int f, int d, int shared_rows, int f_shared,
+    uint32_t* __restrict__ err)
+{
+    __shared__ int s_idx[kSmallPairs];
+    __shared__ int s_cnt[kMaxExperts];
+    __shared__ int s_run[kMaxExperts];
+    __shared__ int warp_sums[32];
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int P = T * k;
+    // 1. top-k, one warp per token
+    for (int t = warp; t < T; t += 32)
+        topk_warp_any(Lp, split_stride, splits, bias, t, E, k, logits_out, topk_idx, topk_w, err, s_idx);
+    for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = 0;
+    __syncthreads();
+    // 2. histogram (the ids come from the top-k above, so they are all in range)
+    for (int q = tid; q < P; q += blockDim.x) atomicAdd(&s_cnt[s_idx[q]], 1);
+    __syncthreads();
+    // 3. scan
+    const int c = tid < E ? s_cnt[tid] : 0;
+    const int incl = block_inclusive_scan(c, warp_sums);
+    const int off = incl - c;
+    if (tid < E) {
+        counts[tid] = c;
+        offsets[tid] = off;
+        s_run[tid] = off;
+    }
+    if (tid == E - 1) offsets[E] = incl;
+    __syncthreads();
+    // 4. stable ranks: pairs in ascending q, 1024 at a time; inside a warp by lane
+    //    order (match_any), warps in turn
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int base = 0; base < P; base += blockDim.x) {
+        const int q = base + tid;
+        const int e = q < P ? s_idx[q] : -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(peers & lt_mask);
+        const int leader = __ffs(peers) - 1;
+        for (int w = 0; w < (int)(blockDim.x >> 5); w++) {
+            if (warp == w && e >= 0) {
+                const int pos = s_run[e] + rank;
+                perm[pos] = q;
+                inv_perm[q] = pos;
+            }
+            __syncwarp();
+            if (warp == w && e >= 0 && lane == leader) s_run[e] += __popc(peers);
+            __syncthreads();
+        }
+    }
+    // 5. tile plan
+    if (plan) build_plan(c, off, E, P, plan, f, d, shared_rows, f_shared, warp_sums);
 }
 
 // ---------------------------------------------------------------- scatter
@@ -212,6 +286,8 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
                                                       const int32_t* __restrict__ block_base,
                                                       int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm)
 {
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
     __shared__ int32_t run[kMaxExperts];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int e = threadIdx.x; e < E; e += blockDim.x) run[e] = block_base[(size_t)blockIdx.x * E + e];
@@ -252,6 +328,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const bf16* __restrict
                                                           const int32_t* __restrict__ offsets, int E, int k, int d,
                                                           bf16* __restrict__ xp)
 {
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
     const int pairs = offsets[E];
     const int nvec = d / 8;
     const int lane = threadIdx.x & 31;
@@ -267,18 +345,20 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const bf16* __restrict
 // ---------------------------------------------------------------- combine
 // out[t, :] = bf16( sum_{j<k} y_p[inv_perm[t*k+j], :]  (+ ys[t, :]) ), summed in
 // fp32 in ascending j, no atomics.  Dropped pairs (inv_perm < 0) add nothing.
-// grid T, block 128; requires d % 8 == 0.
+// grid (T, column blocks), block 64; requires d % 8 == 0.
 __global__ void __launch_bounds__(128) combine_kernel(const bf16* __restrict__ y_p, const int32_t* __restrict__ inv_perm,
                                                       const bf16* __restrict__ ys, int T, int k, int d,
                                                       bf16* __restrict__ out)
 {
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
     const int t = blockIdx.x;
     if (t >= T) return;
     int rows[kMaxTopK];
 #pragma unroll
     for (int j = 0; j < kMaxTopK; j++) rows[j] = j < k ? inv_perm[(size_t)t * k + j] : -1;
     const int nvec = d / 8;
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+    for (int v = blockIdx.y * blockDim.x + threadIdx.x; v < nvec; v += gridDim.y * blockDim.x) {
         float acc[8];
 #pragma unroll
         for (int i = 0; i < 8; i++) acc[i] = 0.f;

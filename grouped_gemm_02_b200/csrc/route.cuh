@@ -9,6 +9,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -31,6 +32,8 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const bf16* __restri
                                                             const float* __restrict__ bias, int T, int d, int E,
                                                             float* __restrict__ L)
 {
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x * kRouterWarps + warp;
     const int t0 = blockIdx.y * kRouterTokens;
@@ -74,29 +77,49 @@ __device__ __forceinline__ uint32_t logit_key(float v)
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// One warp per token; E <= 512 (16 logits per lane), k <= 8.
-__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ L, int T, int E, int k,
-                                                           int32_t* __restrict__ topk_idx,
-                                                           float* __restrict__ topk_w, uint32_t* __restrict__ err)
+// Inverse of logit_key for the values it keeps apart (NaN maps back to a NaN).
+__device__ __forceinline__ float key_logit(uint32_t key)
 {
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// Top-k of one token by one warp; PER logits per lane (E <= 32 * PER).  The
+// token's logit for expert e is
+//   sum_{s < splits} Lp[s * split_stride + t*E + e]  (+ bias[e] when bias != null),
+// summed in ascending s (the split-K partials of the tensor-core router, or the
+// logits themselves when splits == 1).  When logits_out != null that value is
+// stored there.  Writes idx/w for the token (and the ids to s_idx when given).
+template <int PER>
+__device__ __forceinline__ void topk_warp(const float* __restrict__ Lp, size_t split_stride, int splits,
+                                          const float* __restrict__ bias, int t, int E, int k,
+                                          float* __restrict__ logits_out, int32_t* __restrict__ topk_idx,
+                                          float* __restrict__ topk_w, uint32_t* __restrict__ err, int* s_idx)
+{
     const int lane = threadIdx.x & 31;
-    if (warp >= T) return;
-    const float* row = L + (size_t)warp * E;
-    constexpr int kPer = kMaxExperts / 32;
     // Packed candidate: key in the high word, (0xFFFF - expert) in the low word, so
     // the maximum packed value is the largest logit with the lowest index.
-    uint64_t cand[kPer];
+    uint64_t cand[PER];
     bool nan_seen = false;
 #pragma unroll
-    for (int i = 0; i < kPer; i++) {
+    for (int i = 0; i < PER; i++) {
         const int e = lane + 32 * i;
+        cand[i] = 0;   // below every real candidate (real ones have a nonzero low word or key)
         if (e < E) {
-            const float v = row[e];
+            const float* p = Lp + (size_t)t * E + e;
+            float v = p[0];
+            // partials in ascending order, fetched 8 at a time so the loads overlap
+            for (int sp = 1; sp < splits; sp += 8) {
+                float part[8];
+#pragma unroll
+                for (int u = 0; u < 8; u++) part[u] = sp + u < splits ? p[(size_t)(sp + u) * split_stride] : 0.f;
+#pragma unroll
+                for (int u = 0; u < 8; u++)
+                    if (sp + u < splits) v += part[u];
+            }
+            if (bias) v += bias[e];
+            if (logits_out) logits_out[(size_t)t * E + e] = v;
             nan_seen |= (v != v);
             cand[i] = ((uint64_t)logit_key(v) << 32) | (uint64_t)(0xFFFFu - (uint32_t)e);
-        } else {
-            cand[i] = 0;   // below every real candidate (real ones have a nonzero low word or key)
         }
     }
     if (__any_sync(0xffffffffu, nan_seen) && lane == 0) atomicOr(err, DEVERR_NAN_LOGIT);
@@ -107,7 +130,7 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
         if (j < k) {
             uint64_t best = 0;
 #pragma unroll
-            for (int i = 0; i < kPer; i++) best = cand[i] > best ? cand[i] : best;
+            for (int i = 0; i < PER; i++) best = cand[i] > best ? cand[i] : best;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
@@ -115,9 +138,9 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
             }
             const int e = (int)(0xFFFFu - (uint32_t)(best & 0xFFFFu));
             chosen[j] = e;
-            vals[j] = row[e];
+            vals[j] = key_logit((uint32_t)(best >> 32));
 #pragma unroll
-            for (int i = 0; i < kPer; i++)
+            for (int i = 0; i < PER; i++)
                 if (lane + 32 * i == e) cand[i] = 0;   // taken
         }
     }
@@ -135,11 +158,42 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
 #pragma unroll
         for (int j = 0; j < kMaxTopK; j++) {
             if (j < k) {
-                topk_idx[(size_t)warp * k + j] = chosen[j];
-                topk_w[(size_t)warp * k + j] = ex[j] / z;
+                topk_idx[(size_t)t * k + j] = chosen[j];
+                topk_w[(size_t)t * k + j] = ex[j] / z;
+                if (s_idx) s_idx[t * k + j] = chosen[j];
             }
         }
     }
+}
+
+// topk_warp with the smallest per-lane candidate array that holds E logits.
+__device__ __forceinline__ void topk_warp_any(const float* __restrict__ Lp, size_t split_stride, int splits,
+                                              const float* __restrict__ bias, int t, int E, int k,
+                                              float* __restrict__ logits_out, int32_t* __restrict__ topk_idx,
+                                              float* __restrict__ topk_w, uint32_t* __restrict__ err, int* s_idx)
+{
+    if (E <= 64)
+        topk_warp<2>(Lp, split_stride, splits, bias, t, E, k, logits_out, topk_idx, topk_w, err, s_idx);
+    else if (E <= 128)
+        topk_warp<4>(Lp, split_stride, splits, bias, t, E, k, logits_out, topk_idx, topk_w, err, s_idx);
+    else if (E <= 256)
+        topk_warp<8>(Lp, split_stride, splits, bias, t, E, k, logits_out, topk_idx, topk_w, err, s_idx);
+    else
+        topk_warp<16>(Lp, split_stride, splits, bias, t, E, k, logits_out, topk_idx, topk_w, err, s_idx);
+}
+
+// One warp per token; E <= 512 (16 logits per lane), k <= 8.
+__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ Lp, size_t split_stride,
+                                                           int splits, const float* __restrict__ bias, int T, int E,
+                                                           int k, float* __restrict__ logits_out,
+                                                           int32_t* __restrict__ topk_idx,
+                                                           float* __restrict__ topk_w, uint32_t* __restrict__ err)
+{
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (warp >= T) return;
+    topk_warp_any(Lp, split_stride, splits, bias, warp, E, k, logits_out, topk_idx, topk_w, err, nullptr);
 }
 
 }  // namespace moe

@@ -52,7 +52,7 @@ def lib() -> C.CDLL:
         sig = {
             "moe_workspace_size": [i64, i64, i64, i64, i64, i64, C.POINTER(sz)],
             "moe_workspace_init": [vp, sz, i64, i64, i64, vp],
-            "moe_route": [vp, vp, vp, i64, i64, i64, i64, vp, vp, vp, vp, vp],
+            "moe_route": [vp, vp, vp, i64, i64, i64, i64, vp, vp, vp, vp, sz, vp],
             "moe_topk": [vp, i64, i64, i64, vp, vp, vp, vp],
             "moe_permute": [vp, vp, i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_grouped_gemm": [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, vp, vp, sz, vp],
@@ -171,7 +171,7 @@ def moe_route(x: torch.Tensor, Wg: torch.Tensor, bias: Optional[torch.Tensor], k
     topk_idx = torch.empty(T, k, dtype=torch.int32, device=dev) if topk_idx is None else topk_idx
     topk_w = torch.empty(T, k, dtype=torch.float32, device=dev) if topk_w is None else topk_w
     _call("moe_route", _p(x), _p(Wg), _p(bias), T, d, E, k, _p(logits), _p(topk_idx), _p(topk_w), _p(ws),
-          _stream(stream))
+          ws.numel(), _stream(stream))
     return logits, topk_idx, topk_w
 
 

@@ -81,13 +81,17 @@ MOE_API int moe_workspace_size(int64_t T, int64_t d, int64_t f, int64_t E, int64
 MOE_API int moe_workspace_init(void *ws, size_t ws_bytes, int64_t T, int64_t E, int64_t k, void *stream);
 
 /* Router (Decoding the Skew, abstract: the runtime routing distribution).
- * logits [T,E] fp32 = x Wg^T + bias (bias [E] fp32, may be NULL), summed in
- * fp32 in a fixed order; then, per token, the k largest logits in descending
- * order (ties: lower expert id; NaN ranks lowest) -> topk_idx [T,k] int32,
- * and softmax over those k logits -> topk_w [T,k] fp32.  `ws` (required)
- * supplies the device error word. */
-MOE_API int moe_route(const moe_bf16 *x, const moe_bf16 *Wg, const float *bias, int64_t T, int64_t d, int64_t E, int64_t k,
-              float *logits, int32_t *topk_idx, float *topk_w, void *ws, void *stream);
+ * logits [T,E] fp32 = x Wg^T + bias (bias [E] fp32, may be NULL): a bf16
+ * tensor-core GEMM with fp32 accumulation; when T alone cannot fill the GPU
+ * the d-loop is split into fixed ranges whose fp32 partial sums are added in
+ * a fixed order, so the result is deterministic.  Then, per token, the k
+ * largest logits in descending order (ties: lower expert id; NaN ranks
+ * lowest) -> topk_idx [T,k] int32, and softmax over those k logits ->
+ * topk_w [T,k] fp32.  `ws` (required, at least moe_workspace_size(T,d,f,E,k,0)
+ * bytes for any f) holds the device error word and the partial sums. */
+MOE_API int moe_route(const moe_bf16 *x, const moe_bf16 *Wg, const float *bias, int64_t T, int64_t d, int64_t E,
+                      int64_t k, float *logits, int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes,
+                      void *stream);
 
 /* The top-k/softmax step of moe_route alone, on caller-provided fp32 logits
  * [T,E]; same ordering and gate definition.  `ws` (required) supplies the
