@@ -75,7 +75,7 @@ __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + 
 // fp32 partial sums in a fixed order.  The split depends on the sizes only
 // (not on the device), so the workspace size and every result bit do too.
 constexpr int kRouterTargetCtas = 148;
-constexpr int64_t kRouterTileBytes = 256 * 1024;
+constexpr int64_t kRouterTileBytes = 64 * 1024;
 
 struct RouterSplit {
     int units, chunk, mt, splits, kb_per, tiles;

@@ -60,9 +60,8 @@ constexpr int kBlockK = 64;                          // bf16 elements per 128-by
 constexpr int kATileBytes = 128 * kBlockK * 2;       // 16 KB: 128 weight rows
 constexpr int kBRowBytes = kBlockK * 2;              // 128 B per token row
 constexpr int kMaxStages = 12;
-constexpr int kRingBytes = 216 * 1024;
+constexpr int kRingBytes = 208 * 1024;
 constexpr int kBarBytes = 512;
-constexpr int kGemmSmemBytes = 1024 + kRingBytes + kBarBytes;
 constexpr uint32_t kTmemCols = 512;                  // 2 accumulators x 256 columns
 constexpr uint64_t kWaitTimeoutNs = 1000000000ull;   // 1 s
 
@@ -91,6 +90,17 @@ struct Tile {
     bool shared;
 };
 
+// The plan entries this launch reads, copied to shared memory once per CTA so
+// that decoding a tile (a binary search over the tile prefix) costs shared
+// loads instead of a chain of dependent global loads at every tile boundary.
+struct SmemPlan {
+    int tb[kMaxGroups + 1];     // tile prefix of this GEMM
+    int4 blk[kMaxGroups];       // group, row0, rows, chunk
+    int units[kMaxGroups];
+};
+constexpr int kGemmSmemBytes = 1024 + kRingBytes + kBarBytes + (int)sizeof(SmemPlan);
+static_assert(kGemmSmemBytes <= 227 * 1024, "shared memory budget");
+
 template <int MODE>
 __device__ __forceinline__ int total_tiles(const GemmArgs& a, const PlanHeader* hdr)
 {
@@ -99,7 +109,7 @@ __device__ __forceinline__ int total_tiles(const GemmArgs& a, const PlanHeader* 
 }
 
 template <int MODE>
-__device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a)
+__device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a, const SmemPlan* sp)
 {
     Tile tl;
     if (MODE == MODE_ROUTER) {
@@ -119,24 +129,24 @@ __device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a)
         tl.kb1 = min(nk, tl.kb0 + a.kb_per);
         return tl;
     }
-    const PlanArrays pa = plan_arrays(const_cast<int32_t*>(a.plan));
-    const int32_t* tb = MODE == MODE_GATED ? pa.tb1 : pa.tb2;
+    const int* tb = sp->tb;
     int lo = 0, hi = nb - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (__ldg(tb + mid) <= t) lo = mid;
+        if (tb[mid] <= t) lo = mid;
         else hi = mid - 1;
     }
-    const int local = t - __ldg(tb + lo);
-    const int units = __ldg(pa.units + lo);
-    const int chunk = __ldg(pa.chunk + lo);
-    tl.group = __ldg(pa.group + lo);
+    const int local = t - tb[lo];
+    const int units = sp->units[lo];
+    const int4 b = sp->blk[lo];
+    const int chunk = b.w;
+    tl.group = b.x;
     tl.shared = tl.group == a.E;
     tl.m = local / units;
     const int u = local - tl.m * units;
     const int start = u * chunk;
-    tl.rows = min(chunk, __ldg(pa.rows + lo) - start);
-    tl.row0 = __ldg(pa.row0 + lo) + start;
+    tl.rows = min(chunk, b.z - start);
+    tl.row0 = b.y + start;
     tl.n_mma = (tl.rows + 15) & ~15;
     tl.K = tl.shared ? a.K_shared : a.K;
     tl.kb0 = 0;
@@ -185,11 +195,11 @@ struct KIter {
 };
 
 template <int MODE>
-__device__ __forceinline__ bool kiter_begin(KIter& it, int nb, int total, const GemmArgs& a)
+__device__ __forceinline__ bool kiter_begin(KIter& it, int nb, int total, const GemmArgs& a, const SmemPlan* sp)
 {
     it.t = blockIdx.x;
     while (it.t < total) {
-        it.tl = decode_tile<MODE>(nb, it.t, a);
+        it.tl = decode_tile<MODE>(nb, it.t, a, sp);
         if (it.tl.kb0 < it.tl.kb1) {
             it.kb = it.tl.kb0;
             return true;
@@ -200,11 +210,11 @@ __device__ __forceinline__ bool kiter_begin(KIter& it, int nb, int total, const 
 }
 
 template <int MODE>
-__device__ __forceinline__ bool kiter_next(KIter& it, int nb, int total, const GemmArgs& a)
+__device__ __forceinline__ bool kiter_next(KIter& it, int nb, int total, const GemmArgs& a, const SmemPlan* sp)
 {
     if (++it.kb < it.tl.kb1) return true;
     for (it.t += gridDim.x; it.t < total; it.t += gridDim.x) {
-        it.tl = decode_tile<MODE>(nb, it.t, a);
+        it.tl = decode_tile<MODE>(nb, it.t, a, sp);
         if (it.tl.kb0 < it.tl.kb1) {
             it.kb = it.tl.kb0;
             return true;
@@ -269,6 +279,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t stage_bytes = kATileBytes + (uint32_t)n_max * kBRowBytes;
     const int stages = min(kMaxStages, (int)(kRingBytes / stage_bytes));
 
+    SmemPlan* splan = reinterpret_cast<SmemPlan*>(smem + kRingBytes + kBarBytes);
+    if (MODE != MODE_ROUTER) {
+        const PlanArrays pa = plan_arrays(const_cast<int32_t*>(args.plan));
+        const int32_t* tbg = MODE == MODE_GATED ? pa.tb1 : pa.tb2;
+        for (int i = threadIdx.x; i <= nb; i += blockDim.x) {
+            splan->tb[i] = tbg[i];
+            if (i < nb) {
+                splan->blk[i] = make_int4(pa.group[i], pa.row0[i], pa.rows[i], pa.chunk[i]);
+                splan->units[i] = pa.units[i];
+            }
+        }
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; s++) {
             ptx::mbar_init(ptx::smem_u32(&ctl->full[s]), 1);
@@ -307,14 +329,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int pre = 0;
             if (!waited_early) {
                 KIter it;
-                bool more = kiter_begin<MODE>(it, nb, total, args);
+                bool more = kiter_begin<MODE>(it, nb, total, args, splan);
                 while (more && pre < stages) {
                     const uint32_t full = ptx::smem_u32(&ctl->full[pre]);
                     ptx::mbar_arrive_expect_tx(full, kATileBytes + (uint32_t)it.tl.n_mma * kBRowBytes);
                     armed |= 1u << pre;
                     issue_a<MODE>(it, ring + (uint32_t)pre * stage_bytes, full, &mA0, &mA1, &mA0s, &mA1s, args, pol);
                     ++pre;
-                    more = kiter_next<MODE>(it, nb, total, args);
+                    more = kiter_next<MODE>(it, nb, total, args, splan);
                 }
                 ptx::grid_dep_wait();
             }
@@ -323,7 +345,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int s = 0, n = 0;
             uint32_t ph = 0;
             KIter it;
-            bool more = kiter_begin<MODE>(it, nb, total, args);
+            bool more = kiter_begin<MODE>(it, nb, total, args, splan);
             while (more) {
                 const uint32_t a_dst = ring + (uint32_t)s * stage_bytes;
                 const uint32_t full = ptx::smem_u32(&ctl->full[s]);
@@ -346,7 +368,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     s = 0;
                     ph ^= 1u;
                 }
-                more = kiter_next<MODE>(it, nb, total, args);
+                more = kiter_next<MODE>(it, nb, total, args, splan);
             }
             if (!ok) {
                 // drain: wait (bounded) for every load this thread issued
@@ -369,7 +391,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t aph = 0;
             bool ok = true, issued = false;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const Tile tl = decode_tile<MODE>(nb, t, args);
+                const Tile tl = decode_tile<MODE>(nb, t, args, splan);
                 if (tl.kb0 >= tl.kb1) continue;
                 if (!bounded_wait(ptx::smem_u32(&ctl->tempty[acc]), aph ^ 1u, ctl, args.err)) {
                     ok = false;
@@ -419,7 +441,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int acc = 0;
         uint32_t aph = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
-            const Tile tl = decode_tile<MODE>(nb, t, args);
+            const Tile tl = decode_tile<MODE>(nb, t, args, splan);
             if (tl.kb0 >= tl.kb1) continue;
             const bool ok = bounded_wait(ptx::smem_u32(&ctl->tfull[acc]), aph, ctl, args.err);
             if (!__all_sync(0xffffffffu, ok)) break;   // the whole warp leaves together

@@ -190,6 +190,12 @@ TopkSource topk_source(const RouterSplit& rs, float* logits, float* partials, co
 
 int run_topk(const TopkSource& s, int T, int E, int k, int32_t* idx, float* w, uint32_t* err, cudaStream_t st)
 {
+    if (s.splits > 1) {
+        // split router: one CTA per token, one thread per expert sums the partials
+        const int threads = (E + 31) / 32 * 32;
+        return status_of(launch(topk_token_cta_kernel, dim3(T), dim3(threads), 0, st, s.src, s.stride, s.splits,
+                                s.bias, T, E, k, s.logits_out, idx, w, err));
+    }
     return status_of(launch(topk_softmax_kernel, dim3((T + 7) / 8), dim3(256), 0, st, s.src, s.stride, s.splits,
                             s.bias, T, E, k, s.logits_out, idx, w, err));
 }
@@ -471,20 +477,18 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
         return rc;
     const TopkSource src = topk_source(rs, logits, partials, bias, iT, iE);
     const int64_t P = T * k;
-    if (T <= kSmallTokens) {
-        // one CTA: top-k, histogram, scan, stable ranks and the tile plan
-        phase_mark(prof, 1, st);
-        if (launch(route_permute_small_kernel, dim3(1), dim3(1024), 0, st, src.src, src.stride, src.splits, src.bias,
-                   iT, iE, ik, src.logits_out, idx, w, counts, offsets, perm, inv_perm, plan, (int)f, id, shared_rows,
-                   (int)f_shared, err) != cudaSuccess)
+    if ((rc = run_topk(src, iT, iE, ik, idx, w, err, st))) return rc;
+    phase_mark(prof, 1, st);
+    if (P <= kSmallPairs) {
+        // one CTA: histogram, scan, stable ranks and the tile plan
+        if (launch(permute_small_kernel, dim3(1), dim3(1024), 0, st, (const int32_t*)idx, (int)P, iE, counts, offsets,
+                   perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared, err) != cudaSuccess)
             return MOE_ERR_CUDA;
         const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)dev->sm_count * 16));
         if (launch(gather_rows_kernel, dim3(blocks), dim3(256), 0, st, xb, (const int32_t*)perm,
                    (const int32_t*)offsets, iE, ik, id, xp) != cudaSuccess)
             return MOE_ERR_CUDA;
     } else {
-        if ((rc = run_topk(src, iT, iE, ik, idx, w, err, st))) return rc;
-        phase_mark(prof, 1, st);
         if ((rc = run_permute(idx, xb, iT, id, iE, ik, counts, offsets, perm, inv_perm, xp, err,
                               at<int32_t>(ws, L.block_counts), plan, (int)f, shared_rows, (int)f_shared,
                               dev->sm_count, st)))

@@ -211,70 +211,67 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
     build_plan(c, off, E, offsets[E], plan, f, d, shared_rows, f_shared, warp_sums);
 }
 
-// ---------------------------------------------------------------- small-T fused routing + permutation
-// One CTA of 1024 threads does S2-S4 (minus the row gather) and the tile plan
-// when T <= kSmallTokens (then T*k <= 1024 <= kSmallPairs): top-k per token (one warp per token, summing the
-// router's split-K partials), histogram, scan, stable ranks and the plan, so a
-// decode-sized layer pays one launch instead of five.
-constexpr int kSmallTokens = 128;
-constexpr int kSmallPairs = kSmallTokens * kMaxTopK;
+// ---------------------------------------------------------------- small-T permutation
+// One CTA of 1024 threads does S3-S4 (minus the row gather) and the tile plan
+// when T*k <= 1024 (one pair per thread): per-warp expert counts by match_any,
+// histogram, scan, stable positions and the plan, in one launch instead of
+// three.
+constexpr int kSmallPairs = 1024;
 
-__global__ void __launch_bounds__(1024) route_permute_small_kernel(
-    const float* __restrict__ Lp, size_t split_stride, int splits, const float* __restrict__ bias, int T, int E, int k,
-    float* __restrict__ logits_out, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
-    int32_t* __restrict__ inv_perm, int32_t* __restrict__ plan, int f, int d, int shared_rows, int f_shared,
-    uint32_t* __restrict__ err)
+__global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t* __restrict__ topk_idx, int P, int E,
+                                                             int32_t* __restrict__ counts,
+                                                             int32_t* __restrict__ offsets,
+                                                             int32_t* __restrict__ perm,
+                                                             int32_t* __restrict__ inv_perm,
+                                                             int32_t* __restrict__ plan, int f, int d,
+                                                             int shared_rows, int f_shared,
+                                                             uint32_t* __restrict__ err)
 {
-    __shared__ int s_idx[kSmallPairs];
-    __shared__ int s_cnt[kMaxExperts];
-    __shared__ int s_run[kMaxExperts];
+    // s_wcnt[w][e]: pairs of warp w (pairs 32w..32w+31) routed to expert e (<= 32)
+    __shared__ __align__(16) uint8_t s_wcnt[32][kMaxExperts];
+    __shared__ int s_off[kMaxExperts];
     __shared__ int warp_sums[32];
     ptx::grid_dep_wait();
     ptx::grid_dep_launch();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int P = T * k;
-    // 1. top-k, one warp per token
-    for (int t = warp; t < T; t += 32)
-        topk_warp_any(Lp, split_stride, splits, bias, t, E, k, logits_out, topk_idx, topk_w, err, s_idx);
-    for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = 0;
+    reinterpret_cast<uint4*>(&s_wcnt[0][0])[tid] = make_uint4(0, 0, 0, 0);   // 1024 x 16 B = the whole table
+    const int q = tid;
+    int e = q < P ? topk_idx[q] : -1;
+    if (e >= E || (q < P && e < 0)) {
+        atomicOr(err, DEVERR_EXPERT_RANGE);
+        inv_perm[q] = -1;
+        e = -1;
+    }
     __syncthreads();
-    // 2. histogram (the ids come from the top-k above, so they are all in range)
-    for (int q = tid; q < P; q += blockDim.x) atomicAdd(&s_cnt[s_idx[q]], 1);
+    // per-warp counts: pairs of one warp with the same expert are ranked by lane
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (e >= 0 && lane == __ffs(peers) - 1) s_wcnt[warp][e] = (uint8_t)__popc(peers);
     __syncthreads();
-    // 3. scan
-    const int c = tid < E ? s_cnt[tid] : 0;
-    const int incl = block_inclusive_scan(c, warp_sums);
+    // histogram and scan
+    int c = 0;
+    if (tid < E)
+        for (int w = 0; w < 32; w++) c += s_wcnt[w][tid];
+    const int incl = block_inclusive_scan(tid < E ? c : 0, warp_sums);
     const int off = incl - c;
     if (tid < E) {
         counts[tid] = c;
         offsets[tid] = off;
-        s_run[tid] = off;
+        s_off[tid] = off;
     }
     if (tid == E - 1) offsets[E] = incl;
     __syncthreads();
-    // 4. stable ranks: pairs in ascending q, 1024 at a time; inside a warp by lane
-    //    order (match_any), warps in turn
-    const unsigned lt_mask = (1u << lane) - 1u;
-    for (int base = 0; base < P; base += blockDim.x) {
-        const int q = base + tid;
-        const int e = q < P ? s_idx[q] : -1;
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
-        const int rank = __popc(peers & lt_mask);
-        const int leader = __ffs(peers) - 1;
-        for (int w = 0; w < (int)(blockDim.x >> 5); w++) {
-            if (warp == w && e >= 0) {
-                const int pos = s_run[e] + rank;
-                perm[pos] = q;
-                inv_perm[q] = pos;
-            }
-            __syncwarp();
-            if (warp == w && e >= 0 && lane == leader) s_run[e] += __popc(peers);
-            __syncthreads();
-        }
+    // stable position: offsets[e] + pairs of e in earlier warps + rank in the warp
+    if (e >= 0) {
+        int pos = s_off[e] + rank;
+        for (int w = 0; w < warp; w++) pos += s_wcnt[w][e];
+        perm[pos] = q;
+        inv_perm[q] = pos;
     }
-    // 5. tile plan
-    if (plan) build_plan(c, off, E, P, plan, f, d, shared_rows, f_shared, warp_sums);
+    __shared__ int s_pairs;
+    if (tid == E - 1) s_pairs = incl;
+    __syncthreads();
+    if (plan) build_plan(c, off, E, s_pairs, plan, f, d, shared_rows, f_shared, warp_sums);
 }
 
 // ---------------------------------------------------------------- scatter
@@ -333,12 +330,21 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const bf16* __restrict
     const int pairs = offsets[E];
     const int nvec = d / 8;
     const int lane = threadIdx.x & 31;
+    constexpr int kUnroll = 8;
     for (int64_t r = (int64_t)(blockIdx.x * blockDim.x + threadIdx.x) / 32; r < pairs;
          r += (int64_t)gridDim.x * blockDim.x / 32) {
         const int t = perm[r] / k;
         const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
         uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * d);
-        for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+        for (int v0 = lane; v0 < nvec; v0 += 32 * kUnroll) {
+            uint4 buf[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; u++)
+                if (v0 + 32 * u < nvec) buf[u] = __ldg(src + v0 + 32 * u);
+#pragma unroll
+            for (int u = 0; u < kUnroll; u++)
+                if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = buf[u];
+        }
     }
 }
 

@@ -90,7 +90,7 @@ __device__ __forceinline__ float key_logit(uint32_t key)
 // logits themselves when splits == 1).  When logits_out != null that value is
 // stored there.  Writes idx/w for the token (and the ids to s_idx when given).
 template <int PER>
-__device__ __forceinline__ void topk_warp(const float* __restrict__ Lp, size_t split_stride, int splits,
+__device__ __forceinline__ void topk_warp(const float* Lp, size_t split_stride, int splits,
                                           const float* __restrict__ bias, int t, int E, int k,
                                           float* __restrict__ logits_out, int32_t* __restrict__ topk_idx,
                                           float* __restrict__ topk_w, uint32_t* __restrict__ err, int* s_idx)
@@ -105,13 +105,15 @@ __device__ __forceinline__ void topk_warp(const float* __restrict__ Lp, size_t s
         const int e = lane + 32 * i;
         cand[i] = 0;   // below every real candidate (real ones have a nonzero low word or key)
         if (e < E) {
+            // __ldcg: the logits may have been written earlier in this very kernel
             const float* p = Lp + (size_t)t * E + e;
-            float v = p[0];
+            float v = __ldcg(p);
             // partials in ascending order, fetched 8 at a time so the loads overlap
             for (int sp = 1; sp < splits; sp += 8) {
                 float part[8];
 #pragma unroll
-                for (int u = 0; u < 8; u++) part[u] = sp + u < splits ? p[(size_t)(sp + u) * split_stride] : 0.f;
+                for (int u = 0; u < 8; u++)
+                    part[u] = sp + u < splits ? __ldcg(p + (size_t)(sp + u) * split_stride) : 0.f;
 #pragma unroll
                 for (int u = 0; u < 8; u++)
                     if (sp + u < splits) v += part[u];
@@ -167,7 +169,7 @@ __device__ __forceinline__ void topk_warp(const float* __restrict__ Lp, size_t s
 }
 
 // topk_warp with the smallest per-lane candidate array that holds E logits.
-__device__ __forceinline__ void topk_warp_any(const float* __restrict__ Lp, size_t split_stride, int splits,
+__device__ __forceinline__ void topk_warp_any(const float* Lp, size_t split_stride, int splits,
                                               const float* __restrict__ bias, int t, int E, int k,
                                               float* __restrict__ logits_out, int32_t* __restrict__ topk_idx,
                                               float* __restrict__ topk_w, uint32_t* __restrict__ err, int* s_idx)
@@ -180,6 +182,40 @@ __device__ __forceinline__ void topk_warp_any(const float* __restrict__ Lp, size
         topk_warp<8>(Lp, split_stride, splits, bias, t, E, k, logits_out, topk_idx, topk_w, err, s_idx);
     else
         topk_warp<16>(Lp, split_stride, splits, bias, t, E, k, logits_out, topk_idx, topk_w, err, s_idx);
+}
+
+// One CTA per token (blockDim >= E, a multiple of 32) for a split router:
+// thread e adds the token's split-K partials of expert e (ascending order,
+// fetched 8 at a time) and the bias, stores the logit, and warp 0 then runs the
+// top-k on the summed logits.  The partial sums are spread over E threads
+// instead of E/32 per lane, which keeps small-T routing off the latency path.
+__global__ void __launch_bounds__(512) topk_token_cta_kernel(const float* __restrict__ Lp, size_t split_stride,
+                                                             int splits, const float* __restrict__ bias, int T,
+                                                             int E, int k, float* logits_out,
+                                                             int32_t* __restrict__ topk_idx,
+                                                             float* __restrict__ topk_w, uint32_t* __restrict__ err)
+{
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
+    const int t = blockIdx.x;
+    const int e = threadIdx.x;
+    if (e < E) {
+        const float* p = Lp + (size_t)t * E + e;
+        float v = p[0];
+        for (int sp = 1; sp < splits; sp += 8) {
+            float part[8];
+#pragma unroll
+            for (int u = 0; u < 8; u++) part[u] = sp + u < splits ? p[(size_t)(sp + u) * split_stride] : 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; u++)
+                if (sp + u < splits) v += part[u];
+        }
+        if (bias) v += bias[e];
+        logits_out[(size_t)t * E + e] = v;
+    }
+    __syncthreads();   // the block's global writes are visible to its own threads after the barrier
+    if (threadIdx.x < 32)
+        topk_warp_any(logits_out, 0, 1, nullptr, t, E, k, nullptr, topk_idx, topk_w, err, nullptr);
 }
 
 // One warp per token; E <= 512 (16 logits per lane), k <= 8.
