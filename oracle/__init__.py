@@ -38,6 +38,22 @@ def load(path: str) -> C.CDLL:
                                  u16p, u16p, u16p, i64, C.POINTER(i64), i64, f64p, C.c_int]
     for fn in ("oracle_router_logits", "oracle_topk", "oracle_permutation", "oracle_moe_ffn"):
         getattr(L, fn).restype = C.c_int
+    u8p = C.POINTER(C.c_uint8)
+    u8pp, f64pp = C.POINTER(u8p), C.POINTER(f64p)
+    L.oracle_e4m3_decode.argtypes = [C.c_uint8]
+    L.oracle_e4m3_decode.restype = C.c_double
+    L.oracle_e4m3_encode.argtypes = [C.c_double]
+    L.oracle_e4m3_encode.restype = C.c_uint8
+    L.oracle_e4m3_encode_fast.argtypes = [C.c_double]
+    L.oracle_e4m3_encode_fast.restype = C.c_uint8
+    L.oracle_fp8_block_scale.argtypes = [C.c_double]
+    L.oracle_fp8_block_scale.restype = C.c_double
+    L.oracle_quantize_rows_fp8.argtypes = [u16p, i64, i64, u8p, f64p]
+    L.oracle_quantize_blocks_fp8.argtypes = [u16p, i64, i64, u8p, f64p]
+    L.oracle_moe_ffn_fp8.argtypes = [u8p, f64p, u8pp, f64pp, u8pp, f64pp, u8pp, f64pp, i64, i64, i64, i32p, f64p,
+                                     i64, u8p, f64p, u8p, f64p, u8p, f64p, i64, C.POINTER(i64), i64, f64p, C.c_int]
+    for fn in ("oracle_quantize_rows_fp8", "oracle_quantize_blocks_fp8", "oracle_moe_ffn_fp8"):
+        getattr(L, fn).restype = C.c_int
     return L
 
 
@@ -171,3 +187,95 @@ def moe_layer(x, Wg, bias, W1, W3, W2, k: int, shared=None, tokens=None, nthread
     out = moe_ffn(x, W1, W3, W2, idx, w, shared=shared, tokens=tokens, nthreads=nthreads)
     return dict(L64=L64, L32=L32, idx=idx, w=w, counts=counts, offsets=offsets, perm=perm,
                 inv_perm=inv, out=out)
+
+
+# ---------------------------------------------------------------- FP8 (e4m3, power-of-two block scales)
+
+def e4m3_decode(code: int) -> float:
+    return float(lib().oracle_e4m3_decode(int(code)))
+
+
+def e4m3_encode(v: float) -> int:
+    """Nearest e4m3 code (ties to even), saturating to +-448: the definition (walks every code)."""
+    return int(lib().oracle_e4m3_encode(float(v)))
+
+
+def e4m3_encode_fast(v: float) -> int:
+    """The same rounding computed from the binary exponent (used by the quantisers)."""
+    return int(lib().oracle_e4m3_encode_fast(float(v)))
+
+
+def fp8_block_scale(amax: float) -> float:
+    """Smallest power of two s with amax / s <= 448 (1 for amax = 0)."""
+    return float(lib().oracle_fp8_block_scale(float(amax)))
+
+
+def quantize_rows_fp8(x: np.ndarray):
+    """1 x 128 blocks along rows: bf16 bits [R, C] -> (e4m3 codes [R, C], scales [R, C/128])."""
+    x = _u16(x)
+    R, Cc = x.shape
+    q = np.empty((R, Cc), dtype=np.uint8)
+    sc = np.empty((R, Cc // 128), dtype=np.float64)
+    _check(lib().oracle_quantize_rows_fp8(_ptr(x, C.c_uint16), R, Cc, _ptr(q, C.c_uint8), _ptr(sc, C.c_double)),
+           "quantize_rows_fp8")
+    return q, sc
+
+
+def quantize_blocks_fp8(W: np.ndarray):
+    """128 x 128 blocks: bf16 bits [R, C] -> (e4m3 codes [R, C], scales [R/128, C/128])."""
+    W = _u16(W)
+    R, Cc = W.shape
+    q = np.empty((R, Cc), dtype=np.uint8)
+    sc = np.empty((R // 128, Cc // 128), dtype=np.float64)
+    _check(lib().oracle_quantize_blocks_fp8(_ptr(W, C.c_uint16), R, Cc, _ptr(q, C.c_uint8), _ptr(sc, C.c_double)),
+           "quantize_blocks_fp8")
+    return q, sc
+
+
+def moe_ffn_fp8(xq, sx, W1q, s1, W3q, s3, W2q, s2, idx, w, shared=None, tokens=None, nthreads: int = 0):
+    """fp64 y[t] = sum_j w[t,j] FFN8_e(x^_t) (+ shared) on dequantised e4m3 operands, with h
+    requantised in 1 x 128 blocks before the down projection.  Per-expert lists may hold None
+    for experts no listed token uses; shared = dict(W1q, s1, W3q, s3, W2q, s2)."""
+    xq = np.ascontiguousarray(xq, dtype=np.uint8)
+    sx = np.ascontiguousarray(sx, dtype=np.float64)
+    T, d = xq.shape
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    k = idx.shape[1]
+    E = len(W1q)
+    f = next(a.shape[0] for a in W1q if a is not None)
+    up, dp = C.POINTER(C.c_uint8), C.POINTER(C.c_double)
+    keep = []
+
+    def arr(lst, ct, dt):
+        vals = []
+        for a in lst:
+            if a is None:
+                vals.append(C.POINTER(ct)())
+            else:
+                a = np.ascontiguousarray(a, dtype=dt)
+                keep.append(a)
+                vals.append(_ptr(a, ct))
+        return (C.POINTER(ct) * E)(*vals)
+
+    pw1, pw3, pw2 = arr(W1q, C.c_uint8, np.uint8), arr(W3q, C.c_uint8, np.uint8), arr(W2q, C.c_uint8, np.uint8)
+    ps1, ps3, ps2 = arr(s1, C.c_double, np.float64), arr(s3, C.c_double, np.float64), arr(s2, C.c_double, np.float64)
+    fs = 0
+    sh = [None] * 6
+    if shared is not None:
+        sh = [np.ascontiguousarray(shared[n], dtype=(np.uint8 if n.endswith("q") else np.float64))
+              for n in ("W1q", "s1", "W3q", "s3", "W2q", "s2")]
+        fs = sh[0].shape[0]
+    if tokens is None:
+        tok, ntok = None, T
+    else:
+        tok = np.ascontiguousarray(tokens, dtype=np.int64)
+        ntok = tok.size
+    out = np.empty((ntok, d), dtype=np.float64)
+    _check(lib().oracle_moe_ffn_fp8(_ptr(xq, C.c_uint8), _ptr(sx, C.c_double), pw1, ps1, pw3, ps3, pw2, ps2, d, f, E,
+                                    _ptr(idx, C.c_int32), _ptr(w, C.c_double), k,
+                                    _ptr(sh[0], C.c_uint8), _ptr(sh[1], C.c_double), _ptr(sh[2], C.c_uint8),
+                                    _ptr(sh[3], C.c_double), _ptr(sh[4], C.c_uint8), _ptr(sh[5], C.c_double), fs,
+                                    _ptr(tok, C.c_int64), ntok, _ptr(out, C.c_double), int(nthreads)),
+           "moe_ffn_fp8")
+    return out

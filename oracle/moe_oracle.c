@@ -286,3 +286,294 @@ int oracle_moe_ffn(const uint16_t *x,
     free(th);
     return status;
 }
+
+/* ------------------------------------------------------------------------
+ * FP8 block-scaled variant (GC-MoE, abstract: an FP8 MoE operator with
+ * block-scaled MMA and requantisation; the workload table fixes e4m3 codes
+ * with 1x128 activation blocks and 128x128 weight blocks).
+ *
+ * e4m3 (OCP 8-bit floating point, E4M3 variant): 1 sign bit, 4 exponent bits
+ * with bias 7, 3 mantissa bits; no infinities; exponent field 15 with mantissa
+ * 7 is NaN; largest finite value 1.75 * 2^8 = 448; normal values
+ * (1 + m/8) * 2^(e-7) for e = 1..15; subnormals (m/8) * 2^-6.
+ *
+ * Readings taken: a value is encoded by round-to-nearest, ties to the even
+ * code, and magnitudes past 448 saturate to 448.  A block's scale is the
+ * smallest power of two s with amax / s <= 448 (amax = 0 gives s = 1), so
+ * v / s is exact and the dequantised value of code q is decode(q) * s.
+ * ------------------------------------------------------------------------ */
+
+double oracle_e4m3_decode(uint8_t code)
+{
+    int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* Nearest e4m3 code to v (ties to the code with an even mantissa), saturating to 448. */
+uint8_t oracle_e4m3_encode(double v)
+{
+    uint8_t sign = (v < 0 || (v == 0 && signbit(v))) ? 0x80 : 0;
+    double a = fabs(v);
+    if (isnan(v))
+        return 0x7F;
+    if (a >= 448.0)
+        return sign | 0x7E;   /* 448: exponent field 15, mantissa 6 */
+    /* Walk the 127 finite non-negative codes in increasing order; keep the nearest. */
+    uint8_t best = 0;
+    double best_err = a;      /* code 0 is +0 */
+    for (int c = 1; c <= 0x7E; c++) {
+        double err = fabs(oracle_e4m3_decode((uint8_t)c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {
+            best = (uint8_t)c;
+            best_err = err;
+        }
+    }
+    return sign | best;
+}
+
+/* The same rounding computed from the value's binary exponent instead of a
+ * walk over every code (the block quantisers use this one; a test checks it
+ * against oracle_e4m3_encode on every code, every midpoint and random values). */
+uint8_t oracle_e4m3_encode_fast(double v)
+{
+    uint8_t sign = (v < 0 || (v == 0 && signbit(v))) ? 0x80 : 0;
+    double a = fabs(v);
+    if (isnan(v))
+        return 0x7F;
+    if (a >= 448.0)
+        return sign | 0x7E;
+    if (a < ldexp(1.0, -6)) {                 /* subnormal range: steps of 2^-9 */
+        double m = nearbyint(a * 512.0);       /* ties to even (default rounding mode) */
+        return sign | (uint8_t)m;              /* m == 8 is the smallest normal, code 0x08 */
+    }
+    int e;
+    double frac = frexp(a, &e);               /* a = frac * 2^e, frac in [0.5, 1) */
+    int ex = e - 1;                            /* a = (2 frac) * 2^ex, 2 frac in [1, 2) */
+    double m = nearbyint((2.0 * frac - 1.0) * 8.0);
+    if (m == 8.0) {
+        m = 0.0;
+        ex += 1;
+    }
+    int field = ex + 7;
+    if (field > 15 || (field == 15 && m > 6.0))
+        return sign | 0x7E;
+    return sign | (uint8_t)((field << 3) | (int)m);
+}
+
+static double g_e4m3[256];
+static pthread_once_t g_e4m3_once = PTHREAD_ONCE_INIT;
+static void e4m3_table_init(void)
+{
+    for (int c = 0; c < 256; c++)
+        g_e4m3[c] = oracle_e4m3_decode((uint8_t)c);
+}
+static double e4m3_value(uint8_t c)
+{
+    pthread_once(&g_e4m3_once, e4m3_table_init);
+    return g_e4m3[c];
+}
+
+/* Smallest power of two s with amax / s <= 448 (amax = 0: s = 1). */
+double oracle_fp8_block_scale(double amax)
+{
+    if (!(amax > 0))
+        return 1.0;
+    int e = 0;
+    while (amax > ldexp(448.0, e))
+        e++;
+    while (amax <= ldexp(448.0, e - 1))
+        e--;
+    return ldexp(1.0, e);
+}
+
+/* 1 x 128 blocks along each row: x [R, C] bf16 -> q [R, C], s [R, C/128]. C % 128 == 0. */
+int oracle_quantize_rows_fp8(const uint16_t *x, int64_t R, int64_t C, uint8_t *q, double *s)
+{
+    if (R < 0 || C <= 0 || C % 128 || (R > 0 && (!x || !q || !s)))
+        return ORACLE_EARG;
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t b = 0; b < C / 128; b++) {
+            double amax = 0;
+            for (int64_t c = 0; c < 128; c++)
+                amax = fmax(amax, fabs(bf16_value(x[r * C + b * 128 + c])));
+            double sc = oracle_fp8_block_scale(amax);
+            s[r * (C / 128) + b] = sc;
+            for (int64_t c = 0; c < 128; c++)
+                q[r * C + b * 128 + c] = oracle_e4m3_encode_fast(bf16_value(x[r * C + b * 128 + c]) / sc);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* 128 x 128 blocks: W [R, C] bf16 -> q [R, C], s [R/128, C/128].  R, C % 128 == 0. */
+int oracle_quantize_blocks_fp8(const uint16_t *W, int64_t R, int64_t C, uint8_t *q, double *s)
+{
+    if (R <= 0 || C <= 0 || R % 128 || C % 128 || !W || !q || !s)
+        return ORACLE_EARG;
+    for (int64_t br = 0; br < R / 128; br++) {
+        for (int64_t bc = 0; bc < C / 128; bc++) {
+            double amax = 0;
+            for (int64_t r = 0; r < 128; r++)
+                for (int64_t c = 0; c < 128; c++)
+                    amax = fmax(amax, fabs(bf16_value(W[(br * 128 + r) * C + bc * 128 + c])));
+            double sc = oracle_fp8_block_scale(amax);
+            s[br * (C / 128) + bc] = sc;
+            for (int64_t r = 0; r < 128; r++)
+                for (int64_t c = 0; c < 128; c++) {
+                    int64_t i = (br * 128 + r) * C + bc * 128 + c;
+                    q[i] = oracle_e4m3_encode_fast(bf16_value(W[i]) / sc);
+                }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* One FP8 SwiGLU expert on one token (all fp64 on dequantised values):
+ *   g = W1^ x^, u = W3^ x^, h = silu(g) * u,
+ *   h^ = h requantised in 1 x 128 blocks along f, y += gate * W2^ h^.
+ * W1q/W3q [f,d] with scales [f/128, d/128]; W2q [d,f] with [d/128, f/128];
+ * xq [d] with sx [d/128].  h, hq scratch of f doubles / f bytes. */
+static void expert_ffn_fp8_add(const uint8_t *W1q, const double *s1, const uint8_t *W3q, const double *s3,
+                               const uint8_t *W2q, const double *s2, const uint8_t *xq, const double *sx,
+                               int64_t d, int64_t f, double gate, double *h, double *y)
+{
+    const int64_t db = d / 128, fb = f / 128;
+    for (int64_t r = 0; r < f; r++) {
+        double g = 0.0, u = 0.0;
+        for (int64_t c = 0; c < d; c++) {
+            double xc = e4m3_value(xq[c]) * sx[c / 128];
+            g += e4m3_value(W1q[r * d + c]) * s1[(r / 128) * db + c / 128] * xc;
+            u += e4m3_value(W3q[r * d + c]) * s3[(r / 128) * db + c / 128] * xc;
+        }
+        h[r] = g / (1.0 + exp(-g)) * u;
+    }
+    for (int64_t b = 0; b < fb; b++) {          /* requantise h in 1 x 128 blocks */
+        double amax = 0;
+        for (int64_t r = 0; r < 128; r++)
+            amax = fmax(amax, fabs(h[b * 128 + r]));
+        double sc = oracle_fp8_block_scale(amax);
+        for (int64_t r = 0; r < 128; r++)
+            h[b * 128 + r] = e4m3_value(oracle_e4m3_encode_fast(h[b * 128 + r] / sc)) * sc;
+    }
+    for (int64_t c = 0; c < d; c++) {
+        double z = 0.0;
+        for (int64_t r = 0; r < f; r++)
+            z += e4m3_value(W2q[c * f + r]) * s2[(c / 128) * fb + r / 128] * h[r];
+        y[c] += gate * z;
+    }
+}
+
+typedef struct {
+    const uint8_t *xq;
+    const double *sx;
+    const uint8_t *const *W1q, *const *W3q, *const *W2q;
+    const double *const *s1, *const *s3, *const *s2;
+    int64_t d, f, E, k;
+    const int32_t *idx;
+    const double *w;
+    const uint8_t *Ws1q, *Ws3q, *Ws2q;
+    const double *ss1, *ss3, *ss2;
+    int64_t fs;
+    const int64_t *tokens;
+    int64_t ntok;
+    double *out;
+    int nthreads, tid;
+    int status;
+} ffn8_job;
+
+static void *ffn8_worker(void *arg)
+{
+    ffn8_job *J = (ffn8_job *)arg;
+    int64_t hlen = J->f > J->fs ? J->f : J->fs;
+    double *h = (double *)malloc((size_t)(hlen > 0 ? hlen : 1) * sizeof(double));
+    if (!h) {
+        J->status = ORACLE_ENOMEM;
+        return NULL;
+    }
+    const int64_t db = J->d / 128;
+    for (int64_t i = J->tid; i < J->ntok; i += J->nthreads) {
+        int64_t t = J->tokens ? J->tokens[i] : i;
+        const uint8_t *xt = J->xq + t * J->d;
+        const double *st = J->sx + t * db;
+        double *y = J->out + i * J->d;
+        for (int64_t c = 0; c < J->d; c++)
+            y[c] = 0.0;
+        for (int64_t j = 0; j < J->k; j++) {
+            int32_t e = J->idx[t * J->k + j];
+            if (e < 0 || e >= J->E || !J->W1q[e] || !J->W3q[e] || !J->W2q[e]) {
+                J->status = ORACLE_ERANGE;
+                free(h);
+                return NULL;
+            }
+            expert_ffn_fp8_add(J->W1q[e], J->s1[e], J->W3q[e], J->s3[e], J->W2q[e], J->s2[e], xt, st, J->d,
+                               J->f, J->w[t * J->k + j], h, y);
+        }
+        if (J->fs > 0)
+            expert_ffn_fp8_add(J->Ws1q, J->ss1, J->Ws3q, J->ss3, J->Ws2q, J->ss2, xt, st, J->d, J->fs, 1.0, h, y);
+    }
+    free(h);
+    return NULL;
+}
+
+/* FP8 expert FFNs of the listed tokens (the FP8 counterpart of oracle_moe_ffn).
+ * xq [T,d] e4m3 with sx [T, d/128]; per-expert W1q[e], W3q[e] [f,d] with
+ * s1[e], s3[e] [f/128, d/128]; W2q[e] [d,f] with s2[e] [d/128, f/128]; the
+ * shared expert likewise (fs > 0).  d, f, fs multiples of 128. */
+int oracle_moe_ffn_fp8(const uint8_t *xq, const double *sx,
+                       const uint8_t *const *W1q, const double *const *s1,
+                       const uint8_t *const *W3q, const double *const *s3,
+                       const uint8_t *const *W2q, const double *const *s2,
+                       int64_t d, int64_t f, int64_t E, const int32_t *idx, const double *w, int64_t k,
+                       const uint8_t *Ws1q, const double *ss1, const uint8_t *Ws3q, const double *ss3,
+                       const uint8_t *Ws2q, const double *ss2, int64_t fs,
+                       const int64_t *tokens, int64_t ntok, double *out, int nthreads)
+{
+    if (d <= 0 || f <= 0 || E <= 0 || k < 1 || ntok < 0 || fs < 0 || d % 128 || f % 128 || fs % 128)
+        return ORACLE_EARG;
+    if (ntok == 0)
+        return ORACLE_OK;
+    if (!xq || !sx || !W1q || !W3q || !W2q || !s1 || !s3 || !s2 || !idx || !w || !out ||
+        (fs > 0 && (!Ws1q || !Ws3q || !Ws2q || !ss1 || !ss3 || !ss2)))
+        return ORACLE_EARG;
+    if (nthreads <= 0)
+        nthreads = oracle_default_threads();
+    if (nthreads > ntok)
+        nthreads = (int)ntok;
+    ffn8_job *jobs = (ffn8_job *)calloc((size_t)nthreads, sizeof(ffn8_job));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !th) {
+        free(jobs);
+        free(th);
+        return ORACLE_ENOMEM;
+    }
+    for (int i = 0; i < nthreads; i++) {
+        ffn8_job J = {xq, sx, W1q, W3q, W2q, s1, s3, s2, d, f, E, k, idx, w, Ws1q, Ws3q, Ws2q, ss1, ss3, ss2,
+                      fs, tokens, ntok, out, nthreads, i, ORACLE_OK};
+        jobs[i] = J;
+    }
+    int started = 0;
+    for (int i = 1; i < nthreads; i++) {
+        if (pthread_create(&th[i], NULL, ffn8_worker, &jobs[i]) != 0)
+            break;
+        started = i;
+    }
+    for (int i = started + 1; i < nthreads; i++)
+        ffn8_worker(&jobs[i]);
+    ffn8_worker(&jobs[0]);
+    for (int i = 1; i <= started; i++)
+        pthread_join(th[i], NULL);
+    int status = ORACLE_OK;
+    for (int i = 0; i < nthreads; i++)
+        if (jobs[i].status != ORACLE_OK)
+            status = jobs[i].status;
+    free(jobs);
+    free(th);
+    return status;
+}

@@ -255,4 +255,182 @@ def pin_empty_batch():
     assert res["out"].shape == (0, s.d) and res["counts"].sum() == 0 and res["offsets"][-1] == 0
 
 
+# --------------------------------------------------------------------------- FP8
+
+def _torch_e4m3(codes: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.asarray(codes, dtype=np.uint8)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def pin_e4m3_decode_matches_library():
+    """Every one of the 256 codes decodes like torch's float8_e4m3fn (NaN codes included)."""
+    codes = np.arange(256, dtype=np.uint8)
+    mine = np.array([oracle.e4m3_decode(c) for c in codes])
+    ref = _torch_e4m3(codes)
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(mine[ok], ref[ok])
+    assert oracle.e4m3_decode(0x7E) == 448.0 and oracle.e4m3_decode(0x01) == 2.0 ** -9
+
+
+def _e4m3_grid() -> np.ndarray:
+    """Every finite code value, every midpoint between neighbours, tiny offsets around
+    them, random values across the range, both signs."""
+    vals = np.array(sorted({oracle.e4m3_decode(c) for c in range(0x7F)}))
+    mids = (vals[1:] + vals[:-1]) / 2
+    rng = np.random.default_rng(5)
+    rnd = np.exp(rng.uniform(np.log(2.0 ** -12), np.log(460.0), 4000))
+    g = np.concatenate([vals, mids, mids * (1 + 1e-9), mids * (1 - 1e-9), rnd])
+    return np.concatenate([g, -g])
+
+
+def pin_e4m3_encode_matches_library():
+    """Round to nearest, ties to even, against torch's float -> float8_e4m3fn cast (|v| < 464,
+    where torch also saturates to 448); above that the reading saturates to 448."""
+    g = _e4m3_grid()
+    g = g[np.abs(g) < 464]
+    mine = np.array([oracle.e4m3_encode(v) for v in g], dtype=np.uint8)
+    ref = torch.from_numpy(g).to(torch.float32).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    # the fp64 -> fp32 step is exact for the grid's code values and midpoints; compare on those
+    # and on values whose fp32 rounding cannot cross a midpoint
+    exact = g.astype(np.float32).astype(np.float64) == g
+    assert np.array_equal(mine[exact], ref[exact])
+    for v in (500.0, 1e6, -3e4):
+        assert oracle.e4m3_decode(oracle.e4m3_encode(v)) == np.sign(v) * 448.0
+
+
+def pin_e4m3_fast_encoder_equals_definition():
+    g = _e4m3_grid()
+    g = np.concatenate([g, [0.0, -0.0, 448.0, 470.0, 1e9, 2.0 ** -10, 3 * 2.0 ** -10, 2.0 ** -6 - 2.0 ** -10]])
+    a = np.array([oracle.e4m3_encode(v) for v in g])
+    b = np.array([oracle.e4m3_encode_fast(v) for v in g])
+    assert np.array_equal(a, b)
+
+
+def pin_fp8_block_scale():
+    rng = np.random.default_rng(6)
+    for amax in np.concatenate([np.exp(rng.uniform(-30, 30, 500)), [448.0, 449.0, 447.9, 896.0, 1.0, 2.0 ** -20]]):
+        s = oracle.fp8_block_scale(amax)
+        m, e = np.frexp(s)
+        assert m == 0.5                              # a power of two
+        assert amax / s <= 448.0 < amax / (s / 2)    # the smallest such
+    assert oracle.fp8_block_scale(0.0) == 1.0
+
+
+def pin_fp8_quantize_rows_and_blocks():
+    gen = torch.Generator().manual_seed(21)
+    x = (torch.randn(6, 384, generator=gen) * torch.logspace(-3, 3, 6)[:, None]).to(torch.bfloat16)
+    x[2, 128:256] = 0
+    xb = _bits(x)
+    q, sc = oracle.quantize_rows_fp8(xb)
+    xv = x.to(torch.float64).numpy()
+    for r in range(6):
+        for b in range(3):
+            blk = xv[r, 128 * b:128 * (b + 1)]
+            s_ = sc[r, b]
+            assert s_ == oracle.fp8_block_scale(np.abs(blk).max())
+            ref = torch.from_numpy(blk / s_).to(torch.float32).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            assert np.array_equal(q[r, 128 * b:128 * (b + 1)], ref)
+    W = (torch.randn(256, 384, generator=gen) * 0.02).to(torch.bfloat16)
+    W[:128, 256:] *= 1000
+    Wq, Ws = oracle.quantize_blocks_fp8(_bits(W))
+    Wv = W.to(torch.float64).numpy()
+    for br in range(2):
+        for bc in range(3):
+            blk = Wv[128 * br:128 * (br + 1), 128 * bc:128 * (bc + 1)]
+            assert Ws[br, bc] == oracle.fp8_block_scale(np.abs(blk).max())
+            ref = torch.from_numpy(blk / Ws[br, bc]).to(torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)
+            assert np.array_equal(Wq[128 * br:128 * (br + 1), 128 * bc:128 * (bc + 1)], ref.numpy())
+
+
+def _fp8_layer(E=3, k=2, T=5, d=256, f=256, fs=0, seed=30):
+    s = wl.LayerShape("p8", T=T, d=d, f=f, E=E, k=k, alpha=1.0, f_shared=fs)
+    inp = wl.make_inputs(s, seed=seed)
+    xq, sx = oracle.quantize_rows_fp8(_bits(inp["x"]))
+    Q = {}
+    for n in ("W1", "W3", "W2"):
+        Q[n] = [oracle.quantize_blocks_fp8(_bits(inp[n][e])) for e in range(E)]
+    sh = None
+    if fs:
+        sh = {}
+        for n, key in (("Ws1", "1"), ("Ws3", "3"), ("Ws2", "2")):
+            q_, s_ = oracle.quantize_blocks_fp8(_bits(inp[n]))
+            sh["W%sq" % key], sh["s%s" % key] = q_, s_
+    return s, inp, xq, sx, Q, sh
+
+
+def _dq(q, s, rows_per=128, cols_per=128):
+    v = _torch_e4m3(q)
+    return v * np.repeat(np.repeat(s, rows_per, axis=0), cols_per, axis=1)
+
+
+def _requant_h(h):
+    """1 x 128 requantisation of h rows with the library cast (|h / s| <= 448 by construction)."""
+    out = np.empty_like(h)
+    for b in range(h.shape[1] // 128):
+        blk = h[:, 128 * b:128 * (b + 1)]
+        sc = np.array([oracle.fp8_block_scale(a) for a in np.abs(blk).max(axis=1)])
+        c = torch.from_numpy(blk / sc[:, None]).to(torch.float8_e4m3fn)   # direct fp64 -> e4m3 cast
+        out[:, 128 * b:128 * (b + 1)] = c.to(torch.float64).numpy() * sc[:, None]
+    return out
+
+
+def pin_fp8_ffn_expert_major():
+    """Expert-major evaluation with the library's e4m3 decode, float64 matmuls, and the
+    library cast for the requantisation of h; shared expert included."""
+    s, inp, xq, sx, Q, sh = _fp8_layer(fs=128)
+    idx = wl.random_routing(s.T, s.E, s.k, 1.0, 3).numpy()
+    w = wl.random_gates(s.T, s.k, 3).numpy().astype(np.float64)
+    y = oracle.moe_ffn_fp8(xq, sx, [q for q, _ in Q["W1"]], [c for _, c in Q["W1"]], [q for q, _ in Q["W3"]],
+                           [c for _, c in Q["W3"]], [q for q, _ in Q["W2"]], [c for _, c in Q["W2"]], idx, w,
+                           shared=sh)
+    xh = _dq(xq, sx, 1, 128)
+
+    def ffn(W1q, s1, W3q, s3, W2q, s2):
+        g = xh @ _dq(W1q, s1).T
+        u = xh @ _dq(W3q, s3).T
+        h = torch.nn.functional.silu(torch.from_numpy(g)).numpy() * u
+        return _requant_h(h) @ _dq(W2q, s2).T
+
+    ref = np.zeros((s.T, s.d))
+    for e in range(s.E):
+        gate = np.array([w[t][list(idx[t]).index(e)] if e in idx[t] else 0.0 for t in range(s.T)])
+        ref += gate[:, None] * ffn(*Q["W1"][e], *Q["W3"][e], *Q["W2"][e])
+    ref += ffn(sh["W1q"], sh["s1"], sh["W3q"], sh["s3"], sh["W2q"], sh["s2"])
+    assert np.allclose(y, ref, rtol=1e-10, atol=1e-12)
+
+
+def pin_fp8_ffn_exact_operands_match_bf16_path():
+    """With weights and activations that e4m3 holds exactly (scales 1) and h values that the
+    requantisation keeps exactly, the FP8 FFN equals the bf16 FFN on the same values."""
+    E, T, d, f = 2, 3, 128, 128
+    rng = np.random.default_rng(8)
+    pick = lambda shape: rng.choice([0.0, 0.5, -0.5, 0.25, -0.25, 0.125], size=shape)
+    x = torch.from_numpy(pick((T, d))).to(torch.bfloat16)
+    W1 = torch.from_numpy(pick((E, f, d)) / 8).to(torch.bfloat16)
+    W3 = torch.zeros(E, f, d, dtype=torch.bfloat16)
+    W3[:, :, 0] = 1.0                                    # u = x[:, 0], one of the exact values above
+    W2 = torch.from_numpy(pick((E, d, f))).to(torch.bfloat16)
+    idx = np.array([[0, 1], [1, 0], [0, 1]], dtype=np.int32)
+    w = np.array([[0.75, 0.25], [0.5, 0.5], [1.0, 0.0]])
+    y16 = oracle.moe_ffn(_bits(x), _bits(W1), _bits(W3), _bits(W2), idx, w)
+    xq, sx = oracle.quantize_rows_fp8(_bits(x))
+    assert np.array_equal(_dq(xq, sx, 1, 128), x.to(torch.float64).numpy())
+    Qs = {n: [oracle.quantize_blocks_fp8(_bits(t[e])) for e in range(E)] for n, t in (("1", W1), ("3", W3), ("2", W2))}
+    y8 = oracle.moe_ffn_fp8(xq, sx, [q for q, _ in Qs["1"]], [c for _, c in Qs["1"]], [q for q, _ in Qs["3"]],
+                            [c for _, c in Qs["3"]], [q for q, _ in Qs["2"]], [c for _, c in Qs["2"]], idx, w)
+    # h = silu(g) * u is not exact in e4m3, so the two differ only by the requantisation of h:
+    # bound it by the e4m3 half-step (2^-4 relative) times sum |W2| |h|
+    h_bound = np.zeros_like(y16)
+    xv = x.to(torch.float64).numpy()
+    for t in range(T):
+        for j in range(2):
+            e = idx[t, j]
+            g = W1[e].double().numpy() @ xv[t]
+            u = W3[e].double().numpy() @ xv[t]
+            h = torch.nn.functional.silu(torch.from_numpy(g)).numpy() * u
+            h_bound[t] += w[t, j] * (np.abs(W2[e].double().numpy()) @ np.abs(h)) * 2.0 ** -4
+    assert np.all(np.abs(y8 - y16) <= h_bound + 1e-12)
+    assert np.abs(y8 - y16).max() > 0 or np.allclose(h_bound, 0)
+
+
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]
