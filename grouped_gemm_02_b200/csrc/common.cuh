@@ -15,6 +15,7 @@ enum : uint32_t {
     DEVERR_EXPERT_RANGE = 1u,   // a top-k expert id outside [0, E): that pair is dropped
     DEVERR_TIMEOUT = 2u,        // a bounded wait inside a kernel gave up
     DEVERR_NAN_LOGIT = 4u,      // a router logit was NaN (ranked below every number)
+    DEVERR_PLAN = 8u,           // a kernel met a tile plan it cannot run (it did nothing)
 };
 
 constexpr int kMaxExperts = 512;
@@ -146,6 +147,42 @@ __host__ inline WsLayout ws_layout(int64_t T, int64_t d, int64_t f, int64_t E, i
     L.y_p = o; o = align_up(o + (size_t)P * d * 2, 1024);
     L.hs = o; o = align_up(o + (size_t)(fs > 0 ? T : 0) * fs * 2, 1024);
     L.ys = o; o = align_up(o + (size_t)(fs > 0 ? T : 0) * d * 2, 1024);
+    L.total = o;
+    return L;
+}
+
+// Workspace of the FP8 layer: the same control part, then the routing
+// intermediates, e4m3 activations with their 1 x 128 scales, and y_p.
+struct WsLayoutFp8 {
+    WsLayout ctrl;   // err, plan, block_counts, router_partials, ctrl_end
+    size_t logits, topk_idx, topk_w, counts, offsets, perm, inv_perm;
+    size_t x8, sx, xp8, sxp, h8, sh, y_p, hs8, shs, ys;
+    size_t total;
+};
+
+__host__ inline WsLayoutFp8 ws_layout_fp8(int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, int64_t fs)
+{
+    WsLayoutFp8 L{};
+    L.ctrl = ws_layout(T, d, 0, E, k, 0);
+    const int64_t P = T * k, Ts = fs > 0 ? T : 0;
+    size_t o = L.ctrl.ctrl_end;
+    L.logits = o; o = align_up(o + (size_t)T * E * 4, 256);
+    L.topk_idx = o; o = align_up(o + (size_t)P * 4, 256);
+    L.topk_w = o; o = align_up(o + (size_t)P * 4, 256);
+    L.counts = o; o = align_up(o + (size_t)E * 4, 256);
+    L.offsets = o; o = align_up(o + (size_t)(E + 1) * 4, 256);
+    L.perm = o; o = align_up(o + (size_t)P * 4, 256);
+    L.inv_perm = o; o = align_up(o + (size_t)P * 4, 256);
+    L.x8 = o; o = align_up(o + (size_t)T * d, 1024);
+    L.sx = o; o = align_up(o + (size_t)T * (d / 128) * 4, 256);
+    L.xp8 = o; o = align_up(o + (size_t)P * d, 1024);
+    L.sxp = o; o = align_up(o + (size_t)P * (d / 128) * 4, 256);
+    L.h8 = o; o = align_up(o + (size_t)P * f, 1024);
+    L.sh = o; o = align_up(o + (size_t)P * (f / 128) * 4, 256);
+    L.y_p = o; o = align_up(o + (size_t)P * d * 2, 1024);
+    L.hs8 = o; o = align_up(o + (size_t)Ts * fs, 1024);
+    L.shs = o; o = align_up(o + (size_t)Ts * (fs / 128) * 4, 256);
+    L.ys = o; o = align_up(o + (size_t)Ts * d * 2, 1024);
     L.total = o;
     return L;
 }

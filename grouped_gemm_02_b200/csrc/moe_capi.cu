@@ -19,6 +19,7 @@
 
 #include "../../include/moe.h"
 #include "common.cuh"
+#include "fp8.cuh"
 #include "grouped_gemm.cuh"
 #include "permute.cuh"
 #include "ptx.cuh"
@@ -87,7 +88,11 @@ int device_setup(DeviceState** out)
                 cudaFuncSetAttribute(grouped_gemm_kernel<MODE_DOWN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kGemmSmemBytes) != cudaSuccess ||
                 cudaFuncSetAttribute(grouped_gemm_kernel<MODE_ROUTER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     kGemmSmemBytes) != cudaSuccess)
+                                     kGemmSmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(grouped_gemm_fp8_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kFp8SmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(grouped_gemm_fp8_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kFp8SmemBytes) != cudaSuccess)
                 return MOE_ERR_CUDA;
             if (!g_encode) {
                 cudaDriverEntryPointQueryResult q;
@@ -131,6 +136,19 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
     cuuint32_t box[2] = {64, box_rows};
     cuuint32_t estr[2] = {1, 1};
     return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D byte (e4m3) tensor map over a row-major [rows, inner] matrix; box = [128, box_rows].
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows)
+{
+    if (rows == 0) rows = 1;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -200,21 +218,24 @@ int run_topk(const TopkSource& s, int T, int E, int k, int32_t* idx, float* w, u
                             s.bias, T, E, k, s.logits_out, idx, w, err));
 }
 
-// The general (multi-CTA) histogram / scan / scatter / gather.
+// The general (multi-CTA) histogram / scan / scatter (/ gather of bf16 rows
+// into xp when xp is given).  unit_rows / m1_rows shape the tile plan.
 int run_permute(const int32_t* idx, const bf16* x, int T, int d, int E, int k, int32_t* counts, int32_t* offsets,
                 int32_t* perm, int32_t* inv_perm, bf16* xp, uint32_t* err, int32_t* block_counts, int32_t* plan,
-                int f, int shared_rows, int fs, int sms, cudaStream_t st)
+                int f, int shared_rows, int fs, int sms, cudaStream_t st, int unit_rows = kTileRows,
+                int m1_rows = 64)
 {
     const int64_t P = (int64_t)T * k;
     const int nb = hist_blocks(P);
     cudaError_t e = launch(hist_kernel, dim3(nb), dim3(512), 0, st, idx, P, E, block_counts, err);
     if (e == cudaSuccess)
         e = launch(scan_kernel, dim3(1), dim3(1024), 0, st, block_counts, nb, E, counts, offsets, plan, f, d,
-                   shared_rows, fs);
+                   shared_rows, fs, unit_rows, m1_rows);
     if (e == cudaSuccess)
         e = launch(scatter_kernel, dim3(nb), dim3(256), 0, st, idx, P, E, (const int32_t*)block_counts, perm,
                    inv_perm);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (!xp) return MOE_OK;
     const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)sms * 16));
     return status_of(launch(gather_rows_kernel, dim3(blocks), dim3(256), 0, st, x, (const int32_t*)perm,
                             (const int32_t*)offsets, E, k, d, xp));
@@ -394,8 +415,8 @@ int moe_grouped_gemm(const moe_bf16* xp, const int32_t* counts, const int32_t* o
     if ((rc = device_setup(&dev))) return rc;
     cudaStream_t st = as_stream(stream);
     int32_t* plan = at<int32_t>(ws, L.plan);
-    if (launch(plan_kernel, dim3(1), dim3(1024), 0, st, counts, offsets, (int)E, plan, (int)f, (int)d, 0, 0) !=
-        cudaSuccess)
+    if (launch(plan_kernel, dim3(1), dim3(1024), 0, st, counts, offsets, (int)E, plan, (int)f, (int)d, 0, 0,
+               (int)kTileRows, 64) != cudaSuccess)
         return MOE_ERR_CUDA;
     GemmOperands o{};
     o.xp = reinterpret_cast<const bf16*>(xp);
@@ -482,7 +503,8 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     if (P <= kSmallPairs) {
         // one CTA: histogram, scan, stable ranks and the tile plan
         if (launch(permute_small_kernel, dim3(1), dim3(1024), 0, st, (const int32_t*)idx, (int)P, iE, counts, offsets,
-                   perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared, err) != cudaSuccess)
+                   perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared, (int)kTileRows, 64, err) !=
+            cudaSuccess)
             return MOE_ERR_CUDA;
         const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)dev->sm_count * 16));
         if (launch(gather_rows_kernel, dim3(blocks), dim3(256), 0, st, xb, (const int32_t*)perm,
@@ -579,6 +601,256 @@ const char* moe_status_string(int status)
     case MOE_ERR_DEVICE: return "device is not sm_100 (B200)";
     default: return "unknown status";
     }
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- FP8 block-scaled layer
+namespace {
+
+int run_quantize_rows(const bf16* x, int64_t R, int C, uint8_t* q, float* sc, cudaStream_t st)
+{
+    const int64_t warps = R * (C / 128);
+    return status_of(launch(quantize_rows_fp8_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, st, x, R, C, q,
+                            sc));
+}
+
+struct Fp8Operands {
+    const uint8_t *xp8, *x8, *W1q, *W3q, *W2q, *Ws1q, *Ws3q, *Ws2q;
+    const float *sxp, *sx, *s1, *s3, *s2, *ss1, *ss3, *ss2;
+    const int32_t* perm;
+    const float* gate_w;
+    uint8_t *h8, *hs8;
+    float *sh, *shs;
+    bf16 *y_p, *ys;
+    int T, P, d, f, fs, E;
+};
+
+int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int sms, cudaStream_t st, bool prof)
+{
+    CUtensorMap a0, a1, b, a0s, a1s, bs;
+    const uint64_t E = (uint64_t)o.E;
+    if (!make_map_u8(&a0, o.W1q, o.d, E * o.f, 128) || !make_map_u8(&a1, o.W3q, o.d, E * o.f, 128) ||
+        !make_map_u8(&b, o.xp8, o.d, (uint64_t)o.P, 16))
+        return MOE_ERR_CUDA;
+    if (o.fs > 0) {
+        if (!make_map_u8(&a0s, o.Ws1q, o.d, o.fs, 128) || !make_map_u8(&a1s, o.Ws3q, o.d, o.fs, 128) ||
+            !make_map_u8(&bs, o.x8, o.d, (uint64_t)o.T, 16))
+            return MOE_ERR_CUDA;
+    } else {
+        a0s = a0;
+        a1s = a1;
+        bs = b;
+    }
+    Fp8Args g1{};
+    g1.plan = plan;
+    g1.plan_ready = 1;
+    g1.E = o.E;
+    g1.M = o.f;
+    g1.M_shared = o.fs;
+    g1.K = o.d;
+    g1.K_shared = o.d;
+    g1.sA0 = o.s1;
+    g1.sA1 = o.s3;
+    g1.sA0s = o.ss1;
+    g1.sA1s = o.ss3;
+    g1.sB = o.sxp;
+    g1.sBs = o.sx;
+    g1.out8 = o.h8;
+    g1.out8_scale = o.sh;
+    g1.out8_shared = o.hs8;
+    g1.out8_scale_shared = o.shs;
+    g1.perm = o.perm;
+    g1.gate_w = o.gate_w;
+    g1.err = err;
+    if (launch(grouped_gemm_fp8_kernel<true>, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a0, a1, b, a0s, a1s,
+               bs, g1) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    phase_mark(prof, 3, st);
+    if (!make_map_u8(&a0, o.W2q, o.f, E * o.d, 128) || !make_map_u8(&b, o.h8, o.f, (uint64_t)o.P, 16))
+        return MOE_ERR_CUDA;
+    a1 = a0;
+    if (o.fs > 0) {
+        if (!make_map_u8(&a0s, o.Ws2q, o.fs, o.d, 128) || !make_map_u8(&bs, o.hs8, o.fs, (uint64_t)o.T, 16))
+            return MOE_ERR_CUDA;
+        a1s = a0s;
+    } else {
+        a0s = a0;
+        a1s = a0;
+        bs = b;
+    }
+    Fp8Args g2 = g1;
+    g2.M = o.d;
+    g2.M_shared = o.d;
+    g2.K = o.f;
+    g2.K_shared = o.fs;
+    g2.sA0 = o.s2;
+    g2.sA1 = nullptr;
+    g2.sA0s = o.ss2;
+    g2.sA1s = nullptr;
+    g2.sB = o.sh;
+    g2.sBs = o.shs;
+    g2.out = o.y_p;
+    g2.out_shared = o.ys;
+    return status_of(launch(grouped_gemm_fp8_kernel<false>, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a0, a1,
+                            b, a0s, a1s, bs, g2));
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_quantize_fp8_rows(const moe_bf16* x, int64_t rows, int64_t cols, uint8_t* q, float* scales, void* stream)
+{
+    if (rows < 0 || cols <= 0 || cols > (int64_t(1) << 30)) return MOE_ERR_ARG;
+    if (cols % 128 != 0) return MOE_ERR_ALIGN;
+    if (rows == 0) return MOE_OK;
+    if (!x || !q || !scales) return MOE_ERR_ARG;
+    if (!al16(x) || !al16(q)) return MOE_ERR_ALIGN;
+    DeviceState* dev;
+    int rc;
+    if ((rc = device_setup(&dev))) return rc;
+    return run_quantize_rows(reinterpret_cast<const bf16*>(x), rows, (int)cols, q, scales, as_stream(stream));
+}
+
+int moe_quantize_fp8_blocks(const moe_bf16* W, int64_t rows, int64_t cols, uint8_t* q, float* scales, void* stream)
+{
+    if (rows < 0 || cols <= 0) return MOE_ERR_ARG;
+    if (rows % 128 != 0 || cols % 128 != 0) return MOE_ERR_ALIGN;
+    if (rows == 0) return MOE_OK;
+    if (!W || !q || !scales) return MOE_ERR_ARG;
+    if (!al16(W) || !al16(q)) return MOE_ERR_ALIGN;
+    const int64_t blocks = (rows / 128) * (cols / 128);
+    if (blocks >= (int64_t(1) << 31)) return MOE_ERR_ARG;
+    DeviceState* dev;
+    int rc;
+    if ((rc = device_setup(&dev))) return rc;
+    return status_of(launch(quantize_blocks_fp8_kernel, dim3((unsigned)blocks), dim3(256), 0, as_stream(stream),
+                            reinterpret_cast<const bf16*>(W), rows, cols, q, scales));
+}
+
+int moe_workspace_size_fp8(int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, int64_t f_shared, size_t* bytes)
+{
+    if (!bytes || T < 0 || d < 0 || f < 0 || E < 1 || E > kMaxExperts || k < 1 || k > kMaxTopK || f_shared < 0)
+        return MOE_ERR_ARG;
+    *bytes = ws_layout_fp8(T, d, f, E, k, f_shared).total;
+    return MOE_OK;
+}
+
+int moe_workspace_tensor_fp8(void* ws, int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, int64_t f_shared,
+                             int which, void** ptr)
+{
+    if (!ws || !ptr || T < 0 || d < 0 || f < 0 || E < 1 || E > kMaxExperts || k < 1 || k > kMaxTopK || f_shared < 0)
+        return MOE_ERR_ARG;
+    const WsLayoutFp8 L = ws_layout_fp8(T, d, f, E, k, f_shared);
+    const size_t offs[17] = {L.logits, L.topk_idx, L.topk_w, L.counts, L.offsets, L.perm, L.inv_perm, L.x8, L.sx,
+                             L.xp8, L.sxp, L.h8, L.sh, L.y_p, L.hs8, L.shs, L.ys};
+    if (which < 0 || which >= 17) return MOE_ERR_ARG;
+    *ptr = static_cast<uint8_t*>(ws) + offs[which];
+    return MOE_OK;
+}
+
+int moe_layer_forward_fp8(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const uint8_t* W1q,
+                          const float* W1s, const uint8_t* W3q, const float* W3s, const uint8_t* W2q, const float* W2s,
+                          const uint8_t* Ws1q, const float* Ws1s, const uint8_t* Ws3q, const float* Ws3s,
+                          const uint8_t* Ws2q, const float* Ws2s, int64_t f_shared, int64_t T, int64_t d, int64_t f,
+                          int64_t E, int64_t k, moe_bf16* out, void* ws, size_t ws_bytes, void* stream)
+{
+    int rc = check_sizes(T, d, E, k);
+    if (rc) return rc;
+    if (f <= 0 || f_shared < 0) return MOE_ERR_ARG;
+    if (d % 128 != 0 || f % 128 != 0 || f_shared % 128 != 0) return MOE_ERR_ALIGN;
+    if (T == 0) return MOE_OK;
+    if (!x || !Wg || !W1q || !W1s || !W3q || !W3s || !W2q || !W2s || !out || !ws) return MOE_ERR_ARG;
+    if (f_shared > 0 && (!Ws1q || !Ws1s || !Ws3q || !Ws3s || !Ws2q || !Ws2s)) return MOE_ERR_ARG;
+    if (!al16(x) || !al16(Wg) || !al16(W1q) || !al16(W3q) || !al16(W2q) || !al16(out) || !al16(ws))
+        return MOE_ERR_ALIGN;
+    if (f_shared > 0 && (!al16(Ws1q) || !al16(Ws3q) || !al16(Ws2q))) return MOE_ERR_ALIGN;
+    const WsLayoutFp8 L = ws_layout_fp8(T, d, f, E, k, f_shared);
+    if (ws_bytes < L.total) return MOE_ERR_WS;
+    DeviceState* dev;
+    if ((rc = device_setup(&dev))) return rc;
+    cudaStream_t st = as_stream(stream);
+    uint32_t* err = at<uint32_t>(ws, L.ctrl.err);
+    int32_t* plan = at<int32_t>(ws, L.ctrl.plan);
+    float* logits = at<float>(ws, L.logits);
+    float* partials = at<float>(ws, L.ctrl.router_partials);
+    int32_t* idx = at<int32_t>(ws, L.topk_idx);
+    float* w = at<float>(ws, L.topk_w);
+    int32_t* counts = at<int32_t>(ws, L.counts);
+    int32_t* offsets = at<int32_t>(ws, L.offsets);
+    int32_t* perm = at<int32_t>(ws, L.perm);
+    int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
+    uint8_t* x8 = at<uint8_t>(ws, L.x8);
+    float* sx = at<float>(ws, L.sx);
+    uint8_t* xp8 = at<uint8_t>(ws, L.xp8);
+    float* sxp = at<float>(ws, L.sxp);
+    bf16* y_p = at<bf16>(ws, L.y_p);
+    const bf16* xb = reinterpret_cast<const bf16*>(x);
+    const int iT = (int)T, id = (int)d, iE = (int)E, ik = (int)k, shared_rows = f_shared > 0 ? (int)T : 0;
+    const int64_t P = T * k;
+
+    const bool prof = t_phase_armed;
+    t_phase_armed = false;
+    phase_mark(prof, 0, st);
+    RouterSplit rs;
+    if ((rc = run_router_gemm(xb, reinterpret_cast<const bf16*>(Wg), bias, iT, id, iE, logits, partials, err,
+                              dev->sm_count, st, &rs)))
+        return rc;
+    if ((rc = run_quantize_rows(xb, T, id, x8, sx, st))) return rc;
+    if ((rc = run_topk(topk_source(rs, logits, partials, bias, iT, iE), iT, iE, ik, idx, w, err, st))) return rc;
+    phase_mark(prof, 1, st);
+    if (P <= kSmallPairs) {
+        if (launch(permute_small_kernel, dim3(1), dim3(1024), 0, st, (const int32_t*)idx, (int)P, iE, counts, offsets,
+                   perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared, kFp8TileRows, 128, err) !=
+            cudaSuccess)
+            return MOE_ERR_CUDA;
+    } else if ((rc = run_permute(idx, xb, iT, id, iE, ik, counts, offsets, perm, inv_perm, nullptr, err,
+                                 at<int32_t>(ws, L.ctrl.block_counts), plan, (int)f, shared_rows, (int)f_shared,
+                                 dev->sm_count, st, kFp8TileRows, 128))) {
+        return rc;
+    }
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)dev->sm_count * 16));
+    if (launch(gather_rows_fp8_kernel, dim3(blocks), dim3(256), 0, st, (const uint8_t*)x8, (const float*)sx,
+               (const int32_t*)perm, (const int32_t*)offsets, iE, ik, id, xp8, sxp) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    Fp8Operands o{};
+    o.xp8 = xp8;
+    o.x8 = x8;
+    o.sxp = sxp;
+    o.sx = sx;
+    o.W1q = W1q;
+    o.W3q = W3q;
+    o.W2q = W2q;
+    o.s1 = W1s;
+    o.s3 = W3s;
+    o.s2 = W2s;
+    o.Ws1q = Ws1q;
+    o.Ws3q = Ws3q;
+    o.Ws2q = Ws2q;
+    o.ss1 = Ws1s;
+    o.ss3 = Ws3s;
+    o.ss2 = Ws2s;
+    o.perm = perm;
+    o.gate_w = w;
+    o.h8 = at<uint8_t>(ws, L.h8);
+    o.sh = at<float>(ws, L.sh);
+    o.hs8 = f_shared > 0 ? at<uint8_t>(ws, L.hs8) : nullptr;
+    o.shs = f_shared > 0 ? at<float>(ws, L.shs) : nullptr;
+    o.y_p = y_p;
+    o.ys = f_shared > 0 ? at<bf16>(ws, L.ys) : nullptr;
+    o.T = iT;
+    o.P = (int)P;
+    o.d = id;
+    o.f = (int)f;
+    o.fs = (int)f_shared;
+    o.E = iE;
+    phase_mark(prof, 2, st);
+    if ((rc = run_gemms_fp8(o, plan, err, dev->sm_count, st, prof))) return rc;
+    phase_mark(prof, 4, st);
+    rc = run_combine(y_p, inv_perm, o.ys, iT, ik, id, reinterpret_cast<bf16*>(out), st);
+    phase_mark(prof, 5, st);
+    return rc;
 }
 
 }  // extern "C"

@@ -79,16 +79,17 @@ __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b -
 // thread tid < E holds counts[tid] in `c` and offsets[tid] in `off`):
 //   * one block per expert with tokens, plus the shared expert (T rows) when
 //     `shared_rows` > 0;
-//   * a block of n rows is cut into units = ceil(n / 256) chunks of
-//     chunk = roundup16(ceil(n / units)) rows -- the tile width follows the
-//     live count, so a 3-token expert gets a 16-wide tile and a hot expert
-//     256-wide ones;
+//   * a block of n rows is cut into units = ceil(n / unit_rows) chunks of
+//     chunk = roundup16(ceil(n / units)) rows (unit_rows = 256 for bf16, 64
+//     for the FP8 path) -- the tile width follows the live count, so a
+//     3-token expert gets a 16-wide tile and a hot expert the widest ones;
 //   * blocks sorted by n descending (ties: lower expert id), so the heaviest
 //     tiles are dealt first;
-//   * tile prefixes for both GEMMs: units * ceil(M / 64) gate/up tiles and
-//     units * ceil(d / 128) down tiles per block.
+//   * tile prefixes for both GEMMs: units * ceil(M / m1_rows) gate/up tiles
+//     (m1_rows = 64 for bf16, 128 for FP8) and units * ceil(d / 128) down tiles.
 __device__ __forceinline__ void build_plan(int c, int off, int E, int pairs, int32_t* __restrict__ plan, int f, int d,
-                                           int shared_rows, int f_shared, int* warp_sums)
+                                           int shared_rows, int f_shared, int* warp_sums, int unit_rows = kTileRows,
+                                           int m1_rows = 64)
 {
     __shared__ int s_n[kMaxGroups];
     __shared__ int s_order[kMaxGroups];
@@ -121,7 +122,7 @@ __device__ __forceinline__ void build_plan(int c, int off, int E, int pairs, int
     if (tid < nact) {
         const int g = s_order[tid];
         const int n = s_n[g];
-        const int units = ceil_div(n, kTileRows);
+        const int units = ceil_div(n, unit_rows);
         const int chunk = ceil_div(ceil_div(n, units), 16) * 16;
         const int M1 = g < E ? f : f_shared;
         pa.group[tid] = g;
@@ -129,7 +130,7 @@ __device__ __forceinline__ void build_plan(int c, int off, int E, int pairs, int
         pa.rows[tid] = n;
         pa.chunk[tid] = chunk;
         pa.units[tid] = units;
-        my_t1 = units * ceil_div(M1, 64);
+        my_t1 = units * ceil_div(M1, m1_rows);
         my_t2 = units * ceil_div(d, 128);
         my_chunk = chunk;
     }
@@ -166,7 +167,7 @@ __device__ __forceinline__ void build_plan(int c, int off, int E, int pairs, int
 __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ block_counts, int nblk_hist, int E,
                                                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                                     int32_t* __restrict__ plan, int f, int d, int shared_rows,
-                                                    int f_shared)
+                                                    int f_shared, int unit_rows, int m1_rows)
 {
     __shared__ int warp_sums[32];
     __shared__ int s_pairs;
@@ -193,14 +194,14 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ block_
         s_pairs = incl;
     }
     __syncthreads();
-    if (plan) build_plan(c, off, E, s_pairs, plan, f, d, shared_rows, f_shared, warp_sums);
+    if (plan) build_plan(c, off, E, s_pairs, plan, f, d, shared_rows, f_shared, warp_sums, unit_rows, m1_rows);
 }
 
 // Single CTA of 1024 threads: the tile plan from counts/offsets already on the device.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ counts,
                                                     const int32_t* __restrict__ offsets, int E,
                                                     int32_t* __restrict__ plan, int f, int d, int shared_rows,
-                                                    int f_shared)
+                                                    int f_shared, int unit_rows, int m1_rows)
 {
     __shared__ int warp_sums[32];
     ptx::grid_dep_wait();
@@ -208,7 +209,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
     const int tid = threadIdx.x;
     const int c = tid < E ? counts[tid] : 0;
     const int off = tid < E ? offsets[tid] : 0;
-    build_plan(c, off, E, offsets[E], plan, f, d, shared_rows, f_shared, warp_sums);
+    build_plan(c, off, E, offsets[E], plan, f, d, shared_rows, f_shared, warp_sums, unit_rows, m1_rows);
 }
 
 // ---------------------------------------------------------------- small-T permutation
@@ -224,8 +225,8 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t* __re
                                                              int32_t* __restrict__ perm,
                                                              int32_t* __restrict__ inv_perm,
                                                              int32_t* __restrict__ plan, int f, int d,
-                                                             int shared_rows, int f_shared,
-                                                             uint32_t* __restrict__ err)
+                                                             int shared_rows, int f_shared, int unit_rows,
+                                                             int m1_rows, uint32_t* __restrict__ err)
 {
     // s_wcnt[w][e]: pairs of warp w (pairs 32w..32w+31) routed to expert e (<= 32)
     __shared__ __align__(16) uint8_t s_wcnt[32][kMaxExperts];
@@ -271,7 +272,7 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t* __re
     __shared__ int s_pairs;
     if (tid == E - 1) s_pairs = incl;
     __syncthreads();
-    if (plan) build_plan(c, off, E, s_pairs, plan, f, d, shared_rows, f_shared, warp_sums);
+    if (plan) build_plan(c, off, E, s_pairs, plan, f, d, shared_rows, f_shared, warp_sums, unit_rows, m1_rows);
 }
 
 // ---------------------------------------------------------------- scatter

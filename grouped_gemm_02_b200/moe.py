@@ -27,7 +27,8 @@ _lib: Optional[C.CDLL] = None
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_topk", "moe_permute",
            "moe_permute_noalloc", "moe_grouped_gemm", "moe_combine", "moe_layer_forward", "moe_workspace_tensor",
            "moe_record_phase_events", "moe_launch_counter", "moe_get_device_error", "moe_clear_device_error",
-           "moe_status_string")
+           "moe_status_string", "moe_quantize_fp8_rows", "moe_quantize_fp8_blocks", "moe_workspace_size_fp8",
+           "moe_workspace_tensor_fp8", "moe_layer_forward_fp8")
 
 
 class MoEError(RuntimeError):
@@ -64,6 +65,12 @@ def lib() -> C.CDLL:
             "moe_status_string": [C.c_int],
             "moe_record_phase_events": [C.POINTER(vp), C.c_int],
             "moe_launch_counter": [],
+            "moe_quantize_fp8_rows": [vp, i64, i64, vp, vp, vp],
+            "moe_quantize_fp8_blocks": [vp, i64, i64, vp, vp, vp],
+            "moe_workspace_size_fp8": [i64, i64, i64, i64, i64, i64, C.POINTER(sz)],
+            "moe_workspace_tensor_fp8": [vp, i64, i64, i64, i64, i64, i64, C.c_int, C.POINTER(vp)],
+            "moe_layer_forward_fp8": [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
+                                      i64, i64, vp, vp, sz, vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -252,6 +259,93 @@ def workspace_views(ws: torch.Tensor, T: int, d: int, f: int, E: int, k: int, f_
         for s in shape:
             n *= s
         off = ptr - base
+        nbytes = n * torch.tensor([], dtype=dt).element_size()
+        views[name] = ws[off:off + nbytes].view(dt).view(shape)
+    return views
+
+
+# ---------------------------------------------------------------- FP8 path
+
+def moe_quantize_fp8_rows(x: torch.Tensor, stream=None):
+    """1 x 128 blocks along rows: bf16 [R, C] -> (e4m3 codes uint8 [R, C], fp32 scales [R, C/128])."""
+    R, Cc = x.shape
+    _bf16(x)
+    q = torch.empty(R, Cc, dtype=torch.uint8, device=x.device)
+    sc = torch.empty(R, Cc // 128, dtype=torch.float32, device=x.device)
+    _call("moe_quantize_fp8_rows", _p(x), R, Cc, _p(q), _p(sc), _stream(stream))
+    return q, sc
+
+
+def moe_quantize_fp8_blocks(W: torch.Tensor, stream=None):
+    """128 x 128 blocks: bf16 [R, C] (or [E, R', C], taken as [E*R', C]) -> (codes, scales [R/128, C/128])."""
+    W2d = W.reshape(-1, W.shape[-1])
+    _bf16(W2d)
+    R, Cc = W2d.shape
+    q = torch.empty(W.shape, dtype=torch.uint8, device=W.device)
+    sc = torch.empty(R // 128, Cc // 128, dtype=torch.float32, device=W.device)
+    _call("moe_quantize_fp8_blocks", _p(W2d), R, Cc, _p(q), _p(sc), _stream(stream))
+    return q, sc
+
+
+def quantize_layer_fp8(w: dict, stream=None) -> dict:
+    """The expert weights of a layer (W1, W3, W2 and optionally Ws1, Ws3, Ws2) in e4m3 with 128 x 128 scales."""
+    out = {}
+    for n in ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2"):
+        if w.get(n) is not None:
+            out[n + "q"], out[n + "s"] = moe_quantize_fp8_blocks(w[n], stream)
+    return out
+
+
+def moe_workspace_size_fp8(T: int, d: int, f: int, E: int, k: int, f_shared: int = 0) -> int:
+    n = C.c_size_t(0)
+    _call("moe_workspace_size_fp8", T, d, f, E, k, f_shared, C.byref(n))
+    return int(n.value)
+
+
+def new_workspace_fp8(T: int, d: int, f: int, E: int, k: int, f_shared: int = 0, device=None, stream=None):
+    n = moe_workspace_size_fp8(T, d, f, E, k, f_shared)
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device or torch.device("cuda"))
+    moe_workspace_init(ws, T, E, k, stream)
+    return ws
+
+
+def moe_layer_forward_fp8(x, Wg, bias, Q: dict, k: int, ws: torch.Tensor, out=None, stream=None):
+    """FP8 layer; Q holds W1q/W1s, W3q/W3s, W2q/W2s (and Ws1q/Ws1s, ... for the shared expert)."""
+    T, d = x.shape
+    E, f, _ = Q["W1q"].shape
+    fs = 0 if Q.get("Ws1q") is None else Q["Ws1q"].shape[0]
+    _bf16(x), _bf16(Wg, (E, d))
+    out = torch.empty(T, d, dtype=torch.bfloat16, device=x.device) if out is None else out
+    g = lambda n: _p(Q.get(n))
+    _call("moe_layer_forward_fp8", _p(x), _p(Wg), _p(bias), g("W1q"), g("W1s"), g("W3q"), g("W3s"), g("W2q"),
+          g("W2s"), g("Ws1q"), g("Ws1s"), g("Ws3q"), g("Ws3s"), g("Ws2q"), g("Ws2s"), fs, T, d, f, E, k, _p(out),
+          _p(ws), ws.numel(), _stream(stream))
+    return out
+
+
+WS_TENSORS_FP8 = ("logits", "topk_idx", "topk_w", "counts", "offsets", "perm", "inv_perm", "x8", "sx", "xp8", "sxp",
+                  "h8", "sh", "y_p", "hs8", "shs", "ys")
+
+
+def workspace_views_fp8(ws: torch.Tensor, T: int, d: int, f: int, E: int, k: int, f_shared: int = 0):
+    P, Ts = T * k, (T if f_shared else 0)
+    shapes = {"logits": ((T, E), torch.float32), "topk_idx": ((T, k), torch.int32), "topk_w": ((T, k), torch.float32),
+              "counts": ((E,), torch.int32), "offsets": ((E + 1,), torch.int32), "perm": ((P,), torch.int32),
+              "inv_perm": ((P,), torch.int32), "x8": ((T, d), torch.uint8), "sx": ((T, d // 128), torch.float32),
+              "xp8": ((P, d), torch.uint8), "sxp": ((P, d // 128), torch.float32), "h8": ((P, f), torch.uint8),
+              "sh": ((P, f // 128), torch.float32), "y_p": ((P, d), torch.bfloat16),
+              "hs8": ((Ts, f_shared), torch.uint8), "shs": ((Ts, max(f_shared, 128) // 128 if Ts else 0), torch.float32),
+              "ys": ((Ts, d), torch.bfloat16)}
+    base = ws.data_ptr()
+    views = {}
+    for i, name in enumerate(WS_TENSORS_FP8):
+        out = C.c_void_p(0)
+        _call("moe_workspace_tensor_fp8", _p(ws), T, d, f, E, k, f_shared, i, C.byref(out))
+        shape, dt = shapes[name]
+        n = 1
+        for s_ in shape:
+            n *= s_
+        off = int(out.value or 0) - base
         nbytes = n * torch.tensor([], dtype=dt).element_size()
         views[name] = ws[off:off + nbytes].view(dt).view(shape)
     return views

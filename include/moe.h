@@ -68,6 +68,7 @@ typedef uint16_t moe_bf16;
 #define MOE_DEVERR_EXPERT_RANGE 1u  /* an expert id outside [0, E): that pair was dropped */
 #define MOE_DEVERR_TIMEOUT 2u       /* a bounded wait inside a kernel gave up; outputs are invalid */
 #define MOE_DEVERR_NAN_LOGIT 4u     /* a router logit was NaN; it ranked below every number */
+#define MOE_DEVERR_PLAN 8u          /* a GEMM met a tile plan it cannot run and did nothing */
 
 /* Bytes of workspace moe_layer_forward needs for these sizes (f_shared = 0:
  * no shared expert).  The control part of it (error word, tile plan,
@@ -164,6 +165,56 @@ MOE_API int moe_layer_forward(const moe_bf16 *x, const moe_bf16 *Wg, const float
                       const moe_bf16 *W3, const moe_bf16 *W2, const moe_bf16 *Ws1, const moe_bf16 *Ws3,
                       const moe_bf16 *Ws2, int64_t f_shared, int64_t T, int64_t d, int64_t f, int64_t E, int64_t k,
                       moe_bf16 *out, void *ws, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------- FP8 path
+ * The FP8 block-scaled variant (GC-MoE, abstract: an FP8 MoE operator with
+ * block-scaled MMA and requantisation; e4m3 with 1 x 128 activation blocks and
+ * 128 x 128 weight blocks).  Codes are OCP e4m3 (round to nearest, ties to
+ * even, saturating at +-448).  A block's scale is the smallest power of two s
+ * with max|v| / s <= 448 (s = 1 for an all-zero block), stored as fp32, so
+ * code q with scale s stands for e4m3(q) * s exactly.  d, f and f_shared must
+ * be multiples of 128 (MOE_ERR_ALIGN otherwise). */
+
+/* 1 x 128 blocks along each row: x [rows, cols] bf16 -> q [rows, cols] e4m3,
+ * scales [rows, cols/128] fp32.  cols % 128 == 0. */
+MOE_API int moe_quantize_fp8_rows(const moe_bf16 *x, int64_t rows, int64_t cols, uint8_t *q, float *scales,
+                                  void *stream);
+
+/* 128 x 128 blocks: W [rows, cols] bf16 -> q [rows, cols] e4m3, scales
+ * [rows/128, cols/128] fp32 (block (i, j) covers rows 128i.. and cols 128j..).
+ * Expert weights are quantised as one matrix: W1/W3 as [E*f, d] (scales
+ * [E*f/128, d/128]), W2 as [E*d, f] (scales [E*d/128, f/128]). */
+MOE_API int moe_quantize_fp8_blocks(const moe_bf16 *W, int64_t rows, int64_t cols, uint8_t *q, float *scales,
+                                    void *stream);
+
+/* Workspace bytes of moe_layer_forward_fp8 for these sizes. */
+MOE_API int moe_workspace_size_fp8(int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, int64_t f_shared,
+                                   size_t *bytes);
+
+/* Device pointers of the FP8 layer intermediates inside its workspace
+ * (which: 0 logits, 1 topk_idx, 2 topk_w, 3 counts, 4 offsets, 5 perm,
+ * 6 inv_perm, 7 x8, 8 sx, 9 xp8, 10 sxp, 11 h8, 12 sh, 13 y_p, 14 hs8, 15 shs,
+ * 16 ys).  Host-only arithmetic. */
+MOE_API int moe_workspace_tensor_fp8(void *ws, int64_t T, int64_t d, int64_t f, int64_t E, int64_t k,
+                                     int64_t f_shared, int which, void **ptr);
+
+/* The whole layer with FP8 expert GEMMs.  Routing is the bf16 router of
+ * moe_route (same logits, top-k and gates).  x is quantised in 1 x 128 blocks,
+ * gathered into expert order, and multiplied with the pre-quantised weights
+ * (W1q/W3q [E,f,d] with scales W1s/W3s [E*f/128, d/128]; W2q [E,d,f] with W2s
+ * [E*d/128, f/128]; the shared expert Ws1q/Ws3q [f_shared,d], Ws2q
+ * [d,f_shared] with their scales, or all NULL and f_shared = 0):
+ *   h   = silu(x^ W1^T) * (x^ W3^T), requantised in 1 x 128 blocks along f
+ *   y_p = gate * (h^ W2^T)          (bf16), then the combine of moe_combine,
+ * where ^ marks dequantised values; all products accumulate in fp32 (one
+ * 128-wide K block per tensor-core pass, scaled in fp32).  Every intermediate
+ * lives in `ws` (moe_workspace_size_fp8 bytes). */
+MOE_API int moe_layer_forward_fp8(const moe_bf16 *x, const moe_bf16 *Wg, const float *bias, const uint8_t *W1q,
+                                  const float *W1s, const uint8_t *W3q, const float *W3s, const uint8_t *W2q,
+                                  const float *W2s, const uint8_t *Ws1q, const float *Ws1s, const uint8_t *Ws3q,
+                                  const float *Ws3s, const uint8_t *Ws2q, const float *Ws2s, int64_t f_shared,
+                                  int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, moe_bf16 *out, void *ws,
+                                  size_t ws_bytes, void *stream);
 
 /* Per-phase timing of the next moe_layer_forward call made on this host
  * thread: `events` holds n >= 6 cudaEvent_t handles; that call records
