@@ -176,17 +176,31 @@ def workload_label(s: wl.LayerShape) -> str:
     return lab
 
 
-def algorithmic(s: wl.LayerShape, counts: np.ndarray):
-    """Algorithmic bytes and flops of the layer and of the gate/up GEMM launch."""
+def algorithmic(s: wl.LayerShape, counts: np.ndarray, fp8: bool = False):
+    """Algorithmic bytes and flops of the layer and of the gate/up GEMM launch.
+
+    bf16: 2 bytes per weight and activation.  FP8: 1 byte per weight and
+    activation plus one fp32 scale per 128 x 128 weight block and per 1 x 128
+    activation block."""
     active = int((counts > 0).sum())
     P = int(counts.sum())
     fs = s.f_shared
-    w_act = active * 3 * s.d * s.f * 2 + (3 * s.d * fs * 2 if fs else 0)
+    wb = 1 if fp8 else 2
+    wsc = (4.0 / (128 * 128)) if fp8 else 0.0    # weight-scale bytes per weight
+    asc = (4.0 / 128) if fp8 else 0.0            # activation-scale bytes per activation
+
+    def mat(rows, cols):
+        return rows * cols * (wb + wsc)
+
+    def act(rows, cols):
+        return rows * cols * (wb + asc)
+
+    w_act = active * 3 * mat(s.d, s.f) + (3 * mat(s.d, fs) if fs else 0)
     flops = 6.0 * P * s.d * s.f + (6.0 * s.T * s.d * fs if fs else 0)
-    g1_bytes = active * 2 * s.f * s.d * 2 + P * s.d * 2 + P * s.f * 2
+    g1_bytes = active * 2 * mat(s.f, s.d) + act(P, s.d) + act(P, s.f)
     g1_flops = 4.0 * P * s.d * s.f
     if fs:
-        g1_bytes += 2 * fs * s.d * 2 + s.T * s.d * 2 + s.T * fs * 2
+        g1_bytes += 2 * mat(fs, s.d) + act(s.T, s.d) + act(s.T, fs)
         g1_flops += 4.0 * s.T * s.d * fs
     return dict(active=active, pairs=P, w_act=w_act, flops=flops, g1_bytes=g1_bytes, g1_flops=g1_flops)
 
@@ -259,13 +273,24 @@ def run_ours(args, s: wl.LayerShape):
     sets = [one] + [wl.make_weights(s, seed=args.seed + 1000 * (i + 1), device=dev) for i in range(R - 1)]
     base = wl.make_inputs(s, seed=args.seed, device=dev, weights=False)
     x, Wg, bias = base["x"], base["Wg"], base["bias"]
-    ws = moe.new_workspace(s.T, s.d, s.f, s.E, s.k, s.f_shared, device=dev)
     out = torch.empty(s.T, s.d, dtype=torch.bfloat16, device=dev)
+    if args.fp8:
+        # e4m3 weights with 128 x 128 block scales (quantised once, outside the timed region)
+        qsets = [moe.quantize_layer_fp8(w) for w in sets]
+        ws = moe.new_workspace_fp8(s.T, s.d, s.f, s.E, s.k, s.f_shared, device=dev)
+        wbytes = sum(t.numel() * t.element_size() for t in qsets[0].values())
+        sets = one = None                   # the bf16 weights are not used any more
+        torch.cuda.empty_cache()
+    else:
+        ws = moe.new_workspace(s.T, s.d, s.f, s.E, s.k, s.f_shared, device=dev)
 
     def step(i, prof_events=None):
-        w = sets[i % R]
         if prof_events is not None:
             moe.moe_record_phase_events(prof_events)
+        if args.fp8:
+            moe.moe_layer_forward_fp8(x, Wg, bias, qsets[i % R], s.k, ws, out=out)
+            return
+        w = sets[i % R]
         moe.moe_layer_forward(x, Wg, bias, w["W1"], w["W3"], w["W2"], s.k, ws, Ws1=w.get("Ws1"),
                               Ws3=w.get("Ws3"), Ws2=w.get("Ws2"), out=out)
 
@@ -342,24 +367,28 @@ def run_ours(args, s: wl.LayerShape):
                "ms_per_step": e_ms / K}
 
     # realised histogram and roofline
-    views = moe.workspace_views(ws, s.T, s.d, s.f, s.E, s.k, s.f_shared)
+    if args.fp8:
+        views = moe.workspace_views_fp8(ws, s.T, s.d, s.f, s.E, s.k, s.f_shared)
+    else:
+        views = moe.workspace_views(ws, s.T, s.d, s.f, s.E, s.k, s.f_shared)
     counts = views["counts"].cpu().numpy()
-    alg = algorithmic(s, counts)
+    alg = algorithmic(s, counts, fp8=args.fp8)
     pk, pk_kind = peaks()
     bw = pk["hbm_gbs"] * 1e9
-    tc = pk["bf16_tflops_sustained"] * 1e12
+    # FP8 tensor peak: the measured bf16 figure times the nominal fp8 / bf16 ratio (4.5 / 2.25)
+    tc = pk["bf16_tflops_sustained"] * 1e12 * (2.0 if args.fp8 else 1.0)
     t_g1 = phase_ms[2] / 1e3
     g1_hbm = alg["g1_bytes"] / bw
     g1_tc = alg["g1_flops"] / tc
     if g1_hbm >= g1_tc:
         roof = {"bound": "hbm", "achieved": alg["g1_bytes"] / t_g1 / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s"}
     else:
-        roof = {"bound": "tensor", "achieved": alg["g1_flops"] / t_g1 / 1e12, "peak": pk["bf16_tflops_sustained"],
+        roof = {"bound": "tensor", "achieved": alg["g1_flops"] / t_g1 / 1e12, "peak": tc / 1e12,
                 "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = committed_traffic(workload_label(s))
     roof["kernel"] = "grouped_gemm_kernel<gate/up + SwiGLU>"
-    roof["peak_source"] = f"{pk_kind} ({'sustained bf16' if roof['bound'] == 'tensor' else 'HBM copy'})"
+    roof["peak_source"] = f"{pk_kind} ({('2 x sustained bf16 (fp8)' if args.fp8 else 'sustained bf16') if roof['bound'] == 'tensor' else 'HBM copy'})"
     t_roof = max(alg["w_act"] / bw, alg["flops"] / tc)
     layer_roof = {"bound": "hbm" if alg["w_act"] / bw >= alg["flops"] / tc else "tensor",
                   "t_roof_us": t_roof * 1e6, "t_meas_us": ms_per_step * 1e3, "frac": t_roof / (ms_per_step / 1e3),
@@ -367,8 +396,10 @@ def run_ours(args, s: wl.LayerShape):
 
     line = {"metric": METRIC, "value": s.T * K * world / (ms_max / 1e3), "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": workload_label(s), "T": s.T, "d": s.d, "f": s.f, "E": s.E, "k": s.k,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3 (fp32 accumulate)" if args.fp8 else "bf16",
+            "data": "synthetic",
+            "config": {"workload": workload_label(s) + (" fp8" if args.fp8 else ""), "T": s.T, "d": s.d, "f": s.f,
+                       "E": s.E, "k": s.k,
                        "alpha": s.alpha, "f_shared": s.f_shared, "seed": args.seed,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": f"inputs larger than L2: {R} rotating weight sets of {wbytes / 2**20:.0f} MiB",
@@ -379,7 +410,7 @@ def run_ours(args, s: wl.LayerShape):
                                     zip(("route", "permute", "gemm_gate_up", "gemm_down", "combine"), phase_ms)}},
             "roofline": roof, "layer_roofline": layer_roof, "e2e": e2e, "gpu_launches": int(launches),
             "clocks": clocks}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.fp8:
         host = {n: v.cpu() for n, v in base.items()}
         host.update({n: v.cpu() for n, v in one.items()})
         orc = OracleRun(s, host)
@@ -439,6 +470,7 @@ def main(argv=None):
     ap.add_argument("--alpha", type=float, default=None)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--sets", type=int, default=0, help="rotating weight sets (0: enough to exceed 3x L2)")
+    ap.add_argument("--fp8", action="store_true", help="FP8 block-scaled expert GEMMs (moe_layer_forward_fp8)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")

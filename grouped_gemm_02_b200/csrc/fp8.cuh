@@ -31,7 +31,8 @@ namespace moe {
 
 constexpr int kFp8TileRows = 64;                 // most tokens one FP8 tile carries
 constexpr int kFp8BlockK = 128;                  // e4m3 elements per 128-byte swizzle row = one scale block
-constexpr uint32_t kFp8TmemCols = 256;           // 2 partial buffers x (g: 64 + u: 64) columns
+constexpr int kFp8Bufs = 4;                      // TMEM partial buffers between the MMA and the epilogue
+constexpr uint32_t kFp8TmemCols = 512;           // 4 partial buffers x (g: 64 + u: 64) columns
 
 // Smallest power-of-two exponent e with amax <= 448 * 2^e (amax > 0), from the
 // binary exponent of amax: amax = m * 2^x, m in [0.5, 1), 448 = 0.875 * 2^9.
@@ -299,7 +300,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ptx::mbar_init(ptx::smem_u32(&ctl->full[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&ctl->empty[s]), 1);
         }
-        for (int a = 0; a < 2; a++) {
+        for (int a = 0; a < kFp8Bufs; a++) {
             ptx::mbar_init(ptx::smem_u32(&ctl->tfull[a]), 1);
             ptx::mbar_init(ptx::smem_u32(&ctl->tempty[a]), 4);
         }
@@ -432,8 +433,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         s = 0;
                         ph ^= 1u;
                     }
-                    pb ^= 1;
-                    if (pb == 0) pph ^= 1u;
+                    if (++pb == kFp8Bufs) {
+                        pb = 0;
+                        pph ^= 1u;
+                    }
                 }
             }
             if (!ok && issued) {
@@ -446,6 +449,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue: scale, accumulate, finish
+        // The activation scales (sB) come from the kernel right before this one:
+        // wait for it before the first (prefetched) read.
+        if (!waited_early) ptx::grid_dep_wait();
         const int quad = warp & 3;
         const int row_in_tile = quad * 32 + lane;        // weight row of this thread (TMEM lane)
         int pb = 0;
@@ -466,18 +472,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int c = 0; c < kFp8TileRows; c++) acc_g[c] = 0.f;
 #pragma unroll
             for (int c = 0; c < (GATED ? kFp8TileRows : 1); c++) acc_u[c] = 0.f;
+            // scales of K block kb are fetched while K block kb - 1 is being added
+            auto scales = [&](int kb, float& a0, float& a1, float& xa, float& xb) {
+                a0 = __ldg(sA0 + srow * kbl + kb);
+                a1 = GATED ? __ldg(sA1 + srow * kbl + kb) : 0.f;
+                xa = lane < tl.rows ? __ldg(sB + (int64_t)(tl.row0 + lane) * kbl + kb) : 0.f;
+                xb = lane + 32 < tl.rows ? __ldg(sB + (int64_t)(tl.row0 + lane + 32) * kbl + kb) : 0.f;
+            };
+            float s0, s1, sxa, sxb;
+            scales(0, s0, s1, sxa, sxb);
             for (int kb = 0; kb < tl.nkb; kb++) {
+                float n0 = 0.f, n1 = 0.f, nxa = 0.f, nxb = 0.f;
+                if (kb + 1 < tl.nkb) scales(kb + 1, n0, n1, nxa, nxb);
                 const bool good = bounded_wait(ptx::smem_u32(&ctl->tfull[pb]), pph, ctl, args.err);
                 if (!__all_sync(0xffffffffu, good)) {
                     ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
-                const float s0 = __ldg(sA0 + srow * kbl + kb);
-                const float s1 = GATED ? __ldg(sA1 + srow * kbl + kb) : 0.f;
-                // activation-block scales of the tile's columns: lane l holds columns l and l + 32
-                const float sxa = lane < tl.rows ? __ldg(sB + (int64_t)(tl.row0 + lane) * kbl + kb) : 0.f;
-                const float sxb = lane + 32 < tl.rows ? __ldg(sB + (int64_t)(tl.row0 + lane + 32) * kbl + kb) : 0.f;
                 const uint32_t taddr = tmem_base + (uint32_t)pb * 128u + ((uint32_t)(quad * 32) << 16);
 #pragma unroll
                 for (int c0 = 0; c0 < kFp8TileRows; c0 += 16) {
@@ -498,20 +510,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&ctl->tempty[pb]));
-                pb ^= 1;
-                if (pb == 0) pph ^= 1u;
+                if (++pb == kFp8Bufs) {
+                    pb = 0;
+                    pph ^= 1u;
+                }
+                s0 = n0;
+                s1 = n1;
+                sxa = nxa;
+                sxb = nxb;
             }
             if (!ok) break;
             if (GATED) {
                 // h = silu(g) * u, then requantise each token's 128 h values of this tile
 #pragma unroll
                 for (int c = 0; c < kFp8TileRows; c++) {
-                    const float g = acc_g[c];
-                    acc_g[c] = g / (1.0f + __expf(-g)) * acc_u[c];
-                    float a = (c < tl.rows && tl.m * 128 + row_in_tile < Mrows) ? fabsf(acc_g[c]) : 0.f;
+                    if (c < tl.rows) {   // warp-uniform
+                        const float g = acc_g[c];
+                        acc_g[c] = g / (1.0f + __expf(-g)) * acc_u[c];
+                        float a = tl.m * 128 + row_in_tile < Mrows ? fabsf(acc_g[c]) : 0.f;
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-                    if (lane == 0) red[quad * kFp8TileRows + c] = a;
+                        for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+                        if (lane == 0) red[quad * kFp8TileRows + c] = a;
+                    }
                 }
                 named_bar_epilogue();
                 uint8_t* out8 = tl.shared ? args.out8_shared : args.out8;
@@ -538,8 +558,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                       : 1.f;
 #pragma unroll
                 for (int c = 0; c < kFp8TileRows; c++) {
+                    if (c >= tl.rows) continue;   // warp-uniform
                     const float gate = __shfl_sync(0xffffffffu, c < 32 ? gsa : gsb, c & 31);
-                    if (c < tl.rows && drow < Mrows)
+                    if (drow < Mrows)
                         out[(int64_t)(tl.row0 + c) * Mrows + drow] = __float2bfloat16_rn(acc_g[c] * gate);
                 }
             }

@@ -158,8 +158,8 @@ __device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a, co
 struct SmemCtl {
     uint64_t full[kMaxStages];
     uint64_t empty[kMaxStages];
-    uint64_t tfull[2];
-    uint64_t tempty[2];
+    uint64_t tfull[4];     // accumulator buffers: 2 in the bf16 GEMM, 4 partials in the FP8 GEMM
+    uint64_t tempty[4];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
