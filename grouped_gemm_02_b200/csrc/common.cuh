@@ -48,9 +48,10 @@ struct PlanArrays {
     int32_t* units;
     int32_t* tb1;       // tile prefix, gate/up GEMM  [n_blocks + 1]
     int32_t* tb2;       // tile prefix, down GEMM     [n_blocks + 1]
+    int32_t* dep;       // gate/up tiles of the block finished (fused GEMM), zeroed by the plan builder
 };
 
-constexpr size_t kPlanInts = 8 + 5 * kMaxGroups + 2 * (kMaxGroups + 1);
+constexpr size_t kPlanInts = 8 + 6 * kMaxGroups + 2 * (kMaxGroups + 1);
 
 __host__ __device__ inline PlanArrays plan_arrays(int32_t* base)
 {
@@ -62,7 +63,8 @@ __host__ __device__ inline PlanArrays plan_arrays(int32_t* base)
     a.chunk = p; p += kMaxGroups;
     a.units = p; p += kMaxGroups;
     a.tb1 = p; p += kMaxGroups + 1;
-    a.tb2 = p;
+    a.tb2 = p; p += kMaxGroups + 1;
+    a.dep = p;
     return a;
 }
 

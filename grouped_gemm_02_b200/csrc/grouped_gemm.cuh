@@ -16,6 +16,15 @@
 // split over K into fp32 partial sums when the token count alone cannot
 // fill the SMs (the top-k kernel then adds the partials in a fixed order).
 //
+//   MODE_FUSED:  gate/up tiles then down tiles in one persistent launch.  A
+//                down tile of expert block i loads its h rows only after every
+//                gate/up tile of block i has stored them: each gate/up tile's
+//                epilogue bumps a per-block counter (zeroed by the plan
+//                builder) after its stores, and the producer of a down tile
+//                waits for the count (bounded) before its h loads -- its W2
+//                loads go out before the wait.  The down tiles fill the
+//                gate/up tail instead of a second launch ramping up.
+//
 // The MMA is operand-swapped: the weights fill the M = 128 slot and the tokens
 // the N slot (16..256, chosen per expert from its live count by the plan), so
 // a decode expert with 3 tokens costs one 16-wide MMA column block while a hot
@@ -54,6 +63,7 @@ namespace moe {
 constexpr int MODE_DOWN = 0;
 constexpr int MODE_GATED = 1;
 constexpr int MODE_ROUTER = 2;
+constexpr int MODE_FUSED = 3;
 
 constexpr int kGemmThreads = 192;
 constexpr int kBlockK = 64;                          // bf16 elements per 128-byte swizzle row
@@ -87,16 +97,20 @@ struct GemmArgs {
 
 struct Tile {
     int group, m, row0, rows, n_mma, K, kb0, kb1, split;
+    int blk;        // block (plan entry) index
     bool shared;
+    bool gated;     // a gate/up tile (SwiGLU epilogue) rather than a down tile
 };
 
 // The plan entries this launch reads, copied to shared memory once per CTA so
 // that decoding a tile (a binary search over the tile prefix) costs shared
 // loads instead of a chain of dependent global loads at every tile boundary.
 struct SmemPlan {
-    int tb[kMaxGroups + 1];     // tile prefix of this GEMM
+    int tb[kMaxGroups + 1];     // tile prefix of this GEMM (the gate/up one in MODE_FUSED)
+    int tb2[kMaxGroups + 1];    // MODE_FUSED: tile prefix of the down tiles
     int4 blk[kMaxGroups];       // group, row0, rows, chunk
     int units[kMaxGroups];
+    int tiles1;                 // MODE_FUSED: gate/up tiles come first
 };
 constexpr int kGemmSmemBytes = 1024 + kRingBytes + kBarBytes + (int)sizeof(SmemPlan);
 static_assert(kGemmSmemBytes <= 227 * 1024, "shared memory budget");
@@ -105,13 +119,16 @@ template <int MODE>
 __device__ __forceinline__ int total_tiles(const GemmArgs& a, const PlanHeader* hdr)
 {
     if (MODE == MODE_ROUTER) return a.units * a.mt * a.splits;
+    if (MODE == MODE_FUSED) return hdr->tiles1 + hdr->tiles2;
     return MODE == MODE_GATED ? hdr->tiles1 : hdr->tiles2;
 }
 
 template <int MODE>
-__device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a, const SmemPlan* sp)
+__device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a, const GemmArgs& a2, const SmemPlan* sp)
 {
     Tile tl;
+    tl.blk = 0;
+    tl.gated = MODE == MODE_GATED;
     if (MODE == MODE_ROUTER) {
         const int per_unit = a.mt * a.splits;
         const int u = t / per_unit;
@@ -127,9 +144,18 @@ __device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a, co
         const int nk = (a.K + kBlockK - 1) / kBlockK;
         tl.kb0 = tl.split * a.kb_per;
         tl.kb1 = min(nk, tl.kb0 + a.kb_per);
+        tl.gated = false;
         return tl;
     }
+    bool gated = MODE == MODE_GATED;
     const int* tb = sp->tb;
+    if (MODE == MODE_FUSED) {
+        gated = t < sp->tiles1;
+        if (!gated) {
+            t -= sp->tiles1;
+            tb = sp->tb2;
+        }
+    }
     int lo = 0, hi = nb - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -140,6 +166,8 @@ __device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a, co
     const int units = sp->units[lo];
     const int4 b = sp->blk[lo];
     const int chunk = b.w;
+    tl.blk = lo;
+    tl.gated = gated;
     tl.group = b.x;
     tl.shared = tl.group == a.E;
     tl.m = local / units;
@@ -149,6 +177,7 @@ __device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a, co
     tl.row0 = b.y + start;
     tl.n_mma = (tl.rows + 15) & ~15;
     tl.K = tl.shared ? a.K_shared : a.K;
+    if (MODE == MODE_FUSED && !gated) tl.K = tl.shared ? a2.K_shared : a2.K;
     tl.kb0 = 0;
     tl.kb1 = (tl.K + kBlockK - 1) / kBlockK;
     tl.split = 0;
@@ -195,11 +224,12 @@ struct KIter {
 };
 
 template <int MODE>
-__device__ __forceinline__ bool kiter_begin(KIter& it, int nb, int total, const GemmArgs& a, const SmemPlan* sp)
+__device__ __forceinline__ bool kiter_begin(KIter& it, int nb, int total, const GemmArgs& a, const GemmArgs& a2,
+                                            const SmemPlan* sp)
 {
     it.t = blockIdx.x;
     while (it.t < total) {
-        it.tl = decode_tile<MODE>(nb, it.t, a, sp);
+        it.tl = decode_tile<MODE>(nb, it.t, a, a2, sp);
         if (it.tl.kb0 < it.tl.kb1) {
             it.kb = it.tl.kb0;
             return true;
@@ -210,11 +240,12 @@ __device__ __forceinline__ bool kiter_begin(KIter& it, int nb, int total, const 
 }
 
 template <int MODE>
-__device__ __forceinline__ bool kiter_next(KIter& it, int nb, int total, const GemmArgs& a, const SmemPlan* sp)
+__device__ __forceinline__ bool kiter_next(KIter& it, int nb, int total, const GemmArgs& a, const GemmArgs& a2,
+                                           const SmemPlan* sp)
 {
     if (++it.kb < it.tl.kb1) return true;
     for (it.t += gridDim.x; it.t < total; it.t += gridDim.x) {
-        it.tl = decode_tile<MODE>(nb, it.t, a, sp);
+        it.tl = decode_tile<MODE>(nb, it.t, a, a2, sp);
         if (it.tl.kb0 < it.tl.kb1) {
             it.kb = it.tl.kb0;
             return true;
@@ -226,19 +257,23 @@ __device__ __forceinline__ bool kiter_next(KIter& it, int nb, int total, const G
 template <int MODE>
 __device__ __forceinline__ void issue_a(const KIter& it, uint32_t a_dst, uint32_t full, const CUtensorMap* mA0,
                                         const CUtensorMap* mA1, const CUtensorMap* mA0s, const CUtensorMap* mA1s,
-                                        const GemmArgs& a, uint64_t pol)
+                                        const CUtensorMap* mA2, const CUtensorMap* mA2s, const GemmArgs& a,
+                                        const GemmArgs& a2, uint64_t pol)
 {
     const Tile& tl = it.tl;
     const int kc = it.kb * kBlockK;
-    if (MODE == MODE_GATED) {
-        const CUtensorMap* a0 = tl.shared ? mA0s : mA0;
-        const CUtensorMap* a1 = tl.shared ? mA1s : mA1;
+    if (tl.gated) {
+        const CUtensorMap* w1 = tl.shared ? mA0s : mA0;
+        const CUtensorMap* w3 = tl.shared ? mA1s : mA1;
         const int a_row = (tl.shared ? 0 : tl.group * a.M) + tl.m * 64;
 #pragma unroll
         for (int q = 0; q < 4; q++) {
-            ptx::tma_load_2d(a_dst + (32 * q) * 128, a0, full, kc, a_row + 16 * q, pol);
-            ptx::tma_load_2d(a_dst + (32 * q + 16) * 128, a1, full, kc, a_row + 16 * q, pol);
+            ptx::tma_load_2d(a_dst + (32 * q) * 128, w1, full, kc, a_row + 16 * q, pol);
+            ptx::tma_load_2d(a_dst + (32 * q + 16) * 128, w3, full, kc, a_row + 16 * q, pol);
         }
+    } else if (MODE == MODE_FUSED) {
+        const int a_row = (tl.shared ? 0 : tl.group * a2.M) + tl.m * 128;
+        ptx::tma_load_2d(a_dst, tl.shared ? mA2s : mA2, full, kc, a_row, pol);
     } else {
         const CUtensorMap* a0 = tl.shared ? mA0s : mA0;
         const int a_row = (MODE == MODE_ROUTER || tl.shared ? 0 : tl.group * a.M) + tl.m * 128;
@@ -259,8 +294,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mA1,
                         const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mA0s,
                         const __grid_constant__ CUtensorMap mA1s, const __grid_constant__ CUtensorMap mBs,
-                        const GemmArgs args)
+                        const __grid_constant__ CUtensorMap mA2, const __grid_constant__ CUtensorMap mB2,
+                        const __grid_constant__ CUtensorMap mA2s, const __grid_constant__ CUtensorMap mB2s,
+                        const GemmArgs args, const GemmArgs args2)
 {
+    // MODE_FUSED: args describe the gate/up tiles (W1/W3 = mA0/mA1, xp = mB),
+    // args2 the down tiles (W2 = mA2, h = mB2); other modes ignore args2 and mA2..mB2s.
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + kRingBytes);
@@ -282,9 +321,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     SmemPlan* splan = reinterpret_cast<SmemPlan*>(smem + kRingBytes + kBarBytes);
     if (MODE != MODE_ROUTER) {
         const PlanArrays pa = plan_arrays(const_cast<int32_t*>(args.plan));
-        const int32_t* tbg = MODE == MODE_GATED ? pa.tb1 : pa.tb2;
+        const int32_t* tbg = MODE == MODE_DOWN ? pa.tb2 : pa.tb1;
+        if (threadIdx.x == 0) splan->tiles1 = hdr->tiles1;
         for (int i = threadIdx.x; i <= nb; i += blockDim.x) {
             splan->tb[i] = tbg[i];
+            if (MODE == MODE_FUSED) splan->tb2[i] = pa.tb2[i];
             if (i < nb) {
                 splan->blk[i] = make_int4(pa.group[i], pa.row0[i], pa.rows[i], pa.chunk[i]);
                 splan->units[i] = pa.units[i];
@@ -325,18 +366,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint64_t pol = ptx::policy_evict_normal();
             uint32_t armed = 0, armed_ph = 0;   // slots with a load issued, and its phase
             bool ok = true;
+            // MODE_FUSED: all gate/up tiles of the tile's block have stored their h rows
+            auto wait_block_ready = [&](const Tile& tl) -> bool {
+                const int32_t* dep = plan_arrays(const_cast<int32_t*>(args.plan)).dep + tl.blk;
+                const int m1 = tl.shared ? args.M_shared : args.M;
+                const int need = 4 * splan->units[tl.blk] * ((m1 + 63) / 64);   // 4 epilogue warps per tile
+                if (ptx::ld_acquire_gpu(dep) < need) {
+                    const uint64_t t0 = ptx::globaltimer();
+                    while (ptx::ld_acquire_gpu(dep) < need) {
+                        if (*reinterpret_cast<volatile int*>(&ctl->abort)) return false;
+                        if (ptx::globaltimer() - t0 > kWaitTimeoutNs) {
+                            *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
+                            atomicOr(args.err, DEVERR_TIMEOUT);
+                            return false;
+                        }
+                        __nanosleep(64);
+                    }
+                }
+                ptx::fence_proxy_async_global();   // the TMA reads below come after the acquire
+                return true;
+            };
             // pass 1 (before the dependency wait): weight tiles into the free stages
             int pre = 0;
             if (!waited_early) {
                 KIter it;
-                bool more = kiter_begin<MODE>(it, nb, total, args, splan);
+                bool more = kiter_begin<MODE>(it, nb, total, args, args2, splan);
                 while (more && pre < stages) {
                     const uint32_t full = ptx::smem_u32(&ctl->full[pre]);
                     ptx::mbar_arrive_expect_tx(full, kATileBytes + (uint32_t)it.tl.n_mma * kBRowBytes);
                     armed |= 1u << pre;
-                    issue_a<MODE>(it, ring + (uint32_t)pre * stage_bytes, full, &mA0, &mA1, &mA0s, &mA1s, args, pol);
+                    issue_a<MODE>(it, ring + (uint32_t)pre * stage_bytes, full, &mA0, &mA1, &mA0s, &mA1s, &mA2, &mA2s,
+                                  args, args2, pol);
                     ++pre;
-                    more = kiter_next<MODE>(it, nb, total, args, splan);
+                    more = kiter_next<MODE>(it, nb, total, args, args2, splan);
                 }
                 ptx::grid_dep_wait();
             }
@@ -345,11 +407,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int s = 0, n = 0;
             uint32_t ph = 0;
             KIter it;
-            bool more = kiter_begin<MODE>(it, nb, total, args, splan);
+            bool more = kiter_begin<MODE>(it, nb, total, args, args2, splan);
             while (more) {
                 const uint32_t a_dst = ring + (uint32_t)s * stage_bytes;
                 const uint32_t full = ptx::smem_u32(&ctl->full[s]);
-                const CUtensorMap* b = it.tl.shared ? &mBs : &mB;
+                const CUtensorMap* b = it.tl.gated || MODE != MODE_FUSED ? (it.tl.shared ? &mBs : &mB)
+                                                                          : (it.tl.shared ? &mB2s : &mB2);
+                // a down tile of the fused launch reads h only after its block's gate/up tiles stored it
+                if (MODE == MODE_FUSED && !it.tl.gated && it.kb == 0 && !wait_block_ready(it.tl)) {
+                    ok = false;
+                    break;
+                }
                 if (n < pre) {
                     issue_b(it.tl, it.kb, a_dst + kATileBytes, full, b, pol);
                 } else {
@@ -360,7 +428,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     ptx::mbar_arrive_expect_tx(full, kATileBytes + (uint32_t)it.tl.n_mma * kBRowBytes);
                     armed |= 1u << s;
                     armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
-                    issue_a<MODE>(it, a_dst, full, &mA0, &mA1, &mA0s, &mA1s, args, pol);
+                    issue_a<MODE>(it, a_dst, full, &mA0, &mA1, &mA0s, &mA1s, &mA2, &mA2s, args, args2, pol);
                     issue_b(it.tl, it.kb, a_dst + kATileBytes, full, b, pol);
                 }
                 ++n;
@@ -368,7 +436,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     s = 0;
                     ph ^= 1u;
                 }
-                more = kiter_next<MODE>(it, nb, total, args, splan);
+                more = kiter_next<MODE>(it, nb, total, args, args2, splan);
             }
             if (!ok) {
                 // drain: wait (bounded) for every load this thread issued
@@ -391,7 +459,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t aph = 0;
             bool ok = true, issued = false;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const Tile tl = decode_tile<MODE>(nb, t, args, splan);
+                const Tile tl = decode_tile<MODE>(nb, t, args, args2, splan);
                 if (tl.kb0 >= tl.kb1) continue;
                 if (!bounded_wait(ptx::smem_u32(&ctl->tempty[acc]), aph ^ 1u, ctl, args.err)) {
                     ok = false;
@@ -441,20 +509,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int acc = 0;
         uint32_t aph = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
-            const Tile tl = decode_tile<MODE>(nb, t, args, splan);
+            const Tile tl = decode_tile<MODE>(nb, t, args, args2, splan);
             if (tl.kb0 >= tl.kb1) continue;
             const bool ok = bounded_wait(ptx::smem_u32(&ctl->tfull[acc]), aph, ctl, args.err);
             if (!__all_sync(0xffffffffu, ok)) break;   // the whole warp leaves together
             ptx::tc_fence_after();
             const uint32_t taddr = tmem_base + (uint32_t)acc * 256u + ((uint32_t)(quad * 32) << 16);
-            bf16* out = tl.shared ? args.out_shared : args.out;
-            const size_t ld = (size_t)(tl.shared ? args.ld_out_shared : args.ld_out);
-            const int Mrows = tl.shared ? args.M_shared : args.M;
+            const GemmArgs& ea = (MODE == MODE_FUSED && !tl.gated) ? args2 : args;
+            bf16* out = tl.shared ? ea.out_shared : ea.out;
+            const size_t ld = (size_t)(tl.shared ? ea.ld_out_shared : ea.ld_out);
+            const int Mrows = tl.shared ? ea.M_shared : ea.M;
             for (int c0 = 0; c0 < tl.n_mma; c0 += 16) {
                 uint32_t v[16];
                 ptx::tmem_ld16(taddr + (uint32_t)c0, v);
                 ptx::tmem_ld_wait();
-                if (MODE == MODE_GATED) {
+                if (MODE != MODE_ROUTER && tl.gated) {
                     // lanes 0-15: gate of f row 16*quad + lane; lanes 16-31: up of the same row
                     const int half = lane >> 4;
                     const int frow = tl.m * 64 + quad * 16 + (lane & 15);
@@ -468,12 +537,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         if (col < tl.rows && frow < Mrows)
                             out[(size_t)(tl.row0 + col) * ld + frow] = __float2bfloat16_rn(silu_f(g) * u);
                     }
-                } else if (MODE == MODE_DOWN) {
+                } else if (MODE != MODE_ROUTER) {
                     const int drow = tl.m * 128 + quad * 32 + lane;
                     const int my_col = c0 + (lane & 15);
                     float my_scale = 1.0f;
                     if (!tl.shared && my_col < tl.rows)
-                        my_scale = __ldg(args.gate_w + __ldg(args.perm + tl.row0 + my_col));
+                        my_scale = __ldg(ea.gate_w + __ldg(ea.perm + tl.row0 + my_col));
 #pragma unroll
                     for (int j = 0; j < 16; j++) {
                         const float sc = __shfl_sync(0xffffffffu, my_scale, j);
@@ -502,6 +571,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&ctl->tempty[acc]));
             acc ^= 1;
             if (acc == 0) aph ^= 1u;
+            if (MODE == MODE_FUSED && tl.gated) {
+                // publish this warp's h rows of the tile to the down tiles of its
+                // block: each of the 4 epilogue warps adds 1 after its own stores
+                ptx::fence_proxy_async_global();
+                __syncwarp();
+                if (lane == 0) ptx::red_add_release_gpu(plan_arrays(const_cast<int32_t*>(args.plan)).dep + tl.blk, 1);
+            }
         }
     }
 

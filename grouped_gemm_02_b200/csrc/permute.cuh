@@ -130,6 +130,7 @@ __device__ __forceinline__ void build_plan(int c, int off, int E, int pairs, int
         pa.rows[tid] = n;
         pa.chunk[tid] = chunk;
         pa.units[tid] = units;
+        pa.dep[tid] = 0;
         my_t1 = units * ceil_div(M1, m1_rows);
         my_t2 = units * ceil_div(d, 128);
         my_chunk = chunk;

@@ -64,6 +64,8 @@ def test_algorithmic_counts():
     assert a["w_act"] == 4 * 3 * s.d * s.f * 2
     assert a["flops"] == 6.0 * 256 * s.d * s.f
     assert a["g1_bytes"] == 4 * 2 * s.f * s.d * 2 + 256 * s.d * 2 + 256 * s.f * 2
+    assert a["g2_bytes"] == 4 * s.d * s.f * 2 + 256 * s.f * 2 + 256 * s.d * 2
+    assert a["g1_flops"] + a["g2_flops"] == a["flops"]
     sh = wl.DEEPSEEK_V3.with_(T=8)
     c2 = np.zeros(sh.E, dtype=np.int64)
     c2[0] = 64
@@ -109,3 +111,13 @@ def test_workload_label_and_parse():
     s = bench.parse_workload(A)
     assert s.T == 64 and s.alpha == 0.05 and s.f_shared == 2048
     assert "shared_f=2048" in bench.workload_label(s)
+
+
+def test_gemm_launch_rule(monkeypatch):
+    monkeypatch.delenv("MOE_GEMM_SPLIT", raising=False)
+    assert bench.gemm_fused(256, 1024) and bench.gemm_fused(64, 2048)
+    assert not bench.gemm_fused(512, 2048) and not bench.gemm_fused(32, 14336)
+    monkeypatch.setenv("MOE_GEMM_SPLIT", "1")
+    assert not bench.gemm_fused(256, 1024)
+    monkeypatch.setenv("MOE_GEMM_SPLIT", "0")
+    assert bench.gemm_fused(32768, 14336)

@@ -207,6 +207,7 @@ def _layer_check(s: wl.LayerShape, seed: int, n_sample=None, device_inputs=False
     ("mixtral", dict(T=1)),
     ("mixtral", dict(T=16)),
     ("kimi_k2", dict(T=8)),
+    ("deepseek_v3", dict(T=16, alpha=0.05)),    # one launch for both GEMMs, with the shared expert
     ("deepseek_v3", dict(T=64, alpha=0.05)),
 ])
 def test_layer_small(name, kw):
