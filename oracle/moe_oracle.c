@@ -380,15 +380,18 @@ static double e4m3_value(uint8_t c)
     return g_e4m3[c];
 }
 
-/* Smallest power of two s with amax / s <= 448 (amax = 0: s = 1). */
+/* Smallest power of two s with amax / s <= 448 (amax = 0: s = 1), kept in
+ * the range of a UE8M0 scale, 2^-127 .. 2^127: the block-scaled MMA takes
+ * its scales in that format, so a block whose amax lies below 448 * 2^-128
+ * gets the scale 2^-127 (its codes then sit low in the e4m3 range). */
 double oracle_fp8_block_scale(double amax)
 {
     if (!(amax > 0))
         return 1.0;
     int e = 0;
-    while (amax > ldexp(448.0, e))
+    while (amax > ldexp(448.0, e) && e < 127)
         e++;
-    while (amax <= ldexp(448.0, e - 1))
+    while (amax <= ldexp(448.0, e - 1) && e > -127)
         e--;
     return ldexp(1.0, e);
 }

@@ -314,6 +314,20 @@ def pin_fp8_block_scale():
         assert m == 0.5                              # a power of two
         assert amax / s <= 448.0 < amax / (s / 2)    # the smallest such
     assert oracle.fp8_block_scale(0.0) == 1.0
+    # the UE8M0 range ends at 2^-127: every smaller amax gets that scale
+    assert oracle.fp8_block_scale(448.0 * 2.0 ** -127) == 2.0 ** -127
+    assert oracle.fp8_block_scale(448.0 * 2.0 ** -127 * 0.75) == 2.0 ** -127
+    for amax in (2.0 ** -133, 1e-40, 448.0 * 2.0 ** -140):
+        assert oracle.fp8_block_scale(amax) == 2.0 ** -127
+    assert oracle.fp8_block_scale(448.0 * 2.0 ** -126 * 0.75) == 2.0 ** -126
+    # a row whose block holds only values near the bottom of bf16: codes are x / 2^-127
+    xb = np.zeros((1, 128), dtype=np.uint16)
+    xb[0, 0] = 0x0001                                 # 2^-133, the smallest bf16 subnormal
+    xb[0, 1] = 0x0008                                 # 2^-130
+    q, sc = oracle.quantize_rows_fp8(xb)
+    assert sc[0, 0] == 2.0 ** -127
+    assert oracle.e4m3_decode(int(q[0, 1])) == 0.125  # 2^-130 / 2^-127
+    assert oracle.e4m3_decode(int(q[0, 0])) == 2.0 ** -6         # 2^-133 / 2^-127: the smallest e4m3 normal
 
 
 def pin_fp8_quantize_rows_and_blocks():

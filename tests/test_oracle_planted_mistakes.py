@@ -39,7 +39,10 @@ MUTANTS = {
                                     "g += e4m3_value(W1q[r * d + c]) * s1[(c / 128) * db + r / 128] * xc;"),
     "fp8_ties_away_from_zero": ("double m = nearbyint((2.0 * frac - 1.0) * 8.0);",
                                 "double m = round((2.0 * frac - 1.0) * 8.0);"),
-    "fp8_scale_not_smallest": ("while (amax <= ldexp(448.0, e - 1))", "while (amax <= ldexp(448.0, e - 2))"),
+    "fp8_scale_not_smallest": ("while (amax <= ldexp(448.0, e - 1) && e > -127)",
+                               "while (amax <= ldexp(448.0, e - 2) && e > -127)"),
+    "fp8_scale_below_ue8m0": ("while (amax <= ldexp(448.0, e - 1) && e > -127)",
+                              "while (amax <= ldexp(448.0, e - 1) && e > -160)"),
     "fp8_exponent_bias": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
     "fp8_activation_scale_dropped": ("double xc = e4m3_value(xq[c]) * sx[c / 128];", "double xc = e4m3_value(xq[c]);"),
 }
