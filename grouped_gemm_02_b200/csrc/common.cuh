@@ -158,15 +158,22 @@ __host__ inline WsLayout ws_layout(int64_t T, int64_t d, int64_t f, int64_t E, i
 struct WsLayoutFp8 {
     WsLayout ctrl;   // err, plan, block_counts, router_partials, ctrl_end
     size_t logits, topk_idx, topk_w, counts, offsets, perm, inv_perm;
-    size_t x8, sx, xp8, sxp, h8, sh, y_p, hs8, shs, ys;
+    size_t x8, sx, xp8, sxp, h8, sh, y_p, hs8, shs, ys, sxT;
+    int64_t ld_pairs, ld_tokens;   // row length of the K-block-major scale arrays (pairs, tokens rounded up to 4)
     size_t total;
 };
 
+// Token scales the GEMM reads by TMA are stored K-block-major, [K/128][ld]
+// with ld a multiple of 4 (a 16-byte row pitch): sxp [d/128][pairs],
+// sh [f/128][pairs], shs [f_shared/128][T], sxT [d/128][T].  sx keeps the
+// quantiser's row-major [T][d/128].
 __host__ inline WsLayoutFp8 ws_layout_fp8(int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, int64_t fs)
 {
     WsLayoutFp8 L{};
     L.ctrl = ws_layout(T, d, 0, E, k, 0);
     const int64_t P = T * k, Ts = fs > 0 ? T : 0;
+    L.ld_pairs = (P + 3) & ~int64_t(3);
+    L.ld_tokens = (T + 3) & ~int64_t(3);
     size_t o = L.ctrl.ctrl_end;
     L.logits = o; o = align_up(o + (size_t)T * E * 4, 256);
     L.topk_idx = o; o = align_up(o + (size_t)P * 4, 256);
@@ -178,13 +185,14 @@ __host__ inline WsLayoutFp8 ws_layout_fp8(int64_t T, int64_t d, int64_t f, int64
     L.x8 = o; o = align_up(o + (size_t)T * d, 1024);
     L.sx = o; o = align_up(o + (size_t)T * (d / 128) * 4, 256);
     L.xp8 = o; o = align_up(o + (size_t)P * d, 1024);
-    L.sxp = o; o = align_up(o + (size_t)P * (d / 128) * 4, 256);
+    L.sxp = o; o = align_up(o + (size_t)(d / 128) * L.ld_pairs * 4, 256);
     L.h8 = o; o = align_up(o + (size_t)P * f, 1024);
-    L.sh = o; o = align_up(o + (size_t)P * (f / 128) * 4, 256);
+    L.sh = o; o = align_up(o + (size_t)(f / 128) * L.ld_pairs * 4, 256);
     L.y_p = o; o = align_up(o + (size_t)P * d * 2, 1024);
     L.hs8 = o; o = align_up(o + (size_t)Ts * fs, 1024);
-    L.shs = o; o = align_up(o + (size_t)Ts * (fs / 128) * 4, 256);
+    L.shs = o; o = align_up(o + (size_t)(fs / 128) * (Ts ? L.ld_tokens : 0) * 4, 256);
     L.ys = o; o = align_up(o + (size_t)Ts * d * 2, 1024);
+    L.sxT = o; o = align_up(o + (size_t)(d / 128) * (Ts ? L.ld_tokens : 0) * 4, 256);
     L.total = o;
     return L;
 }

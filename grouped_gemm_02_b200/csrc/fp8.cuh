@@ -1,24 +1,29 @@
 // fp8.cuh -- the FP8 block-scaled expert path (S9): e4m3 quantisers, the e4m3
-// row gather, and a persistent tcgen05 grouped GEMM on e4m3 operands.
+// row gather, and a persistent grouped GEMM on tcgen05 block-scaled MMAs.
 //
-// GC-MoE (abstract) runs its expert GEMMs as block-scaled FP8 MMAs with a
-// requantisation step; the workload table fixes e4m3 codes with 1 x 128
-// activation blocks and 128 x 128 weight blocks.  Readings: a block's scale is
-// the smallest power of two s with amax / s <= 448 (amax = 0: s = 1); codes are
-// round-to-nearest-even with saturation to +-448.  Because every scale is a
-// power of two, scaling is exact: the GEMM multiplies e4m3 codes on the tensor
-// cores one 128-wide K block at a time (tcgen05.mma kind::f8f6f4, fp32
-// accumulate into a fresh TMEM partial) and the epilogue warps add each partial
-// times (weight-block scale x activation-block scale) into fp32 running sums --
-// the dequantised product the definition asks for.
+// GC-MoE (abstract) runs its expert GEMMs as operand-swapped tcgen05
+// block-scaled MMAs with a requantisation step; the workload table fixes e4m3
+// codes with 1 x 128 activation blocks and 128 x 128 weight blocks.  Readings:
+// a block's scale is the smallest power of two s with amax / s <= 448 (amax =
+// 0: s = 1), held to the UE8M0 range 2^-127 .. 2^127 that the MMA takes;
+// codes are round-to-nearest-even with saturation to +-448.
 //
-//   MODE gate/up:  h = silu(sum_kb P_g * s_W1 * s_x) * (sum_kb P_u * s_W3 * s_x),
-//                  then h is requantised in 1 x 128 blocks along f (the tile's
-//                  128 f rows are one block) -> h8 [pairs, f] + sh [pairs, f/128]
-//   MODE down:     y_p = gate * sum_kb P * s_W2 * s_h  -> bf16
+// Because every scale is a power of two it is exactly a UE8M0 exponent, and
+// the MMA (kind::mxf8f6f4.block_scale, one scale per row per 32-wide K
+// sub-block, fp32 accumulate) applies it to each product inside the tensor
+// core: the TMEM accumulator holds sum_k (a_k s_a)(b_k s_b) over the whole K
+// range, the dequantised product the definition asks for, and the epilogue
+// reads it once.  A 128 x 128 weight block and a 1 x 128 activation block
+// each give one exponent repeated over their four 32-wide sub-blocks.
 //
-// One tile = 128 weight rows (W1 and W3 rows side by side for gate/up) x at
-// most 64 tokens; the epilogue keeps the tile's running sums in registers.
+//   gate/up:  h = silu(x W1^T) * (x W3^T) per tile of 128 f rows, then h is
+//             requantised in 1 x 128 blocks along f (the tile's 128 f rows are
+//             one block) -> h8 [pairs, f] + scales [f/128, pairs]
+//   down:     y_p = gate * (h W2^T) -> bf16
+//
+// One tile = 128 weight rows (W1 and W3 side by side for gate/up: two MMAs
+// into two accumulators) x at most 112 tokens, so that two tiles' accumulators
+// (2 x (112 + 112) columns) and the scale factors fit the 512 TMEM columns.
 #pragma once
 
 #include <cuda_fp8.h>
@@ -29,19 +34,58 @@
 
 namespace moe {
 
-constexpr int kFp8TileRows = 64;                 // most tokens one FP8 tile carries
+constexpr int kFp8TileRows = 112;                // most tokens one FP8 tile carries
 constexpr int kFp8BlockK = 128;                  // e4m3 elements per 128-byte swizzle row = one scale block
-constexpr int kFp8Bufs = 4;                      // TMEM partial buffers between the MMA and the epilogue
-constexpr uint32_t kFp8TmemCols = 512;           // 4 partial buffers x (g: 64 + u: 64) columns
+constexpr int kFp8MaxK = 128 * kFp8BlockK;       // reduction length limit: 4 weight scales per lane of a warp
+constexpr uint32_t kFp8TmemCols = 512;
+constexpr uint32_t kFp8AccCols = 256;            // accumulator set b at column 256 b: g at +0, u at +112
+constexpr uint32_t kSfColA0 = 480;               // scale factors: W1 (or W2) at 480, W3 at 484, tokens at 488
+constexpr uint32_t kSfColA1 = 484;
+constexpr uint32_t kSfColB = 488;
+constexpr int kFp8RingBytes = kRingBytes - 4096;
+constexpr uint32_t kSfStageBytes = 2048;         // per stage: 128 token scales (fp32, by TMA) + 3 scale atoms
 
 // Smallest power-of-two exponent e with amax <= 448 * 2^e (amax > 0), from the
-// binary exponent of amax: amax = m * 2^x, m in [0.5, 1), 448 = 0.875 * 2^9.
+// binary exponent of amax: amax = m * 2^x, m in [0.5, 1), 448 = 0.875 * 2^9;
+// held to the UE8M0 range [-127, 127].
 __device__ __forceinline__ int fp8_scale_exp(float amax)
 {
     if (!(amax > 0.f)) return 0;
     int x;
     const float m = frexpf(amax, &x);
-    return m <= 0.875f ? x - 9 : x - 8;
+    return max(-127, min(127, m <= 0.875f ? x - 9 : x - 8));
+}
+
+// 2^k as fp32 for k in [-127, 127] (2^-127 is the subnormal 0x00400000).
+__device__ __forceinline__ float pow2f(int k)
+{
+    return k >= -126 ? __int_as_float((k + 127) << 23) : __int_as_float(0x00400000);
+}
+
+// Per-column maximum over the 32 lanes of 16 columns held one per register:
+// a butterfly that halves the columns at every step (16 shuffles instead of
+// 5 per column).  On return, lanes 2c and 2c + 1 hold column c's maximum in v[0].
+__device__ __forceinline__ void warp_colmax16(float (&v)[16], int lane)
+{
+#pragma unroll
+    for (int step = 0; step < 4; step++) {
+        const int m = 16 >> step, half = 8 >> step;
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < half; i++) {
+            const float keep = upper ? v[i + half] : v[i];
+            const float send = upper ? v[i] : v[i + half];
+            v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, m));
+        }
+    }
+    v[0] = fmaxf(v[0], __shfl_xor_sync(0xffffffffu, v[0], 1));
+}
+
+// UE8M0 code of a power-of-two fp32 scale in [2^-127, 2^127]: its biased
+// exponent (2^-127 is the fp32 subnormal 0x00400000, exponent field 0).
+__device__ __forceinline__ uint32_t ue8m0_of(float s)
+{
+    return (__float_as_uint(s) >> 23) & 0xFFu;
 }
 
 __device__ __forceinline__ uint8_t e4m3_of(float v)
@@ -51,8 +95,10 @@ __device__ __forceinline__ uint8_t e4m3_of(float v)
 
 // ---------------------------------------------------------------- quantisers
 // 1 x 128 blocks along rows: one warp per (row, block); lane l holds 4 values.
+// scale_t (may be null) also receives the scales K-block-major: scale_t[b * ld_t + r].
 __global__ void __launch_bounds__(256) quantize_rows_fp8_kernel(const bf16* __restrict__ src, int64_t R, int C,
-                                                                uint8_t* __restrict__ dst, float* __restrict__ scale)
+                                                                uint8_t* __restrict__ dst, float* __restrict__ scale,
+                                                                float* __restrict__ scale_t, int64_t ld_t)
 {
     ptx::grid_dep_wait();
     ptx::grid_dep_launch();
@@ -73,7 +119,10 @@ __global__ void __launch_bounds__(256) quantize_rows_fp8_kernel(const bf16* __re
 #pragma unroll
     for (int i = 0; i < 4; i++) packed |= (uint32_t)e4m3_of(ldexpf(v[i], -e)) << (8 * i);
     *reinterpret_cast<uint32_t*>(dst + r * C + b * 128 + lane * 4) = packed;
-    if (lane == 0) scale[r * nb + b] = ldexpf(1.f, e);
+    if (lane == 0) {
+        scale[r * nb + b] = ldexpf(1.f, e);
+        if (scale_t) scale_t[b * ld_t + r] = ldexpf(1.f, e);
+    }
 }
 
 // 128 x 128 blocks: one CTA of 256 threads per block; thread t covers half of row t/2.
@@ -126,12 +175,14 @@ __global__ void __launch_bounds__(256) quantize_blocks_fp8_kernel(const bf16* __
     if (threadIdx.x == 0) scale[br * nbc + bc] = ldexpf(1.f, e);
 }
 
-// xp8[pos, :] = x8[perm[pos] / k, :], sxp[pos, :] = sx[perm[pos] / k, :]; one warp per row.
+// xp8[pos, :] = x8[perm[pos] / k, :], and the row's scales K-block-major:
+// sxpT[b * ld + pos] = sx[perm[pos] / k, b]; one warp per row.
 __global__ void __launch_bounds__(256) gather_rows_fp8_kernel(const uint8_t* __restrict__ x8,
                                                               const float* __restrict__ sx,
                                                               const int32_t* __restrict__ perm,
                                                               const int32_t* __restrict__ offsets, int E, int k, int d,
-                                                              uint8_t* __restrict__ xp8, float* __restrict__ sxp)
+                                                              uint8_t* __restrict__ xp8, float* __restrict__ sxpT,
+                                                              int64_t ld)
 {
     ptx::grid_dep_wait();
     ptx::grid_dep_launch();
@@ -152,9 +203,10 @@ __global__ void __launch_bounds__(256) gather_rows_fp8_kernel(const uint8_t* __r
             for (int u = 0; u < 4; u++)
                 if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = buf[u];
         }
-        for (int b = lane; b < nsb; b += 32) sxp[(size_t)r * nsb + b] = sx[(size_t)t * nsb + b];
+        for (int b = lane; b < nsb; b += 32) sxpT[(size_t)b * ld + r] = sx[(size_t)t * nsb + b];
     }
 }
+
 
 // ---------------------------------------------------------------- FP8 grouped GEMM
 struct Fp8Args {
@@ -167,12 +219,12 @@ struct Fp8Args {
     const float* sA1;               // W3 (gate/up)
     const float* sA0s;              // shared expert: Ws1 or Ws2
     const float* sA1s;              // Ws3
-    const float* sB;                // activation-block scales of the B rows [pairs, K/128]
-    const float* sBs;               // shared rows [T, K_shared/128]
     uint8_t* out8;                  // gate/up: h8 [pairs, f]
-    float* out8_scale;              // sh [pairs, f/128]
+    float* out8_scale;              // its scales, K-block-major [f/128, ld_scale]
+    int ld_scale;
     uint8_t* out8_shared;           // hs8 [T, f_shared]
-    float* out8_scale_shared;       // shs [T, f_shared/128]
+    float* out8_scale_shared;       // [f_shared/128, ld_scale_shared]
+    int ld_scale_shared;
     bf16* out;                      // down: y_p [pairs, d]
     bf16* out_shared;               // ys [T, d]
     const int32_t* perm;
@@ -185,7 +237,6 @@ struct Fp8Tile {
     bool shared;
 };
 
-template <bool GATED>
 __device__ __forceinline__ Fp8Tile fp8_decode(int nb, int t, const Fp8Args& a, const SmemPlan* sp)
 {
     const int* tb = sp->tb;
@@ -207,7 +258,7 @@ __device__ __forceinline__ Fp8Tile fp8_decode(int nb, int t, const Fp8Args& a, c
     tl.rows = min(b.w, b.z - start);
     tl.row0 = b.y + start;
     tl.n_mma = (tl.rows + 15) & ~15;
-    tl.nkb = ((tl.shared ? a.K_shared : a.K) + kFp8BlockK - 1) / kFp8BlockK;
+    tl.nkb = (tl.shared ? a.K_shared : a.K) / kFp8BlockK;
     return tl;
 }
 
@@ -216,59 +267,92 @@ struct Fp8Iter {
     Fp8Tile tl;
 };
 
-template <bool GATED>
 __device__ __forceinline__ bool fp8_iter_begin(Fp8Iter& it, int nb, int total, const Fp8Args& a, const SmemPlan* sp)
 {
-    it.t = blockIdx.x;
-    if (it.t >= total) return false;
-    it.tl = fp8_decode<GATED>(nb, it.t, a, sp);
-    it.kb = 0;
-    return true;
+    for (it.t = blockIdx.x; it.t < total; it.t += gridDim.x) {
+        it.tl = fp8_decode(nb, it.t, a, sp);
+        if (it.tl.nkb > 0) {
+            it.kb = 0;
+            return true;
+        }
+    }
+    return false;
 }
 
-template <bool GATED>
 __device__ __forceinline__ bool fp8_iter_next(Fp8Iter& it, int nb, int total, const Fp8Args& a, const SmemPlan* sp)
 {
     if (++it.kb < it.tl.nkb) return true;
-    it.t += gridDim.x;
-    if (it.t >= total) return false;
-    it.tl = fp8_decode<GATED>(nb, it.t, a, sp);
-    it.kb = 0;
-    return true;
+    for (it.t += gridDim.x; it.t < total; it.t += gridDim.x) {
+        it.tl = fp8_decode(nb, it.t, a, sp);
+        if (it.tl.nkb > 0) {
+            it.kb = 0;
+            return true;
+        }
+    }
+    return false;
 }
 
-__device__ __forceinline__ void named_bar_epilogue() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
-// Instruction descriptor for kind::f8f6f4 with e4m3 A and B (format 0), fp32 accumulator.
-__host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t M, uint32_t N)
+// Instruction descriptor for kind::mxf8f6f4 with block scaling: A and B e4m3
+// (format 0, bits 7-9 and 10-12), both K-major, N >> 3 in bits 17-22, scale
+// format UE8M0 (bit 23), M >> 4 in bits 24-28, scale-factor byte 0 for A
+// (bits 29-30) and B (bits 4-5), dense K = 32.  The accumulator is fp32.
+__host__ __device__ constexpr uint32_t idesc_mxf8_ue8m0(uint32_t M, uint32_t N)
 {
-    return (1u << 4) | ((N >> 3) << 17) | ((M >> 4) << 24);
+    return ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_fp8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                           uint32_t accumulate)
+// D[tmem] (+)= (A * 2^sfa) (B * 2^sfb)^T over one 32-wide K step: sfa / sfb
+// are the TMEM addresses of the scale-factor columns.
+__device__ __forceinline__ void mma_mxf8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t sfa, uint32_t sfb, uint32_t accumulate)
 {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
         : "memory");
 }
 
+__device__ __forceinline__ uint32_t pick4(const uint32_t (&v)[4], int i)
+{
+    return i == 0 ? v[0] : i == 1 ? v[1] : i == 2 ? v[2] : v[3];
+}
+
+__device__ __forceinline__ float pick4f(const float (&v)[4], int i)
+{
+    return i == 0 ? v[0] : i == 1 ? v[1] : i == 2 ? v[2] : v[3];
+}
+
+// Persistent grouped GEMM on e4m3 operands with UE8M0 block scales.
+//
+// Warp roles as in the bf16 GEMM: warp 0 TMA producer, warp 1 MMA issuer,
+// warps 2-5 epilogue.  A ring stage holds the A tile(s) (128 weight rows x 128
+// K bytes each), the token rows (n x 128 bytes), the tokens' 128 fp32 scales of
+// that K block (one TMA box starting at row0 rounded down to 4 tokens, the
+// 16-byte rule for a TMA start) and three 512-byte scale-factor atoms.  The MMA
+// warp turns the staged token scales and the tile's weight scales into UE8M0
+// atoms -- 32 rows of 16 bytes, token n = n0 + 32 n1 at byte 16 n0 + 4 n1,
+// its exponent repeated in the four bytes of the 32-bit word, one per 32-wide
+// K sub-block -- copies them into TMEM with tcgen05.cp (32x128b, repeated over
+// the four lane quadrants) and issues the MMAs.  tcgen05.cp and tcgen05.mma
+// from one thread execute in issue order, so one set of scale-factor columns
+// serves every K block.
 template <bool GATED>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mA1,
                             const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mA0s,
                             const __grid_constant__ CUtensorMap mA1s, const __grid_constant__ CUtensorMap mBs,
+                            const __grid_constant__ CUtensorMap mSB, const __grid_constant__ CUtensorMap mSBs,
                             const Fp8Args args)
 {
     constexpr uint32_t kABytes = GATED ? 2 * 128 * kFp8BlockK : 128 * kFp8BlockK;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + kRingBytes);
-    SmemPlan* splan = reinterpret_cast<SmemPlan*>(smem + kRingBytes + kBarBytes);
-    float* red = reinterpret_cast<float*>(smem + kRingBytes + kBarBytes + sizeof(SmemPlan));   // [4][64]
+    SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + kFp8RingBytes);
+    SmemPlan* splan = reinterpret_cast<SmemPlan*>(smem + kFp8RingBytes + kBarBytes);
+    // per-token amax of h from each epilogue warp, two tiles deep: [2][4][kFp8TileRows]
+    float* red = reinterpret_cast<float*>(smem + kFp8RingBytes + kBarBytes + sizeof(SmemPlan));
     const uint32_t ring = ptx::smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -282,8 +366,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int nb = hdr->n_blocks;
     const int total = GATED ? hdr->tiles1 : hdr->tiles2;
     const int n_max = max(16, hdr->n_max);
-    const uint32_t stage_bytes = kABytes + (uint32_t)n_max * kFp8BlockK;
-    const int stages = min(kMaxStages, (int)(kRingBytes / stage_bytes));
+    const uint32_t b_bytes = (uint32_t)n_max * kFp8BlockK;       // B region of a stage (largest tile)
+    const uint32_t stage_bytes = kABytes + b_bytes + kSfStageBytes;
+    const int stages = min(kMaxStages, (int)(kFp8RingBytes / stage_bytes));
     {
         const PlanArrays pa = plan_arrays(const_cast<int32_t*>(args.plan));
         const int32_t* tbg = GATED ? pa.tb1 : pa.tb2;
@@ -300,10 +385,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ptx::mbar_init(ptx::smem_u32(&ctl->full[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&ctl->empty[s]), 1);
         }
-        for (int a = 0; a < kFp8Bufs; a++) {
+        for (int a = 0; a < 2; a++) {
             ptx::mbar_init(ptx::smem_u32(&ctl->tfull[a]), 1);
             ptx::mbar_init(ptx::smem_u32(&ctl->tempty[a]), 4);
         }
+        ptx::mbar_init(ptx::smem_u32(&ctl->tfull[2]), 4);   // the epilogue warps' per-tile amax exchange
         ptx::mbar_init(ptx::smem_u32(&ctl->drain), 1);
         ctl->abort = 0;
         ptx::fence_mbar_init();
@@ -312,6 +398,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == 0 && lane == 0) {
         ptx::prefetch_tensormap(&mA0);
         ptx::prefetch_tensormap(&mB);
+        ptx::prefetch_tensormap(&mSB);
         if (GATED) ptx::prefetch_tensormap(&mA1);
     }
     if (warp == 1) {
@@ -329,6 +416,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint64_t pol = ptx::policy_evict_normal();
             uint32_t armed = 0, armed_ph = 0;
             bool ok = true;
+            auto tx_bytes = [&](const Fp8Tile& tl) { return kABytes + (uint32_t)tl.n_mma * kFp8BlockK + 512u; };
             auto issue_a = [&](const Fp8Iter& it, uint32_t a_dst, uint32_t full) {
                 const Fp8Tile& tl = it.tl;
                 const int kc = it.kb * kFp8BlockK;
@@ -337,24 +425,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 ptx::tma_load_2d(a_dst, tl.shared ? &mA0s : &mA0, full, kc, a_row, pol);
                 if (GATED) ptx::tma_load_2d(a_dst + 128 * kFp8BlockK, tl.shared ? &mA1s : &mA1, full, kc, a_row, pol);
             };
-            auto issue_b = [&](const Fp8Iter& it, uint32_t b_dst, uint32_t full) {
+            auto issue_b = [&](const Fp8Iter& it, uint32_t stage, uint32_t full) {
                 const Fp8Tile& tl = it.tl;
                 const int kc = it.kb * kFp8BlockK;
+                const uint32_t b_dst = stage + kABytes;
                 for (int i = 0; i < tl.n_mma / 16; i++)
                     ptx::tma_load_2d(b_dst + i * 16 * kFp8BlockK, tl.shared ? &mBs : &mB, full, kc, tl.row0 + 16 * i,
                                      pol);
+                // the tokens' scales of this K block: 128 fp32 from row0 rounded down to 4
+                ptx::tma_load_2d(b_dst + b_bytes, tl.shared ? &mSBs : &mSB, full, tl.row0 & ~3, it.kb, pol);
             };
             int pre = 0;
             if (!waited_early) {
                 Fp8Iter it;
-                bool more = fp8_iter_begin<GATED>(it, nb, total, args, splan);
+                bool more = fp8_iter_begin(it, nb, total, args, splan);
                 while (more && pre < stages) {
                     const uint32_t full = ptx::smem_u32(&ctl->full[pre]);
-                    ptx::mbar_arrive_expect_tx(full, kABytes + (uint32_t)it.tl.n_mma * kFp8BlockK);
+                    ptx::mbar_arrive_expect_tx(full, tx_bytes(it.tl));
                     armed |= 1u << pre;
                     issue_a(it, ring + (uint32_t)pre * stage_bytes, full);
                     ++pre;
-                    more = fp8_iter_next<GATED>(it, nb, total, args, splan);
+                    more = fp8_iter_next(it, nb, total, args, splan);
                 }
                 ptx::grid_dep_wait();
             }
@@ -362,29 +453,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int s = 0, n = 0;
             uint32_t ph = 0;
             Fp8Iter it;
-            bool more = fp8_iter_begin<GATED>(it, nb, total, args, splan);
+            bool more = fp8_iter_begin(it, nb, total, args, splan);
             while (more) {
-                const uint32_t a_dst = ring + (uint32_t)s * stage_bytes;
+                const uint32_t stage = ring + (uint32_t)s * stage_bytes;
                 const uint32_t full = ptx::smem_u32(&ctl->full[s]);
                 if (n < pre) {
-                    issue_b(it, a_dst + kABytes, full);
+                    issue_b(it, stage, full);
                 } else {
                     if (!bounded_wait(ptx::smem_u32(&ctl->empty[s]), ph ^ 1u, ctl, args.err)) {
                         ok = false;
                         break;
                     }
-                    ptx::mbar_arrive_expect_tx(full, kABytes + (uint32_t)it.tl.n_mma * kFp8BlockK);
+                    ptx::mbar_arrive_expect_tx(full, tx_bytes(it.tl));
                     armed |= 1u << s;
                     armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
-                    issue_a(it, a_dst, full);
-                    issue_b(it, a_dst + kABytes, full);
+                    issue_a(it, stage, full);
+                    issue_b(it, stage, full);
                 }
                 ++n;
                 if (++s == stages) {
                     s = 0;
                     ph ^= 1u;
                 }
-                more = fp8_iter_next<GATED>(it, nb, total, args, splan);
+                more = fp8_iter_next(it, nb, total, args, splan);
             }
             if (!ok) {
                 const uint64_t t0 = ptx::globaltimer();
@@ -398,172 +489,220 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer: one fresh partial per K block
-        if (ptx::elect_one()) {
-            int s = 0, pb = 0;
-            uint32_t ph = 0, pph = 0;
-            bool ok = true, issued = false;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const Fp8Tile tl = fp8_decode<GATED>(nb, t, args, splan);
-                const uint32_t idesc = idesc_e4m3_f32(128, (uint32_t)tl.n_mma);
-                for (int kb = 0; kb < tl.nkb; kb++) {
-                    if (!bounded_wait(ptx::smem_u32(&ctl->tempty[pb]), pph ^ 1u, ctl, args.err) ||
-                        !bounded_wait(ptx::smem_u32(&ctl->full[s]), ph, ctl, args.err)) {
-                        ok = false;
-                        break;
-                    }
+        // ------------------------------------------------------------ scale factors + MMA issue (whole warp)
+        int s = 0, acc = 0;
+        uint32_t ph = 0, aph = 0;
+        bool ok = true, issued = false;
+        // The weight-block scales of a tile (lane l: K blocks l, l + 32, l + 64, l + 96)
+        // are loaded one tile ahead, so their latency hides behind the previous tile.
+        auto next_tile = [&](int t) {
+            for (; t < total; t += gridDim.x)
+                if (fp8_decode(nb, t, args, splan).nkb > 0) break;
+            return t;
+        };
+        auto load_scales = [&](int t, float (&wa)[4], float (&wb)[4]) {
+            if (t >= total) return;
+            const Fp8Tile tl = fp8_decode(nb, t, args, splan);
+            const int Mrows = tl.shared ? args.M_shared : args.M;
+            const int64_t srow = (int64_t)(tl.shared ? 0 : tl.group * (Mrows / 128)) + tl.m;
+            const float* sA0 = (tl.shared ? args.sA0s : args.sA0) + srow * tl.nkb;
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const int kb = 32 * i + lane;
+                wa[i] = kb < tl.nkb ? __ldg(sA0 + kb) : 1.f;
+            }
+            if (GATED) {
+                const float* sA1 = (tl.shared ? args.sA1s : args.sA1) + srow * tl.nkb;
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const int kb = 32 * i + lane;
+                    wb[i] = kb < tl.nkb ? __ldg(sA1 + kb) : 1.f;
+                }
+            }
+        };
+        float nwa[4] = {1.f, 1.f, 1.f, 1.f}, nwb[4] = {1.f, 1.f, 1.f, 1.f};
+        int t = next_tile(blockIdx.x);
+        load_scales(t, nwa, nwb);
+        for (; t < total && ok;) {
+            const Fp8Tile tl = fp8_decode(nb, t, args, splan);
+            uint32_t ea[4], eb[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                ea[i] = __float_as_uint(nwa[i]);
+                eb[i] = __float_as_uint(nwb[i]);
+            }
+            const int t_next = next_tile(t + gridDim.x);
+            load_scales(t_next, nwa, nwb);
+            ok = __all_sync(0xffffffffu, bounded_wait(ptx::smem_u32(&ctl->tempty[acc]), aph ^ 1u, ctl, args.err));
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const uint32_t d_g = tmem_base + (uint32_t)acc * kFp8AccCols;
+            const uint32_t idesc = idesc_mxf8_ue8m0(128, (uint32_t)tl.n_mma);
+            const int shift = tl.row0 & 3;
+            for (int kb = 0; kb < tl.nkb; kb++) {
+                ok = __all_sync(0xffffffffu, bounded_wait(ptx::smem_u32(&ctl->full[s]), ph, ctl, args.err));
+                if (!ok) break;
+                uint8_t* stage_p = smem + (size_t)s * stage_bytes;
+                const float* staged = reinterpret_cast<const float*>(stage_p + kABytes + b_bytes);
+                uint8_t* atoms = stage_p + kABytes + b_bytes + 512;   // A0, A1, B: 512 bytes each
+                uint32_t w[4];
+#pragma unroll
+                for (int m1 = 0; m1 < 4; m1++) {
+                    const int c = lane + 32 * m1;
+                    const uint32_t e = c < tl.rows ? ue8m0_of(staged[shift + c]) : 127u;
+                    w[m1] = e * 0x01010101u;
+                }
+                *reinterpret_cast<uint4*>(atoms + 1024 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+                const uint32_t a0 = ue8m0_of(__uint_as_float(__shfl_sync(0xffffffffu, pick4(ea, kb >> 5), kb & 31))) *
+                                    0x01010101u;
+                *reinterpret_cast<uint4*>(atoms + 16 * lane) = make_uint4(a0, a0, a0, a0);
+                if (GATED) {
+                    const uint32_t a1 =
+                        ue8m0_of(__uint_as_float(__shfl_sync(0xffffffffu, pick4(eb, kb >> 5), kb & 31))) * 0x01010101u;
+                    *reinterpret_cast<uint4*>(atoms + 512 + 16 * lane) = make_uint4(a1, a1, a1, a1);
+                }
+                ptx::fence_proxy_async_smem();   // the atoms are read by tcgen05.cp (async proxy)
+                __syncwarp();
+                if (lane == 0) {
                     ptx::tc_fence_after();
                     const uint32_t a_addr = ring + (uint32_t)s * stage_bytes;
                     const uint32_t b_addr = a_addr + kABytes;
-                    const uint32_t d_g = tmem_base + (uint32_t)pb * 128u;
+                    const uint32_t atoms_addr = b_addr + b_bytes + 512;
+                    ptx::tmem_cp_32x128b_warpx4(tmem_base + kSfColA0, ptx::plain_rows16_desc(atoms_addr));
+                    if (GATED) ptx::tmem_cp_32x128b_warpx4(tmem_base + kSfColA1, ptx::plain_rows16_desc(atoms_addr + 512));
+                    ptx::tmem_cp_32x128b_warpx4(tmem_base + kSfColB, ptx::plain_rows16_desc(atoms_addr + 1024));
 #pragma unroll
                     for (int kk = 0; kk < kFp8BlockK / 32; kk++)
-                        mma_fp8_ss(d_g, ptx::sw128_kmajor_desc(a_addr + kk * 32),
-                                   ptx::sw128_kmajor_desc(b_addr + kk * 32), idesc, kk > 0 ? 1u : 0u);
+                        mma_mxf8_ss(d_g, ptx::sw128_kmajor_desc(a_addr + kk * 32), ptx::sw128_kmajor_desc(b_addr + kk * 32),
+                                    idesc, tmem_base + kSfColA0, tmem_base + kSfColB, (kb > 0 || kk > 0) ? 1u : 0u);
                     if (GATED) {
 #pragma unroll
                         for (int kk = 0; kk < kFp8BlockK / 32; kk++)
-                            mma_fp8_ss(d_g + 64u, ptx::sw128_kmajor_desc(a_addr + 128 * kFp8BlockK + kk * 32),
-                                       ptx::sw128_kmajor_desc(b_addr + kk * 32), idesc, kk > 0 ? 1u : 0u);
+                            mma_mxf8_ss(d_g + (uint32_t)kFp8TileRows,
+                                        ptx::sw128_kmajor_desc(a_addr + 128 * kFp8BlockK + kk * 32),
+                                        ptx::sw128_kmajor_desc(b_addr + kk * 32), idesc, tmem_base + kSfColA1,
+                                        tmem_base + kSfColB, (kb > 0 || kk > 0) ? 1u : 0u);
                     }
-                    issued = true;
                     ptx::mma_commit(ptx::smem_u32(&ctl->empty[s]));
-                    ptx::mma_commit(ptx::smem_u32(&ctl->tfull[pb]));
-                    if (++s == stages) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
-                    if (++pb == kFp8Bufs) {
-                        pb = 0;
-                        pph ^= 1u;
-                    }
+                }
+                __syncwarp();
+                issued = true;
+                if (++s == stages) {
+                    s = 0;
+                    ph ^= 1u;
                 }
             }
-            if (!ok && issued) {
-                ptx::mma_commit(ptx::smem_u32(&ctl->drain));
-                const uint64_t t0 = ptx::globaltimer();
-                while (!ptx::mbar_try_wait(ptx::smem_u32(&ctl->drain), 0) &&
-                       ptx::globaltimer() - t0 < kWaitTimeoutNs) {
-                }
+            if (!ok) break;
+            if (lane == 0) ptx::mma_commit(ptx::smem_u32(&ctl->tfull[acc]));
+            __syncwarp();
+            acc ^= 1;
+            if (acc == 0) aph ^= 1u;
+            t = t_next;
+        }
+        if (!ok && issued && lane == 0) {
+            // drain: every tcgen05 op issued so far completes before TMEM is freed
+            ptx::mma_commit(ptx::smem_u32(&ctl->drain));
+            const uint64_t t0 = ptx::globaltimer();
+            while (!ptx::mbar_try_wait(ptx::smem_u32(&ctl->drain), 0) && ptx::globaltimer() - t0 < kWaitTimeoutNs) {
             }
         }
     } else {
-        // ------------------------------------------------------------ epilogue: scale, accumulate, finish
-        // The activation scales (sB) come from the kernel right before this one:
-        // wait for it before the first (prefetched) read.
-        if (!waited_early) ptx::grid_dep_wait();
+        // ------------------------------------------------------------ epilogue (warps 2-5)
         const int quad = warp & 3;
-        const int row_in_tile = quad * 32 + lane;        // weight row of this thread (TMEM lane)
-        int pb = 0;
-        uint32_t pph = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const Fp8Tile tl = fp8_decode<GATED>(nb, t, args, splan);
-            const int Mrows = tl.shared ? args.M_shared : args.M;
-            const int K = tl.shared ? args.K_shared : args.K;
-            const int kbl = K / 128;                          // scale blocks along K
-            const float* sB = tl.shared ? args.sBs : args.sB;
-            const float* sA0 = tl.shared ? args.sA0s : args.sA0;
-            const float* sA1 = tl.shared ? args.sA1s : args.sA1;
-            // row of the weight-scale table for this tile's 128 weight rows
-            const int64_t srow = (int64_t)(tl.shared ? 0 : tl.group * (Mrows / 128)) + tl.m;
-            float acc_g[kFp8TileRows], acc_u[GATED ? kFp8TileRows : 1];
+        int acc = 0, tcount = 0;
+        uint32_t aph = 0, xph = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+            const Fp8Tile tl = fp8_decode(nb, t, args, splan);
+            if (tl.nkb <= 0) continue;
+            // down: the tile's gates (lane l: columns l, l + 32, l + 64, l + 96), fetched before the wait
+            float gates[4] = {1.f, 1.f, 1.f, 1.f};
+            if (!GATED && !tl.shared) {
 #pragma unroll
-            for (int c = 0; c < kFp8TileRows; c++) acc_g[c] = 0.f;
-#pragma unroll
-            for (int c = 0; c < (GATED ? kFp8TileRows : 1); c++) acc_u[c] = 0.f;
-            // scales of K block kb are fetched while K block kb - 1 is being added
-            auto scales = [&](int kb, float& a0, float& a1, float& xa, float& xb) {
-                a0 = __ldg(sA0 + srow * kbl + kb);
-                a1 = GATED ? __ldg(sA1 + srow * kbl + kb) : 0.f;
-                xa = lane < tl.rows ? __ldg(sB + (int64_t)(tl.row0 + lane) * kbl + kb) : 0.f;
-                xb = lane + 32 < tl.rows ? __ldg(sB + (int64_t)(tl.row0 + lane + 32) * kbl + kb) : 0.f;
-            };
-            float s0, s1, sxa, sxb;
-            scales(0, s0, s1, sxa, sxb);
-            for (int kb = 0; kb < tl.nkb; kb++) {
-                float n0 = 0.f, n1 = 0.f, nxa = 0.f, nxb = 0.f;
-                if (kb + 1 < tl.nkb) scales(kb + 1, n0, n1, nxa, nxb);
-                const bool good = bounded_wait(ptx::smem_u32(&ctl->tfull[pb]), pph, ctl, args.err);
-                if (!__all_sync(0xffffffffu, good)) {
-                    ok = false;
-                    break;
+                for (int i = 0; i < 4; i++) {
+                    const int col = 32 * i + lane;
+                    if (col < tl.rows) gates[i] = __ldg(args.gate_w + __ldg(args.perm + tl.row0 + col));
                 }
-                ptx::tc_fence_after();
-                const uint32_t taddr = tmem_base + (uint32_t)pb * 128u + ((uint32_t)(quad * 32) << 16);
+            }
+            if (!__all_sync(0xffffffffu, bounded_wait(ptx::smem_u32(&ctl->tfull[acc]), aph, ctl, args.err))) break;
+            ptx::tc_fence_after();
+            const uint32_t taddr = tmem_base + (uint32_t)acc * kFp8AccCols + ((uint32_t)(quad * 32) << 16);
+            const int Mrows = tl.shared ? args.M_shared : args.M;
+            const int mrow = tl.m * 128 + quad * 32 + lane;   // weight row of this thread (TMEM lane)
+            bool ok = true;
+            if (GATED) {
+                float* rb = red + (tcount & 1) * 4 * kFp8TileRows;
+                // pass 1: h = silu(g) * u, written back over g in TMEM, and per token
+                // the largest |h| over this warp's 32 f rows
+                for (int c0 = 0; c0 < tl.n_mma; c0 += 16) {
+                    uint32_t g[16], u[16];
+                    ptx::tmem_ld16(taddr + (uint32_t)c0, g);
+                    ptx::tmem_ld16(taddr + (uint32_t)kFp8TileRows + (uint32_t)c0, u);
+                    ptx::tmem_ld_wait();
+                    float a[16];
 #pragma unroll
-                for (int c0 = 0; c0 < kFp8TileRows; c0 += 16) {
-                    if (c0 < tl.n_mma) {
-                        uint32_t v[16], w[16];
-                        ptx::tmem_ld16(taddr + (uint32_t)c0, v);
-                        if (GATED) ptx::tmem_ld16(taddr + 64u + (uint32_t)c0, w);
+                    for (int j = 0; j < 16; j++) {
+                        const float h = silu_f(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+                        g[j] = __float_as_uint(h);
+                        a[j] = mrow < Mrows ? fabsf(h) : 0.f;
+                    }
+                    ptx::tmem_st16(taddr + (uint32_t)c0, g);
+                    warp_colmax16(a, lane);
+                    if ((lane & 1) == 0) rb[quad * kFp8TileRows + c0 + (lane >> 1)] = a[0];
+                }
+                ptx::tmem_st_wait();
+                // exchange among the four epilogue warps (bounded; a warp that gives up stops the others)
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&ctl->tfull[2]));
+                ok = __all_sync(0xffffffffu, bounded_wait(ptx::smem_u32(&ctl->tfull[2]), xph, ctl, args.err));
+                xph ^= 1u;
+                if (ok) {
+                    // pass 2: each token's 128 h values of this tile are one block: scale, encode, store
+                    uint8_t* out8 = tl.shared ? args.out8_shared : args.out8;
+                    float* osc = tl.shared ? args.out8_scale_shared : args.out8_scale;
+                    const int lds = tl.shared ? args.ld_scale_shared : args.ld_scale;
+                    for (int c0 = 0; c0 < tl.n_mma; c0 += 16) {
+                        uint32_t h[16];
+                        ptx::tmem_ld16(taddr + (uint32_t)c0, h);
+                        // lane j < 16: the block scale 2^e of token c0 + j
+                        const int mc = c0 + (lane & 15);
+                        const float amax = fmaxf(fmaxf(rb[mc], rb[kFp8TileRows + mc]),
+                                                 fmaxf(rb[2 * kFp8TileRows + mc], rb[3 * kFp8TileRows + mc]));
+                        const int e = fp8_scale_exp(amax);
+                        const float inv = pow2f(-e);
+                        if (quad == 0 && lane < 16 && mc < tl.rows) osc[(int64_t)tl.m * lds + tl.row0 + mc] = pow2f(e);
                         ptx::tmem_ld_wait();
 #pragma unroll
                         for (int j = 0; j < 16; j++) {
-                            const int c = c0 + j;
-                            const float sx = __shfl_sync(0xffffffffu, c < 32 ? sxa : sxb, c & 31);
-                            acc_g[c] = fmaf(__uint_as_float(v[j]), s0 * sx, acc_g[c]);
-                            if (GATED) acc_u[c] = fmaf(__uint_as_float(w[j]), s1 * sx, acc_u[c]);
+                            const float m = __shfl_sync(0xffffffffu, inv, j);
+                            const int col = c0 + j;
+                            if (col < tl.rows && mrow < Mrows)
+                                out8[(int64_t)(tl.row0 + col) * Mrows + mrow] = e4m3_of(__uint_as_float(h[j]) * m);
                         }
                     }
                 }
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&ctl->tempty[pb]));
-                if (++pb == kFp8Bufs) {
-                    pb = 0;
-                    pph ^= 1u;
-                }
-                s0 = n0;
-                s1 = n1;
-                sxa = nxa;
-                sxb = nxb;
-            }
-            if (!ok) break;
-            if (GATED) {
-                // h = silu(g) * u, then requantise each token's 128 h values of this tile
-#pragma unroll
-                for (int c = 0; c < kFp8TileRows; c++) {
-                    if (c < tl.rows) {   // warp-uniform
-                        const float g = acc_g[c];
-                        acc_g[c] = g / (1.0f + __expf(-g)) * acc_u[c];
-                        float a = tl.m * 128 + row_in_tile < Mrows ? fabsf(acc_g[c]) : 0.f;
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-                        if (lane == 0) red[quad * kFp8TileRows + c] = a;
-                    }
-                }
-                named_bar_epilogue();
-                uint8_t* out8 = tl.shared ? args.out8_shared : args.out8;
-                float* osc = tl.shared ? args.out8_scale_shared : args.out8_scale;
-                const int frow = tl.m * 128 + row_in_tile;
-#pragma unroll
-                for (int c = 0; c < kFp8TileRows; c++) {
-                    if (c < tl.rows) {
-                        const float amax = fmaxf(fmaxf(red[c], red[kFp8TileRows + c]),
-                                                 fmaxf(red[2 * kFp8TileRows + c], red[3 * kFp8TileRows + c]));
-                        const int e = fp8_scale_exp(amax);
-                        const int64_t r = tl.row0 + c;
-                        if (frow < Mrows) out8[r * Mrows + frow] = e4m3_of(ldexpf(acc_g[c], -e));
-                        if (row_in_tile == 0) osc[r * (Mrows / 128) + tl.m] = ldexpf(1.f, e);
-                    }
-                }
-                named_bar_epilogue();   // red[] is reused by the next tile
             } else {
                 bf16* out = tl.shared ? args.out_shared : args.out;
-                const int drow = tl.m * 128 + row_in_tile;
-                const float gsa = (!tl.shared && lane < tl.rows) ? __ldg(args.gate_w + __ldg(args.perm + tl.row0 + lane)) : 1.f;
-                const float gsb = (!tl.shared && lane + 32 < tl.rows)
-                                      ? __ldg(args.gate_w + __ldg(args.perm + tl.row0 + lane + 32))
-                                      : 1.f;
+                for (int c0 = 0; c0 < tl.n_mma; c0 += 16) {
+                    uint32_t v[16];
+                    ptx::tmem_ld16(taddr + (uint32_t)c0, v);
+                    ptx::tmem_ld_wait();
+                    const float mine = pick4f(gates, c0 >> 5);
 #pragma unroll
-                for (int c = 0; c < kFp8TileRows; c++) {
-                    if (c >= tl.rows) continue;   // warp-uniform
-                    const float gate = __shfl_sync(0xffffffffu, c < 32 ? gsa : gsb, c & 31);
-                    if (drow < Mrows)
-                        out[(int64_t)(tl.row0 + c) * Mrows + drow] = __float2bfloat16_rn(acc_g[c] * gate);
+                    for (int j = 0; j < 16; j++) {
+                        const float gate = __shfl_sync(0xffffffffu, mine, (c0 & 31) + j);
+                        const int col = c0 + j;
+                        if (col < tl.rows && mrow < Mrows)
+                            out[(int64_t)(tl.row0 + col) * Mrows + mrow] = __float2bfloat16_rn(__uint_as_float(v[j]) * gate);
+                    }
                 }
             }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&ctl->tempty[acc]));
+            if (!ok) break;
+            acc ^= 1;
+            if (acc == 0) aph ^= 1u;
+            ++tcount;
         }
     }
 
@@ -575,7 +714,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
 }
 
-constexpr int kFp8SmemBytes = kGemmSmemBytes + 4 * kFp8TileRows * 4;
+constexpr int kFp8SmemBytes = 1024 + kFp8RingBytes + kBarBytes + (int)sizeof(SmemPlan) + 2 * 4 * kFp8TileRows * 4;
 static_assert(kFp8SmemBytes <= 227 * 1024, "shared memory budget (fp8)");
 
 }  // namespace moe

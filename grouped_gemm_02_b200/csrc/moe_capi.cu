@@ -156,6 +156,20 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D fp32 tensor map over a row-major [rows, inner] matrix; box = [128, 1], no swizzle.
+bool make_map_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows)
+{
+    if (rows == 0) rows = 1;
+    if (inner == 0) inner = 4;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 4};
+    cuuint32_t box[2] = {128, 1};
+    cuuint32_t estr[2] = {1, 1};
+    return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <class T>
 T* at(void* ws, size_t off)
 {
@@ -626,39 +640,43 @@ const char* moe_status_string(int status)
 // ---------------------------------------------------------------- FP8 block-scaled layer
 namespace {
 
-int run_quantize_rows(const bf16* x, int64_t R, int C, uint8_t* q, float* sc, cudaStream_t st)
+int run_quantize_rows(const bf16* x, int64_t R, int C, uint8_t* q, float* sc, cudaStream_t st,
+                      float* sc_t = nullptr, int64_t ld_t = 0)
 {
     const int64_t warps = R * (C / 128);
     return status_of(launch(quantize_rows_fp8_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, st, x, R, C, q,
-                            sc));
+                            sc, sc_t, ld_t));
 }
 
 struct Fp8Operands {
     const uint8_t *xp8, *x8, *W1q, *W3q, *W2q, *Ws1q, *Ws3q, *Ws2q;
-    const float *sxp, *sx, *s1, *s3, *s2, *ss1, *ss3, *ss2;
+    const float *sxp, *sxT, *s1, *s3, *s2, *ss1, *ss3, *ss2;   // sxp / sxT K-block-major
     const int32_t* perm;
     const float* gate_w;
     uint8_t *h8, *hs8;
-    float *sh, *shs;
+    float *sh, *shs;                                           // K-block-major
     bf16 *y_p, *ys;
     int T, P, d, f, fs, E;
+    int64_t ld_pairs, ld_tokens;
 };
 
 int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int sms, cudaStream_t st, bool prof)
 {
-    CUtensorMap a0, a1, b, a0s, a1s, bs;
+    CUtensorMap a0, a1, b, a0s, a1s, bs, sb, sbs;
     const uint64_t E = (uint64_t)o.E;
+    const uint64_t lp = (uint64_t)o.ld_pairs, lt = (uint64_t)o.ld_tokens;
     if (!make_map_u8(&a0, o.W1q, o.d, E * o.f, 128) || !make_map_u8(&a1, o.W3q, o.d, E * o.f, 128) ||
-        !make_map_u8(&b, o.xp8, o.d, (uint64_t)o.P, 16))
+        !make_map_u8(&b, o.xp8, o.d, (uint64_t)o.P, 16) || !make_map_f32(&sb, o.sxp, lp, o.d / 128))
         return MOE_ERR_CUDA;
     if (o.fs > 0) {
         if (!make_map_u8(&a0s, o.Ws1q, o.d, o.fs, 128) || !make_map_u8(&a1s, o.Ws3q, o.d, o.fs, 128) ||
-            !make_map_u8(&bs, o.x8, o.d, (uint64_t)o.T, 16))
+            !make_map_u8(&bs, o.x8, o.d, (uint64_t)o.T, 16) || !make_map_f32(&sbs, o.sxT, lt, o.d / 128))
             return MOE_ERR_CUDA;
     } else {
         a0s = a0;
         a1s = a1;
         bs = b;
+        sbs = sb;
     }
     Fp8Args g1{};
     g1.plan = plan;
@@ -672,30 +690,33 @@ int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int 
     g1.sA1 = o.s3;
     g1.sA0s = o.ss1;
     g1.sA1s = o.ss3;
-    g1.sB = o.sxp;
-    g1.sBs = o.sx;
     g1.out8 = o.h8;
     g1.out8_scale = o.sh;
+    g1.ld_scale = (int)o.ld_pairs;
     g1.out8_shared = o.hs8;
     g1.out8_scale_shared = o.shs;
+    g1.ld_scale_shared = (int)o.ld_tokens;
     g1.perm = o.perm;
     g1.gate_w = o.gate_w;
     g1.err = err;
     if (launch(grouped_gemm_fp8_kernel<true>, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a0, a1, b, a0s, a1s,
-               bs, g1) != cudaSuccess)
+               bs, sb, sbs, g1) != cudaSuccess)
         return MOE_ERR_CUDA;
     phase_mark(prof, 3, st);
-    if (!make_map_u8(&a0, o.W2q, o.f, E * o.d, 128) || !make_map_u8(&b, o.h8, o.f, (uint64_t)o.P, 16))
+    if (!make_map_u8(&a0, o.W2q, o.f, E * o.d, 128) || !make_map_u8(&b, o.h8, o.f, (uint64_t)o.P, 16) ||
+        !make_map_f32(&sb, o.sh, lp, o.f / 128))
         return MOE_ERR_CUDA;
     a1 = a0;
     if (o.fs > 0) {
-        if (!make_map_u8(&a0s, o.Ws2q, o.fs, o.d, 128) || !make_map_u8(&bs, o.hs8, o.fs, (uint64_t)o.T, 16))
+        if (!make_map_u8(&a0s, o.Ws2q, o.fs, o.d, 128) || !make_map_u8(&bs, o.hs8, o.fs, (uint64_t)o.T, 16) ||
+            !make_map_f32(&sbs, o.shs, lt, o.fs / 128))
             return MOE_ERR_CUDA;
         a1s = a0s;
     } else {
         a0s = a0;
         a1s = a0;
         bs = b;
+        sbs = sb;
     }
     Fp8Args g2 = g1;
     g2.M = o.d;
@@ -706,12 +727,10 @@ int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int 
     g2.sA1 = nullptr;
     g2.sA0s = o.ss2;
     g2.sA1s = nullptr;
-    g2.sB = o.sh;
-    g2.sBs = o.shs;
     g2.out = o.y_p;
     g2.out_shared = o.ys;
     return status_of(launch(grouped_gemm_fp8_kernel<false>, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a0, a1,
-                            b, a0s, a1s, bs, g2));
+                            b, a0s, a1s, bs, sb, sbs, g2));
 }
 
 }  // namespace
@@ -761,9 +780,9 @@ int moe_workspace_tensor_fp8(void* ws, int64_t T, int64_t d, int64_t f, int64_t 
     if (!ws || !ptr || T < 0 || d < 0 || f < 0 || E < 1 || E > kMaxExperts || k < 1 || k > kMaxTopK || f_shared < 0)
         return MOE_ERR_ARG;
     const WsLayoutFp8 L = ws_layout_fp8(T, d, f, E, k, f_shared);
-    const size_t offs[17] = {L.logits, L.topk_idx, L.topk_w, L.counts, L.offsets, L.perm, L.inv_perm, L.x8, L.sx,
-                             L.xp8, L.sxp, L.h8, L.sh, L.y_p, L.hs8, L.shs, L.ys};
-    if (which < 0 || which >= 17) return MOE_ERR_ARG;
+    const size_t offs[18] = {L.logits, L.topk_idx, L.topk_w, L.counts, L.offsets, L.perm, L.inv_perm, L.x8, L.sx,
+                             L.xp8, L.sxp, L.h8, L.sh, L.y_p, L.hs8, L.shs, L.ys, L.sxT};
+    if (which < 0 || which >= 18) return MOE_ERR_ARG;
     *ptr = static_cast<uint8_t*>(ws) + offs[which];
     return MOE_OK;
 }
@@ -778,6 +797,7 @@ int moe_layer_forward_fp8(const moe_bf16* x, const moe_bf16* Wg, const float* bi
     if (rc) return rc;
     if (f <= 0 || f_shared < 0) return MOE_ERR_ARG;
     if (d % 128 != 0 || f % 128 != 0 || f_shared % 128 != 0) return MOE_ERR_ALIGN;
+    if (d > kFp8MaxK || f > kFp8MaxK || f_shared > kFp8MaxK) return MOE_ERR_ARG;
     if (T == 0) return MOE_OK;
     if (!x || !Wg || !W1q || !W1s || !W3q || !W3s || !W2q || !W2s || !out || !ws) return MOE_ERR_ARG;
     if (f_shared > 0 && (!Ws1q || !Ws1s || !Ws3q || !Ws3s || !Ws2q || !Ws2s)) return MOE_ERR_ARG;
@@ -815,7 +835,8 @@ int moe_layer_forward_fp8(const moe_bf16* x, const moe_bf16* Wg, const float* bi
     if ((rc = run_router_gemm(xb, reinterpret_cast<const bf16*>(Wg), bias, iT, id, iE, logits, partials, err,
                               dev->sm_count, st, &rs)))
         return rc;
-    if ((rc = run_quantize_rows(xb, T, id, x8, sx, st))) return rc;
+    float* sxT = f_shared > 0 ? at<float>(ws, L.sxT) : nullptr;   // the shared expert's token scales
+    if ((rc = run_quantize_rows(xb, T, id, x8, sx, st, sxT, L.ld_tokens))) return rc;
     if ((rc = run_topk(topk_source(rs, logits, partials, bias, iT, iE), iT, iE, ik, idx, w, err, st))) return rc;
     phase_mark(prof, 1, st);
     if (P <= kSmallPairs) {
@@ -830,13 +851,15 @@ int moe_layer_forward_fp8(const moe_bf16* x, const moe_bf16* Wg, const float* bi
     }
     const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)dev->sm_count * 16));
     if (launch(gather_rows_fp8_kernel, dim3(blocks), dim3(256), 0, st, (const uint8_t*)x8, (const float*)sx,
-               (const int32_t*)perm, (const int32_t*)offsets, iE, ik, id, xp8, sxp) != cudaSuccess)
+               (const int32_t*)perm, (const int32_t*)offsets, iE, ik, id, xp8, sxp, L.ld_pairs) != cudaSuccess)
         return MOE_ERR_CUDA;
     Fp8Operands o{};
     o.xp8 = xp8;
     o.x8 = x8;
     o.sxp = sxp;
-    o.sx = sx;
+    o.sxT = sxT;
+    o.ld_pairs = L.ld_pairs;
+    o.ld_tokens = L.ld_tokens;
     o.W1q = W1q;
     o.W3q = W3q;
     o.W2q = W2q;

@@ -324,18 +324,19 @@ def moe_layer_forward_fp8(x, Wg, bias, Q: dict, k: int, ws: torch.Tensor, out=No
 
 
 WS_TENSORS_FP8 = ("logits", "topk_idx", "topk_w", "counts", "offsets", "perm", "inv_perm", "x8", "sx", "xp8", "sxp",
-                  "h8", "sh", "y_p", "hs8", "shs", "ys")
+                  "h8", "sh", "y_p", "hs8", "shs", "ys", "sxT")
 
 
 def workspace_views_fp8(ws: torch.Tensor, T: int, d: int, f: int, E: int, k: int, f_shared: int = 0):
     P, Ts = T * k, (T if f_shared else 0)
+    P4, T4 = (P + 3) // 4 * 4, (T + 3) // 4 * 4     # K-block-major scale rows are padded to 4 entries
     shapes = {"logits": ((T, E), torch.float32), "topk_idx": ((T, k), torch.int32), "topk_w": ((T, k), torch.float32),
               "counts": ((E,), torch.int32), "offsets": ((E + 1,), torch.int32), "perm": ((P,), torch.int32),
               "inv_perm": ((P,), torch.int32), "x8": ((T, d), torch.uint8), "sx": ((T, d // 128), torch.float32),
-              "xp8": ((P, d), torch.uint8), "sxp": ((P, d // 128), torch.float32), "h8": ((P, f), torch.uint8),
-              "sh": ((P, f // 128), torch.float32), "y_p": ((P, d), torch.bfloat16),
-              "hs8": ((Ts, f_shared), torch.uint8), "shs": ((Ts, max(f_shared, 128) // 128 if Ts else 0), torch.float32),
-              "ys": ((Ts, d), torch.bfloat16)}
+              "xp8": ((P, d), torch.uint8), "sxp": ((d // 128, P4), torch.float32), "h8": ((P, f), torch.uint8),
+              "sh": ((f // 128, P4), torch.float32), "y_p": ((P, d), torch.bfloat16),
+              "hs8": ((Ts, f_shared), torch.uint8), "shs": ((f_shared // 128, T4 if Ts else 0), torch.float32),
+              "ys": ((Ts, d), torch.bfloat16), "sxT": ((d // 128, T4 if Ts else 0), torch.float32)}
     base = ws.data_ptr()
     views = {}
     for i, name in enumerate(WS_TENSORS_FP8):

@@ -171,9 +171,11 @@ MOE_API int moe_layer_forward(const moe_bf16 *x, const moe_bf16 *Wg, const float
  * block-scaled MMA and requantisation; e4m3 with 1 x 128 activation blocks and
  * 128 x 128 weight blocks).  Codes are OCP e4m3 (round to nearest, ties to
  * even, saturating at +-448).  A block's scale is the smallest power of two s
- * with max|v| / s <= 448 (s = 1 for an all-zero block), stored as fp32, so
+ * with max|v| / s <= 448 (s = 1 for an all-zero block), held to the UE8M0
+ * range 2^-127 .. 2^127 that the block-scaled MMA takes, stored as fp32, so
  * code q with scale s stands for e4m3(q) * s exactly.  d, f and f_shared must
- * be multiples of 128 (MOE_ERR_ALIGN otherwise). */
+ * be multiples of 128 (MOE_ERR_ALIGN otherwise) and at most 16384
+ * (MOE_ERR_ARG otherwise). */
 
 /* 1 x 128 blocks along each row: x [rows, cols] bf16 -> q [rows, cols] e4m3,
  * scales [rows, cols/128] fp32.  cols % 128 == 0. */
@@ -194,7 +196,10 @@ MOE_API int moe_workspace_size_fp8(int64_t T, int64_t d, int64_t f, int64_t E, i
 /* Device pointers of the FP8 layer intermediates inside its workspace
  * (which: 0 logits, 1 topk_idx, 2 topk_w, 3 counts, 4 offsets, 5 perm,
  * 6 inv_perm, 7 x8, 8 sx, 9 xp8, 10 sxp, 11 h8, 12 sh, 13 y_p, 14 hs8, 15 shs,
- * 16 ys).  Host-only arithmetic. */
+ * 16 ys, 17 sxT).  sx is [T, d/128]; the scale arrays the GEMMs read are
+ * K-block-major with rows padded to a multiple of 4 entries: sxp
+ * [d/128, P4], sh [f/128, P4], shs [f_shared/128, T4], sxT [d/128, T4]
+ * (P4 = T*k and T4 = T rounded up to a multiple of 4).  Host-only arithmetic. */
 MOE_API int moe_workspace_tensor_fp8(void *ws, int64_t T, int64_t d, int64_t f, int64_t E, int64_t k,
                                      int64_t f_shared, int which, void **ptr);
 
@@ -206,9 +211,9 @@ MOE_API int moe_workspace_tensor_fp8(void *ws, int64_t T, int64_t d, int64_t f, 
  * [d,f_shared] with their scales, or all NULL and f_shared = 0):
  *   h   = silu(x^ W1^T) * (x^ W3^T), requantised in 1 x 128 blocks along f
  *   y_p = gate * (h^ W2^T)          (bf16), then the combine of moe_combine,
- * where ^ marks dequantised values; all products accumulate in fp32 (one
- * 128-wide K block per tensor-core pass, scaled in fp32).  Every intermediate
- * lives in `ws` (moe_workspace_size_fp8 bytes). */
+ * where ^ marks dequantised values; all products accumulate in fp32 (the
+ * tensor cores apply the power-of-two block scales as UE8M0 exponents inside
+ * the MMA).  Every intermediate lives in `ws` (moe_workspace_size_fp8 bytes). */
 MOE_API int moe_layer_forward_fp8(const moe_bf16 *x, const moe_bf16 *Wg, const float *bias, const uint8_t *W1q,
                                   const float *W1s, const uint8_t *W3q, const float *W3s, const uint8_t *W2q,
                                   const float *W2s, const uint8_t *Ws1q, const float *Ws1s, const uint8_t *Ws3q,
