@@ -214,6 +214,24 @@ __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, Smem
     }
 }
 
+// Spin until the global counter reaches `need` (acquire), with the same
+// deadline; on timeout or another role's abort, flag the CTA and return false.
+__device__ __forceinline__ bool bounded_count_wait(const int* cnt, int need, SmemCtl* ctl, uint32_t* err)
+{
+    if (ptx::ld_acquire_gpu(cnt) >= need) return true;
+    const uint64_t t0 = ptx::globaltimer();
+    while (ptx::ld_acquire_gpu(cnt) < need) {
+        if (*reinterpret_cast<volatile int*>(&ctl->abort)) return false;
+        if (ptx::globaltimer() - t0 > kWaitTimeoutNs) {
+            *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
+            atomicOr(err, DEVERR_TIMEOUT);
+            return false;
+        }
+        __nanosleep(64);
+    }
+    return true;
+}
+
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
 // Walks this CTA's (tile, k-block) sequence in order; shared by the two
@@ -371,18 +389,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int32_t* dep = plan_arrays(const_cast<int32_t*>(args.plan)).dep + tl.blk;
                 const int m1 = tl.shared ? args.M_shared : args.M;
                 const int need = 4 * splan->units[tl.blk] * ((m1 + 63) / 64);   // 4 epilogue warps per tile
-                if (ptx::ld_acquire_gpu(dep) < need) {
-                    const uint64_t t0 = ptx::globaltimer();
-                    while (ptx::ld_acquire_gpu(dep) < need) {
-                        if (*reinterpret_cast<volatile int*>(&ctl->abort)) return false;
-                        if (ptx::globaltimer() - t0 > kWaitTimeoutNs) {
-                            *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
-                            atomicOr(args.err, DEVERR_TIMEOUT);
-                            return false;
-                        }
-                        __nanosleep(64);
-                    }
-                }
+                if (!bounded_count_wait(dep, need, ctl, args.err)) return false;
                 ptx::fence_proxy_async_global();   // the TMA reads below come after the acquire
                 return true;
             };
@@ -511,6 +518,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
             const Tile tl = decode_tile<MODE>(nb, t, args, args2, splan);
             if (tl.kb0 >= tl.kb1) continue;
+            // a down tile's gates (lane l: columns l + 32 i), fetched before the accumulator wait
+            float gates[8];
+#pragma unroll
+            for (int i = 0; i < 8; i++) gates[i] = 1.f;
+            if (MODE != MODE_ROUTER && !tl.gated && !tl.shared) {
+                const GemmArgs& ga = MODE == MODE_FUSED ? args2 : args;
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    const int col = 32 * i + lane;
+                    if (col < tl.rows) gates[i] = __ldg(ga.gate_w + __ldg(ga.perm + tl.row0 + col));
+                }
+            }
             const bool ok = bounded_wait(ptx::smem_u32(&ctl->tfull[acc]), aph, ctl, args.err);
             if (!__all_sync(0xffffffffu, ok)) break;   // the whole warp leaves together
             ptx::tc_fence_after();
@@ -539,13 +558,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 } else if (MODE != MODE_ROUTER) {
                     const int drow = tl.m * 128 + quad * 32 + lane;
-                    const int my_col = c0 + (lane & 15);
-                    float my_scale = 1.0f;
-                    if (!tl.shared && my_col < tl.rows)
-                        my_scale = __ldg(ea.gate_w + __ldg(ea.perm + tl.row0 + my_col));
+                    const int gi = c0 >> 5;
+                    const float mine = gi == 0 ? gates[0] : gi == 1 ? gates[1] : gi == 2 ? gates[2] : gi == 3 ? gates[3]
+                                     : gi == 4 ? gates[4] : gi == 5 ? gates[5] : gi == 6 ? gates[6] : gates[7];
 #pragma unroll
                     for (int j = 0; j < 16; j++) {
-                        const float sc = __shfl_sync(0xffffffffu, my_scale, j);
+                        const float sc = __shfl_sync(0xffffffffu, mine, (c0 & 31) + j);
                         const int col = c0 + j;
                         if (col < tl.rows && drow < Mrows)
                             out[(size_t)(tl.row0 + col) * ld + drow] =
@@ -587,6 +605,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem_base, kTmemCols);
     }
+}
+
+// Diagnostic: one CTA waits, through the two bounded waits the GEMMs use, on
+// an mbarrier nobody arrives on and on a counter nobody increments.  Each
+// wait gives up after its deadline and sets DEVERR_TIMEOUT; the kernel then
+// returns normally, so the context stays usable.
+__global__ void __launch_bounds__(32) wait_timeout_probe_kernel(const int* never, uint32_t* err)
+{
+    __shared__ SmemCtl ctl;
+    if (threadIdx.x != 0) return;
+    ctl.abort = 0;
+    ptx::mbar_init(ptx::smem_u32(&ctl.full[0]), 1);
+    ptx::fence_mbar_init();
+    const bool a = bounded_wait(ptx::smem_u32(&ctl.full[0]), 0u, &ctl, err);
+    ctl.abort = 0;
+    const bool b = bounded_count_wait(never, 1, &ctl, err);
+    if (a || b) atomicOr(err, DEVERR_PLAN);   // a wait that should not have ended did
 }
 
 }  // namespace moe

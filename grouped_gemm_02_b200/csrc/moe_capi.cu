@@ -616,6 +616,21 @@ int moe_get_device_error(const void* ws, uint32_t* code, void* stream)
     return cudaStreamSynchronize(st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+int moe_selftest_wait_timeout(void* ws, void* stream)
+{
+    if (!ws || !al16(ws)) return MOE_ERR_ARG;
+    DeviceState* dev;
+    int rc;
+    if ((rc = device_setup(&dev))) return rc;
+    cudaStream_t st = as_stream(stream);
+    // the workspace's error word is followed by the plan; the probe's counter is the
+    // error word's neighbour, zeroed here and never incremented
+    int* never = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + sizeof(uint32_t));
+    if (cudaMemsetAsync(never, 0, sizeof(int), st) != cudaSuccess) return MOE_ERR_CUDA;
+    return status_of(launch(wait_timeout_probe_kernel, dim3(1), dim3(32), 0, st, (const int*)never,
+                            static_cast<uint32_t*>(ws)));
+}
+
 int moe_clear_device_error(void* ws, void* stream)
 {
     if (!ws) return MOE_ERR_ARG;

@@ -20,13 +20,14 @@ from . import build as _build
 MOE_OK = 0
 STATUS = {0: "ok", -1: "invalid argument", -2: "size or pointer alignment", -3: "workspace too small",
           -4: "CUDA launch or runtime error", -5: "device is not sm_100 (B200)"}
-DEVERR_EXPERT_RANGE, DEVERR_TIMEOUT, DEVERR_NAN_LOGIT = 1, 2, 4
+DEVERR_EXPERT_RANGE, DEVERR_TIMEOUT, DEVERR_NAN_LOGIT, DEVERR_PLAN = 1, 2, 4, 8
 
 _lib: Optional[C.CDLL] = None
 
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_topk", "moe_permute",
            "moe_permute_noalloc", "moe_grouped_gemm", "moe_combine", "moe_layer_forward", "moe_workspace_tensor",
            "moe_record_phase_events", "moe_launch_counter", "moe_get_device_error", "moe_clear_device_error",
+           "moe_selftest_wait_timeout",
            "moe_status_string", "moe_quantize_fp8_rows", "moe_quantize_fp8_blocks", "moe_workspace_size_fp8",
            "moe_workspace_tensor_fp8", "moe_layer_forward_fp8")
 
@@ -62,6 +63,7 @@ def lib() -> C.CDLL:
             "moe_workspace_tensor": [vp, i64, i64, i64, i64, i64, i64, C.c_int, C.POINTER(vp)],
             "moe_get_device_error": [vp, C.POINTER(C.c_uint32), vp],
             "moe_clear_device_error": [vp, vp],
+            "moe_selftest_wait_timeout": [vp, vp],
             "moe_status_string": [C.c_int],
             "moe_record_phase_events": [C.POINTER(vp), C.c_int],
             "moe_launch_counter": [],
@@ -139,6 +141,11 @@ def moe_get_device_error(ws: torch.Tensor, stream=None) -> int:
 
 def moe_clear_device_error(ws: torch.Tensor, stream=None) -> None:
     _call("moe_clear_device_error", _p(ws), _stream(stream))
+
+
+def moe_selftest_wait_timeout(ws: torch.Tensor, stream=None) -> None:
+    """Run the bounded-wait diagnostic (about 2 s); read the result with moe_get_device_error."""
+    _call("moe_selftest_wait_timeout", _p(ws), _stream(stream))
 
 
 def moe_record_phase_events(events) -> None:

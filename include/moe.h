@@ -244,6 +244,16 @@ MOE_API int moe_get_device_error(const void *ws, uint32_t *code, void *stream);
 /* Clears the sticky device error word; enqueued on `stream`. */
 MOE_API int moe_clear_device_error(void *ws, void *stream);
 
+/* Diagnostic of the failure path (the pages have no counterpart): one CTA
+ * runs the two bounded waits the GEMM kernels use -- on an mbarrier nobody
+ * arrives on, then on a counter nobody increments (the int after the error
+ * word in `ws`, zeroed by this call) -- and each gives up after its 1 s
+ * deadline.  Afterwards the error word holds MOE_DEVERR_TIMEOUT (and
+ * MOE_DEVERR_PLAN only if a wait ended that should not have) and the CUDA
+ * context is still usable.  Takes about 2 s of GPU time; `ws` is any layer
+ * workspace. */
+MOE_API int moe_selftest_wait_timeout(void *ws, void *stream);
+
 /* Human-readable name of a status code. */
 MOE_API const char *moe_status_string(int status);
 
