@@ -90,6 +90,9 @@ struct GemmArgs {
     // MODE_ROUTER: tokens split into `units` chunks of `chunk` rows, `mt` tiles of
     // 128 experts, K split into `splits` ranges of `kb_per` 64-wide blocks.
     int T, units, chunk, mt, splits, kb_per;
+    // MODE_FUSED: down tiles an SM with one gate/up tile fewer takes first (the
+    // ratio of gate/up to down k-blocks per tile, rounded; see cta_tile)
+    int comp;
     float* out_f32;             // splits == 1: logits [T, E] (+ bias); else partials [splits, T, E]
     const float* bias;          // may be null
     uint32_t* err;
@@ -234,27 +237,66 @@ __device__ __forceinline__ bool bounded_count_wait(const int* cnt, int need, Sme
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
+// The i-th tile of this CTA, or -1.  Every mode but MODE_FUSED deals tiles
+// round-robin.  MODE_FUSED deals its G gate/up tiles round-robin; when G is
+// not a multiple of the grid, the SMs left one gate/up tile short first take
+// `comp` down tiles each (one gate/up tile weighs about `comp` down tiles), and
+// the remaining down tiles are dealt round-robin.  The compensating tiles are
+// the first down tiles, whose blocks' gate/up tiles ran in the first round.
+template <int MODE>
+__device__ __forceinline__ int cta_tile(int i, int total, int G, int comp)
+{
+    const int b = blockIdx.x, grid = gridDim.x;
+    if (MODE != MODE_FUSED) {
+        const int t = b + grid * i;
+        return t < total ? t : -1;
+    }
+    const int D = total - G;
+    const int grem = G % grid;
+    const int gb = G / grid + (b < grem ? 1 : 0);
+    if (i < gb) return b + grid * i;
+    int j = i - gb;
+    int comp_total = 0, my_comp = 0, comp0 = 0;
+    if (grem > 0) {
+        comp_total = min(D, (grid - grem) * comp);
+        if (b >= grem) {
+            comp0 = (b - grem) * comp;
+            my_comp = max(0, min(comp, comp_total - comp0));
+        }
+    }
+    if (j < my_comp) return G + comp0 + j;
+    j -= my_comp;
+    const int dj = comp_total + b + grid * j;
+    return dj < D ? G + dj : -1;
+}
+
 // Walks this CTA's (tile, k-block) sequence in order; shared by the two
 // passes of the producer.
 struct KIter {
-    int t, kb;
+    int i, t, kb;
     Tile tl;
 };
 
 template <int MODE>
-__device__ __forceinline__ bool kiter_begin(KIter& it, int nb, int total, const GemmArgs& a, const GemmArgs& a2,
-                                            const SmemPlan* sp)
+__device__ __forceinline__ bool kiter_seek(KIter& it, int nb, int total, const GemmArgs& a, const GemmArgs& a2,
+                                           const SmemPlan* sp)
 {
-    it.t = blockIdx.x;
-    while (it.t < total) {
+    for (; (it.t = cta_tile<MODE>(it.i, total, sp->tiles1, a.comp)) >= 0; it.i++) {
         it.tl = decode_tile<MODE>(nb, it.t, a, a2, sp);
         if (it.tl.kb0 < it.tl.kb1) {
             it.kb = it.tl.kb0;
             return true;
         }
-        it.t += gridDim.x;
     }
     return false;
+}
+
+template <int MODE>
+__device__ __forceinline__ bool kiter_begin(KIter& it, int nb, int total, const GemmArgs& a, const GemmArgs& a2,
+                                            const SmemPlan* sp)
+{
+    it.i = 0;
+    return kiter_seek<MODE>(it, nb, total, a, a2, sp);
 }
 
 template <int MODE>
@@ -262,14 +304,8 @@ __device__ __forceinline__ bool kiter_next(KIter& it, int nb, int total, const G
                                            const SmemPlan* sp)
 {
     if (++it.kb < it.tl.kb1) return true;
-    for (it.t += gridDim.x; it.t < total; it.t += gridDim.x) {
-        it.tl = decode_tile<MODE>(nb, it.t, a, a2, sp);
-        if (it.tl.kb0 < it.tl.kb1) {
-            it.kb = it.tl.kb0;
-            return true;
-        }
-    }
-    return false;
+    ++it.i;
+    return kiter_seek<MODE>(it, nb, total, a, a2, sp);
 }
 
 template <int MODE>
@@ -465,7 +501,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int acc = 0;
             uint32_t aph = 0;
             bool ok = true, issued = false;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (int i = 0, t; ok && (t = cta_tile<MODE>(i, total, splan->tiles1, args.comp)) >= 0; i++) {
                 const Tile tl = decode_tile<MODE>(nb, t, args, args2, splan);
                 if (tl.kb0 >= tl.kb1) continue;
                 if (!bounded_wait(ptx::smem_u32(&ctl->tempty[acc]), aph ^ 1u, ctl, args.err)) {
@@ -515,7 +551,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int quad = warp & 3;            // TMEM lane quadrant this warp may access
         int acc = 0;
         uint32_t aph = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        for (int i = 0, t; (t = cta_tile<MODE>(i, total, splan->tiles1, args.comp)) >= 0; i++) {
             const Tile tl = decode_tile<MODE>(nb, t, args, args2, splan);
             if (tl.kb0 >= tl.kb1) continue;
             // a down tile's gates (lane l: columns l + 32 i), fetched before the accumulator wait

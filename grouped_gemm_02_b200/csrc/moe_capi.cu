@@ -332,6 +332,9 @@ int run_gemms(const GemmOperands& o, const int32_t* plan, bool plan_ready, uint3
     g2.out_shared = o.ys;
     g2.ld_out_shared = o.d;
     if (gemm_fused(o.P, o.f)) {
+        // a gate/up tile streams d/64 k-blocks, a down tile f/64
+        const int kb1 = (o.d + 63) / 64, kb2 = (o.f + 63) / 64;
+        g1.comp = std::max(1, (kb1 + kb2 / 2) / kb2);
         const cudaError_t e = launch(grouped_gemm_kernel<MODE_FUSED>, dim3(sms), dim3(kGemmThreads), kGemmSmemBytes,
                                      st, a0, a1, b, a0s, a1s, bs, a2, b2, a2s, b2s, g1, g2);
         phase_mark(prof, 3, st);   // the fused launch has no boundary: the down phase reads as zero
