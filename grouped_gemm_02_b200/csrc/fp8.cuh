@@ -230,16 +230,35 @@ struct Fp8Args {
     const int32_t* perm;
     const float* gate_w;
     uint32_t* err;
+    int comp;                       // FP8_FUSED: down tiles per gate/up tile, for the balanced order (cta_tile)
 };
+
+// What one launch of the FP8 GEMM runs: the down tiles, the gate/up tiles, or
+// both (gate/up tiles first; a block's down tiles wait for its h, as in the
+// bf16 MODE_FUSED launch).
+constexpr int FP8_DOWN = 0;
+constexpr int FP8_GATED = 1;
+constexpr int FP8_FUSED = 2;
 
 struct Fp8Tile {
-    int group, m, row0, rows, n_mma, nkb;
-    bool shared;
+    int group, m, row0, rows, n_mma, nkb, blk;
+    bool shared, gated;
 };
 
-__device__ __forceinline__ Fp8Tile fp8_decode(int nb, int t, const Fp8Args& a, const SmemPlan* sp)
+// Tile t of the launch; in FP8_FUSED the first tiles1 are gate/up tiles
+// (prefix sp->tb, args a) and the rest down tiles (prefix sp->tb2, args a2).
+template <int KIND>
+__device__ __forceinline__ Fp8Tile fp8_decode(int nb, int t, const Fp8Args& a, const Fp8Args& a2, const SmemPlan* sp)
 {
+    bool gated = KIND == FP8_GATED;
     const int* tb = sp->tb;
+    if (KIND == FP8_FUSED) {
+        gated = t < sp->tiles1;
+        if (!gated) {
+            t -= sp->tiles1;
+            tb = sp->tb2;
+        }
+    }
     int lo = 0, hi = nb - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -249,28 +268,41 @@ __device__ __forceinline__ Fp8Tile fp8_decode(int nb, int t, const Fp8Args& a, c
     const int local = t - tb[lo];
     const int units = sp->units[lo];
     const int4 b = sp->blk[lo];
+    const Fp8Args& ta = (KIND == FP8_FUSED && !gated) ? a2 : a;
     Fp8Tile tl;
+    tl.blk = lo;
+    tl.gated = gated;
     tl.group = b.x;
-    tl.shared = tl.group == a.E;
+    tl.shared = tl.group == ta.E;
     tl.m = local / units;
     const int u = local - tl.m * units;
     const int start = u * b.w;
     tl.rows = min(b.w, b.z - start);
     tl.row0 = b.y + start;
     tl.n_mma = (tl.rows + 15) & ~15;
-    tl.nkb = (tl.shared ? a.K_shared : a.K) / kFp8BlockK;
+    tl.nkb = (tl.shared ? ta.K_shared : ta.K) / kFp8BlockK;
     return tl;
 }
 
+// The i-th tile of this CTA (-1 past the end): round-robin, or the balanced
+// gate/up-then-down order of the single launch.
+template <int KIND>
+__device__ __forceinline__ int fp8_cta_tile(int i, int total, const Fp8Args& a, const SmemPlan* sp)
+{
+    return KIND == FP8_FUSED ? cta_tile<MODE_FUSED>(i, total, sp->tiles1, a.comp) : cta_tile<MODE_DOWN>(i, total, 0, 0);
+}
+
 struct Fp8Iter {
-    int t, kb;
+    int i, t, kb;
     Fp8Tile tl;
 };
 
-__device__ __forceinline__ bool fp8_iter_begin(Fp8Iter& it, int nb, int total, const Fp8Args& a, const SmemPlan* sp)
+template <int KIND>
+__device__ __forceinline__ bool fp8_iter_seek(Fp8Iter& it, int nb, int total, const Fp8Args& a, const Fp8Args& a2,
+                                              const SmemPlan* sp)
 {
-    for (it.t = blockIdx.x; it.t < total; it.t += gridDim.x) {
-        it.tl = fp8_decode(nb, it.t, a, sp);
+    for (; (it.t = fp8_cta_tile<KIND>(it.i, total, a, sp)) >= 0; it.i++) {
+        it.tl = fp8_decode<KIND>(nb, it.t, a, a2, sp);
         if (it.tl.nkb > 0) {
             it.kb = 0;
             return true;
@@ -279,17 +311,21 @@ __device__ __forceinline__ bool fp8_iter_begin(Fp8Iter& it, int nb, int total, c
     return false;
 }
 
-__device__ __forceinline__ bool fp8_iter_next(Fp8Iter& it, int nb, int total, const Fp8Args& a, const SmemPlan* sp)
+template <int KIND>
+__device__ __forceinline__ bool fp8_iter_begin(Fp8Iter& it, int nb, int total, const Fp8Args& a, const Fp8Args& a2,
+                                               const SmemPlan* sp)
+{
+    it.i = 0;
+    return fp8_iter_seek<KIND>(it, nb, total, a, a2, sp);
+}
+
+template <int KIND>
+__device__ __forceinline__ bool fp8_iter_next(Fp8Iter& it, int nb, int total, const Fp8Args& a, const Fp8Args& a2,
+                                              const SmemPlan* sp)
 {
     if (++it.kb < it.tl.nkb) return true;
-    for (it.t += gridDim.x; it.t < total; it.t += gridDim.x) {
-        it.tl = fp8_decode(nb, it.t, a, sp);
-        if (it.tl.nkb > 0) {
-            it.kb = 0;
-            return true;
-        }
-    }
-    return false;
+    ++it.i;
+    return fp8_iter_seek<KIND>(it, nb, total, a, a2, sp);
 }
 
 // Instruction descriptor for kind::mxf8f6f4 with block scaling: A and B e4m3
@@ -338,15 +374,21 @@ __device__ __forceinline__ float pick4f(const float (&v)[4], int i)
 // the four lane quadrants) and issues the MMAs.  tcgen05.cp and tcgen05.mma
 // from one thread execute in issue order, so one set of scale-factor columns
 // serves every K block.
-template <bool GATED>
+template <int KIND>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mA1,
                             const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mA0s,
                             const __grid_constant__ CUtensorMap mA1s, const __grid_constant__ CUtensorMap mBs,
                             const __grid_constant__ CUtensorMap mSB, const __grid_constant__ CUtensorMap mSBs,
-                            const Fp8Args args)
+                            const __grid_constant__ CUtensorMap mA2, const __grid_constant__ CUtensorMap mB2,
+                            const __grid_constant__ CUtensorMap mA2s, const __grid_constant__ CUtensorMap mB2s,
+                            const __grid_constant__ CUtensorMap mSB2, const __grid_constant__ CUtensorMap mSB2s,
+                            const Fp8Args args, const Fp8Args args2)
 {
-    constexpr uint32_t kABytes = GATED ? 2 * 128 * kFp8BlockK : 128 * kFp8BlockK;
+    // FP8_FUSED: args and mA0..mSBs describe the gate/up tiles (W1/W3, xp8, its
+    // scales), args2 and mA2..mSB2s the down tiles (W2, h8, its scales).  The
+    // other kinds use args and mA0..mSBs only.
+    constexpr uint32_t kABytes = KIND != FP8_DOWN ? 2 * 128 * kFp8BlockK : 128 * kFp8BlockK;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + kFp8RingBytes);
@@ -364,16 +406,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         return;
     }
     const int nb = hdr->n_blocks;
-    const int total = GATED ? hdr->tiles1 : hdr->tiles2;
+    const int total = KIND == FP8_FUSED ? hdr->tiles1 + hdr->tiles2 : KIND == FP8_GATED ? hdr->tiles1 : hdr->tiles2;
     const int n_max = max(16, hdr->n_max);
     const uint32_t b_bytes = (uint32_t)n_max * kFp8BlockK;       // B region of a stage (largest tile)
     const uint32_t stage_bytes = kABytes + b_bytes + kSfStageBytes;
     const int stages = min(kMaxStages, (int)(kFp8RingBytes / stage_bytes));
     {
         const PlanArrays pa = plan_arrays(const_cast<int32_t*>(args.plan));
-        const int32_t* tbg = GATED ? pa.tb1 : pa.tb2;
+        const int32_t* tbg = KIND == FP8_DOWN ? pa.tb2 : pa.tb1;
+        if (threadIdx.x == 0) splan->tiles1 = hdr->tiles1;
         for (int i = threadIdx.x; i <= nb; i += blockDim.x) {
             splan->tb[i] = tbg[i];
+            if (KIND == FP8_FUSED) splan->tb2[i] = pa.tb2[i];
             if (i < nb) {
                 splan->blk[i] = make_int4(pa.group[i], pa.row0[i], pa.rows[i], pa.chunk[i]);
                 splan->units[i] = pa.units[i];
@@ -399,7 +443,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         ptx::prefetch_tensormap(&mA0);
         ptx::prefetch_tensormap(&mB);
         ptx::prefetch_tensormap(&mSB);
-        if (GATED) ptx::prefetch_tensormap(&mA1);
+        if (KIND != FP8_DOWN) ptx::prefetch_tensormap(&mA1);
+        if (KIND == FP8_FUSED) {
+            ptx::prefetch_tensormap(&mA2);
+            ptx::prefetch_tensormap(&mB2);
+            ptx::prefetch_tensormap(&mSB2);
+        }
     }
     if (warp == 1) {
         ptx::tmem_alloc(ptx::smem_u32(&ctl->tmem_base), kFp8TmemCols);
@@ -416,36 +465,51 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint64_t pol = ptx::policy_evict_normal();
             uint32_t armed = 0, armed_ph = 0;
             bool ok = true;
-            auto tx_bytes = [&](const Fp8Tile& tl) { return kABytes + (uint32_t)tl.n_mma * kFp8BlockK + 512u; };
-            auto issue_a = [&](const Fp8Iter& it, uint32_t a_dst, uint32_t full) {
-                const Fp8Tile& tl = it.tl;
-                const int kc = it.kb * kFp8BlockK;
-                const int Mrows = tl.shared ? args.M_shared : args.M;
-                const int a_row = (tl.shared ? 0 : tl.group * Mrows) + tl.m * 128;
-                ptx::tma_load_2d(a_dst, tl.shared ? &mA0s : &mA0, full, kc, a_row, pol);
-                if (GATED) ptx::tma_load_2d(a_dst + 128 * kFp8BlockK, tl.shared ? &mA1s : &mA1, full, kc, a_row, pol);
+            auto tx_bytes = [&](const Fp8Tile& tl) {
+                return (tl.gated ? 2u : 1u) * 128u * kFp8BlockK + (uint32_t)tl.n_mma * kFp8BlockK + 512u;
             };
-            auto issue_b = [&](const Fp8Iter& it, uint32_t stage, uint32_t full) {
-                const Fp8Tile& tl = it.tl;
-                const int kc = it.kb * kFp8BlockK;
+            // the down tiles of the single launch read the second set of maps and args
+            auto down2 = [&](const Fp8Tile& tl) { return KIND == FP8_FUSED && !tl.gated; };
+            auto issue_a = [&](const Fp8Tile& tl, int kb, uint32_t a_dst, uint32_t full) {
+                const int kc = kb * kFp8BlockK;
+                const Fp8Args& ta = down2(tl) ? args2 : args;
+                const int Mrows = tl.shared ? ta.M_shared : ta.M;
+                const int a_row = (tl.shared ? 0 : tl.group * Mrows) + tl.m * 128;
+                const CUtensorMap* a0 = down2(tl) ? (tl.shared ? &mA2s : &mA2) : (tl.shared ? &mA0s : &mA0);
+                ptx::tma_load_2d(a_dst, a0, full, kc, a_row, pol);
+                if (tl.gated) ptx::tma_load_2d(a_dst + 128 * kFp8BlockK, tl.shared ? &mA1s : &mA1, full, kc, a_row, pol);
+            };
+            auto issue_b = [&](const Fp8Tile& tl, int kb, uint32_t stage, uint32_t full) {
+                const int kc = kb * kFp8BlockK;
                 const uint32_t b_dst = stage + kABytes;
+                const CUtensorMap* bm = down2(tl) ? (tl.shared ? &mB2s : &mB2) : (tl.shared ? &mBs : &mB);
+                const CUtensorMap* sm = down2(tl) ? (tl.shared ? &mSB2s : &mSB2) : (tl.shared ? &mSBs : &mSB);
                 for (int i = 0; i < tl.n_mma / 16; i++)
-                    ptx::tma_load_2d(b_dst + i * 16 * kFp8BlockK, tl.shared ? &mBs : &mB, full, kc, tl.row0 + 16 * i,
-                                     pol);
+                    ptx::tma_load_2d(b_dst + i * 16 * kFp8BlockK, bm, full, kc, tl.row0 + 16 * i, pol);
                 // the tokens' scales of this K block: 128 fp32 from row0 rounded down to 4
-                ptx::tma_load_2d(b_dst + b_bytes, tl.shared ? &mSBs : &mSB, full, tl.row0 & ~3, it.kb, pol);
+                ptx::tma_load_2d(b_dst + b_bytes, sm, full, tl.row0 & ~3, kb, pol);
+            };
+            // FP8_FUSED: a down tile reads h8 and its scales only after every gate/up
+            // tile of its block has published them (4 epilogue warps per tile)
+            auto wait_block_ready = [&](const Fp8Tile& tl) -> bool {
+                const int32_t* dep = plan_arrays(const_cast<int32_t*>(args.plan)).dep + tl.blk;
+                const int m1 = tl.shared ? args.M_shared : args.M;
+                const int need = 4 * splan->units[tl.blk] * ((m1 + 127) / 128);
+                if (!bounded_count_wait(dep, need, ctl, args.err)) return false;
+                ptx::fence_proxy_async_global();   // the TMA reads below come after the acquire
+                return true;
             };
             int pre = 0;
             if (!waited_early) {
                 Fp8Iter it;
-                bool more = fp8_iter_begin(it, nb, total, args, splan);
+                bool more = fp8_iter_begin<KIND>(it, nb, total, args, args2, splan);
                 while (more && pre < stages) {
                     const uint32_t full = ptx::smem_u32(&ctl->full[pre]);
                     ptx::mbar_arrive_expect_tx(full, tx_bytes(it.tl));
                     armed |= 1u << pre;
-                    issue_a(it, ring + (uint32_t)pre * stage_bytes, full);
+                    issue_a(it.tl, it.kb, ring + (uint32_t)pre * stage_bytes, full);
                     ++pre;
-                    more = fp8_iter_next(it, nb, total, args, splan);
+                    more = fp8_iter_next<KIND>(it, nb, total, args, args2, splan);
                 }
                 ptx::grid_dep_wait();
             }
@@ -453,13 +517,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int s = 0, n = 0;
             uint32_t ph = 0;
             Fp8Iter it;
-            bool more = fp8_iter_begin(it, nb, total, args, splan);
+            bool more = fp8_iter_begin<KIND>(it, nb, total, args, args2, splan);
             while (more) {
                 const uint32_t stage = ring + (uint32_t)s * stage_bytes;
                 const uint32_t full = ptx::smem_u32(&ctl->full[s]);
-                if (n < pre) {
-                    issue_b(it, stage, full);
-                } else {
+                if (n >= pre) {
                     if (!bounded_wait(ptx::smem_u32(&ctl->empty[s]), ph ^ 1u, ctl, args.err)) {
                         ok = false;
                         break;
@@ -467,15 +529,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     ptx::mbar_arrive_expect_tx(full, tx_bytes(it.tl));
                     armed |= 1u << s;
                     armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
-                    issue_a(it, stage, full);
-                    issue_b(it, stage, full);
+                    issue_a(it.tl, it.kb, stage, full);
                 }
+                if (KIND == FP8_FUSED && !it.tl.gated && it.kb == 0 && !wait_block_ready(it.tl)) {
+                    ok = false;
+                    break;
+                }
+                issue_b(it.tl, it.kb, stage, full);
                 ++n;
                 if (++s == stages) {
                     s = 0;
                     ph ^= 1u;
                 }
-                more = fp8_iter_next(it, nb, total, args, splan);
+                more = fp8_iter_next<KIND>(it, nb, total, args, args2, splan);
             }
             if (!ok) {
                 const uint64_t t0 = ptx::globaltimer();
@@ -495,23 +561,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         bool ok = true, issued = false;
         // The weight-block scales of a tile (lane l: K blocks l, l + 32, l + 64, l + 96)
         // are loaded one tile ahead, so their latency hides behind the previous tile.
-        auto next_tile = [&](int t) {
-            for (; t < total; t += gridDim.x)
-                if (fp8_decode(nb, t, args, splan).nkb > 0) break;
-            return t;
-        };
         auto load_scales = [&](int t, float (&wa)[4], float (&wb)[4]) {
-            if (t >= total) return;
-            const Fp8Tile tl = fp8_decode(nb, t, args, splan);
-            const int Mrows = tl.shared ? args.M_shared : args.M;
+            if (t < 0) return;
+            const Fp8Tile tl = fp8_decode<KIND>(nb, t, args, args2, splan);
+            const Fp8Args& ta = (KIND == FP8_FUSED && !tl.gated) ? args2 : args;
+            const int Mrows = tl.shared ? ta.M_shared : ta.M;
             const int64_t srow = (int64_t)(tl.shared ? 0 : tl.group * (Mrows / 128)) + tl.m;
-            const float* sA0 = (tl.shared ? args.sA0s : args.sA0) + srow * tl.nkb;
+            const float* sA0 = (tl.shared ? ta.sA0s : ta.sA0) + srow * tl.nkb;
 #pragma unroll
             for (int i = 0; i < 4; i++) {
                 const int kb = 32 * i + lane;
                 wa[i] = kb < tl.nkb ? __ldg(sA0 + kb) : 1.f;
             }
-            if (GATED) {
+            if (tl.gated) {
                 const float* sA1 = (tl.shared ? args.sA1s : args.sA1) + srow * tl.nkb;
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
@@ -521,17 +583,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         };
         float nwa[4] = {1.f, 1.f, 1.f, 1.f}, nwb[4] = {1.f, 1.f, 1.f, 1.f};
-        int t = next_tile(blockIdx.x);
+        int ti = 0;
+        int t = fp8_cta_tile<KIND>(ti, total, args, splan);
         load_scales(t, nwa, nwb);
-        for (; t < total && ok;) {
-            const Fp8Tile tl = fp8_decode(nb, t, args, splan);
+        while (t >= 0 && ok) {
+            const Fp8Tile tl = fp8_decode<KIND>(nb, t, args, args2, splan);
             uint32_t ea[4], eb[4];
 #pragma unroll
             for (int i = 0; i < 4; i++) {
                 ea[i] = __float_as_uint(nwa[i]);
                 eb[i] = __float_as_uint(nwb[i]);
             }
-            const int t_next = next_tile(t + gridDim.x);
+            const int t_next = fp8_cta_tile<KIND>(++ti, total, args, splan);
             load_scales(t_next, nwa, nwb);
             ok = __all_sync(0xffffffffu, bounded_wait(ptx::smem_u32(&ctl->tempty[acc]), aph ^ 1u, ctl, args.err));
             if (!ok) break;
@@ -556,7 +619,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const uint32_t a0 = ue8m0_of(__uint_as_float(__shfl_sync(0xffffffffu, pick4(ea, kb >> 5), kb & 31))) *
                                     0x01010101u;
                 *reinterpret_cast<uint4*>(atoms + 16 * lane) = make_uint4(a0, a0, a0, a0);
-                if (GATED) {
+                if (tl.gated) {
                     const uint32_t a1 =
                         ue8m0_of(__uint_as_float(__shfl_sync(0xffffffffu, pick4(eb, kb >> 5), kb & 31))) * 0x01010101u;
                     *reinterpret_cast<uint4*>(atoms + 512 + 16 * lane) = make_uint4(a1, a1, a1, a1);
@@ -569,13 +632,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t b_addr = a_addr + kABytes;
                     const uint32_t atoms_addr = b_addr + b_bytes + 512;
                     ptx::tmem_cp_32x128b_warpx4(tmem_base + kSfColA0, ptx::plain_rows16_desc(atoms_addr));
-                    if (GATED) ptx::tmem_cp_32x128b_warpx4(tmem_base + kSfColA1, ptx::plain_rows16_desc(atoms_addr + 512));
+                    if (tl.gated)
+                        ptx::tmem_cp_32x128b_warpx4(tmem_base + kSfColA1, ptx::plain_rows16_desc(atoms_addr + 512));
                     ptx::tmem_cp_32x128b_warpx4(tmem_base + kSfColB, ptx::plain_rows16_desc(atoms_addr + 1024));
 #pragma unroll
                     for (int kk = 0; kk < kFp8BlockK / 32; kk++)
                         mma_mxf8_ss(d_g, ptx::sw128_kmajor_desc(a_addr + kk * 32), ptx::sw128_kmajor_desc(b_addr + kk * 32),
                                     idesc, tmem_base + kSfColA0, tmem_base + kSfColB, (kb > 0 || kk > 0) ? 1u : 0u);
-                    if (GATED) {
+                    if (tl.gated) {
 #pragma unroll
                         for (int kk = 0; kk < kFp8BlockK / 32; kk++)
                             mma_mxf8_ss(d_g + (uint32_t)kFp8TileRows,
@@ -609,28 +673,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue (warps 2-5)
         const int quad = warp & 3;
-        int acc = 0, tcount = 0;
+        int acc = 0, gcount = 0;   // gcount: gate/up tiles so far (their amax buffers alternate)
         uint32_t aph = 0, xph = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x) {
-            const Fp8Tile tl = fp8_decode(nb, t, args, splan);
+        for (int ti = 0, t; (t = fp8_cta_tile<KIND>(ti, total, args, splan)) >= 0; ti++) {
+            const Fp8Tile tl = fp8_decode<KIND>(nb, t, args, args2, splan);
             if (tl.nkb <= 0) continue;
+            const Fp8Args& ea = (KIND == FP8_FUSED && !tl.gated) ? args2 : args;
             // down: the tile's gates (lane l: columns l, l + 32, l + 64, l + 96), fetched before the wait
             float gates[4] = {1.f, 1.f, 1.f, 1.f};
-            if (!GATED && !tl.shared) {
+            if (!tl.gated && !tl.shared) {
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
                     const int col = 32 * i + lane;
-                    if (col < tl.rows) gates[i] = __ldg(args.gate_w + __ldg(args.perm + tl.row0 + col));
+                    if (col < tl.rows) gates[i] = __ldg(ea.gate_w + __ldg(ea.perm + tl.row0 + col));
                 }
             }
             if (!__all_sync(0xffffffffu, bounded_wait(ptx::smem_u32(&ctl->tfull[acc]), aph, ctl, args.err))) break;
             ptx::tc_fence_after();
             const uint32_t taddr = tmem_base + (uint32_t)acc * kFp8AccCols + ((uint32_t)(quad * 32) << 16);
-            const int Mrows = tl.shared ? args.M_shared : args.M;
+            const int Mrows = tl.shared ? ea.M_shared : ea.M;
             const int mrow = tl.m * 128 + quad * 32 + lane;   // weight row of this thread (TMEM lane)
             bool ok = true;
-            if (GATED) {
-                float* rb = red + (tcount & 1) * 4 * kFp8TileRows;
+            if (tl.gated) {
+                float* rb = red + (gcount++ & 1) * 4 * kFp8TileRows;
                 // pass 1: h = silu(g) * u, written back over g in TMEM, and per token
                 // the largest |h| over this warp's 32 f rows
                 for (int c0 = 0; c0 < tl.n_mma; c0 += 16) {
@@ -681,7 +746,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
             } else {
-                bf16* out = tl.shared ? args.out_shared : args.out;
+                bf16* out = tl.shared ? ea.out_shared : ea.out;
                 for (int c0 = 0; c0 < tl.n_mma; c0 += 16) {
                     uint32_t v[16];
                     ptx::tmem_ld16(taddr + (uint32_t)c0, v);
@@ -702,7 +767,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!ok) break;
             acc ^= 1;
             if (acc == 0) aph ^= 1u;
-            ++tcount;
+            if (KIND == FP8_FUSED && tl.gated) {
+                // publish this warp's h8 rows and scales of the tile to the down tiles of
+                // its block: each of the 4 epilogue warps adds 1 after its own stores
+                ptx::fence_proxy_async_global();
+                __syncwarp();
+                if (lane == 0) ptx::red_add_release_gpu(plan_arrays(const_cast<int32_t*>(args.plan)).dep + tl.blk, 1);
+            }
         }
     }
 

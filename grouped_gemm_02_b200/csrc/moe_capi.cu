@@ -92,9 +92,11 @@ int device_setup(DeviceState** out)
                                      kGemmSmemBytes) != cudaSuccess ||
                 cudaFuncSetAttribute(grouped_gemm_kernel<MODE_FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kGemmSmemBytes) != cudaSuccess ||
-                cudaFuncSetAttribute(grouped_gemm_fp8_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                cudaFuncSetAttribute(grouped_gemm_fp8_kernel<FP8_GATED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kFp8SmemBytes) != cudaSuccess ||
-                cudaFuncSetAttribute(grouped_gemm_fp8_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                cudaFuncSetAttribute(grouped_gemm_fp8_kernel<FP8_DOWN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kFp8SmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(grouped_gemm_fp8_kernel<FP8_FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kFp8SmemBytes) != cudaSuccess)
                 return MOE_ERR_CUDA;
             if (!g_encode) {
@@ -680,21 +682,31 @@ struct Fp8Operands {
 
 int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int sms, cudaStream_t st, bool prof)
 {
+    // gate/up operands: W1/W3, xp8 and its scales (shared: Ws1/Ws3, x8, sxT)
     CUtensorMap a0, a1, b, a0s, a1s, bs, sb, sbs;
+    // down operands: W2, h8 and its scales (shared: Ws2, hs8, shs)
+    CUtensorMap a2, b2, a2s, b2s, sb2, sb2s;
     const uint64_t E = (uint64_t)o.E;
     const uint64_t lp = (uint64_t)o.ld_pairs, lt = (uint64_t)o.ld_tokens;
     if (!make_map_u8(&a0, o.W1q, o.d, E * o.f, 128) || !make_map_u8(&a1, o.W3q, o.d, E * o.f, 128) ||
-        !make_map_u8(&b, o.xp8, o.d, (uint64_t)o.P, 16) || !make_map_f32(&sb, o.sxp, lp, o.d / 128))
+        !make_map_u8(&b, o.xp8, o.d, (uint64_t)o.P, 16) || !make_map_f32(&sb, o.sxp, lp, o.d / 128) ||
+        !make_map_u8(&a2, o.W2q, o.f, E * o.d, 128) || !make_map_u8(&b2, o.h8, o.f, (uint64_t)o.P, 16) ||
+        !make_map_f32(&sb2, o.sh, lp, o.f / 128))
         return MOE_ERR_CUDA;
     if (o.fs > 0) {
         if (!make_map_u8(&a0s, o.Ws1q, o.d, o.fs, 128) || !make_map_u8(&a1s, o.Ws3q, o.d, o.fs, 128) ||
-            !make_map_u8(&bs, o.x8, o.d, (uint64_t)o.T, 16) || !make_map_f32(&sbs, o.sxT, lt, o.d / 128))
+            !make_map_u8(&bs, o.x8, o.d, (uint64_t)o.T, 16) || !make_map_f32(&sbs, o.sxT, lt, o.d / 128) ||
+            !make_map_u8(&a2s, o.Ws2q, o.fs, o.d, 128) || !make_map_u8(&b2s, o.hs8, o.fs, (uint64_t)o.T, 16) ||
+            !make_map_f32(&sb2s, o.shs, lt, o.fs / 128))
             return MOE_ERR_CUDA;
     } else {
         a0s = a0;
         a1s = a1;
         bs = b;
         sbs = sb;
+        a2s = a2;
+        b2s = b2;
+        sb2s = sb2;
     }
     Fp8Args g1{};
     g1.plan = plan;
@@ -717,25 +729,6 @@ int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int 
     g1.perm = o.perm;
     g1.gate_w = o.gate_w;
     g1.err = err;
-    if (launch(grouped_gemm_fp8_kernel<true>, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a0, a1, b, a0s, a1s,
-               bs, sb, sbs, g1) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    phase_mark(prof, 3, st);
-    if (!make_map_u8(&a0, o.W2q, o.f, E * o.d, 128) || !make_map_u8(&b, o.h8, o.f, (uint64_t)o.P, 16) ||
-        !make_map_f32(&sb, o.sh, lp, o.f / 128))
-        return MOE_ERR_CUDA;
-    a1 = a0;
-    if (o.fs > 0) {
-        if (!make_map_u8(&a0s, o.Ws2q, o.fs, o.d, 128) || !make_map_u8(&bs, o.hs8, o.fs, (uint64_t)o.T, 16) ||
-            !make_map_f32(&sbs, o.shs, lt, o.fs / 128))
-            return MOE_ERR_CUDA;
-        a1s = a0s;
-    } else {
-        a0s = a0;
-        a1s = a0;
-        bs = b;
-        sbs = sb;
-    }
     Fp8Args g2 = g1;
     g2.M = o.d;
     g2.M_shared = o.d;
@@ -747,8 +740,21 @@ int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int 
     g2.sA1s = nullptr;
     g2.out = o.y_p;
     g2.out_shared = o.ys;
-    return status_of(launch(grouped_gemm_fp8_kernel<false>, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a0, a1,
-                            b, a0s, a1s, bs, sb, sbs, g2));
+    if (gemm_fused(o.P, o.f)) {
+        // one launch: a gate/up tile streams d/128 k-blocks, a down tile f/128
+        const int kb1 = o.d / 128, kb2 = o.f / 128;
+        g1.comp = std::max(1, (kb1 + kb2 / 2) / kb2);
+        const cudaError_t e = launch(grouped_gemm_fp8_kernel<FP8_FUSED>, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes,
+                                     st, a0, a1, b, a0s, a1s, bs, sb, sbs, a2, b2, a2s, b2s, sb2, sb2s, g1, g2);
+        phase_mark(prof, 3, st);   // the single launch has no boundary: the down phase reads as zero
+        return status_of(e);
+    }
+    if (launch(grouped_gemm_fp8_kernel<FP8_GATED>, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a0, a1, b, a0s,
+               a1s, bs, sb, sbs, a2, b2, a2s, b2s, sb2, sb2s, g1, g1) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    phase_mark(prof, 3, st);
+    return status_of(launch(grouped_gemm_fp8_kernel<FP8_DOWN>, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a2,
+                            a2, b2, a2s, a2s, b2s, sb2, sb2s, a2, b2, a2s, b2s, sb2, sb2s, g2, g2));
 }
 
 }  // namespace
