@@ -109,6 +109,7 @@ def _fp8_layer_check(s: wl.LayerShape, seed: int, n_sample=None, device_inputs=F
     ("decode64", dict(alpha=0.1)),
     ("decode64", dict(alpha=1.0)),
     ("kimi_k2", dict(T=8)),
+    ("deepseek_v3", dict(T=16, alpha=0.05)),    # one launch for both GEMMs, with the shared expert
     ("deepseek_v3", dict(T=64, alpha=0.5)),
 ])
 def test_fp8_layer_small(name, kw):
