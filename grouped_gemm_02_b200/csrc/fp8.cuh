@@ -24,6 +24,9 @@
 // One tile = 128 weight rows (W1 and W3 side by side for gate/up: two MMAs
 // into two accumulators) x at most 112 tokens, so that two tiles' accumulators
 // (2 x (112 + 112) columns) and the scale factors fit the 512 TMEM columns.
+// A launch runs the gate/up tiles, the down tiles, or both (FP8_FUSED: the
+// down tiles of a block wait, bounded, on a counter its gate/up tiles' epilogue
+// warps bump after storing h8 and its scales).
 #pragma once
 
 #include <cuda_fp8.h>

@@ -21,9 +21,10 @@
 //                gate/up tile of block i has stored them: each gate/up tile's
 //                epilogue bumps a per-block counter (zeroed by the plan
 //                builder) after its stores, and the producer of a down tile
-//                waits for the count (bounded) before its h loads -- its W2
-//                loads go out before the wait.  The down tiles fill the
-//                gate/up tail instead of a second launch ramping up.
+//                waits for the count (bounded) before that tile's loads (W2
+//                tiles it prefetched before griddepcontrol.wait are already
+//                in flight).  The down tiles fill the gate/up tail instead of
+//                a second launch ramping up.
 //
 // The MMA is operand-swapped: the weights fill the M = 128 slot and the tokens
 // the N slot (16..256, chosen per expert from its live count by the plan), so
