@@ -92,3 +92,50 @@ def test_product_path_refuses_missing_library(monkeypatch, tmp_path):
     monkeypatch.setattr(moe, "library_path", lambda: str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError, match="missing"):
         moe.lib()
+
+
+# ------------------------------------------------------------------ workspace layout (host arithmetic only)
+
+def _bf16_layout(T, d, f, E, k, fs):
+    """Byte sizes and alignments of the layer intermediates, from the header's shapes."""
+    P, Ts = T * k, (T if fs else 0)
+    return [("logits", T * E * 4, 4), ("topk_idx", P * 4, 4), ("topk_w", P * 4, 4), ("counts", E * 4, 4),
+            ("offsets", (E + 1) * 4, 4), ("perm", P * 4, 4), ("inv_perm", P * 4, 4), ("xp", P * d * 2, 256),
+            ("h", P * f * 2, 256), ("y_p", P * d * 2, 256), ("hs", Ts * fs * 2, 256), ("ys", Ts * d * 2, 256)]
+
+
+def _fp8_layout(T, d, f, E, k, fs):
+    P, Ts = T * k, (T if fs else 0)
+    P4, T4 = (P + 3) // 4 * 4, (T + 3) // 4 * 4
+    return [("logits", T * E * 4, 4), ("topk_idx", P * 4, 4), ("topk_w", P * 4, 4), ("counts", E * 4, 4),
+            ("offsets", (E + 1) * 4, 4), ("perm", P * 4, 4), ("inv_perm", P * 4, 4), ("x8", T * d, 256),
+            ("sx", T * (d // 128) * 4, 16), ("xp8", P * d, 256), ("sxp", (d // 128) * P4 * 4, 16),
+            ("h8", P * f, 256), ("sh", (f // 128) * P4 * 4, 16), ("y_p", P * d * 2, 256),
+            ("hs8", Ts * fs, 256), ("shs", (fs // 128) * (T4 if Ts else 0) * 4, 16), ("ys", Ts * d * 2, 256),
+            ("sxT", (d // 128) * (T4 if Ts else 0) * 4, 16)]
+
+
+@pytest.mark.parametrize("T,d,f,E,k,fs", [(32, 2048, 1024, 64, 8, 0), (1, 256, 512, 8, 2, 0), (37, 7168, 2048, 256, 8, 2048),
+                                          (16384, 7168, 2048, 256, 8, 2048), (5, 4096, 14336, 8, 2, 0)])
+@pytest.mark.parametrize("fp8", [False, True])
+def test_workspace_tensors_disjoint_aligned_inside(L, T, d, f, E, k, fs, fp8):
+    layout = (_fp8_layout if fp8 else _bf16_layout)(T, d, f, E, k, fs)
+    total = C.c_size_t(0)
+    rc = (L.moe_workspace_size_fp8 if fp8 else L.moe_workspace_size)(T, d, f, E, k, fs, C.byref(total))
+    assert rc == 0
+    base = 1 << 40                      # any 1 KiB-aligned address: the call only adds offsets
+    fn = L.moe_workspace_tensor_fp8 if fp8 else L.moe_workspace_tensor
+    spans = []
+    for which, (name, nbytes, align) in enumerate(layout):
+        out = C.c_void_p(0)
+        assert fn(C.c_void_p(base), T, d, f, E, k, fs, which, C.byref(out)) == 0
+        off = out.value - base
+        assert off % align == 0, name
+        assert 0 <= off and off + nbytes <= total.value, name
+        if nbytes:
+            spans.append((off, off + nbytes, name))
+    spans.sort()
+    for (a0, a1, an), (b0, b1, bn) in zip(spans, spans[1:]):
+        assert a1 <= b0, f"{an} overlaps {bn}"
+    out = C.c_void_p(0)
+    assert fn(C.c_void_p(base), T, d, f, E, k, fs, len(layout), C.byref(out)) != 0   # past the last tensor
