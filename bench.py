@@ -402,7 +402,8 @@ def run_ours(args, s: wl.LayerShape):
         roof = {"bound": "tensor", "achieved": g_flops / t_g / 1e12, "peak": tc / 1e12,
                 "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = committed_traffic(workload_label(s))
+    # the record names the workload as the JSON line does (" fp8" for the FP8 kernels)
+    roof["traffic"] = committed_traffic(workload_label(s) + (" fp8" if args.fp8 else ""))
     roof["kernel"] = ("grouped_gemm_fp8_kernel<gate/up>+<down>" if args.fp8 else
                       ("grouped_gemm_kernel<fused gate/up + down>" if gemm_fused(s.P, s.f)
                        else "grouped_gemm_kernel<gate/up>+<down>"))

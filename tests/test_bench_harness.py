@@ -80,6 +80,7 @@ def test_traffic_record_tied_to_kernel_source(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(p))
     assert bench.committed_traffic("w") == 123
     assert bench.committed_traffic("other") is None
+    assert bench.committed_traffic("w fp8") is None          # another kernel's record
     rec["source_sha"] = "0" * 16
     p.write_text(json.dumps(rec))
     assert bench.committed_traffic("w") is None
