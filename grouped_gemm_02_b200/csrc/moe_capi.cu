@@ -352,12 +352,13 @@ int run_gemms(const GemmOperands& o, const int32_t* plan, bool plan_ready, uint3
 }
 
 int run_combine(const bf16* y_p, const int32_t* inv_perm, const bf16* ys, int T, int k, int d, bf16* out,
-                cudaStream_t st)
+                cudaStream_t st, bool inv_perm_ready = false)
 {
     constexpr int kThreads = 64;
     const int nvec = d / 8;
     const int gy = std::max(1, std::min((nvec + kThreads - 1) / kThreads, 65535));
-    return status_of(launch(combine_kernel, dim3(T, gy), dim3(kThreads), 0, st, y_p, inv_perm, ys, T, k, d, out));
+    return status_of(launch(combine_kernel, dim3(T, gy), dim3(kThreads), 0, st, y_p, inv_perm, ys, T, k, d, out,
+                            inv_perm_ready ? 1 : 0));
 }
 
 }  // namespace
@@ -578,7 +579,7 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     // the plan was written two or more launches before the gate/up GEMM (the gather is in between)
     if ((rc = run_gemms(o, plan, /*plan_ready=*/true, err, dev->sm_count, st, prof))) return rc;
     phase_mark(prof, 4, st);
-    rc = run_combine(y_p, inv_perm, ys, iT, ik, id, reinterpret_cast<bf16*>(out), st);
+    rc = run_combine(y_p, inv_perm, ys, iT, ik, id, reinterpret_cast<bf16*>(out), st, /*inv_perm_ready=*/true);
     phase_mark(prof, 5, st);
     return rc;
 }
@@ -913,7 +914,7 @@ int moe_layer_forward_fp8(const moe_bf16* x, const moe_bf16* Wg, const float* bi
     phase_mark(prof, 2, st);
     if ((rc = run_gemms_fp8(o, plan, err, dev->sm_count, st, prof))) return rc;
     phase_mark(prof, 4, st);
-    rc = run_combine(y_p, inv_perm, o.ys, iT, ik, id, reinterpret_cast<bf16*>(out), st);
+    rc = run_combine(y_p, inv_perm, o.ys, iT, ik, id, reinterpret_cast<bf16*>(out), st, /*inv_perm_ready=*/true);
     phase_mark(prof, 5, st);
     return rc;
 }

@@ -354,17 +354,20 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const bf16* __restrict
 // out[t, :] = bf16( sum_{j<k} y_p[inv_perm[t*k+j], :]  (+ ys[t, :]) ), summed in
 // fp32 in ascending j, no atomics.  Dropped pairs (inv_perm < 0) add nothing.
 // grid (T, column blocks), block 64; requires d % 8 == 0.
+// inv_perm_ready: inv_perm was written two or more launches earlier (the layer
+// forward), so it is read before griddepcontrol.wait.
 __global__ void __launch_bounds__(128) combine_kernel(const bf16* __restrict__ y_p, const int32_t* __restrict__ inv_perm,
                                                       const bf16* __restrict__ ys, int T, int k, int d,
-                                                      bf16* __restrict__ out)
+                                                      bf16* __restrict__ out, int inv_perm_ready)
 {
-    ptx::grid_dep_wait();
-    ptx::grid_dep_launch();
+    if (!inv_perm_ready) ptx::grid_dep_wait();
     const int t = blockIdx.x;
-    if (t >= T) return;
     int rows[kMaxTopK];
 #pragma unroll
-    for (int j = 0; j < kMaxTopK; j++) rows[j] = j < k ? inv_perm[(size_t)t * k + j] : -1;
+    for (int j = 0; j < kMaxTopK; j++) rows[j] = (t < T && j < k) ? inv_perm[(size_t)t * k + j] : -1;
+    if (inv_perm_ready) ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
+    if (t >= T) return;
     const int nvec = d / 8;
     for (int v = blockIdx.y * blockDim.x + threadIdx.x; v < nvec; v += gridDim.y * blockDim.x) {
         float acc[8];
