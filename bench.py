@@ -7,7 +7,10 @@ grouped GEMM, combine) over one batch of seeded synthetic tokens, through
 moe_layer_forward.  Prints ONE JSON line on rank 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode64]
-                    [--T ..] [--alpha ..] [--impl ours|reference]
+                    [--T ..] [--alpha ..] [--fp8] [--impl ours|reference]
+
+``--fp8`` times moe_layer_forward_fp8 (e4m3 expert weights with 128 x 128
+block scales, quantised once before the timed region).
 
 Multi-GPU (torchrun) runs independent replicas: the layer has no exchange
 step, so every rank times its own copy and the value is the tokens of all
