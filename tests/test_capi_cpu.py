@@ -87,6 +87,36 @@ def test_host_argument_checks(L):
     assert L.moe_permute(FAKE, FAKE, 4, 128, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, None) == -3
 
 
+def _layer_fp8(L, **kw):
+    a = dict(x=FAKE, Wg=FAKE, bias=None, W1q=FAKE, W1s=FAKE, W3q=FAKE, W3s=FAKE, W2q=FAKE, W2s=FAKE, Ws1q=None,
+             Ws1s=None, Ws3q=None, Ws3s=None, Ws2q=None, Ws2s=None, fs=0, T=4, d=256, f=256, E=4, k=2, out=FAKE,
+             ws=FAKE, ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    return L.moe_layer_forward_fp8(a["x"], a["Wg"], a["bias"], a["W1q"], a["W1s"], a["W3q"], a["W3s"], a["W2q"],
+                                   a["W2s"], a["Ws1q"], a["Ws1s"], a["Ws3q"], a["Ws3s"], a["Ws2q"], a["Ws2s"], a["fs"],
+                                   a["T"], a["d"], a["f"], a["E"], a["k"], a["out"], a["ws"], a["ws_bytes"],
+                                   a["stream"])
+
+
+def test_fp8_host_argument_checks(L):
+    assert _layer_fp8(L, d=192) == -2          # a multiple of 64 but not of 128
+    assert _layer_fp8(L, f=64) == -2
+    assert _layer_fp8(L, fs=64) == -2
+    assert _layer_fp8(L, d=16512) == -1        # past the 16384 limit of the weight-scale registers
+    assert _layer_fp8(L, f=16512) == -1
+    assert _layer_fp8(L, W2s=None) == -1
+    assert _layer_fp8(L, fs=128) == -1         # shared expert without weights
+    assert _layer_fp8(L, x=C.c_void_p(0x10008)) == -2
+    assert _layer_fp8(L, ws_bytes=1024) == -3
+    assert _layer_fp8(L, T=0) == 0
+    assert L.moe_quantize_fp8_rows(FAKE, 4, 100, FAKE, FAKE, None) == -2
+    assert L.moe_quantize_fp8_rows(FAKE, -1, 128, FAKE, FAKE, None) == -1
+    assert L.moe_quantize_fp8_rows(FAKE, 4, 128, None, FAKE, None) == -1
+    assert L.moe_quantize_fp8_rows(FAKE, 0, 128, FAKE, FAKE, None) == 0
+    assert L.moe_quantize_fp8_blocks(FAKE, 100, 128, FAKE, FAKE, None) == -2
+    assert L.moe_quantize_fp8_blocks(FAKE, 128, 128, FAKE, None, None) == -1
+
+
 def test_product_path_refuses_missing_library(monkeypatch, tmp_path):
     monkeypatch.setattr(moe, "_lib", None)
     monkeypatch.setattr(moe, "library_path", lambda: str(tmp_path / "absent.so"))
