@@ -356,9 +356,28 @@ def pin_fp8_quantize_rows_and_blocks():
             assert np.array_equal(Wq[128 * br:128 * (br + 1), 128 * bc:128 * (bc + 1)], ref.numpy())
 
 
-def _fp8_layer(E=3, k=2, T=5, d=256, f=256, fs=0, seed=30):
+def _skew_blocks(t: torch.Tensor, row_scale: float, col_scale: float) -> torch.Tensor:
+    """Scale the second 128-row block by row_scale and the second 128-column block by
+    col_scale (powers of two: exact in bf16), so neighbouring blocks get different,
+    asymmetric scales and a block-index slip changes the result."""
+    t = t.clone()
+    t[..., 128:256, :] *= row_scale
+    t[..., :, 128:256] *= col_scale
+    return t
+
+
+def _fp8_layer(E=3, k=2, T=5, d=256, f=256, fs=0, seed=30, skew=False):
     s = wl.LayerShape("p8", T=T, d=d, f=f, E=E, k=k, alpha=1.0, f_shared=fs)
     inp = wl.make_inputs(s, seed=seed)
+    if skew:
+        inp["x"] = inp["x"].clone()
+        inp["x"][:, 128:256] *= 32.0
+        for n in ("W1", "W3", "Ws1", "Ws3"):
+            if inp.get(n) is not None:
+                inp[n] = _skew_blocks(inp[n], 0.125, 4.0)
+        for n in ("W2", "Ws2"):
+            if inp.get(n) is not None:
+                inp[n] = _skew_blocks(inp[n], 0.0625, 8.0)
     xq, sx = oracle.quantize_rows_fp8(_bits(inp["x"]))
     Q = {}
     for n in ("W1", "W3", "W2"):
@@ -390,8 +409,11 @@ def _requant_h(h):
 
 def pin_fp8_ffn_expert_major():
     """Expert-major evaluation with the library's e4m3 decode, float64 matmuls, and the
-    library cast for the requantisation of h; shared expert included."""
-    s, inp, xq, sx, Q, sh = _fp8_layer(fs=128)
+    library cast for the requantisation of h; shared expert included.  Neighbouring
+    128-wide blocks of x and of every weight differ by powers of two, so each block
+    scale is used where it belongs."""
+    s, inp, xq, sx, Q, sh = _fp8_layer(fs=128, skew=True)
+    assert len(np.unique(sx[:, :2])) > 1 and not np.allclose(Q["W2"][0][1], Q["W2"][0][1].T)
     idx = wl.random_routing(s.T, s.E, s.k, 1.0, 3).numpy()
     w = wl.random_gates(s.T, s.k, 3).numpy().astype(np.float64)
     y = oracle.moe_ffn_fp8(xq, sx, [q for q, _ in Q["W1"]], [c for _, c in Q["W1"]], [q for q, _ in Q["W3"]],

@@ -45,6 +45,11 @@ MUTANTS = {
                               "while (amax <= ldexp(448.0, e - 1) && e > -160)"),
     "fp8_exponent_bias": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
     "fp8_activation_scale_dropped": ("double xc = e4m3_value(xq[c]) * sx[c / 128];", "double xc = e4m3_value(xq[c]);"),
+    "fp8_activation_first_block_scale": ("double xc = e4m3_value(xq[c]) * sx[c / 128];",
+                                         "double xc = e4m3_value(xq[c]) * sx[0];"),
+    "fp8_h_requant_block0_amax": ("amax = fmax(amax, fabs(h[b * 128 + r]));", "amax = fmax(amax, fabs(h[r]));"),
+    "fp8_down_scale_transposed": ("z += e4m3_value(W2q[c * f + r]) * s2[(c / 128) * fb + r / 128] * h[r];",
+                                  "z += e4m3_value(W2q[c * f + r]) * s2[(r / 128) * fb + c / 128] * h[r];"),
 }
 
 
