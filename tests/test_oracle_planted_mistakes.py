@@ -32,6 +32,11 @@ MUTANTS = {
     "permutation_unstable": ("for (int64_t q = 0; q < P; q++) {      /* ascending q keeps each segment stable */",
                              "for (int64_t q = P - 1; q >= 0; q--) {"),
     "shared_expert_dropped": ("if (J->fs > 0)\n            expert_ffn_add", "if (0)\n            expert_ffn_add"),
+    "up_uses_gate_weights": ("u += bf16_value(W3[r * d + c]) * xc;", "u += bf16_value(W1[r * d + c]) * xc;"),
+    "gate_proj_transposed": ("g += bf16_value(W1[r * d + c]) * xc;", "g += bf16_value(W1[c * f + r]) * xc;"),
+    "shared_expert_gated": ("expert_ffn_add(J->Ws1, J->Ws3, J->Ws2, xt, J->d, J->fs, 1.0, h, y);",
+                            "expert_ffn_add(J->Ws1, J->Ws3, J->Ws2, xt, J->d, J->fs, J->w[t * J->k], h, y);"),
+    "gate_of_first_pair_for_all": ("J->f, J->w[t * J->k + j], h, y);", "J->f, J->w[t * J->k], h, y);"),
     "x_row_stride": ("const uint16_t *xt = J->x + t * J->d;", "const uint16_t *xt = J->x + t;"),
     "fp8_h_requant_dropped": ("h[b * 128 + r] = e4m3_value(oracle_e4m3_encode_fast(h[b * 128 + r] / sc)) * sc;",
                               "h[b * 128 + r] = h[b * 128 + r];"),
