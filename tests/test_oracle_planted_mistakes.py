@@ -37,6 +37,11 @@ MUTANTS = {
     "shared_expert_gated": ("expert_ffn_add(J->Ws1, J->Ws3, J->Ws2, xt, J->d, J->fs, 1.0, h, y);",
                             "expert_ffn_add(J->Ws1, J->Ws3, J->Ws2, xt, J->d, J->fs, J->w[t * J->k], h, y);"),
     "gate_of_first_pair_for_all": ("J->f, J->w[t * J->k + j], h, y);", "J->f, J->w[t * J->k], h, y);"),
+    "router_weights_transposed": ("s += bf16_value(x[t * d + c]) * bf16_value(Wg[e * d + c]);",
+                                  "s += bf16_value(x[t * d + c]) * bf16_value(Wg[c * E + e]);"),
+    "bias_subtracted": ("s += (double)bias[e];", "s -= (double)bias[e];"),
+    "perm_holds_token_not_pair": ("perm[pos] = (int32_t)q;", "perm[pos] = (int32_t)(q / k * k);"),
+    "inv_perm_is_perm": ("inv_perm[q] = pos;", "inv_perm[q] = (int32_t)q;"),
     "x_row_stride": ("const uint16_t *xt = J->x + t * J->d;", "const uint16_t *xt = J->x + t;"),
     "fp8_h_requant_dropped": ("h[b * 128 + r] = e4m3_value(oracle_e4m3_encode_fast(h[b * 128 + r] / sc)) * sc;",
                               "h[b * 128 + r] = h[b * 128 + r];"),
