@@ -248,6 +248,35 @@ def pin_hand_worked_layer():
     assert np.allclose(out_s[0], [y[0] + hs * 1.0, y[1] + hs * 2.0], rtol=1e-14, atol=0)
 
 
+def pin_hand_worked_fp8_layer():
+    """An FP8 expert FFN small enough to work by hand (tests/golden/hand_worked_fp8_layer.json):
+    the scale choice, the round to nearest of h's requantisation and the absolute output."""
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "hand_worked_fp8_layer.json")
+    g = json.load(open(path))
+    d, f, split = g["d"], g["f"], g["W2_split_row"]
+    bf = lambda a: torch.tensor(a, dtype=torch.float32).to(torch.bfloat16)
+    x = bf(np.full((1, d), g["x_fill"]))
+    W1 = bf(np.full((f, d), g["W1_fill"]))
+    W3 = bf(np.full((f, d), g["W3_fill"]))
+    W2 = np.full((d, f), g["W2_rows_lo"])
+    W2[split:] = g["W2_rows_hi"]
+    W2 = bf(W2)
+    xq, sx = oracle.quantize_rows_fp8(_bits(x))
+    W1q, s1 = oracle.quantize_blocks_fp8(_bits(W1))
+    W3q, s3 = oracle.quantize_blocks_fp8(_bits(W3))
+    W2q, s2 = oracle.quantize_blocks_fp8(_bits(W2))
+    exp = g["expected_scales"]
+    assert (sx[0, 0], s1[0, 0], s3[0, 0], s2[0, 0]) == (exp["x"], exp["W1"], exp["W3"], exp["W2"])
+    assert oracle.e4m3_decode(int(xq[0, 0])) == 256.0 and oracle.e4m3_decode(int(W1q[0, 0])) == 256.0
+    # h = silu(1) * 2 = 1.4621...; / 2^-8 = 374.3 -> nearest e4m3 value 384 -> 1.5
+    assert oracle.fp8_block_scale(2.0 / (1.0 + math.exp(-1.0))) == 2.0 ** -8
+    y = oracle.moe_ffn_fp8(xq, sx, [W1q], [s1], [W3q], [s3], [W2q], [s2], np.zeros((1, 1), dtype=np.int32),
+                           np.ones((1, 1)))
+    assert np.all(y[0, :split] == g["expected_y_lo"]) and np.all(y[0, split:] == g["expected_y_hi"])
+
+
 def pin_empty_batch():
     s, inp = _small_layer(T=0, E=3, k=2, seed=13)
     res = oracle.moe_layer(_bits(inp["x"]), _bits(inp["Wg"]), inp["bias"].numpy(), _bits(inp["W1"]),
