@@ -136,3 +136,26 @@ def test_fp8_deterministic():
     a = moe.moe_layer_forward_fp8(d["x"], d["Wg"], d["bias"], Q, s.k, ws)
     b = moe.moe_layer_forward_fp8(d["x"], d["Wg"], d["bias"], Q, s.k, ws)
     assert torch.equal(a, b)
+
+
+def test_fp8_hand_worked_layer_exact():
+    """The hand-worked FP8 layer of tests/golden/hand_worked_fp8_layer.json through the C ABI:
+    every intermediate is exact in fp32, so the GPU reproduces y = 1.5 / -3.0 exactly."""
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hand_worked_fp8_layer.json")))
+    d, f, split = g["d"], g["f"], g["W2_split_row"]
+    bf = lambda a: torch.tensor(a, dtype=torch.float32).to(torch.bfloat16).to(DEV)
+    x = bf(np.full((1, d), g["x_fill"]))
+    W2 = np.full((1, d, f), g["W2_rows_lo"])
+    W2[:, split:] = g["W2_rows_hi"]
+    w = {"W1": bf(np.full((1, f, d), g["W1_fill"])), "W3": bf(np.full((1, f, d), g["W3_fill"])), "W2": bf(W2)}
+    Wg = bf(np.zeros((1, d)))
+    bias = torch.zeros(1, dtype=torch.float32, device=DEV)
+    Q = moe.quantize_layer_fp8(w)
+    ws = moe.new_workspace_fp8(1, d, f, 1, 1)
+    out = moe.moe_layer_forward_fp8(x, Wg, bias, Q, 1, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_error(ws) == 0
+    y = out.float().cpu().numpy()[0]
+    assert np.all(y[:split] == g["expected_y_lo"]) and np.all(y[split:] == g["expected_y_hi"])
