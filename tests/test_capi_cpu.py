@@ -169,3 +169,20 @@ def test_workspace_tensors_disjoint_aligned_inside(L, T, d, f, E, k, fs, fp8):
         assert a1 <= b0, f"{an} overlaps {bn}"
     out = C.c_void_p(0)
     assert fn(C.c_void_p(base), T, d, f, E, k, fs, len(layout), C.byref(out)) != 0   # past the last tensor
+
+
+def test_status_and_error_codes_agree_across_header_binding_and_library(L):
+    src = open(HEADER).read()
+    defs = {m.group(1): int(m.group(2)) for m in re.finditer(r"#define (MOE_(?:OK|ERR_\w+|DEVERR_\w+))\s+\(?(-?\d+)u?\)?", src)}
+    assert defs["MOE_OK"] == moe.MOE_OK
+    for name, val in defs.items():
+        if name.startswith("MOE_ERR") or name == "MOE_OK":
+            assert val in moe.STATUS, name
+            assert L.moe_status_string(val).decode() == moe.STATUS[val], name
+        else:
+            assert getattr(moe, name[len("MOE_"):]) == val, name
+    kernel = open(os.path.join(ROOT, "grouped_gemm_02_b200", "csrc", "common.cuh")).read()
+    for name, val in defs.items():
+        if name.startswith("MOE_DEVERR"):
+            m = re.search(name[len("MOE_"):] + r"\s*=\s*(\d+)", kernel)
+            assert m and int(m.group(1)) == val, name
