@@ -52,7 +52,9 @@ def load(path: str) -> C.CDLL:
     L.oracle_quantize_blocks_fp8.argtypes = [u16p, i64, i64, u8p, f64p]
     L.oracle_moe_ffn_fp8.argtypes = [u8p, f64p, u8pp, f64pp, u8pp, f64pp, u8pp, f64pp, i64, i64, i64, i32p, f64p,
                                      i64, u8p, f64p, u8p, f64p, u8p, f64p, i64, C.POINTER(i64), i64, f64p, C.c_int]
-    for fn in ("oracle_quantize_rows_fp8", "oracle_quantize_blocks_fp8", "oracle_moe_ffn_fp8"):
+    L.oracle_expert_h_fp8.argtypes = [u8p, f64p, u8p, f64p, u8p, f64p, i64, i64, u8p, f64p]
+    for fn in ("oracle_quantize_rows_fp8", "oracle_quantize_blocks_fp8", "oracle_moe_ffn_fp8",
+               "oracle_expert_h_fp8"):
         getattr(L, fn).restype = C.c_int
     return L
 
@@ -279,3 +281,22 @@ def moe_ffn_fp8(xq, sx, W1q, s1, W3q, s3, W2q, s2, idx, w, shared=None, tokens=N
                                     _ptr(tok, C.c_int64), ntok, _ptr(out, C.c_double), int(nthreads)),
            "moe_ffn_fp8")
     return out
+
+
+def expert_h_fp8(xq, sx, W1q, s1, W3q, s3):
+    """The requantised h of one FP8 expert on one token: h = silu(W1^ x^) * (W3^ x^) in fp64
+    on dequantised operands, then 1 x 128 blocks along f -> (codes [f], scales [f/128]).
+    xq [d] codes with sx [d/128]; W1q/W3q [f, d] with s1/s3 [f/128, d/128]."""
+    xq = np.ascontiguousarray(xq, dtype=np.uint8).ravel()
+    sx = np.ascontiguousarray(sx, dtype=np.float64).ravel()
+    W1q = np.ascontiguousarray(W1q, dtype=np.uint8)
+    W3q = np.ascontiguousarray(W3q, dtype=np.uint8)
+    s1 = np.ascontiguousarray(s1, dtype=np.float64)
+    s3 = np.ascontiguousarray(s3, dtype=np.float64)
+    f, d = W1q.shape
+    hq = np.empty(f, dtype=np.uint8)
+    sh = np.empty(f // 128, dtype=np.float64)
+    _check(lib().oracle_expert_h_fp8(_ptr(W1q, C.c_uint8), _ptr(s1, C.c_double), _ptr(W3q, C.c_uint8),
+                                     _ptr(s3, C.c_double), _ptr(xq, C.c_uint8), _ptr(sx, C.c_double), d, f,
+                                     _ptr(hq, C.c_uint8), _ptr(sh, C.c_double)), "expert_h_fp8")
+    return hq, sh

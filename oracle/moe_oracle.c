@@ -438,14 +438,14 @@ int oracle_quantize_blocks_fp8(const uint16_t *W, int64_t R, int64_t C, uint8_t 
     return ORACLE_OK;
 }
 
-/* One FP8 SwiGLU expert on one token (all fp64 on dequantised values):
- *   g = W1^ x^, u = W3^ x^, h = silu(g) * u,
- *   h^ = h requantised in 1 x 128 blocks along f, y += gate * W2^ h^.
- * W1q/W3q [f,d] with scales [f/128, d/128]; W2q [d,f] with [d/128, f/128];
- * xq [d] with sx [d/128].  h, hq scratch of f doubles / f bytes. */
-static void expert_ffn_fp8_add(const uint8_t *W1q, const double *s1, const uint8_t *W3q, const double *s3,
-                               const uint8_t *W2q, const double *s2, const uint8_t *xq, const double *sx,
-                               int64_t d, int64_t f, double gate, double *h, double *y)
+/* The first half of one FP8 SwiGLU expert on one token (fp64 on dequantised
+ * values): g = W1^ x^, u = W3^ x^, h = silu(g) * u, then h requantised in
+ * 1 x 128 blocks along f -> codes hq [f] and scales sh [f/128].
+ * W1q/W3q [f,d] with scales [f/128, d/128]; xq [d] with sx [d/128]; h is
+ * scratch of f doubles. */
+static void expert_h_fp8(const uint8_t *W1q, const double *s1, const uint8_t *W3q, const double *s3,
+                         const uint8_t *xq, const double *sx, int64_t d, int64_t f, double *h, uint8_t *hq,
+                         double *sh)
 {
     const int64_t db = d / 128, fb = f / 128;
     for (int64_t r = 0; r < f; r++) {
@@ -462,15 +462,45 @@ static void expert_ffn_fp8_add(const uint8_t *W1q, const double *s1, const uint8
         for (int64_t r = 0; r < 128; r++)
             amax = fmax(amax, fabs(h[b * 128 + r]));
         double sc = oracle_fp8_block_scale(amax);
+        sh[b] = sc;
         for (int64_t r = 0; r < 128; r++)
-            h[b * 128 + r] = e4m3_value(oracle_e4m3_encode_fast(h[b * 128 + r] / sc)) * sc;
+            hq[b * 128 + r] = oracle_e4m3_encode_fast(h[b * 128 + r] / sc);
     }
+}
+
+/* One FP8 SwiGLU expert on one token: h^ from expert_h_fp8, then
+ * y += gate * W2^ h^ (W2q [d,f] with scales [d/128, f/128]).  h, hq, sh are
+ * scratch of f doubles, f bytes and f/128 doubles. */
+static void expert_ffn_fp8_add(const uint8_t *W1q, const double *s1, const uint8_t *W3q, const double *s3,
+                               const uint8_t *W2q, const double *s2, const uint8_t *xq, const double *sx,
+                               int64_t d, int64_t f, double gate, double *h, uint8_t *hq, double *sh, double *y)
+{
+    const int64_t fb = f / 128;
+    expert_h_fp8(W1q, s1, W3q, s3, xq, sx, d, f, h, hq, sh);
+    for (int64_t r = 0; r < f; r++)
+        h[r] = e4m3_value(hq[r]) * sh[r / 128];
     for (int64_t c = 0; c < d; c++) {
         double z = 0.0;
         for (int64_t r = 0; r < f; r++)
             z += e4m3_value(W2q[c * f + r]) * s2[(c / 128) * fb + r / 128] * h[r];
         y[c] += gate * z;
     }
+}
+
+/* The requantised h of one FP8 expert on one token (the intermediate the
+ * down projection reads): codes hq [f] and scales sh [f/128].  W1q/W3q [f,d]
+ * with s1/s3 [f/128, d/128]; xq [d] with sx [d/128]; d, f multiples of 128. */
+int oracle_expert_h_fp8(const uint8_t *W1q, const double *s1, const uint8_t *W3q, const double *s3,
+                        const uint8_t *xq, const double *sx, int64_t d, int64_t f, uint8_t *hq, double *sh)
+{
+    if (d <= 0 || f <= 0 || d % 128 || f % 128 || !W1q || !s1 || !W3q || !s3 || !xq || !sx || !hq || !sh)
+        return ORACLE_EARG;
+    double *h = (double *)malloc((size_t)f * sizeof(double));
+    if (!h)
+        return ORACLE_ENOMEM;
+    expert_h_fp8(W1q, s1, W3q, s3, xq, sx, d, f, h, hq, sh);
+    free(h);
+    return ORACLE_OK;
 }
 
 typedef struct {
@@ -495,8 +525,15 @@ static void *ffn8_worker(void *arg)
 {
     ffn8_job *J = (ffn8_job *)arg;
     int64_t hlen = J->f > J->fs ? J->f : J->fs;
-    double *h = (double *)malloc((size_t)(hlen > 0 ? hlen : 1) * sizeof(double));
-    if (!h) {
+    if (hlen <= 0)
+        hlen = 128;
+    double *h = (double *)malloc((size_t)hlen * sizeof(double));
+    uint8_t *hq = (uint8_t *)malloc((size_t)hlen);
+    double *sh = (double *)malloc((size_t)(hlen / 128) * sizeof(double));
+    if (!h || !hq || !sh) {
+        free(h);
+        free(hq);
+        free(sh);
         J->status = ORACLE_ENOMEM;
         return NULL;
     }
@@ -513,15 +550,20 @@ static void *ffn8_worker(void *arg)
             if (e < 0 || e >= J->E || !J->W1q[e] || !J->W3q[e] || !J->W2q[e]) {
                 J->status = ORACLE_ERANGE;
                 free(h);
+                free(hq);
+                free(sh);
                 return NULL;
             }
             expert_ffn_fp8_add(J->W1q[e], J->s1[e], J->W3q[e], J->s3[e], J->W2q[e], J->s2[e], xt, st, J->d,
-                               J->f, J->w[t * J->k + j], h, y);
+                               J->f, J->w[t * J->k + j], h, hq, sh, y);
         }
         if (J->fs > 0)
-            expert_ffn_fp8_add(J->Ws1q, J->ss1, J->Ws3q, J->ss3, J->Ws2q, J->ss2, xt, st, J->d, J->fs, 1.0, h, y);
+            expert_ffn_fp8_add(J->Ws1q, J->ss1, J->Ws3q, J->ss3, J->Ws2q, J->ss2, xt, st, J->d, J->fs, 1.0, h, hq,
+                               sh, y);
     }
     free(h);
+    free(hq);
+    free(sh);
     return NULL;
 }
 

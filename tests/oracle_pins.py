@@ -464,6 +464,39 @@ def pin_fp8_ffn_expert_major():
     assert np.allclose(y, ref, rtol=1e-10, atol=1e-12)
 
 
+def pin_fp8_expert_h():
+    """The requantised h of one FP8 expert on one token (what the down projection reads):
+    codes and scales against float64 matmuls on the library's e4m3 decode and the library's
+    fp64 -> e4m3 cast, on skewed blocks; and the hand-worked fixture's h = 1.5 exactly."""
+    s, inp, xq, sx, Q, _ = _fp8_layer(skew=True)
+    xh = _dq(xq, sx, 1, 128)
+    for e in range(s.E):
+        (W1q, s1), (W3q, s3) = Q["W1"][e], Q["W3"][e]
+        g = xh @ _dq(W1q, s1).T
+        u = xh @ _dq(W3q, s3).T
+        h = torch.nn.functional.silu(torch.from_numpy(g)).numpy() * u
+        for t in range(s.T):
+            hq, sh = oracle.expert_h_fp8(xq[t], sx[t], W1q, s1, W3q, s3)
+            for b in range(s.f // 128):
+                blk = h[t, 128 * b:128 * (b + 1)]
+                sc = oracle.fp8_block_scale(np.abs(blk).max())
+                assert sh[b] == sc
+                ref = torch.from_numpy(blk / sc).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+                assert np.array_equal(hq[128 * b:128 * (b + 1)], ref), (e, t, b)
+    # the hand-worked layer: h = 2 silu(1) = 1.462..., scale 2^-8, code of 384
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hand_worked_fp8_layer.json")))
+    d, f = g["d"], g["f"]
+    bf = lambda a: torch.tensor(a, dtype=torch.float32).to(torch.bfloat16)
+    xq, sx = oracle.quantize_rows_fp8(_bits(bf(np.full((1, d), g["x_fill"]))))
+    W1q, s1 = oracle.quantize_blocks_fp8(_bits(bf(np.full((f, d), g["W1_fill"]))))
+    W3q, s3 = oracle.quantize_blocks_fp8(_bits(bf(np.full((f, d), g["W3_fill"]))))
+    hq, sh = oracle.expert_h_fp8(xq[0], sx[0], W1q, s1, W3q, s3)
+    assert np.all(sh == 2.0 ** -8)
+    assert all(oracle.e4m3_decode(int(c)) * sh[0] == g["expected_h_after_requant"] for c in hq)
+
+
 def pin_fp8_ffn_exact_operands_match_bf16_path():
     """With weights and activations that e4m3 holds exactly (scales 1) and h values that the
     requantisation keeps exactly, the FP8 FFN equals the bf16 FFN on the same values."""

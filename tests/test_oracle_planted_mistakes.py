@@ -43,8 +43,10 @@ MUTANTS = {
     "perm_holds_token_not_pair": ("perm[pos] = (int32_t)q;", "perm[pos] = (int32_t)(q / k * k);"),
     "inv_perm_is_perm": ("inv_perm[q] = pos;", "inv_perm[q] = (int32_t)q;"),
     "x_row_stride": ("const uint16_t *xt = J->x + t * J->d;", "const uint16_t *xt = J->x + t;"),
-    "fp8_h_requant_dropped": ("h[b * 128 + r] = e4m3_value(oracle_e4m3_encode_fast(h[b * 128 + r] / sc)) * sc;",
-                              "h[b * 128 + r] = h[b * 128 + r];"),
+    "fp8_h_requant_dropped": ("h[r] = e4m3_value(hq[r]) * sh[r / 128];", "h[r] = h[r];"),
+    "fp8_h_scale_not_stored": ("sh[b] = sc;", "sh[b] = 1.0;"),
+    "fp8_h_codes_unscaled": ("hq[b * 128 + r] = oracle_e4m3_encode_fast(h[b * 128 + r] / sc);",
+                             "hq[b * 128 + r] = oracle_e4m3_encode_fast(h[b * 128 + r]);"),
     "fp8_weight_scale_transposed": ("g += e4m3_value(W1q[r * d + c]) * s1[(r / 128) * db + c / 128] * xc;",
                                     "g += e4m3_value(W1q[r * d + c]) * s1[(c / 128) * db + r / 128] * xc;"),
     "fp8_ties_away_from_zero": ("double m = nearbyint((2.0 * frac - 1.0) * 8.0);",
