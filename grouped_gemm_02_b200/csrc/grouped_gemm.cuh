@@ -58,6 +58,7 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "schedule.h"
 
 namespace moe {
 
@@ -238,37 +239,12 @@ __device__ __forceinline__ bool bounded_count_wait(const int* cnt, int need, Sme
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
-// The i-th tile of this CTA, or -1.  Every mode but MODE_FUSED deals tiles
-// round-robin.  MODE_FUSED deals its G gate/up tiles round-robin; when G is
-// not a multiple of the grid, the SMs left one gate/up tile short first take
-// `comp` down tiles each (one gate/up tile weighs about `comp` down tiles), and
-// the remaining down tiles are dealt round-robin.  The compensating tiles are
-// the first down tiles, whose blocks' gate/up tiles ran in the first round.
+// The i-th tile of this CTA, or -1: the balanced deal of schedule.h in
+// MODE_FUSED, round-robin in every other mode.
 template <int MODE>
 __device__ __forceinline__ int cta_tile(int i, int total, int G, int comp)
 {
-    const int b = blockIdx.x, grid = gridDim.x;
-    if (MODE != MODE_FUSED) {
-        const int t = b + grid * i;
-        return t < total ? t : -1;
-    }
-    const int D = total - G;
-    const int grem = G % grid;
-    const int gb = G / grid + (b < grem ? 1 : 0);
-    if (i < gb) return b + grid * i;
-    int j = i - gb;
-    int comp_total = 0, my_comp = 0, comp0 = 0;
-    if (grem > 0) {
-        comp_total = min(D, (grid - grem) * comp);
-        if (b >= grem) {
-            comp0 = (b - grem) * comp;
-            my_comp = max(0, min(comp, comp_total - comp0));
-        }
-    }
-    if (j < my_comp) return G + comp0 + j;
-    j -= my_comp;
-    const int dj = comp_total + b + grid * j;
-    return dj < D ? G + dj : -1;
+    return deal_tile((int)blockIdx.x, (int)gridDim.x, i, total, G, comp, MODE == MODE_FUSED);
 }
 
 // Walks this CTA's (tile, k-block) sequence in order; shared by the two
@@ -446,6 +422,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 ptx::grid_dep_wait();
             }
+            // After the wait, never before it: the layer's later kernels read data
+            // written two launches back (the combine reads inv_perm before its own
+            // wait), which holds only if every kernel waits before it triggers.
             ptx::grid_dep_launch();
             // pass 2: the same sequence again; the first `pre` stages only need their token tiles
             int s = 0, n = 0;
