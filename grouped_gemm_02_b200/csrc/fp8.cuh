@@ -516,6 +516,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 ptx::grid_dep_wait();
             }
+            // After the wait, never before it: the layer's later kernels read data
+            // written two launches back (the combine reads inv_perm before its own
+            // wait), which holds only if every kernel waits before it triggers.
             ptx::grid_dep_launch();
             int s = 0, n = 0;
             uint32_t ph = 0;

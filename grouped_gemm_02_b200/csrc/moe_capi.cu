@@ -42,6 +42,7 @@ std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::atomic<int64_t> g_launches{0};
+thread_local int64_t t_launches = 0;   // kernels this host thread has launched (orders a layer's launches)
 thread_local cudaEvent_t t_phase[6] = {};
 thread_local bool t_phase_armed = false;
 
@@ -65,6 +66,7 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     g_launches.fetch_add(1, std::memory_order_relaxed);
+    ++t_launches;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
@@ -242,7 +244,7 @@ int run_topk(const TopkSource& s, int T, int E, int k, int32_t* idx, float* w, u
 int run_permute(const int32_t* idx, const bf16* x, int T, int d, int E, int k, int32_t* counts, int32_t* offsets,
                 int32_t* perm, int32_t* inv_perm, bf16* xp, uint32_t* err, int32_t* block_counts, int32_t* plan,
                 int f, int shared_rows, int fs, int sms, cudaStream_t st, int unit_rows = kTileRows,
-                int m1_rows = 64)
+                int m1_rows = 64, int64_t* inv_perm_launch = nullptr)
 {
     const int64_t P = (int64_t)T * k;
     const int nb = hist_blocks(P);
@@ -254,6 +256,7 @@ int run_permute(const int32_t* idx, const bf16* x, int T, int d, int E, int k, i
         e = launch(scatter_kernel, dim3(nb), dim3(256), 0, st, idx, P, E, (const int32_t*)block_counts, perm,
                    inv_perm);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (inv_perm_launch) *inv_perm_launch = t_launches;
     if (!xp) return MOE_OK;
     const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)sms * 16));
     return status_of(launch(gather_rows_kernel, dim3(blocks), dim3(256), 0, st, x, (const int32_t*)perm,
@@ -351,9 +354,15 @@ int run_gemms(const GemmOperands& o, const int32_t* plan, bool plan_ready, uint3
                             a2, b2, a2s, a2s, b2s, a2, b2, a2s, b2s, g2, g2));
 }
 
+// inv_perm_launch: this thread's launch count right after the kernel that wrote
+// inv_perm (0: unknown).  The combine may read inv_perm before its
+// griddepcontrol.wait only when two or more launches separate it from that
+// kernel: every kernel waits before it lets its successor start, so the
+// writer has then completed before the combine begins.
 int run_combine(const bf16* y_p, const int32_t* inv_perm, const bf16* ys, int T, int k, int d, bf16* out,
-                cudaStream_t st, bool inv_perm_ready = false)
+                cudaStream_t st, int64_t inv_perm_launch = 0)
 {
+    const bool inv_perm_ready = inv_perm_launch > 0 && t_launches - inv_perm_launch >= 2;
     constexpr int kThreads = 64;
     const int nvec = d / 8;
     const int gy = std::max(1, std::min((nvec + kThreads - 1) / kThreads, 65535));
@@ -529,6 +538,7 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
 
     const bool prof = t_phase_armed;   // the armed events serve this call only
     t_phase_armed = false;
+    int64_t inv_perm_launch = 0;
     phase_mark(prof, 0, st);
     RouterSplit rs;
     if ((rc = run_router_gemm(xb, reinterpret_cast<const bf16*>(Wg), bias, iT, id, iE, logits, partials, err,
@@ -544,6 +554,7 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
                    perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared, (int)kTileRows, 64, err) !=
             cudaSuccess)
             return MOE_ERR_CUDA;
+        inv_perm_launch = t_launches;
         const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)dev->sm_count * 16));
         if (launch(gather_rows_kernel, dim3(blocks), dim3(256), 0, st, xb, (const int32_t*)perm,
                    (const int32_t*)offsets, iE, ik, id, xp) != cudaSuccess)
@@ -551,7 +562,7 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     } else {
         if ((rc = run_permute(idx, xb, iT, id, iE, ik, counts, offsets, perm, inv_perm, xp, err,
                               at<int32_t>(ws, L.block_counts), plan, (int)f, shared_rows, (int)f_shared,
-                              dev->sm_count, st)))
+                              dev->sm_count, st, kTileRows, 64, &inv_perm_launch)))
             return rc;
     }
     GemmOperands o{};
@@ -579,7 +590,7 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     // the plan was written two or more launches before the gate/up GEMM (the gather is in between)
     if ((rc = run_gemms(o, plan, /*plan_ready=*/true, err, dev->sm_count, st, prof))) return rc;
     phase_mark(prof, 4, st);
-    rc = run_combine(y_p, inv_perm, ys, iT, ik, id, reinterpret_cast<bf16*>(out), st, /*inv_perm_ready=*/true);
+    rc = run_combine(y_p, inv_perm, ys, iT, ik, id, reinterpret_cast<bf16*>(out), st, inv_perm_launch);
     phase_mark(prof, 5, st);
     return rc;
 }
@@ -607,9 +618,9 @@ int moe_workspace_tensor(void* ws, int64_t T, int64_t d, int64_t f, int64_t E, i
     if (!ws || !ptr || T < 0 || d < 0 || f < 0 || E < 1 || E > kMaxExperts || k < 1 || k > kMaxTopK || f_shared < 0)
         return MOE_ERR_ARG;
     const WsLayout L = ws_layout(T, d, f, E, k, f_shared);
-    const size_t offs[12] = {L.logits, L.topk_idx, L.topk_w, L.counts, L.offsets, L.perm,
-                             L.inv_perm, L.xp, L.h, L.y_p, L.hs, L.ys};
-    if (which < 0 || which >= 12) return MOE_ERR_ARG;
+    const size_t offs[13] = {L.logits, L.topk_idx, L.topk_w, L.counts, L.offsets, L.perm,
+                             L.inv_perm, L.xp, L.h, L.y_p, L.hs, L.ys, L.plan};
+    if (which < 0 || which >= 13) return MOE_ERR_ARG;
     *ptr = static_cast<uint8_t*>(ws) + offs[which];
     return MOE_OK;
 }
@@ -805,9 +816,9 @@ int moe_workspace_tensor_fp8(void* ws, int64_t T, int64_t d, int64_t f, int64_t 
     if (!ws || !ptr || T < 0 || d < 0 || f < 0 || E < 1 || E > kMaxExperts || k < 1 || k > kMaxTopK || f_shared < 0)
         return MOE_ERR_ARG;
     const WsLayoutFp8 L = ws_layout_fp8(T, d, f, E, k, f_shared);
-    const size_t offs[18] = {L.logits, L.topk_idx, L.topk_w, L.counts, L.offsets, L.perm, L.inv_perm, L.x8, L.sx,
-                             L.xp8, L.sxp, L.h8, L.sh, L.y_p, L.hs8, L.shs, L.ys, L.sxT};
-    if (which < 0 || which >= 18) return MOE_ERR_ARG;
+    const size_t offs[19] = {L.logits, L.topk_idx, L.topk_w, L.counts, L.offsets, L.perm, L.inv_perm, L.x8, L.sx,
+                             L.xp8, L.sxp, L.h8, L.sh, L.y_p, L.hs8, L.shs, L.ys, L.sxT, L.ctrl.plan};
+    if (which < 0 || which >= 19) return MOE_ERR_ARG;
     *ptr = static_cast<uint8_t*>(ws) + offs[which];
     return MOE_OK;
 }
@@ -855,6 +866,7 @@ int moe_layer_forward_fp8(const moe_bf16* x, const moe_bf16* Wg, const float* bi
 
     const bool prof = t_phase_armed;
     t_phase_armed = false;
+    int64_t inv_perm_launch = 0;
     phase_mark(prof, 0, st);
     RouterSplit rs;
     if ((rc = run_router_gemm(xb, reinterpret_cast<const bf16*>(Wg), bias, iT, id, iE, logits, partials, err,
@@ -869,9 +881,10 @@ int moe_layer_forward_fp8(const moe_bf16* x, const moe_bf16* Wg, const float* bi
                    perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared, kFp8TileRows, 128, err) !=
             cudaSuccess)
             return MOE_ERR_CUDA;
+        inv_perm_launch = t_launches;
     } else if ((rc = run_permute(idx, xb, iT, id, iE, ik, counts, offsets, perm, inv_perm, nullptr, err,
                                  at<int32_t>(ws, L.ctrl.block_counts), plan, (int)f, shared_rows, (int)f_shared,
-                                 dev->sm_count, st, kFp8TileRows, 128))) {
+                                 dev->sm_count, st, kFp8TileRows, 128, &inv_perm_launch))) {
         return rc;
     }
     const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)dev->sm_count * 16));
@@ -914,7 +927,7 @@ int moe_layer_forward_fp8(const moe_bf16* x, const moe_bf16* Wg, const float* bi
     phase_mark(prof, 2, st);
     if ((rc = run_gemms_fp8(o, plan, err, dev->sm_count, st, prof))) return rc;
     phase_mark(prof, 4, st);
-    rc = run_combine(y_p, inv_perm, o.ys, iT, ik, id, reinterpret_cast<bf16*>(out), st, /*inv_perm_ready=*/true);
+    rc = run_combine(y_p, inv_perm, o.ys, iT, ik, id, reinterpret_cast<bf16*>(out), st, inv_perm_launch);
     phase_mark(prof, 5, st);
     return rc;
 }

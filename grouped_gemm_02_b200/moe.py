@@ -246,7 +246,9 @@ def moe_layer_forward(x, Wg, bias, W1, W3, W2, k: int, ws: torch.Tensor, Ws1=Non
     return out
 
 
-WS_TENSORS = ("logits", "topk_idx", "topk_w", "counts", "offsets", "perm", "inv_perm", "xp", "h", "y_p", "hs", "ys")
+WS_TENSORS = ("logits", "topk_idx", "topk_w", "counts", "offsets", "perm", "inv_perm", "xp", "h", "y_p", "hs", "ys",
+              "plan")
+PLAN_INTS = 8 + 6 * 513 + 2 * 514       # MOE_PLAN_INTS
 
 
 def workspace_views(ws: torch.Tensor, T: int, d: int, f: int, E: int, k: int, f_shared: int = 0):
@@ -256,7 +258,7 @@ def workspace_views(ws: torch.Tensor, T: int, d: int, f: int, E: int, k: int, f_
               "counts": ((E,), torch.int32), "offsets": ((E + 1,), torch.int32), "perm": ((P,), torch.int32),
               "inv_perm": ((P,), torch.int32), "xp": ((P, d), torch.bfloat16), "h": ((P, f), torch.bfloat16),
               "y_p": ((P, d), torch.bfloat16), "hs": ((T if f_shared else 0, f_shared), torch.bfloat16),
-              "ys": ((T if f_shared else 0, d), torch.bfloat16)}
+              "ys": ((T if f_shared else 0, d), torch.bfloat16), "plan": ((PLAN_INTS,), torch.int32)}
     base = ws.data_ptr()
     views = {}
     for i, name in enumerate(WS_TENSORS):
@@ -331,7 +333,7 @@ def moe_layer_forward_fp8(x, Wg, bias, Q: dict, k: int, ws: torch.Tensor, out=No
 
 
 WS_TENSORS_FP8 = ("logits", "topk_idx", "topk_w", "counts", "offsets", "perm", "inv_perm", "x8", "sx", "xp8", "sxp",
-                  "h8", "sh", "y_p", "hs8", "shs", "ys", "sxT")
+                  "h8", "sh", "y_p", "hs8", "shs", "ys", "sxT", "plan")
 
 
 def workspace_views_fp8(ws: torch.Tensor, T: int, d: int, f: int, E: int, k: int, f_shared: int = 0):
@@ -343,7 +345,8 @@ def workspace_views_fp8(ws: torch.Tensor, T: int, d: int, f: int, E: int, k: int
               "xp8": ((P, d), torch.uint8), "sxp": ((d // 128, P4), torch.float32), "h8": ((P, f), torch.uint8),
               "sh": ((f // 128, P4), torch.float32), "y_p": ((P, d), torch.bfloat16),
               "hs8": ((Ts, f_shared), torch.uint8), "shs": ((f_shared // 128, T4 if Ts else 0), torch.float32),
-              "ys": ((Ts, d), torch.bfloat16), "sxT": ((d // 128, T4 if Ts else 0), torch.float32)}
+              "ys": ((Ts, d), torch.bfloat16), "sxT": ((d // 128, T4 if Ts else 0), torch.float32),
+              "plan": ((PLAN_INTS,), torch.int32)}
     base = ws.data_ptr()
     views = {}
     for i, name in enumerate(WS_TENSORS_FP8):

@@ -64,6 +64,9 @@ typedef uint16_t moe_bf16;
 #define MOE_ERR_CUDA (-4)    /* a CUDA launch or attribute call failed */
 #define MOE_ERR_DEVICE (-5)  /* current device is not sm_100 */
 
+/* int32 entries of the tile plan (moe_workspace_tensor which = 12). */
+#define MOE_PLAN_INTS (8 + 6 * 513 + 2 * 514)
+
 /* Device error bits (OR-ed, sticky until moe_clear_device_error). */
 #define MOE_DEVERR_EXPERT_RANGE 1u  /* an expert id outside [0, E): that pair was dropped */
 #define MOE_DEVERR_TIMEOUT 2u       /* a bounded wait inside a kernel gave up; outputs are invalid */
@@ -196,7 +199,7 @@ MOE_API int moe_workspace_size_fp8(int64_t T, int64_t d, int64_t f, int64_t E, i
 /* Device pointers of the FP8 layer intermediates inside its workspace
  * (which: 0 logits, 1 topk_idx, 2 topk_w, 3 counts, 4 offsets, 5 perm,
  * 6 inv_perm, 7 x8, 8 sx, 9 xp8, 10 sxp, 11 h8, 12 sh, 13 y_p, 14 hs8, 15 shs,
- * 16 ys, 17 sxT).  sx is [T, d/128]; the scale arrays the GEMMs read are
+ * 16 ys, 17 sxT, 18 the tile plan).  sx is [T, d/128]; the scale arrays the GEMMs read are
  * K-block-major with rows padded to a multiple of 4 entries: sxp
  * [d/128, P4], sh [f/128, P4], shs [f_shared/128, T4], sxT [d/128, T4]
  * (P4 = T*k and T4 = T rounded up to a multiple of 4).  Host-only arithmetic. */
@@ -233,7 +236,12 @@ MOE_API int64_t moe_launch_counter(void);
 
 /* Device pointers of the layer intermediates inside a layer workspace
  * (which: 0 logits, 1 topk_idx, 2 topk_w, 3 counts, 4 offsets, 5 perm,
- * 6 inv_perm, 7 xp, 8 h, 9 y_p, 10 hs, 11 ys).  Host-only arithmetic. */
+ * 6 inv_perm, 7 xp, 8 h, 9 y_p, 10 hs, 11 ys, 12 the tile plan).  The tile plan is
+ * MOE_PLAN_INTS int32: a header {n_blocks, tiles1, tiles2, n_max, pairs, 3 x 0},
+ * then arrays of 513 entries group, row0, rows, chunk, units, two tile
+ * prefixes of 514 entries (gate/up, down) and 513 per-block counters of
+ * finished gate/up tiles (see the tile plan in the grouped-GEMM comment).
+ * Host-only arithmetic. */
 MOE_API int moe_workspace_tensor(void *ws, int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, int64_t f_shared,
                          int which, void **ptr);
 

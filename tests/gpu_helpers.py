@@ -91,3 +91,99 @@ def sample_tokens(idx: np.ndarray, E: int, n_random: int, seed: int) -> np.ndarr
             toks = np.nonzero((idx == e).any(axis=1))[0][:4]
             pick.update(toks.tolist())
     return np.array(sorted(pick), dtype=np.int64)
+
+
+PLAN_GROUPS = 513          # kMaxGroups: routed experts (<= 512) + the shared expert
+
+
+def decode_plan(plan) -> dict:
+    """The tile plan a layer leaves in its workspace (int32 [MOE_PLAN_INTS]) as host arrays."""
+    p = plan.cpu().numpy() if hasattr(plan, "cpu") else np.asarray(plan)
+    G = PLAN_GROUPS
+    nb, tiles1, tiles2, n_max, pairs = (int(v) for v in p[:5])
+    o = 8
+    out = {"n_blocks": nb, "tiles1": tiles1, "tiles2": tiles2, "n_max": n_max, "pairs": pairs}
+    for name in ("group", "row0", "rows", "chunk", "units"):
+        out[name] = p[o:o + nb].astype(np.int64)
+        o += G
+    out["tb1"] = p[o:o + nb + 1].astype(np.int64)
+    o += G + 1
+    out["tb2"] = p[o:o + nb + 1].astype(np.int64)
+    o += G + 1
+    out["dep"] = p[o:o + nb].astype(np.int64)
+    return out
+
+
+def check_plan(plan: dict, counts: np.ndarray, offsets: np.ndarray, T: int, f: int, d: int, f_shared: int,
+               unit_max: int, m1_rows: int, what: str = "") -> None:
+    """The invariants of a tile plan built from the live histogram:
+    * one block per expert with tokens (+ the shared expert over all T tokens),
+      heaviest first (ties: lower group id);
+    * each block's rows [row0, row0 + rows) are cut into `units` chunks of
+      `chunk` rows, a multiple of 16 and at most unit_max, every chunk non-empty,
+      so the tiles of a block cover its rows exactly once;
+    * the routed blocks' rows tile [0, offsets[E]) exactly once;
+    * the tile prefixes count units x M-tiles of each GEMM, and n_max is the
+      widest chunk."""
+    E = counts.size
+    active = np.nonzero(counts > 0)[0]
+    n_blocks = active.size + (1 if f_shared else 0)
+    assert plan["n_blocks"] == n_blocks, (what, plan["n_blocks"], n_blocks)
+    g, r0, rows, ch, un = plan["group"], plan["row0"], plan["rows"], plan["chunk"], plan["units"]
+    assert sorted(g.tolist()) == sorted(active.tolist() + ([E] if f_shared else [])), what
+    for i in range(n_blocks):
+        if g[i] < E:
+            assert rows[i] == counts[g[i]] and r0[i] == offsets[g[i]], (what, i)
+        else:
+            assert rows[i] == T and r0[i] == 0, (what, i)
+    key = [(-int(rows[i]), int(g[i])) for i in range(n_blocks)]
+    assert key == sorted(key), f"{what}: blocks not heaviest first"
+    assert np.all(ch % 16 == 0) and np.all(ch >= 16) and np.all(ch <= unit_max), what
+    assert np.all(ch * un >= rows) and np.all(ch * (un - 1) < rows), f"{what}: an empty or missing unit"
+    cover = np.zeros(int(offsets[-1]), dtype=np.int64)
+    for i in range(n_blocks):
+        if g[i] == E:
+            continue
+        for u in range(int(un[i])):
+            a = r0[i] + u * ch[i]
+            b = r0[i] + min((u + 1) * ch[i], rows[i])
+            cover[a:b] += 1
+    assert np.all(cover == 1), f"{what}: routed rows not covered exactly once"
+    m1 = np.array([-(-(f if gi < E else f_shared) // m1_rows) for gi in g], dtype=np.int64)
+    m2 = -(-d // 128)
+    assert np.array_equal(plan["tb1"], np.concatenate([[0], np.cumsum(un * m1)])), what
+    assert np.array_equal(plan["tb2"], np.concatenate([[0], np.cumsum(un * m2)])), what
+    assert plan["tiles1"] == plan["tb1"][-1] and plan["tiles2"] == plan["tb2"][-1], what
+    assert plan["n_max"] == (int(ch.max()) if n_blocks else 0), what
+    assert plan["pairs"] == int(offsets[-1]), what
+
+
+def fused_gemms(P: int, f: int) -> bool:
+    """The library's rule: both expert GEMMs in one launch for P <= 256 pairs and f <= 4096."""
+    return P <= 256 and f <= 4096
+
+
+def check_routing(views, s: wl.LayerShape, what: str):
+    """Routing on identical fp32 logits: the oracle's top-k of the GPU's own logits
+    equals the GPU's indices for every token (gates within 1e-6), and counts,
+    offsets, perm and inv_perm equal the oracle's permutation of those indices."""
+    g_L = views["logits"].cpu().numpy()
+    g_idx = views["topk_idx"].cpu().numpy()
+    o_idx, o_w = oracle.topk(g_L, s.k)
+    assert np.array_equal(g_idx, o_idx), f"{what}: top-k differs on identical logits"
+    assert np.max(np.abs(views["topk_w"].cpu().numpy() - o_w)) <= 1e-6, what
+    rc, ro, rp, ri = oracle.permutation(g_idx, s.E)
+    assert np.array_equal(views["counts"].cpu().numpy(), rc), what
+    assert np.array_equal(views["offsets"].cpu().numpy(), ro), what
+    assert np.array_equal(views["perm"].cpu().numpy(), rp), what
+    assert np.array_equal(views["inv_perm"].cpu().numpy(), ri), what
+    return g_L, o_idx, o_w, rc, ro
+
+
+def check_layer_plan(views, s: wl.LayerShape, counts, offsets, unit_max, m1_rows, what):
+    plan = decode_plan(views["plan"])
+    check_plan(plan, counts, offsets, s.T, s.f, s.d, s.f_shared, unit_max, m1_rows, what)
+    # the single launch counts its finished gate/up tiles per block (4 epilogue warps per tile)
+    m1 = np.array([-(-(s.f if g < s.E else s.f_shared) // m1_rows) for g in plan["group"]], dtype=np.int64)
+    need = 4 * plan["units"] * m1 if fused_gemms(s.P, s.f) else np.zeros_like(m1)
+    assert np.array_equal(plan["dep"], need), f"{what}: gate/up tiles published {plan['dep']} != {need}"

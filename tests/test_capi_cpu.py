@@ -126,12 +126,16 @@ def test_product_path_refuses_missing_library(monkeypatch, tmp_path):
 
 # ------------------------------------------------------------------ workspace layout (host arithmetic only)
 
+PLAN_BYTES = moe.PLAN_INTS * 4
+
+
 def _bf16_layout(T, d, f, E, k, fs):
     """Byte sizes and alignments of the layer intermediates, from the header's shapes."""
     P, Ts = T * k, (T if fs else 0)
     return [("logits", T * E * 4, 4), ("topk_idx", P * 4, 4), ("topk_w", P * 4, 4), ("counts", E * 4, 4),
             ("offsets", (E + 1) * 4, 4), ("perm", P * 4, 4), ("inv_perm", P * 4, 4), ("xp", P * d * 2, 256),
-            ("h", P * f * 2, 256), ("y_p", P * d * 2, 256), ("hs", Ts * fs * 2, 256), ("ys", Ts * d * 2, 256)]
+            ("h", P * f * 2, 256), ("y_p", P * d * 2, 256), ("hs", Ts * fs * 2, 256), ("ys", Ts * d * 2, 256),
+            ("plan", PLAN_BYTES, 256)]
 
 
 def _fp8_layout(T, d, f, E, k, fs):
@@ -142,7 +146,7 @@ def _fp8_layout(T, d, f, E, k, fs):
             ("sx", T * (d // 128) * 4, 16), ("xp8", P * d, 256), ("sxp", (d // 128) * P4 * 4, 16),
             ("h8", P * f, 256), ("sh", (f // 128) * P4 * 4, 16), ("y_p", P * d * 2, 256),
             ("hs8", Ts * fs, 256), ("shs", (fs // 128) * (T4 if Ts else 0) * 4, 16), ("ys", Ts * d * 2, 256),
-            ("sxT", (d // 128) * (T4 if Ts else 0) * 4, 16)]
+            ("sxT", (d // 128) * (T4 if Ts else 0) * 4, 16), ("plan", PLAN_BYTES, 256)]
 
 
 @pytest.mark.parametrize("T,d,f,E,k,fs", [(32, 2048, 1024, 64, 8, 0), (1, 256, 512, 8, 2, 0), (37, 7168, 2048, 256, 8, 2048),
@@ -186,3 +190,15 @@ def test_status_and_error_codes_agree_across_header_binding_and_library(L):
         if name.startswith("MOE_DEVERR"):
             m = re.search(name[len("MOE_"):] + r"\s*=\s*(\d+)", kernel)
             assert m and int(m.group(1)) == val, name
+
+
+def test_plan_size_agrees_across_header_binding_and_kernels():
+    src = open(HEADER).read()
+    m = re.search(r"#define MOE_PLAN_INTS \((\d+) \+ (\d+) \* (\d+) \+ (\d+) \* (\d+)\)", src)
+    assert m
+    a, b, c, d_, e = (int(v) for v in m.groups())
+    assert a + b * c + d_ * e == moe.PLAN_INTS
+    common = open(os.path.join(ROOT, "grouped_gemm_02_b200", "csrc", "common.cuh")).read()
+    assert "constexpr int kMaxExperts = 512;" in common
+    assert "kPlanInts = 8 + 6 * kMaxGroups + 2 * (kMaxGroups + 1)" in common
+    assert moe.PLAN_INTS == 8 + 6 * 513 + 2 * 514

@@ -58,6 +58,53 @@ def _oracle_weights(W: torch.Tensor, experts):
     return codes, scales
 
 
+def _e4m3_grid():
+    """Every finite e4m3 value, ascending, and each code's index on that grid."""
+    vals = np.array([oracle.e4m3_decode(c) for c in range(256)])
+    fin = np.isfinite(vals)
+    grid = np.unique(vals[fin])
+    pos = np.full(256, -10**6, dtype=np.int64)
+    pos[fin] = np.searchsorted(grid, vals[fin])
+    return vals, pos
+
+
+def check_h8(views, s, g_idx, tokens, xq, sx, W1q, s1, W3q, s3, sh_w, what):
+    """The GPU's requantised h (codes h8, K-block-major scales sh) for every pair of the
+    sampled tokens against the oracle's: h is formed in fp32 on the GPU and in fp64 in
+    the oracle, so a block's scale may differ only where its amax sits at a power-of-two
+    boundary, and a code by at most one e4m3 step."""
+    vals, pos = _e4m3_grid()
+    inv = views["inv_perm"].cpu().numpy()
+    h8 = views["h8"].cpu().numpy()
+    shg = views["sh"].cpu().numpy()
+    nb = s.f // 128
+    n_blocks = n_scale_diff = 0
+    for i, t in enumerate(tokens):
+        for j in range(s.k):
+            e = int(g_idx[t, j])
+            r = int(inv[t * s.k + j])
+            hq, shq = oracle.expert_h_fp8(xq[i], sx[i], W1q[e], s1[e], W3q[e], s3[e])
+            for b in range(nb):
+                n_blocks += 1
+                gs = float(shg[b, r])
+                if gs != shq[b]:
+                    n_scale_diff += 1
+                    assert gs in (2 * shq[b], shq[b] / 2), f"{what}: h scale {gs} vs {shq[b]}"
+                    continue
+                d = np.abs(pos[h8[r, 128 * b:128 * (b + 1)]] - pos[hq[128 * b:128 * (b + 1)]])
+                assert d.max() <= 1, f"{what}: h code off by {d.max()} steps (token {t}, expert {e})"
+    assert n_scale_diff <= max(1, n_blocks // 100), f"{what}: {n_scale_diff}/{n_blocks} h scales differ"
+    if s.f_shared:
+        hs8 = views["hs8"].cpu().numpy()
+        shs = views["shs"].cpu().numpy()
+        for i, t in enumerate(tokens[:4]):
+            hq, shq = oracle.expert_h_fp8(xq[i], sx[i], *sh_w)
+            for b in range(s.f_shared // 128):
+                if float(shs[b, t]) == shq[b]:
+                    d = np.abs(pos[hs8[t, 128 * b:128 * (b + 1)]] - pos[hq[128 * b:128 * (b + 1)]])
+                    assert d.max() <= 1, f"{what}: shared h code off by {d.max()} steps"
+
+
 def _fp8_layer_check(s: wl.LayerShape, seed: int, n_sample=None, device_inputs=False):
     inp = wl.make_inputs(s, seed=seed, device=DEV if device_inputs else "cpu")
     d_inp = {n: v.to(DEV) for n, v in inp.items()}
@@ -67,24 +114,20 @@ def _fp8_layer_check(s: wl.LayerShape, seed: int, n_sample=None, device_inputs=F
     torch.cuda.synchronize()
     assert moe.moe_get_device_error(ws) == 0
     views = moe.workspace_views_fp8(ws, s.T, s.d, s.f, s.E, s.k, s.f_shared)
-    g_idx = views["topk_idx"].cpu().numpy()
-    g_L = views["logits"].cpu().numpy()
+    what = f"fp8 layer {s}"
+    # routing (the bf16 router, as in the bf16 layer): bit-exact on identical fp32 logits
+    g_L, o_idx, o_w, counts, offsets = H.check_routing(views, s, what)
+    H.check_layer_plan(views, s, counts, offsets, 112, 128, what)
     x_h = inp["x"].cpu()
-    tokens = np.arange(s.T) if n_sample is None else H.sample_tokens(g_idx, s.E, n_sample, seed)
+    tokens = np.arange(s.T) if n_sample is None else H.sample_tokens(o_idx, s.E, n_sample, seed)
+    L64 = oracle.router_logits(H.bits(x_h[tokens]), H.bits(inp["Wg"].cpu()), inp["bias"].cpu().numpy())
+    dL = np.abs(g_L[tokens].astype(np.float64) - L64)
+    assert np.all(dL <= 1e-3 + 1e-3 * np.abs(L64)), f"router logits off by {dL.max()}"
     # activations: GPU codes and scales equal the oracle's
     xq, sx = oracle.quantize_rows_fp8(H.bits(x_h[tokens]))
     assert np.array_equal(views["x8"].cpu().numpy()[tokens], xq)
     assert np.array_equal(views["sx"].cpu().numpy()[tokens].astype(np.float64), sx)
-    # routing (bf16 router, as in the bf16 layer)
-    L64 = oracle.router_logits(H.bits(x_h[tokens]), H.bits(inp["Wg"].cpu()), inp["bias"].cpu().numpy())
-    L32 = L64.astype(np.float32)
-    o_idx, o_w = oracle.topk(L32, s.k)
-    dL = np.abs(g_L[tokens].astype(np.float64) - L64)
-    delta = 4 * dL.max(axis=1) + 1e-6 * (1 + np.abs(L64).max(axis=1))
-    clear = H.clear_margin_tokens(L32.astype(np.float64), s.k, delta)
-    assert np.array_equal(g_idx[tokens][clear], o_idx[clear])
-    keep = clear
-    used = np.unique(o_idx[keep])
+    used = np.unique(o_idx[tokens])
     W1q, s1 = _oracle_weights(inp["W1"], used)
     W3q, s3 = _oracle_weights(inp["W3"], used)
     W2q, s2 = _oracle_weights(inp["W2"], used)
@@ -94,14 +137,17 @@ def _fp8_layer_check(s: wl.LayerShape, seed: int, n_sample=None, device_inputs=F
     assert np.array_equal(Q["W1q"][e0].cpu().numpy(), W1q[e0])
     assert np.array_equal(Q["W1s"][e0 * rows1:(e0 + 1) * rows1].cpu().numpy().astype(np.float64), s1[e0])
     sh = None
+    sh_w = None
     if s.f_shared:
         sh = {}
         for n, key in (("Ws1", "1"), ("Ws3", "3"), ("Ws2", "2")):
             q_, s_ = oracle.quantize_blocks_fp8(H.bits(inp[n].cpu()))
             sh["W%sq" % key], sh["s%s" % key] = q_, s_
-    ref = oracle.moe_ffn_fp8(xq[keep], sx[keep], W1q, s1, W3q, s3, W2q, s2, o_idx[keep], o_w[keep], shared=sh)
-    H.assert_close(out.float().cpu().numpy()[tokens[keep]], ref, f"fp8 layer {s}", atol=1e-2, rtol=FP8_RTOL,
-                   frob=FP8_RTOL)
+        sh_w = (sh["W1q"], sh["s1"], sh["W3q"], sh["s3"])
+    # the requantised h the down projection reads
+    check_h8(views, s, o_idx, tokens, xq, sx, W1q, s1, W3q, s3, sh_w, what)
+    ref = oracle.moe_ffn_fp8(xq, sx, W1q, s1, W3q, s3, W2q, s2, o_idx[tokens], o_w[tokens], shared=sh)
+    H.assert_close(out.float().cpu().numpy()[tokens], ref, what, atol=1e-2, rtol=FP8_RTOL, frob=FP8_RTOL)
 
 
 @pytest.mark.parametrize("name,kw", [

@@ -55,6 +55,27 @@ def test_permute_noalloc_matches_workspace_entry_point():
         torch.cuda.synchronize()
         for name, a, b in zip(("counts", "offsets", "perm", "inv_perm", "xp"), got, ref):
             assert torch.equal(a, b), f"{name} differs from moe_permute (T={T} E={E})"
+    # out-of-range expert ids are dropped as moe_permute drops them: no error word to read,
+    # so the drop shows as offsets[E] == T*k - (dropped pairs) and inv_perm == -1 there
+    T, E, k, d = 300, 64, 4, 128
+    idx = wl.random_routing(T, E, k, 1.0, seed=5)
+    bad = [(3, 1, E + 2), (17, 0, -1), (299, 3, 1 << 20)]
+    for t, j, v in bad:
+        idx[t, j] = v
+    idx = idx.cuda()
+    x = wl.make_inputs(wl.LayerShape("p", T=T, d=d, f=64, E=E, k=k, alpha=1.0), seed=5,
+                       weights=False)["x"].cuda()
+    rc, got = _noalloc(L, idx, x, E, k)
+    assert rc == 0, moe.moe_status_string(rc)
+    ws = moe.new_workspace(T, d, 64, E, k)
+    ref = moe.moe_permute(idx, x, E, ws)
+    torch.cuda.synchronize()
+    counts, offsets, perm, inv, xp = got
+    n_valid = T * k - len(bad)
+    assert int(offsets[E]) == n_valid
+    assert all(int(inv[t * k + j]) == -1 for t, j, _ in bad)
+    assert torch.equal(counts, ref[0]) and torch.equal(offsets, ref[1]) and torch.equal(inv, ref[3])
+    assert torch.equal(perm[:n_valid], ref[2][:n_valid]) and torch.equal(xp, ref[4])
     # a size beyond the static scratch is refused on the host, before any work
     big_T = (65536 // 512 + 1) * 4096 // 8
     rc, _ = _noalloc(L, torch.zeros(big_T, 8, dtype=torch.int32, device="cuda"),
