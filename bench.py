@@ -6,8 +6,15 @@ scan, permutation and row gather, gate/up grouped GEMM with SwiGLU, down
 grouped GEMM, combine) over one batch of seeded synthetic tokens, through
 moe_layer_forward.  Prints ONE JSON line on rank 0.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode64]
-                    [--T ..] [--alpha ..] [--fp8] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--T ..] [--alpha ..] [--E ..] [--fp8] [--impl ours|reference]
+
+With no --workload the line times the largest layer of the workload table
+that fits one GPU: the DeepSeek-V3-shaped layer at T=16384 (d=7168, f=2048,
+E=256 routed experts, top-8, Dirichlet alpha=0.5, plus the always-on shared
+expert of f=2048), in bf16.  The same line carries a sub-record for the
+decode-shaped layer (decode64: T=32, d=2048, f=1024, E=64, top-8, alpha=1),
+the small-T, weight-streaming end of the table.
 
 ``--fp8`` times moe_layer_forward_fp8 (e4m3 expert weights with 128 x 128
 block scales, quantised once before the timed region).
@@ -44,9 +51,17 @@ METRIC = "fused MoE layer µs & tokens/s on 1 B200; % of HBM / tensor-core roofl
 UNIT = "tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# The round figures the layer's targets are stated against: about 8 TB/s of HBM3e and
+# 2.25 PFLOP/s of dense bf16 (4.5 fp8).  Fractions of these are reported beside the
+# fractions of the measured peaks.
+NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+HEADLINE = dict(workload="deepseek_v3", T=16384, alpha=0.5)
+DECODE_SUB = dict(workload="decode64", T=32, alpha=1.0)
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "roofline_traffic.json")
 KERNEL_SOURCES = ["grouped_gemm_02_b200/csrc/grouped_gemm.cuh", "grouped_gemm_02_b200/csrc/ptx.cuh",
                   "grouped_gemm_02_b200/csrc/common.cuh"]
+FP8_KERNEL_SOURCES = ["grouped_gemm_02_b200/csrc/fp8.cuh", "grouped_gemm_02_b200/csrc/ptx.cuh",
+                      "grouped_gemm_02_b200/csrc/common.cuh"]
 
 
 def log(*a):
@@ -82,23 +97,36 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(fp8: bool = False) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in (FP8_KERNEL_SOURCES if fp8 else KERNEL_SOURCES):
         h.update(open(os.path.join(ROOT, rel), "rb").read())
     return h.hexdigest()[:16]
 
 
-def committed_traffic(workload_name: str):
-    """DRAM bytes per launch of the gate/up GEMM from the committed ncu summary,
-    or None when absent, for another workload, or taken on older kernel source."""
+def traffic_records():
     try:
         rec = json.load(open(PROFILE_TRAFFIC))
     except Exception:
-        return None
-    if rec.get("workload") != workload_name or rec.get("source_sha") != kernel_source_hash():
-        return None
-    return rec.get("dram_bytes_per_launch")
+        return []
+    return rec if isinstance(rec, list) else [rec]
+
+
+def committed_traffic(workload_name: str, kernel: str = None):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
+    or None when absent, for another workload or kernel, or taken on older kernel
+    source.  A record taken on a reduced case carries the full launch's bytes
+    scaled from it (its "scaled_from" says how)."""
+    fp8 = workload_name.endswith(" fp8")
+    for rec in traffic_records():
+        if rec.get("workload") != workload_name:
+            continue
+        if kernel is not None and rec.get("kernel_role", kernel) != kernel:
+            continue
+        if rec.get("source_sha") != kernel_source_hash(fp8):
+            return None
+        return rec.get("dram_bytes_per_launch")
+    return None
 
 
 class ClockSampler:
@@ -164,12 +192,17 @@ class ClockSampler:
 
 def parse_workload(args) -> wl.LayerShape:
     kw = {}
-    if args.T is not None:
+    name = getattr(args, "workload", None)
+    if name is None:
+        name = HEADLINE["workload"]
+        kw.update(T=HEADLINE["T"], alpha=HEADLINE["alpha"])
+    if getattr(args, "T", None) is not None:
         kw["T"] = args.T
-    if args.alpha is not None:
+    if getattr(args, "alpha", None) is not None:
         kw["alpha"] = args.alpha
-    s = wl.shape(args.workload, **kw)
-    return s
+    if getattr(args, "E", None) is not None:
+        kw["E"] = args.E
+    return wl.shape(name, **kw)
 
 
 def workload_label(s: wl.LayerShape) -> str:
@@ -221,36 +254,122 @@ def algorithmic(s: wl.LayerShape, counts: np.ndarray, fp8: bool = False):
                 g2_bytes=g2_bytes, g2_flops=g2_flops)
 
 
+def weight_sets(wbytes: int) -> int:
+    """Rotating weight sets so that no step finds its weights in L2: enough sets to
+    exceed 3x L2, and at least two unless one set alone is ten times L2."""
+    want = max(1, math.ceil(3 * L2_BYTES / max(wbytes, 1)))
+    if wbytes < 10 * L2_BYTES:
+        want = max(want, 2)
+    return want
+
+
+def kernel_roofline(s, alg, phase_ms, fp8, pk, pk_kind):
+    """The dominant kernel's roofline: the single expert-GEMM launch when the
+    library fuses both GEMMs, else the gate/up launch (2/3 of the flops and the
+    largest launch of the layer)."""
+    bw = pk["hbm_gbs"] * 1e9
+    tc = pk["bf16_tflops_sustained"] * 1e12 * (2.0 if fp8 else 1.0)
+    tc_nom = NOMINAL_PEAKS["bf16_tflops"] * 1e12 * (2.0 if fp8 else 1.0)
+    bw_nom = NOMINAL_PEAKS["hbm_gbs"] * 1e9
+    fused = gemm_fused(s.P, s.f)
+    if fused:
+        t = (phase_ms[2] + phase_ms[3]) / 1e3
+        nbytes = alg["g1_bytes"] + alg["g2_bytes"]
+        nflops = alg["g1_flops"] + alg["g2_flops"]
+        role = "fused"
+    else:
+        t = phase_ms[2] / 1e3
+        nbytes = alg["g1_bytes"]
+        nflops = alg["g1_flops"]
+        role = "gate_up"
+    if nbytes / bw >= nflops / tc:
+        roof = {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s"}
+        roof["frac_nominal"] = nbytes / t / bw_nom
+    else:
+        roof = {"bound": "tensor", "achieved": nflops / t / 1e12, "peak": tc / 1e12, "unit": "TFLOP/s"}
+        roof["frac_nominal"] = nflops / t / tc_nom
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    name = ("grouped_gemm_fp8_kernel" if fp8 else "grouped_gemm_kernel")
+    roof["kernel"] = f"{name}<{'fused gate/up + down' if fused else 'gate/up + SwiGLU'}>"
+    roof["kernel_role"] = role
+    roof["scope"] = "one expert-GEMM launch (the layer's fraction is layer_roofline.frac)"
+    roof["algorithmic_bytes_per_launch"] = nbytes
+    roof["algorithmic_flops_per_launch"] = nflops
+    roof["launch_us"] = t * 1e6
+    if roof["bound"] == "tensor":
+        roof["peak_source"] = f"{pk_kind} ({'2 x sustained bf16 (fp8)' if fp8 else 'sustained bf16'})"
+    else:
+        roof["peak_source"] = f"{pk_kind} (HBM copy)"
+    roof["nominal_peak"] = (tc_nom / 1e12 if roof["bound"] == "tensor" else bw_nom / 1e9)
+    roof["traffic"] = committed_traffic(workload_label(s) + (" fp8" if fp8 else ""), role)
+    return roof
+
+
+def layer_roofline(alg, ms_per_step, fp8, pk, pk_kind):
+    """t_roof = max(active weight bytes / HBM, layer flops / tensor peak) over the layer time."""
+    bw = pk["hbm_gbs"] * 1e9
+    tc = pk["bf16_tflops_sustained"] * 1e12 * (2.0 if fp8 else 1.0)
+    bw_nom = NOMINAL_PEAKS["hbm_gbs"] * 1e9
+    tc_nom = NOMINAL_PEAKS["bf16_tflops"] * 1e12 * (2.0 if fp8 else 1.0)
+    t_meas = ms_per_step / 1e3
+    t_roof = max(alg["w_act"] / bw, alg["flops"] / tc)
+    t_nom = max(alg["w_act"] / bw_nom, alg["flops"] / tc_nom)
+    return {"bound": "hbm" if alg["w_act"] / bw >= alg["flops"] / tc else "tensor",
+            "t_roof_us": t_roof * 1e6, "t_meas_us": t_meas * 1e6, "frac": t_roof / t_meas,
+            "t_roof_nominal_us": t_nom * 1e6, "frac_nominal": t_nom / t_meas,
+            "w_act_bytes": alg["w_act"], "flops": alg["flops"],
+            "peak_source": f"{pk_kind}; nominal = {NOMINAL_PEAKS['hbm_gbs']:.0f} GB/s and "
+                           f"{NOMINAL_PEAKS['bf16_tflops'] * (2 if fp8 else 1):.0f} TFLOP/s"}
+
+
 # ------------------------------------------------------------------ CPU oracle timing
 
 class OracleRun:
-    """The CPU oracle on a token sample of a workload (host arrays prepared once)."""
+    """The CPU oracle on a token sample of a layer: per batch, fp64 router logits,
+    top-k, the permutation and the per-token expert FFNs (+ shared expert).
 
-    def __init__(self, s: wl.LayerShape, inp_host: dict):
+    Host memory stays bounded: the sample is drawn from a pool of tokens whose k
+    experts all lie in a small set of experts, and only those experts' weights
+    are brought to the host (``expert_fn(e)`` returns W1[e], W3[e], W2[e] as
+    host bf16 tensors, on first use).  Every token costs the same k expert FFNs
+    of the same shape, so the oracle's time per token does not depend on which
+    experts the pool holds."""
+
+    def __init__(self, s: wl.LayerShape, x: torch.Tensor, Wg: torch.Tensor, bias: torch.Tensor,
+                 expert_fn, shared=None, pool=None):
         import oracle
         self.oracle = oracle
         self.s = s
         self.threads = oracle.default_threads()
-        self.x = wl.bf16_bits(inp_host["x"])
-        self.Wg = wl.bf16_bits(inp_host["Wg"])
-        self.bias = inp_host["bias"].numpy()
-        self.W1 = [wl.bf16_bits(inp_host["W1"][e]) for e in range(s.E)]
-        self.W3 = [wl.bf16_bits(inp_host["W3"][e]) for e in range(s.E)]
-        self.W2 = [wl.bf16_bits(inp_host["W2"][e]) for e in range(s.E)]
+        self.pool = np.arange(x.shape[0]) if pool is None else np.asarray(pool, dtype=np.int64)
+        self.x = wl.bf16_bits(x)
+        self.Wg = wl.bf16_bits(Wg)
+        self.bias = bias.numpy()
+        self.expert_fn = expert_fn
+        self.W1 = [None] * s.E
+        self.W3 = [None] * s.E
+        self.W2 = [None] * s.E
         self.shared = None
-        if s.f_shared:
-            self.shared = {n: wl.bf16_bits(inp_host[n]) for n in ("Ws1", "Ws3", "Ws2")}
+        if shared:
+            self.shared = {n: wl.bf16_bits(shared[n]) for n in ("Ws1", "Ws3", "Ws2")}
         self.next = 0
 
+    def load(self, experts):
+        for e in sorted(set(int(v) for v in experts)):
+            if self.W1[e] is None:
+                w = self.expert_fn(e)
+                self.W1[e], self.W3[e], self.W2[e] = (wl.bf16_bits(w[n]) for n in ("W1", "W3", "W2"))
+
     def batch(self, n: int) -> int:
-        """Routing and expert FFNs of the next n tokens (wrapping around T)."""
+        """Routing and expert FFNs of the next n pool tokens (wrapping around)."""
         o = self.oracle
-        toks = np.arange(self.next, self.next + n) % self.s.T
+        toks = self.pool[np.arange(self.next, self.next + n) % self.pool.size]
         self.next += n
         xs = np.ascontiguousarray(self.x[toks])
         L = o.router_logits(xs, self.Wg, self.bias).astype(np.float32)
         idx, w = o.topk(L, self.s.k)
         o.permutation(idx, self.s.E)
+        self.load(idx.ravel())
         o.moe_ffn(xs, self.W1, self.W3, self.W2, idx, w, shared=self.shared, nthreads=self.threads)
         return n
 
@@ -265,54 +384,74 @@ class OracleRun:
                 return done, el, min(self.threads, n)
 
 
+def token_pool(idx: np.ndarray, E: int, want: int = 256, max_experts: int = 48):
+    """Tokens whose k experts all lie among the most-used experts: grows the expert
+    set (by count, descending) until `want` tokens qualify or it holds
+    `max_experts`.  Returns (pool tokens, expert set); the pool may be small."""
+    counts = np.bincount(idx.ravel(), minlength=E)
+    order = np.argsort(-counts, kind="stable")
+    m = min(E, max(idx.shape[1], 8))
+    while True:
+        allowed = np.zeros(E, dtype=bool)
+        allowed[order[:m]] = True
+        ok = np.nonzero(allowed[idx].all(axis=1))[0]
+        if ok.size >= want or m >= min(E, max_experts):
+            break
+        m = min(E, m + 8)
+    if ok.size == 0:                     # no token fits: take the first token's experts
+        ok = np.array([0])
+    return ok, order[:m]
+
+
+def pool_note(pool, experts, s):
+    return (f"tokens drawn from a pool of {pool.size} tokens whose {s.k} experts lie among the "
+            f"{len(experts)} most-used experts (host copies of those experts only; every token costs the "
+            f"same {s.k} expert FFNs{' + the shared expert' if s.f_shared else ''})")
+
+
 # ------------------------------------------------------------------ GPU arm
 
-def run_ours(args, s: wl.LayerShape):
-    from grouped_gemm_02_b200 import moe
-    rank, local_rank, world = dist_env()
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    dev = torch.device("cuda", torch.cuda.current_device())
-    torch.cuda.set_device(dev)
-    stream = torch.cuda.current_stream()
-
-    # inputs: R rotating weight sets so that consecutive steps never find their
-    # weights in L2 (each set is larger than L2 already for the default layer)
-    one = wl.make_weights(s, seed=args.seed, device=dev)
-    wbytes = sum(t.numel() * t.element_size() for t in one.values())
-    free, _ = torch.cuda.mem_get_info(dev)
-    want = max(2, math.ceil(3 * L2_BYTES / max(wbytes, 1)))
-    R = int(max(1, min(want, args.sets or want, (free * 0.6) // max(wbytes, 1))))
-    sets = [one] + [wl.make_weights(s, seed=args.seed + 1000 * (i + 1), device=dev) for i in range(R - 1)]
-    base = wl.make_inputs(s, seed=args.seed, device=dev, weights=False)
-    x, Wg, bias = base["x"], base["Wg"], base["bias"]
-    out = torch.empty(s.T, s.d, dtype=torch.bfloat16, device=dev)
-    if args.fp8:
-        # e4m3 weights with 128 x 128 block scales (quantised once, outside the timed region)
-        qsets = [moe.quantize_layer_fp8(w) for w in sets]
-        ws = moe.new_workspace_fp8(s.T, s.d, s.f, s.E, s.k, s.f_shared, device=dev)
-        wbytes = sum(t.numel() * t.element_size() for t in qsets[0].values())
-        sets = one = None                   # the bf16 weights are not used any more
-        torch.cuda.empty_cache()
-    else:
-        ws = moe.new_workspace(s.T, s.d, s.f, s.E, s.k, s.f_shared, device=dev)
-
+def _make_step(moe, s, fp8, x, Wg, bias, sets, qsets, ws, out, R):
     def step(i, prof_events=None):
         if prof_events is not None:
             moe.moe_record_phase_events(prof_events)
-        if args.fp8:
+        if fp8:
             moe.moe_layer_forward_fp8(x, Wg, bias, qsets[i % R], s.k, ws, out=out)
             return
         w = sets[i % R]
         moe.moe_layer_forward(x, Wg, bias, w["W1"], w["W3"], w["W2"], s.k, ws, Ws1=w.get("Ws1"),
                               Ws3=w.get("Ws3"), Ws2=w.get("Ws2"), out=out)
+    return step
 
-    sampler = ClockSampler([torch.cuda.current_device()]) if rank == 0 else None
-    # warm-up (at least 3 steps; also lets the clock sampler start)
-    for i in range(max(3, args.warmup)):
+
+def measure_layer(s: wl.LayerShape, args, steps: int, warmup: int, world: int, dev, sampler=None,
+                  phases_in_timed: bool = True, with_e2e: bool = True, sets_override: int = 0):
+    """Times `steps` layer forwards after `warmup`; returns the measured record
+    (and the host-side handles the CPU baseline needs)."""
+    from grouped_gemm_02_b200 import moe
+    stream = torch.cuda.current_stream()
+    one = wl.make_weights(s, seed=args.seed, device=dev)
+    wbytes = sum(t.numel() * t.element_size() for t in one.values())
+    free, _ = torch.cuda.mem_get_info(dev)
+    R = int(max(1, min(weight_sets(wbytes), sets_override or weight_sets(wbytes),
+                       (free * 0.6) // max(wbytes, 1))))
+    sets = [one] + [wl.make_weights(s, seed=args.seed + 1000 * (i + 1), device=dev) for i in range(R - 1)]
+    base = wl.make_inputs(s, seed=args.seed, device=dev, weights=False)
+    x, Wg, bias = base["x"], base["Wg"], base["bias"]
+    out = torch.empty(s.T, s.d, dtype=torch.bfloat16, device=dev)
+    qsets = None
+    if args.fp8:
+        # e4m3 weights with 128 x 128 block scales (quantised once, outside the timed region)
+        qsets = [moe.quantize_layer_fp8(w) for w in sets]
+        ws = moe.new_workspace_fp8(s.T, s.d, s.f, s.E, s.k, s.f_shared, device=dev)
+        wbytes = sum(t.numel() * t.element_size() for t in qsets[0].values())
+        sets = None
+        torch.cuda.empty_cache()
+    else:
+        ws = moe.new_workspace(s.T, s.d, s.f, s.E, s.k, s.f_shared, device=dev)
+    step = _make_step(moe, s, args.fp8, x, Wg, bias, sets, qsets, ws, out, R)
+
+    for i in range(warmup):
         step(i)
     if sampler:
         sampler.wait_first_sample()
@@ -320,8 +459,15 @@ def run_ours(args, s: wl.LayerShape):
     if moe.moe_get_device_error(ws) != 0:
         raise RuntimeError("device error after warm-up")
 
-    # timed region: K steps of the layer, nothing else on the stream
-    K = args.steps
+    # CUDA events for the per-phase split: inside the timed region itself (each
+    # step records six events on the layer's stream), or in a second pass
+    n_ev = steps if phases_in_timed else min(steps, 500)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(n_ev)]
+    for row in ev:          # torch creates the CUDA event on its first record
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         import torch.distributed as dist
@@ -329,39 +475,32 @@ def run_ours(args, s: wl.LayerShape):
     torch.cuda.synchronize()
     n0 = moe.moe_launch_counter()
     start.record(stream)
-    for i in range(K):
-        step(i)
+    for i in range(steps):
+        step(i, ev[i] if phases_in_timed else None)
     end.record(stream)
     torch.cuda.synchronize()
     launches = moe.moe_launch_counter() - n0
-    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        dist.barrier()
     ms = start.elapsed_time(end)
     ms_max = reduce_max(ms, world, dev)
-    ms_per_step = ms_max / K
     if moe.moe_get_device_error(ws) != 0:
         raise RuntimeError("device error in the timed region")
-
-    # per-phase pass: the same steps with CUDA events between the phases (an event
-    # between two kernels keeps the second from starting early, so these phase
-    # times are upper bounds); gives the gate/up GEMM's own duration
-    Kp = min(K, 500)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(Kp)]
-    for row in ev:          # torch creates the CUDA event on its first record
-        for e in row:
-            e.record(stream)
-    torch.cuda.synchronize()
-    for i in range(Kp):
-        step(i, ev[i])
-    torch.cuda.synchronize()
-    phase = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(5)] for i in range(Kp)])
+    if not phases_in_timed:
+        # events between phases keep the next kernel from starting early, so
+        # these phase times are upper bounds
+        for i in range(n_ev):
+            step(i, ev[i])
+        torch.cuda.synchronize()
+    phase = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(5)] for i in range(n_ev)])
     phase_ms = phase.mean(axis=0)
 
-    # end to end through the C ABI: pinned host x -> device, layer, device out -> pinned host
     e2e = None
-    if not args.no_e2e:
+    if with_e2e:
+        # end to end through the C ABI: pinned host x -> device, layer, device out -> pinned host
         x_host = x.cpu().pin_memory()
         out_host = torch.empty(s.T, s.d, dtype=torch.bfloat16).pin_memory()
-        for i in range(3):
+        for i in range(min(3, warmup)):
             x.copy_(x_host, non_blocking=True)
             step(i)
             out_host.copy_(out, non_blocking=True)
@@ -371,77 +510,104 @@ def run_ours(args, s: wl.LayerShape):
         torch.cuda.synchronize()
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s0.record(stream)
-        for i in range(K):
+        for i in range(steps):
             x.copy_(x_host, non_blocking=True)
             step(i)
             out_host.copy_(out, non_blocking=True)
         s1.record(stream)
         torch.cuda.synchronize()
         e_ms = reduce_max(s0.elapsed_time(s1), world, dev)
-        e2e = {"value": s.T * K * world / (e_ms / 1e3), "unit": UNIT,
+        e2e = {"value": s.T * steps * world / (e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": s.T * s.d * 2, "d2h_bytes_per_step": s.T * s.d * 2,
-               "ms_per_step": e_ms / K}
+               "ms_per_step": e_ms / steps}
 
-    # realised histogram and roofline
     if args.fp8:
         views = moe.workspace_views_fp8(ws, s.T, s.d, s.f, s.E, s.k, s.f_shared)
     else:
         views = moe.workspace_views(ws, s.T, s.d, s.f, s.E, s.k, s.f_shared)
     counts = views["counts"].cpu().numpy()
+    idx = views["topk_idx"].cpu().numpy()
     alg = algorithmic(s, counts, fp8=args.fp8)
     pk, pk_kind = peaks()
-    bw = pk["hbm_gbs"] * 1e9
-    # FP8 tensor peak: the measured bf16 figure times the nominal fp8 / bf16 ratio (4.5 / 2.25)
-    tc = pk["bf16_tflops_sustained"] * 1e12 * (2.0 if args.fp8 else 1.0)
-    # the dominant kernel is the expert GEMM: one launch (gate/up + SwiGLU, then down) for
-    # P <= 256 and f <= 4096, else the two launches together (the library's rule; the
-    # MOE_GEMM_SPLIT variable overrides it there and here)
-    t_g = (phase_ms[2] + phase_ms[3]) / 1e3
-    g_bytes = alg["g1_bytes"] + alg["g2_bytes"]
-    g_flops = alg["g1_flops"] + alg["g2_flops"]
-    if g_bytes / bw >= g_flops / tc:
-        roof = {"bound": "hbm", "achieved": g_bytes / t_g / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s"}
-    else:
-        roof = {"bound": "tensor", "achieved": g_flops / t_g / 1e12, "peak": tc / 1e12,
-                "unit": "TFLOP/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    # the record names the workload as the JSON line does (" fp8" for the FP8 kernels)
-    roof["traffic"] = committed_traffic(workload_label(s) + (" fp8" if args.fp8 else ""))
-    roof["kernel"] = ("grouped_gemm_fp8_kernel<gate/up>+<down>" if args.fp8 else
-                      ("grouped_gemm_kernel<fused gate/up + down>" if gemm_fused(s.P, s.f)
-                       else "grouped_gemm_kernel<gate/up>+<down>"))
-    roof["algorithmic_bytes_per_launch"] = g_bytes
-    roof["launch_us"] = t_g * 1e6
-    roof["peak_source"] = f"{pk_kind} ({('2 x sustained bf16 (fp8)' if args.fp8 else 'sustained bf16') if roof['bound'] == 'tensor' else 'HBM copy'})"
-    t_roof = max(alg["w_act"] / bw, alg["flops"] / tc)
-    layer_roof = {"bound": "hbm" if alg["w_act"] / bw >= alg["flops"] / tc else "tensor",
-                  "t_roof_us": t_roof * 1e6, "t_meas_us": ms_per_step * 1e3, "frac": t_roof / (ms_per_step / 1e3),
-                  "w_act_bytes": alg["w_act"], "flops": alg["flops"], "peak_source": pk_kind}
+    ms_per_step = ms_max / steps
+    rec = {"ms_per_step": ms_per_step, "ms_total": ms_max, "launches": int(launches), "phase_ms": phase_ms,
+           "phases_in_timed": phases_in_timed, "counts": counts, "alg": alg, "e2e": e2e, "R": R,
+           "wbytes": wbytes,
+           "roofline": kernel_roofline(s, alg, phase_ms, args.fp8, pk, pk_kind),
+           "layer_roofline": layer_roofline(alg, ms_per_step, args.fp8, pk, pk_kind)}
+    host = None
+    if not args.fp8:
+        host = {"x": x, "Wg": Wg, "bias": bias, "weights": one, "idx": idx}
+    return rec, host
 
-    line = {"metric": METRIC, "value": s.T * K * world / (ms_max / 1e3), "unit": UNIT, "n_gpus": world,
+
+def sub_record(s, rec, fp8):
+    """The compact form of a second workload measured in the same run."""
+    return {"workload": workload_label(s) + (" fp8" if fp8 else ""), "value": s.T / (rec["ms_per_step"] / 1e3),
+            "unit": UNIT, "us_per_layer": rec["ms_per_step"] * 1e3, "steps": rec["steps"],
+            "layer_roofline": rec["layer_roofline"], "roofline": rec["roofline"],
+            "histogram": stats.histogram_stats(rec["counts"]),
+            "phase_us": {n: float(v * 1e3) for n, v in
+                         zip(("route", "permute", "gemm_gate_up", "gemm_down", "combine"), rec["phase_ms"])},
+            "phase_note": "per-phase means from a second pass with CUDA events between phases"}
+
+
+def cpu_baseline(s, host, budget_s):
+    """The oracle, as it stands, on the host cores for about budget_s seconds."""
+    pool, experts = token_pool(host["idx"], s.E)
+    W = host["weights"]
+    shared = {n: W[n].cpu() for n in ("Ws1", "Ws3", "Ws2")} if s.f_shared else None
+    orc = OracleRun(s, host["x"].cpu(), host["Wg"].cpu(), host["bias"].cpu(),
+                    lambda e: {n: W[n][e].cpu() for n in ("W1", "W3", "W2")}, shared=shared, pool=pool)
+    orc.load(experts)
+    toks, secs, cores = orc.timed(budget_s, orc.threads)
+    return {"value": toks / secs, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{toks} tokens of {workload_label(s)} (fp64 router logits, top-k, permutation and expert "
+                      f"FFNs per token), {secs:.1f} s on {cores} host threads; {pool_note(pool, experts, s)}"}
+
+
+def run_ours(args, s: wl.LayerShape):
+    rank, local_rank, world = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+
+    sampler = ClockSampler([torch.cuda.current_device()]) if rank == 0 else None
+    rec, host = measure_layer(s, args, args.steps, args.warmup, world, dev, sampler=sampler,
+                              phases_in_timed=True, with_e2e=not args.no_e2e, sets_override=args.sets)
+    clocks = sampler.stop() if sampler else None
+    K = args.steps
+    ms_per_step = rec["ms_per_step"]
+    line = {"metric": METRIC, "value": s.T * K * world / (rec["ms_total"] / 1e3), "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3 (fp32 accumulate)" if args.fp8 else "bf16",
-            "data": "synthetic",
+            "data": "synthetic (seeded; Dirichlet routing skew; random-init weights of the layer's shape)",
             "config": {"workload": workload_label(s) + (" fp8" if args.fp8 else ""), "T": s.T, "d": s.d, "f": s.f,
                        "E": s.E, "k": s.k,
                        "alpha": s.alpha, "f_shared": s.f_shared, "seed": args.seed,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": f"inputs larger than L2: {R} rotating weight sets of {wbytes / 2**20:.0f} MiB",
-                       "histogram": stats.histogram_stats(counts),
+                       "l2": f"inputs larger than L2: {rec['R']} rotating weight set(s) of "
+                             f"{rec['wbytes'] / 2**20:.0f} MiB",
+                       "histogram": stats.histogram_stats(rec["counts"]),
                        "us_per_layer": ms_per_step * 1e3,
-                       "phase_note": "per-phase means from a second pass with CUDA events between phases",
+                       "phase_note": "per-phase means from CUDA events recorded between the phases inside the "
+                                     "timed region",
                        "phase_us": {n: float(v * 1e3) for n, v in
-                                    zip(("route", "permute", "gemm_gate_up", "gemm_down", "combine"), phase_ms)}},
-            "roofline": roof, "layer_roofline": layer_roof, "e2e": e2e, "gpu_launches": int(launches),
-            "clocks": clocks}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.fp8:
-        host = {n: v.cpu() for n, v in base.items()}
-        host.update({n: v.cpu() for n, v in one.items()})
-        orc = OracleRun(s, host)
-        toks, secs, cores = orc.timed(args.cpu_budget, orc.threads)
-        line["cpu_baseline"] = {"value": toks / secs, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": f"{toks} tokens of {workload_label(s)} (full routing + expert FFNs per "
-                                          f"token, fp64), {secs:.1f} s on {cores} host threads"}
+                                    zip(("route", "permute", "gemm_gate_up", "gemm_down", "combine"),
+                                        rec["phase_ms"])}},
+            "roofline": rec["roofline"], "layer_roofline": rec["layer_roofline"], "e2e": rec["e2e"],
+            "gpu_launches": rec["launches"], "clocks": clocks}
+    if not args.no_sub and s.name != DECODE_SUB["workload"]:
+        ds = wl.shape(DECODE_SUB["workload"], T=DECODE_SUB["T"], alpha=DECODE_SUB["alpha"])
+        drec, _ = measure_layer(ds, args, args.sub_steps, 20, world, dev, phases_in_timed=False, with_e2e=False)
+        drec["steps"] = args.sub_steps
+        line["decode64"] = sub_record(ds, drec, args.fp8)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and host is not None:
+        line["cpu_baseline"] = cpu_baseline(s, host, args.cpu_budget)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -451,11 +617,27 @@ def run_ours(args, s: wl.LayerShape):
 
 # ------------------------------------------------------------------ reference arm (the CPU oracle)
 
+def reference_setup(s: wl.LayerShape, seed: int):
+    """Host inputs for the oracle's timed sample: x, Wg and bias as the workload
+    draws them, a token pool picked from a float32 routing of every token, and
+    the routed experts drawn one by one on first use."""
+    inp = wl.make_inputs(s, seed=seed, weights=False)
+    # the pool selection only picks which tokens to sample; the timed oracle routes them itself
+    L = inp["x"].float() @ inp["Wg"].float().T + inp["bias"]
+    idx = torch.topk(L, s.k, dim=1).indices.numpy()
+    pool, experts = token_pool(idx, s.E)
+    shared = wl.make_shared_weights(s, seed) if s.f_shared else None
+    orc = OracleRun(s, inp["x"], inp["Wg"], inp["bias"], lambda e: wl.make_expert_weights(s, seed, e),
+                    shared=shared, pool=pool)
+    orc.load(experts)
+    return orc, pool, experts
+
+
 def run_reference(args, s: wl.LayerShape):
     rank, _, world = dist_env()
     if rank != 0:
         return None
-    orc = OracleRun(s, wl.make_inputs(s, seed=args.seed))
+    orc, pool, experts = reference_setup(s, args.seed)
     # calibrate one batch, then size each step so the whole run stays within a few minutes
     t0 = time.perf_counter()
     orc.batch(orc.threads)
@@ -478,27 +660,35 @@ def run_reference(args, s: wl.LayerShape):
             "config": {"workload": workload_label(s), "T": s.T, "d": s.d, "f": s.f, "E": s.E, "k": s.k,
                        "alpha": s.alpha, "f_shared": s.f_shared, "seed": args.seed},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": f"{tokens_per_step} tokens per step of {workload_label(s)} "
-                                       f"(full routing + expert FFNs, fp64)"},
+                             "sample": f"{tokens_per_step} tokens per step of {workload_label(s)} (fp64 router "
+                                       f"logits, top-k, permutation and expert FFNs); {pool_note(pool, experts, s)}"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-def main(argv=None):
+def build_parser():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default="decode64", choices=sorted(wl.FAMILIES))
+    ap.add_argument("--workload", default=None, choices=sorted(wl.FAMILIES),
+                    help="layer family (default: deepseek_v3 at T=16384, alpha=0.5)")
     ap.add_argument("--T", type=int, default=None)
     ap.add_argument("--alpha", type=float, default=None)
+    ap.add_argument("--E", type=int, default=None, help="override the number of routed experts (profiling cases)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--sets", type=int, default=0, help="rotating weight sets (0: enough to exceed 3x L2)")
     ap.add_argument("--fp8", action="store_true", help="FP8 block-scaled expert GEMMs (moe_layer_forward_fp8)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sub", action="store_true", help="skip the decode64 sub-record")
+    ap.add_argument("--sub-steps", type=int, default=2000, help="timed steps of the decode64 sub-record")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
-    args = ap.parse_args(argv)
+    return ap
+
+
+def main(argv=None):
+    args = build_parser().parse_args(argv)
     args.warmup = max(3, args.warmup)
     s = parse_workload(args)
     line = run_reference(args, s) if args.impl == "reference" else run_ours(args, s)

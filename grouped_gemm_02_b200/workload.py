@@ -136,12 +136,32 @@ def make_weights(s: LayerShape, seed: int = 0, device="cpu") -> Dict[str, torch.
     w["W1"] = _normal_bf16((s.E, s.f, s.d), 1.0 / math.sqrt(s.d), seed, "W1", device)
     w["W3"] = _normal_bf16((s.E, s.f, s.d), 1.0 / math.sqrt(s.d), seed, "W3", device)
     w["W2"] = _normal_bf16((s.E, s.d, s.f), 1.0 / math.sqrt(s.f), seed, "W2", device)
-    if s.f_shared:
-        fs = s.f_shared
-        w["Ws1"] = _normal_bf16((fs, s.d), 1.0 / math.sqrt(s.d), seed, "Ws1", device)
-        w["Ws3"] = _normal_bf16((fs, s.d), 1.0 / math.sqrt(s.d), seed, "Ws3", device)
-        w["Ws2"] = _normal_bf16((s.d, fs), 1.0 / math.sqrt(fs), seed, "Ws2", device)
+    w.update(make_shared_weights(s, seed, device))
     return w
+
+
+def make_expert_weights(s: LayerShape, seed: int, e: int, device="cpu") -> Dict[str, torch.Tensor]:
+    """One routed expert's W1[e] [f,d], W3[e] [f,d], W2[e] [d,f], each drawn from a
+    generator of its own (seeded from (seed, name, e)): the same distribution as
+    ``make_weights``, different values.  Lets a host-side sample of a very large
+    layer draw only the experts its tokens use."""
+    return {
+        "W1": _normal_bf16((s.f, s.d), 1.0 / math.sqrt(s.d), seed, f"W1/{e}", device),
+        "W3": _normal_bf16((s.f, s.d), 1.0 / math.sqrt(s.d), seed, f"W3/{e}", device),
+        "W2": _normal_bf16((s.d, s.f), 1.0 / math.sqrt(s.f), seed, f"W2/{e}", device),
+    }
+
+
+def make_shared_weights(s: LayerShape, seed: int = 0, device="cpu") -> Dict[str, torch.Tensor]:
+    """The shared expert's Ws1/Ws3 [f_shared,d] and Ws2 [d,f_shared] (as ``make_weights`` draws them)."""
+    fs = s.f_shared
+    if not fs:
+        return {}
+    return {
+        "Ws1": _normal_bf16((fs, s.d), 1.0 / math.sqrt(s.d), seed, "Ws1", device),
+        "Ws3": _normal_bf16((fs, s.d), 1.0 / math.sqrt(s.d), seed, "Ws3", device),
+        "Ws2": _normal_bf16((s.d, fs), 1.0 / math.sqrt(fs), seed, "Ws2", device),
+    }
 
 
 def random_logits(T: int, E: int, seed: int, ties: bool = False, device="cpu") -> torch.Tensor:

@@ -122,3 +122,52 @@ def test_gemm_launch_rule(monkeypatch):
     assert not bench.gemm_fused(256, 1024)
     monkeypatch.setenv("MOE_GEMM_SPLIT", "0")
     assert bench.gemm_fused(32768, 14336)
+
+
+def test_default_workload_is_the_largest_single_gpu_layer():
+    args = bench.build_parser().parse_args([])
+    s = bench.parse_workload(args)
+    assert (s.name, s.T, s.d, s.f, s.E, s.k, s.alpha, s.f_shared) == ("deepseek_v3", 16384, 7168, 2048, 256, 8, 0.5,
+                                                                       2048)
+    args = bench.build_parser().parse_args(["--workload", "deepseek_v3", "--T", "1024", "--E", "16"])
+    s = bench.parse_workload(args)
+    assert (s.T, s.E, s.alpha) == (1024, 16, 0.5)
+
+
+def test_weight_sets_exceed_l2():
+    L2 = bench.L2_BYTES
+    assert bench.weight_sets(22 * 2**30) == 1                  # one set is far larger than L2
+    assert bench.weight_sets(805 * 2**20) == 2                 # decode64: at least two sets
+    assert bench.weight_sets(6 * 2**20) * 6 * 2**20 >= 3 * L2   # the tiny layer: enough sets for 3x L2
+
+
+def test_token_pool_keeps_experts_bounded():
+    idx = wl.random_routing(4096, 256, 8, 0.5, seed=3).numpy()
+    pool, experts = bench.token_pool(idx, 256, want=64, max_experts=48)
+    assert len(experts) <= 48 and pool.size >= 1
+    allowed = np.zeros(256, dtype=bool)
+    allowed[experts] = True
+    assert allowed[idx[pool]].all()
+    # a pool that cannot be filled still returns at least one token
+    pool, experts = bench.token_pool(idx, 256, want=10**6, max_experts=16)
+    assert pool.size >= 1 and len(experts) <= 16
+
+
+def test_layer_roofline_fractions():
+    pk = {"hbm_gbs": 6531.0, "bf16_tflops": 1668.8, "bf16_tflops_sustained": 1403.8}
+    alg = {"w_act": 6.531e9, "flops": 1e9}
+    r = bench.layer_roofline(alg, 2.0, False, pk, "measured")           # 1 ms roofline over 2 ms
+    assert r["bound"] == "hbm" and abs(r["frac"] - 0.5) < 1e-12
+    assert abs(r["frac_nominal"] - 6.531e9 / 8e12 / 2e-3) < 1e-12
+    alg = {"w_act": 1e6, "flops": 1.4038e12}
+    r = bench.layer_roofline(alg, 4.0, False, pk, "measured")
+    assert r["bound"] == "tensor" and abs(r["frac"] - 0.25) < 1e-12
+    assert abs(r["frac_nominal"] - 1.4038e12 / 2.25e15 / 4e-3) < 1e-12
+
+
+def test_reference_sample_on_a_small_layer():
+    s = wl.TINY.with_(T=32)
+    orc, pool, experts = bench.reference_setup(s, seed=0)
+    assert pool.size >= 1
+    assert orc.batch(4) == 4
+    assert all(orc.W1[e] is not None for e in experts)
