@@ -1,72 +1,16 @@
-// route.cuh -- router logits (S1) and warp-per-token top-k with softmax gates (S2).
+// route.cuh -- top-k with softmax gates (S2) over the router logits (S1, which
+// run on the tensor cores as grouped_gemm_kernel<MODE_ROUTER>).
 //
-// Router: L[t,e] = sum_c x[t,c] * Wg[e,c] + b[e], fp32 accumulation in a fixed
-// order (each lane sums its 8-element slices in ascending order, then a fixed
-// butterfly over the warp).  Top-k: the k largest fp32 logits of a token in
-// descending order, ties to the lower expert index, NaN below every number;
-// gates are the softmax over the k chosen logits (Decoding the Skew, abstract:
-// the routing distribution decided at run time drives the expert GEMMs).
+// Top-k: the k largest fp32 logits of a token in descending order, ties to the
+// lower expert index, NaN below every number; gates are the softmax over the k
+// chosen logits (Decoding the Skew, abstract: the routing distribution decided
+// at run time drives the expert GEMMs).
 #pragma once
 
 #include "common.cuh"
 #include "ptx.cuh"
 
 namespace moe {
-
-constexpr int kRouterTokens = 8;     // tokens per warp in the router kernel
-constexpr int kRouterWarps = 8;      // experts per CTA (one per warp)
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&o)[8])
-{
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        o[2 * i] = __uint_as_float(w[i] << 16);
-        o[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-}
-
-// grid (ceil(E / 8), ceil(T / 8)), block 256: warp w of CTA (bx, by) computes
-// expert bx*8+w for tokens by*8 .. by*8+7.  Requires d % 8 == 0.
-__global__ void __launch_bounds__(256) router_logits_kernel(const bf16* __restrict__ x, const bf16* __restrict__ Wg,
-                                                            const float* __restrict__ bias, int T, int d, int E,
-                                                            float* __restrict__ L)
-{
-    ptx::grid_dep_wait();
-    ptx::grid_dep_launch();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e = blockIdx.x * kRouterWarps + warp;
-    const int t0 = blockIdx.y * kRouterTokens;
-    if (e >= E) return;
-    const int nt = min(kRouterTokens, T - t0);
-    float acc[kRouterTokens];
-#pragma unroll
-    for (int i = 0; i < kRouterTokens; i++) acc[i] = 0.f;
-    const uint4* wrow = reinterpret_cast<const uint4*>(Wg + (size_t)e * d);
-    const int nvec = d / 8;
-    for (int v = lane; v < nvec; v += 32) {
-        float wv[8];
-        bf16x8_to_f32(__ldg(wrow + v), wv);
-#pragma unroll
-        for (int i = 0; i < kRouterTokens; i++) {
-            if (i < nt) {
-                float xv[8];
-                bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + i) * d) + v), xv);
-#pragma unroll
-                for (int j = 0; j < 8; j++) acc[i] = fmaf(xv[j], wv[j], acc[i]);
-            }
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < kRouterTokens; i++) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
-    }
-    if (lane == 0) {
-        const float b = bias ? bias[e] : 0.f;
-        for (int i = 0; i < nt; i++) L[(size_t)(t0 + i) * E + e] = acc[i] + b;
-    }
-}
 
 // Order-preserving key: larger logit -> larger key; -0 and +0 equal; NaN lowest (0).
 __device__ __forceinline__ uint32_t logit_key(float v)
