@@ -36,7 +36,16 @@ struct PlanHeader {
     int32_t tiles2;     // tiles of the down GEMM (M-tile = 128 rows of W2)
     int32_t n_max;      // widest tile (tokens) in this launch
     int32_t pairs;      // routed pairs with a valid expert id (== offsets[E])
-    int32_t pad[3];
+    int32_t pair;       // 1: tiles cut for CTA pairs (2 x 128 weight rows, widths a multiple of 32)
+    int32_t pad[2];
+};
+
+// How the plan cuts blocks into tiles: at most unit_rows tokens per tile, tile
+// widths a multiple of `align`; m1_rows f rows per gate/up tile and m2_rows d
+// rows per down tile.  Single CTAs: (256, 64, 128, 16, 0) for bf16 and
+// (112, 128, 128, 16, 0) for FP8; CTA pairs: (256, 128, 256, 32, 1).
+struct PlanShape {
+    int unit_rows, m1_rows, m2_rows, align, pair;
 };
 
 struct PlanArrays {

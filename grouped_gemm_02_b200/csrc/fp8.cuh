@@ -38,6 +38,7 @@
 namespace moe {
 
 constexpr int kFp8TileRows = 112;                // most tokens one FP8 tile carries
+constexpr PlanShape kPlanFp8{kFp8TileRows, 128, 128, 16, 0};
 constexpr int kFp8BlockK = 128;                  // e4m3 elements per 128-byte swizzle row = one scale block
 constexpr int kFp8MaxK = 128 * kFp8BlockK;       // reduction length limit: 4 weight scales per lane of a warp
 constexpr uint32_t kFp8TmemCols = 512;

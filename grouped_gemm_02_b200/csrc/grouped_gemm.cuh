@@ -103,6 +103,9 @@ struct GemmArgs {
 struct Tile {
     int group, m, row0, rows, n_mma, K, kb0, kb1, split;
     int blk;        // block (plan entry) index
+    int ma;         // this CTA's M-tile of the weights: m, or 2m + rank for a CTA pair
+    int b_row0;     // first B row this CTA loads, and how many (n_mma, or n_mma / 2 for a pair)
+    int b_n;
     bool shared;
     bool gated;     // a gate/up tile (SwiGLU epilogue) rather than a down tile
 };
@@ -128,8 +131,9 @@ __device__ __forceinline__ int total_tiles(const GemmArgs& a, const PlanHeader* 
     return MODE == MODE_GATED ? hdr->tiles1 : hdr->tiles2;
 }
 
-template <int MODE>
-__device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a, const GemmArgs& a2, const SmemPlan* sp)
+template <int MODE, bool PAIR = false>
+__device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a, const GemmArgs& a2, const SmemPlan* sp,
+                                            int rank = 0)
 {
     Tile tl;
     tl.blk = 0;
@@ -150,6 +154,9 @@ __device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a, co
         tl.kb0 = tl.split * a.kb_per;
         tl.kb1 = min(nk, tl.kb0 + a.kb_per);
         tl.gated = false;
+        tl.ma = tl.m;
+        tl.b_row0 = tl.row0;
+        tl.b_n = tl.n_mma;
         return tl;
     }
     bool gated = MODE == MODE_GATED;
@@ -180,12 +187,24 @@ __device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a, co
     const int start = u * chunk;
     tl.rows = min(chunk, b.z - start);
     tl.row0 = b.y + start;
-    tl.n_mma = (tl.rows + 15) & ~15;
+    // MMA width: a multiple of 16, of 32 for a pair (each CTA loads N/2 rows in 16-row boxes)
+    tl.n_mma = PAIR ? (tl.rows + 31) & ~31 : (tl.rows + 15) & ~15;
     tl.K = tl.shared ? a.K_shared : a.K;
     if (MODE == MODE_FUSED && !gated) tl.K = tl.shared ? a2.K_shared : a2.K;
     tl.kb0 = 0;
     tl.kb1 = (tl.K + kBlockK - 1) / kBlockK;
     tl.split = 0;
+    if (PAIR) {
+        // a pair tile: 2 x 128 weight rows, the CTA of rank r takes M-tile 2m + r
+        // and B rows [row0 + r n/2, row0 + (r + 1) n/2)
+        tl.ma = 2 * tl.m + rank;
+        tl.b_n = tl.n_mma >> 1;
+        tl.b_row0 = tl.row0 + rank * tl.b_n;
+    } else {
+        tl.ma = tl.m;
+        tl.b_n = tl.n_mma;
+        tl.b_row0 = tl.row0;
+    }
     return tl;
 }
 
@@ -241,9 +260,11 @@ __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)
 
 // The i-th tile of this CTA, or -1: the balanced deal of schedule.h in
 // MODE_FUSED, round-robin in every other mode.
-template <int MODE>
+// A CTA pair deals by cluster: both CTAs of a cluster take the same tiles.
+template <int MODE, bool PAIR = false>
 __device__ __forceinline__ int cta_tile(int i, int total, int G, int comp)
 {
+    if (PAIR) return deal_tile((int)ptx::cluster_id_x(), (int)ptx::nclusters_x(), i, total, G, comp, MODE == MODE_FUSED);
     return deal_tile((int)blockIdx.x, (int)gridDim.x, i, total, G, comp, MODE == MODE_FUSED);
 }
 
@@ -254,12 +275,12 @@ struct KIter {
     Tile tl;
 };
 
-template <int MODE>
+template <int MODE, bool PAIR>
 __device__ __forceinline__ bool kiter_seek(KIter& it, int nb, int total, const GemmArgs& a, const GemmArgs& a2,
-                                           const SmemPlan* sp)
+                                           const SmemPlan* sp, int rank)
 {
-    for (; (it.t = cta_tile<MODE>(it.i, total, sp->tiles1, a.comp)) >= 0; it.i++) {
-        it.tl = decode_tile<MODE>(nb, it.t, a, a2, sp);
+    for (; (it.t = cta_tile<MODE, PAIR>(it.i, total, sp->tiles1, a.comp)) >= 0; it.i++) {
+        it.tl = decode_tile<MODE, PAIR>(nb, it.t, a, a2, sp, rank);
         if (it.tl.kb0 < it.tl.kb1) {
             it.kb = it.tl.kb0;
             return true;
@@ -268,24 +289,34 @@ __device__ __forceinline__ bool kiter_seek(KIter& it, int nb, int total, const G
     return false;
 }
 
-template <int MODE>
+template <int MODE, bool PAIR>
 __device__ __forceinline__ bool kiter_begin(KIter& it, int nb, int total, const GemmArgs& a, const GemmArgs& a2,
-                                            const SmemPlan* sp)
+                                            const SmemPlan* sp, int rank)
 {
     it.i = 0;
-    return kiter_seek<MODE>(it, nb, total, a, a2, sp);
+    return kiter_seek<MODE, PAIR>(it, nb, total, a, a2, sp, rank);
 }
 
-template <int MODE>
+template <int MODE, bool PAIR>
 __device__ __forceinline__ bool kiter_next(KIter& it, int nb, int total, const GemmArgs& a, const GemmArgs& a2,
-                                           const SmemPlan* sp)
+                                           const SmemPlan* sp, int rank)
 {
     if (++it.kb < it.tl.kb1) return true;
     ++it.i;
-    return kiter_seek<MODE>(it, nb, total, a, a2, sp);
+    return kiter_seek<MODE, PAIR>(it, nb, total, a, a2, sp, rank);
 }
 
-template <int MODE>
+// One TMA tile load; a CTA of a pair counts its bytes on the leader's barrier
+// (`full` is then a shared::cluster address).
+template <bool PAIR>
+__device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, uint32_t full, int c0, int c1,
+                                         uint64_t pol)
+{
+    if (PAIR) ptx::tma_load_2d_pair(dst, map, full, c0, c1, pol);
+    else ptx::tma_load_2d(dst, map, full, c0, c1, pol);
+}
+
+template <int MODE, bool PAIR>
 __device__ __forceinline__ void issue_a(const KIter& it, uint32_t a_dst, uint32_t full, const CUtensorMap* mA0,
                                         const CUtensorMap* mA1, const CUtensorMap* mA0s, const CUtensorMap* mA1s,
                                         const CUtensorMap* mA2, const CUtensorMap* mA2s, const GemmArgs& a,
@@ -296,31 +327,32 @@ __device__ __forceinline__ void issue_a(const KIter& it, uint32_t a_dst, uint32_
     if (tl.gated) {
         const CUtensorMap* w1 = tl.shared ? mA0s : mA0;
         const CUtensorMap* w3 = tl.shared ? mA1s : mA1;
-        const int a_row = (tl.shared ? 0 : tl.group * a.M) + tl.m * 64;
+        const int a_row = (tl.shared ? 0 : tl.group * a.M) + tl.ma * 64;
 #pragma unroll
         for (int q = 0; q < 4; q++) {
-            ptx::tma_load_2d(a_dst + (32 * q) * 128, w1, full, kc, a_row + 16 * q, pol);
-            ptx::tma_load_2d(a_dst + (32 * q + 16) * 128, w3, full, kc, a_row + 16 * q, pol);
+            tma_load<PAIR>(a_dst + (32 * q) * 128, w1, full, kc, a_row + 16 * q, pol);
+            tma_load<PAIR>(a_dst + (32 * q + 16) * 128, w3, full, kc, a_row + 16 * q, pol);
         }
     } else if (MODE == MODE_FUSED) {
-        const int a_row = (tl.shared ? 0 : tl.group * a2.M) + tl.m * 128;
-        ptx::tma_load_2d(a_dst, tl.shared ? mA2s : mA2, full, kc, a_row, pol);
+        const int a_row = (tl.shared ? 0 : tl.group * a2.M) + tl.ma * 128;
+        tma_load<PAIR>(a_dst, tl.shared ? mA2s : mA2, full, kc, a_row, pol);
     } else {
         const CUtensorMap* a0 = tl.shared ? mA0s : mA0;
-        const int a_row = (MODE == MODE_ROUTER || tl.shared ? 0 : tl.group * a.M) + tl.m * 128;
-        ptx::tma_load_2d(a_dst, a0, full, kc, a_row, pol);
+        const int a_row = (MODE == MODE_ROUTER || tl.shared ? 0 : tl.group * a.M) + tl.ma * 128;
+        tma_load<PAIR>(a_dst, a0, full, kc, a_row, pol);
     }
 }
 
+template <bool PAIR>
 __device__ __forceinline__ void issue_b(const Tile& tl, int kb, uint32_t b_dst, uint32_t full, const CUtensorMap* b,
                                         uint64_t pol)
 {
     const int kc = kb * kBlockK;
-    for (int i = 0; i < tl.n_mma / 16; i++)
-        ptx::tma_load_2d(b_dst + i * 16 * kBRowBytes, b, full, kc, tl.row0 + 16 * i, pol);
+    for (int i = 0; i < tl.b_n / 16; i++)
+        tma_load<PAIR>(b_dst + i * 16 * kBRowBytes, b, full, kc, tl.b_row0 + 16 * i, pol);
 }
 
-template <int MODE>
+template <int MODE, bool PAIR = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mA1,
                         const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mA0s,
@@ -331,11 +363,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 {
     // MODE_FUSED: args describe the gate/up tiles (W1/W3 = mA0/mA1, xp = mB),
     // args2 the down tiles (W2 = mA2, h = mB2); other modes ignore args2 and mA2..mB2s.
+    // PAIR: launched in clusters of two CTAs; a tile is 2 x 128 weight rows and
+    // the leader (rank 0) issues its MMAs for both CTAs (cta_group::2).
+    static_assert(!(PAIR && MODE == MODE_ROUTER), "the router runs on single CTAs");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + kRingBytes);
     const uint32_t ring = ptx::smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rank = PAIR ? (int)ptx::cluster_ctarank() : 0;
+    const bool leader = rank == 0;
 
     // The plan comes from an earlier kernel; when that kernel is the one right
     // before this launch, wait for it before reading anything.
@@ -343,10 +380,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (waited_early) ptx::grid_dep_wait();
 
     const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(args.plan);
+    // a plan cut for the other tile shape (pair or single CTA) cannot be run:
+    // every CTA of the launch sees the same header and leaves before any barrier
+    if (MODE != MODE_ROUTER && hdr->pair != (PAIR ? 1 : 0)) {
+        if (threadIdx.x == 0) atomicOr(args.err, DEVERR_PLAN);
+        if (!waited_early) ptx::grid_dep_wait();
+        ptx::grid_dep_launch();
+        return;
+    }
     const int nb = MODE == MODE_ROUTER ? 0 : hdr->n_blocks;
     const int total = total_tiles<MODE>(args, hdr);
     const int n_max = MODE == MODE_ROUTER ? max(16, (min(args.chunk, args.T) + 15) & ~15) : max(16, hdr->n_max);
-    const uint32_t stage_bytes = kATileBytes + (uint32_t)n_max * kBRowBytes;
+    const uint32_t stage_bytes = kATileBytes + (uint32_t)(PAIR ? n_max / 2 : n_max) * kBRowBytes;
     const int stages = min(kMaxStages, (int)(kRingBytes / stage_bytes));
 
     SmemPlan* splan = reinterpret_cast<SmemPlan*>(smem + kRingBytes + kBarBytes);
@@ -370,7 +415,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int a = 0; a < 2; a++) {
             ptx::mbar_init(ptx::smem_u32(&ctl->tfull[a]), 1);
-            ptx::mbar_init(ptx::smem_u32(&ctl->tempty[a]), 4);
+            // the epilogue warps of both CTAs of a pair free the leader's accumulator
+            ptx::mbar_init(ptx::smem_u32(&ctl->tempty[a]), PAIR ? 8 : 4);
         }
         ptx::mbar_init(ptx::smem_u32(&ctl->drain), 1);
         ctl->abort = 0;
@@ -383,25 +429,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (MODE == MODE_GATED) ptx::prefetch_tensormap(&mA1);
     }
     if (warp == 1) {
-        ptx::tmem_alloc(ptx::smem_u32(&ctl->tmem_base), kTmemCols);
-        ptx::tmem_relinquish();
+        if (PAIR) {
+            ptx::tmem_alloc_pair(ptx::smem_u32(&ctl->tmem_base), kTmemCols);
+            ptx::tmem_relinquish_pair();
+        } else {
+            ptx::tmem_alloc(ptx::smem_u32(&ctl->tmem_base), kTmemCols);
+            ptx::tmem_relinquish();
+        }
     }
     ptx::tc_fence_before();
-    __syncthreads();
+    // a pair's barriers are signalled across the two CTAs: both must be initialised first
+    if (PAIR) ptx::cluster_sync();
+    else __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
+    // the leader's barrier of a given offset, as the peer addresses it
+    auto leader_bar = [&](uint64_t* bar) -> uint32_t {
+        return PAIR ? ptx::mapa_shared(ptx::smem_u32(bar), 0) : ptx::smem_u32(bar);
+    };
+    // bytes one stage brings: this CTA's A and B tiles, or both CTAs' for a pair (the leader counts them)
+    auto stage_tx = [&](const Tile& tl) -> uint32_t {
+        return PAIR ? 2u * (kATileBytes + (uint32_t)tl.b_n * kBRowBytes) : kATileBytes + (uint32_t)tl.b_n * kBRowBytes;
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (ptx::elect_one()) {
             const uint64_t pol = ptx::policy_evict_normal();
-            uint32_t armed = 0, armed_ph = 0;   // slots with a load issued, and its phase
+            uint32_t armed = 0, armed_ph = 0;   // slots with a load issued (leader's count), and its phase
             bool ok = true;
             // MODE_FUSED: all gate/up tiles of the tile's block have stored their h rows
             auto wait_block_ready = [&](const Tile& tl) -> bool {
                 const int32_t* dep = plan_arrays(const_cast<int32_t*>(args.plan)).dep + tl.blk;
                 const int m1 = tl.shared ? args.M_shared : args.M;
-                const int need = 4 * splan->units[tl.blk] * ((m1 + 63) / 64);   // 4 epilogue warps per tile
+                // 4 epilogue warps per CTA and gate/up tile (two CTAs per pair tile of 128 f rows)
+                const int need = PAIR ? 8 * splan->units[tl.blk] * ((m1 + 127) / 128)
+                                      : 4 * splan->units[tl.blk] * ((m1 + 63) / 64);
                 if (!bounded_count_wait(dep, need, ctl, args.err)) return false;
                 ptx::fence_proxy_async_global();   // the TMA reads below come after the acquire
                 return true;
@@ -410,15 +473,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int pre = 0;
             if (!waited_early) {
                 KIter it;
-                bool more = kiter_begin<MODE>(it, nb, total, args, args2, splan);
+                bool more = kiter_begin<MODE, PAIR>(it, nb, total, args, args2, splan, rank);
                 while (more && pre < stages) {
-                    const uint32_t full = ptx::smem_u32(&ctl->full[pre]);
-                    ptx::mbar_arrive_expect_tx(full, kATileBytes + (uint32_t)it.tl.n_mma * kBRowBytes);
-                    armed |= 1u << pre;
-                    issue_a<MODE>(it, ring + (uint32_t)pre * stage_bytes, full, &mA0, &mA1, &mA0s, &mA1s, &mA2, &mA2s,
-                                  args, args2, pol);
+                    const uint32_t full = leader_bar(&ctl->full[pre]);
+                    if (leader) {
+                        ptx::mbar_arrive_expect_tx(ptx::smem_u32(&ctl->full[pre]), stage_tx(it.tl));
+                        armed |= 1u << pre;
+                    }
+                    issue_a<MODE, PAIR>(it, ring + (uint32_t)pre * stage_bytes, full, &mA0, &mA1, &mA0s, &mA1s, &mA2,
+                                        &mA2s, args, args2, pol);
                     ++pre;
-                    more = kiter_next<MODE>(it, nb, total, args, args2, splan);
+                    more = kiter_next<MODE, PAIR>(it, nb, total, args, args2, splan, rank);
                 }
                 ptx::grid_dep_wait();
             }
@@ -430,10 +495,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int s = 0, n = 0;
             uint32_t ph = 0;
             KIter it;
-            bool more = kiter_begin<MODE>(it, nb, total, args, args2, splan);
+            bool more = kiter_begin<MODE, PAIR>(it, nb, total, args, args2, splan, rank);
             while (more) {
                 const uint32_t a_dst = ring + (uint32_t)s * stage_bytes;
-                const uint32_t full = ptx::smem_u32(&ctl->full[s]);
+                const uint32_t full = leader_bar(&ctl->full[s]);
                 const CUtensorMap* b = it.tl.gated || MODE != MODE_FUSED ? (it.tl.shared ? &mBs : &mB)
                                                                           : (it.tl.shared ? &mB2s : &mB2);
                 // a down tile of the fused launch reads h only after its block's gate/up tiles stored it
@@ -442,27 +507,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     break;
                 }
                 if (n < pre) {
-                    issue_b(it.tl, it.kb, a_dst + kATileBytes, full, b, pol);
+                    issue_b<PAIR>(it.tl, it.kb, a_dst + kATileBytes, full, b, pol);
                 } else {
                     if (!bounded_wait(ptx::smem_u32(&ctl->empty[s]), ph ^ 1u, ctl, args.err)) {
                         ok = false;
                         break;
                     }
-                    ptx::mbar_arrive_expect_tx(full, kATileBytes + (uint32_t)it.tl.n_mma * kBRowBytes);
-                    armed |= 1u << s;
-                    armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
-                    issue_a<MODE>(it, a_dst, full, &mA0, &mA1, &mA0s, &mA1s, &mA2, &mA2s, args, args2, pol);
-                    issue_b(it.tl, it.kb, a_dst + kATileBytes, full, b, pol);
+                    if (leader) {
+                        ptx::mbar_arrive_expect_tx(ptx::smem_u32(&ctl->full[s]), stage_tx(it.tl));
+                        armed |= 1u << s;
+                        armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
+                    }
+                    issue_a<MODE, PAIR>(it, a_dst, full, &mA0, &mA1, &mA0s, &mA1s, &mA2, &mA2s, args, args2, pol);
+                    issue_b<PAIR>(it.tl, it.kb, a_dst + kATileBytes, full, b, pol);
                 }
                 ++n;
                 if (++s == stages) {
                     s = 0;
                     ph ^= 1u;
                 }
-                more = kiter_next<MODE>(it, nb, total, args, args2, splan);
+                more = kiter_next<MODE, PAIR>(it, nb, total, args, args2, splan, rank);
             }
             if (!ok) {
-                // drain: wait (bounded) for every load this thread issued
+                // drain: wait (bounded) for every stage the leader armed; a pair's
+                // loads from both CTAs complete on the leader's barriers, and the
+                // peer does not leave before the leader (cluster barrier below)
                 const uint64_t t0 = ptx::globaltimer();
                 for (int i = 0; i < stages; i++) {
                     if (!(armed >> i & 1u)) continue;
@@ -474,15 +543,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (ptx::elect_one()) {
+        // ------------------------------------------------------------ MMA issuer (the leader of a pair)
+        if (leader && ptx::elect_one()) {
             int s = 0;
             uint32_t ph = 0;
             int acc = 0;
             uint32_t aph = 0;
             bool ok = true, issued = false;
-            for (int i = 0, t; ok && (t = cta_tile<MODE>(i, total, splan->tiles1, args.comp)) >= 0; i++) {
-                const Tile tl = decode_tile<MODE>(nb, t, args, args2, splan);
+            for (int i = 0, t; ok && (t = cta_tile<MODE, PAIR>(i, total, splan->tiles1, args.comp)) >= 0; i++) {
+                const Tile tl = decode_tile<MODE, PAIR>(nb, t, args, args2, splan, rank);
                 if (tl.kb0 >= tl.kb1) continue;
                 if (!bounded_wait(ptx::smem_u32(&ctl->tempty[acc]), aph ^ 1u, ctl, args.err)) {
                     ok = false;
@@ -490,7 +559,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 ptx::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)acc * 256u;
-                const uint32_t idesc = ptx::idesc_bf16_f32(128, (uint32_t)tl.n_mma);
+                const uint32_t idesc = ptx::idesc_bf16_f32(PAIR ? 256 : 128, (uint32_t)tl.n_mma);
                 for (int kb = tl.kb0; kb < tl.kb1; kb++) {
                     if (!bounded_wait(ptx::smem_u32(&ctl->full[s]), ph, ctl, args.err)) {
                         ok = false;
@@ -501,25 +570,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t b_addr = a_addr + kATileBytes;
 #pragma unroll
                     for (int kk = 0; kk < kBlockK / 16; kk++) {
-                        ptx::mma_bf16_ss(d_tmem, ptx::sw128_kmajor_desc(a_addr + kk * 32),
-                                         ptx::sw128_kmajor_desc(b_addr + kk * 32), idesc,
-                                         (kb > tl.kb0 || kk > 0) ? 1u : 0u);
+                        const uint64_t ad = ptx::sw128_kmajor_desc(a_addr + kk * 32);
+                        const uint64_t bd = ptx::sw128_kmajor_desc(b_addr + kk * 32);
+                        const uint32_t accum = (kb > tl.kb0 || kk > 0) ? 1u : 0u;
+                        if (PAIR) ptx::mma_bf16_ss_pair(d_tmem, ad, bd, idesc, accum);
+                        else ptx::mma_bf16_ss(d_tmem, ad, bd, idesc, accum);
                     }
                     issued = true;
-                    ptx::mma_commit(ptx::smem_u32(&ctl->empty[s]));
+                    // the stage is free in both CTAs once these MMAs have read it
+                    if (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&ctl->empty[s]), 3);
+                    else ptx::mma_commit(ptx::smem_u32(&ctl->empty[s]));
                     if (++s == stages) {
                         s = 0;
                         ph ^= 1u;
                     }
                 }
                 if (!ok) break;
-                ptx::mma_commit(ptx::smem_u32(&ctl->tfull[acc]));
+                if (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&ctl->tfull[acc]), 3);
+                else ptx::mma_commit(ptx::smem_u32(&ctl->tfull[acc]));
                 acc ^= 1;
                 if (acc == 0) aph ^= 1u;
             }
             if (!ok && issued) {
                 // drain: every MMA issued so far completes before TMEM is freed
-                ptx::mma_commit(ptx::smem_u32(&ctl->drain));
+                if (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&ctl->drain), 1);
+                else ptx::mma_commit(ptx::smem_u32(&ctl->drain));
                 const uint64_t t0 = ptx::globaltimer();
                 while (!ptx::mbar_try_wait(ptx::smem_u32(&ctl->drain), 0) &&
                        ptx::globaltimer() - t0 < kWaitTimeoutNs) {
@@ -531,8 +606,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int quad = warp & 3;            // TMEM lane quadrant this warp may access
         int acc = 0;
         uint32_t aph = 0;
-        for (int i = 0, t; (t = cta_tile<MODE>(i, total, splan->tiles1, args.comp)) >= 0; i++) {
-            const Tile tl = decode_tile<MODE>(nb, t, args, args2, splan);
+        for (int i = 0, t; (t = cta_tile<MODE, PAIR>(i, total, splan->tiles1, args.comp)) >= 0; i++) {
+            const Tile tl = decode_tile<MODE, PAIR>(nb, t, args, args2, splan, rank);
             if (tl.kb0 >= tl.kb1) continue;
             // a down tile's gates (lane l: columns l + 32 i), fetched before the accumulator wait
             float gates[8];
@@ -561,7 +636,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (MODE != MODE_ROUTER && tl.gated) {
                     // lanes 0-15: gate of f row 16*quad + lane; lanes 16-31: up of the same row
                     const int half = lane >> 4;
-                    const int frow = tl.m * 64 + quad * 16 + (lane & 15);
+                    const int frow = tl.ma * 64 + quad * 16 + (lane & 15);
 #pragma unroll
                     for (int p = 0; p < 8; p++) {
                         const float send = __uint_as_float(half ? v[2 * p] : v[2 * p + 1]);
@@ -573,7 +648,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             out[(size_t)(tl.row0 + col) * ld + frow] = __float2bfloat16_rn(silu_f(g) * u);
                     }
                 } else if (MODE != MODE_ROUTER) {
-                    const int drow = tl.m * 128 + quad * 32 + lane;
+                    const int drow = tl.ma * 128 + quad * 32 + lane;
                     const int gi = c0 >> 5;
                     const float mine = gi == 0 ? gates[0] : gi == 1 ? gates[1] : gi == 2 ? gates[2] : gi == 3 ? gates[3]
                                      : gi == 4 ? gates[4] : gi == 5 ? gates[5] : gi == 6 ? gates[6] : gates[7];
@@ -602,7 +677,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&ctl->tempty[acc]));
+            if (lane == 0) {
+                // the accumulator is free again: tell the MMA issuer (the leader's, for a pair)
+                if (PAIR) ptx::mbar_arrive_cluster(leader_bar(&ctl->tempty[acc]));
+                else ptx::mbar_arrive(ptx::smem_u32(&ctl->tempty[acc]));
+            }
             acc ^= 1;
             if (acc == 0) aph ^= 1u;
             if (MODE == MODE_FUSED && tl.gated) {
@@ -616,10 +695,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
 
     ptx::tc_fence_before();
-    __syncthreads();
+    // neither CTA of a pair leaves (or frees TMEM) while the other may still
+    // signal its barriers or the leader's MMAs may still write its TMEM
+    if (PAIR) ptx::cluster_sync();
+    else __syncthreads();
+    __syncwarp();   // the dealloc below is .sync.aligned: warp 1 converged
     if (warp == 1) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem_base, kTmemCols);
+        if (PAIR) ptx::tmem_dealloc_pair(tmem_base, kTmemCols);
+        else ptx::tmem_dealloc(tmem_base, kTmemCols);
     }
 }
 

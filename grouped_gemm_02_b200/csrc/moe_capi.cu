@@ -36,6 +36,7 @@ struct DeviceState {
     bool ready = false;
     bool supported = false;
     int sm_count = 0;
+    int pair_grid = 0;   // CTAs of a CTA-pair GEMM launch: 2 x the clusters that fit at once (0: none)
 };
 
 std::mutex g_mu;
@@ -70,6 +71,53 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// The same with clusters of two CTAs (the CTA-pair GEMMs).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pair(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                        Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    ++t_launches;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// How many clusters of two CTAs of `kernel` can be resident at once (0 on error).
+template <typename... KArgs>
+int max_pair_clusters(void (*kernel)(KArgs...), size_t smem)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
 // Per-device one-time set-up: architecture check, SM count, kernel attributes.
 int device_setup(DeviceState** out)
 {
@@ -99,8 +147,20 @@ int device_setup(DeviceState** out)
                 cudaFuncSetAttribute(grouped_gemm_fp8_kernel<FP8_DOWN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kFp8SmemBytes) != cudaSuccess ||
                 cudaFuncSetAttribute(grouped_gemm_fp8_kernel<FP8_FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     kFp8SmemBytes) != cudaSuccess)
+                                     kFp8SmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(grouped_gemm_kernel<MODE_GATED, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(grouped_gemm_kernel<MODE_DOWN, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(grouped_gemm_kernel<MODE_FUSED, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) != cudaSuccess)
                 return MOE_ERR_CUDA;
+            // CTA pairs: a grid of exactly the clusters that fit at once, so the
+            // persistent pairs all start together (the same count for every mode)
+            int pc = max_pair_clusters(grouped_gemm_kernel<MODE_GATED, true>, kGemmSmemBytes);
+            pc = std::min(pc, max_pair_clusters(grouped_gemm_kernel<MODE_DOWN, true>, kGemmSmemBytes));
+            pc = std::min(pc, max_pair_clusters(grouped_gemm_kernel<MODE_FUSED, true>, kGemmSmemBytes));
+            st.pair_grid = 2 * std::min(pc, sms / 2);
             if (!g_encode) {
                 cudaDriverEntryPointQueryResult q;
                 void* fn = nullptr;
@@ -240,18 +300,18 @@ int run_topk(const TopkSource& s, int T, int E, int k, int32_t* idx, float* w, u
 }
 
 // The general (multi-CTA) histogram / scan / scatter (/ gather of bf16 rows
-// into xp when xp is given).  unit_rows / m1_rows shape the tile plan.
+// into xp when xp is given).  `ps` shapes the tile plan.
 int run_permute(const int32_t* idx, const bf16* x, int T, int d, int E, int k, int32_t* counts, int32_t* offsets,
                 int32_t* perm, int32_t* inv_perm, bf16* xp, uint32_t* err, int32_t* block_counts, int32_t* plan,
-                int f, int shared_rows, int fs, int sms, cudaStream_t st, int unit_rows = kTileRows,
-                int m1_rows = 64, int64_t* inv_perm_launch = nullptr)
+                int f, int shared_rows, int fs, int sms, cudaStream_t st, PlanShape ps,
+                int64_t* inv_perm_launch = nullptr)
 {
     const int64_t P = (int64_t)T * k;
     const int nb = hist_blocks(P);
     cudaError_t e = launch(hist_kernel, dim3(nb), dim3(512), 0, st, idx, P, E, block_counts, err);
     if (e == cudaSuccess)
         e = launch(scan_kernel, dim3(1), dim3(1024), 0, st, block_counts, nb, E, counts, offsets, plan, f, d,
-                   shared_rows, fs, unit_rows, m1_rows);
+                   shared_rows, fs, ps);
     if (e == cudaSuccess)
         e = launch(scatter_kernel, dim3(nb), dim3(256), 0, st, idx, P, E, (const int32_t*)block_counts, perm,
                    inv_perm);
@@ -271,27 +331,66 @@ struct GemmOperands {
     int T, P, d, f, fs, E;
 };
 
+// Process-wide choices of the expert-GEMM launch form (moe_set_policy; -1 =
+// the library's rule).  Their first values come from MOE_GEMM_SPLIT (0: one
+// launch, 1: two) and MOE_GEMM_PAIR (0/1) when those are set.
+std::atomic<int> g_policy_fused{-2};
+std::atomic<int> g_policy_pair{-2};
+
+int env_switch(const char* name)
+{
+    const char* e = getenv(name);
+    return (e && (e[0] == '0' || e[0] == '1')) ? e[0] - '0' : -1;
+}
+
+int policy(std::atomic<int>& slot, const char* env, bool invert)
+{
+    int v = slot.load(std::memory_order_relaxed);
+    if (v == -2) {
+        int e = env_switch(env);
+        if (e >= 0 && invert) e = 1 - e;
+        int expect = -2;
+        slot.compare_exchange_strong(expect, e);
+        v = slot.load(std::memory_order_relaxed);
+    }
+    return v;
+}
+
 // One launch for both expert GEMMs (down tiles wait on per-block counters of
 // finished gate/up tiles) or two launches with a kernel boundary between them.
 // Measured on B200: the single launch saves the boundary's tail when few
 // token-expert pairs spread over many weight tiles (P <= 256 with f <= 4096:
 // 3-5% faster), and loses 4-10% once blocks hold more tokens, where the down
-// tiles' waits on the counters cost more than the boundary.  MOE_GEMM_SPLIT=1
-// forces two launches, MOE_GEMM_SPLIT=0 one; it is read once per process.
+// tiles' waits on the counters cost more than the boundary.
 bool gemm_fused(int P, int f)
 {
-    static const int forced = [] {
-        const char* e = getenv("MOE_GEMM_SPLIT");
-        return (e && (e[0] == '0' || e[0] == '1')) ? e[0] - '0' : -1;
-    }();
-    if (forced >= 0) return forced == 0;
+    const int forced = policy(g_policy_fused, "MOE_GEMM_SPLIT", /*invert=*/true);
+    if (forced >= 0) return forced == 1;
     return P <= 256 && f <= 4096;
 }
 
-// plan_ready: the plan was written two or more launches before the gate/up GEMM.
-int run_gemms(const GemmOperands& o, const int32_t* plan, bool plan_ready, uint32_t* err, int sms, cudaStream_t st,
-              bool prof = false)
+// CTA pairs (cta_group::2, 2 x 128 weight rows per tile, each SM loading half
+// of the token tile) halve each SM's operand traffic per MMA, which is what
+// limits the single-CTA tiles once experts hold hundreds of tokens; they are
+// taken whenever both expert GEMMs run as two launches (P > 256 or f > 4096)
+// and the device can hold the pair grid.
+bool gemm_pair(int P, int f, const DeviceState* dev)
 {
+    if (dev->pair_grid < 2) return false;
+    const int forced = policy(g_policy_pair, "MOE_GEMM_PAIR", /*invert=*/false);
+    if (forced >= 0) return forced == 1;
+    return !gemm_fused(P, f);
+}
+
+constexpr PlanShape kPlanSingle{kTileRows, 64, 128, 16, 0};
+constexpr PlanShape kPlanPair{kTileRows, 128, 256, 32, 1};
+
+// plan_ready: the plan was written two or more launches before the gate/up GEMM.
+// pair: the plan was cut for CTA pairs (kPlanPair) and the pair kernels run.
+int run_gemms(const GemmOperands& o, const int32_t* plan, bool plan_ready, uint32_t* err, const DeviceState* dev,
+              bool pair, cudaStream_t st, bool prof = false)
+{
+    const int sms = dev->sm_count;
     CUtensorMap a0, a1, b, a0s, a1s, bs, a2, b2, a2s, b2s;
     const uint64_t E = (uint64_t)o.E;
     // gate/up: A = W1/W3 rows (16-row boxes), B = xp rows; shared: Ws1/Ws3 and x
@@ -336,22 +435,31 @@ int run_gemms(const GemmOperands& o, const int32_t* plan, bool plan_ready, uint3
     g2.ld_out = o.d;
     g2.out_shared = o.ys;
     g2.ld_out_shared = o.d;
+    const dim3 grid(pair ? dev->pair_grid : sms), block(kGemmThreads);
     if (gemm_fused(o.P, o.f)) {
         // a gate/up tile streams d/64 k-blocks, a down tile f/64
         const int kb1 = (o.d + 63) / 64, kb2 = (o.f + 63) / 64;
         g1.comp = std::max(1, (kb1 + kb2 / 2) / kb2);
-        const cudaError_t e = launch(grouped_gemm_kernel<MODE_FUSED>, dim3(sms), dim3(kGemmThreads), kGemmSmemBytes,
-                                     st, a0, a1, b, a0s, a1s, bs, a2, b2, a2s, b2s, g1, g2);
+        const cudaError_t e =
+            pair ? launch_pair(grouped_gemm_kernel<MODE_FUSED, true>, grid, block, kGemmSmemBytes, st, a0, a1, b, a0s,
+                               a1s, bs, a2, b2, a2s, b2s, g1, g2)
+                 : launch(grouped_gemm_kernel<MODE_FUSED>, grid, block, kGemmSmemBytes, st, a0, a1, b, a0s, a1s, bs,
+                          a2, b2, a2s, b2s, g1, g2);
         phase_mark(prof, 3, st);   // the fused launch has no boundary: the down phase reads as zero
         return status_of(e);
     }
-    if (launch(grouped_gemm_kernel<MODE_GATED>, dim3(sms), dim3(kGemmThreads), kGemmSmemBytes, st, a0, a1, b, a0s,
-               a1s, bs, a0, b, a0, b, g1, g1) != cudaSuccess)
-        return MOE_ERR_CUDA;
+    const cudaError_t e1 =
+        pair ? launch_pair(grouped_gemm_kernel<MODE_GATED, true>, grid, block, kGemmSmemBytes, st, a0, a1, b, a0s,
+                           a1s, bs, a0, b, a0, b, g1, g1)
+             : launch(grouped_gemm_kernel<MODE_GATED>, grid, block, kGemmSmemBytes, st, a0, a1, b, a0s, a1s, bs, a0,
+                      b, a0, b, g1, g1);
+    if (e1 != cudaSuccess) return MOE_ERR_CUDA;
     phase_mark(prof, 3, st);
     g2.plan_ready = 1;   // written before the gate/up GEMM
-    return status_of(launch(grouped_gemm_kernel<MODE_DOWN>, dim3(sms), dim3(kGemmThreads), kGemmSmemBytes, st, a2,
-                            a2, b2, a2s, a2s, b2s, a2, b2, a2s, b2s, g2, g2));
+    return status_of(pair ? launch_pair(grouped_gemm_kernel<MODE_DOWN, true>, grid, block, kGemmSmemBytes, st, a2, a2,
+                                        b2, a2s, a2s, b2s, a2, b2, a2s, b2s, g2, g2)
+                          : launch(grouped_gemm_kernel<MODE_DOWN>, grid, block, kGemmSmemBytes, st, a2, a2, b2, a2s,
+                                   a2s, b2s, a2, b2, a2s, b2s, g2, g2));
 }
 
 // inv_perm_launch: this thread's launch count right after the kernel that wrote
@@ -441,7 +549,8 @@ int moe_permute(const int32_t* topk_idx, const moe_bf16* x, int64_t T, int64_t d
     if ((rc = device_setup(&dev))) return rc;
     return run_permute(topk_idx, reinterpret_cast<const bf16*>(x), (int)T, (int)d, (int)E, (int)k, counts, offsets,
                        perm, inv_perm, reinterpret_cast<bf16*>(xp), at<uint32_t>(ws, L.err),
-                       at<int32_t>(ws, L.block_counts), nullptr, 0, 0, 0, dev->sm_count, as_stream(stream));
+                       at<int32_t>(ws, L.block_counts), nullptr, 0, 0, 0, dev->sm_count, as_stream(stream),
+                       kPlanSingle);
 }
 
 int moe_grouped_gemm(const moe_bf16* xp, const int32_t* counts, const int32_t* offsets, const int32_t* perm,
@@ -462,8 +571,9 @@ int moe_grouped_gemm(const moe_bf16* xp, const int32_t* counts, const int32_t* o
     if ((rc = device_setup(&dev))) return rc;
     cudaStream_t st = as_stream(stream);
     int32_t* plan = at<int32_t>(ws, L.plan);
+    const bool pair = gemm_pair((int)(T * k), (int)f, dev);
     if (launch(plan_kernel, dim3(1), dim3(1024), 0, st, counts, offsets, (int)E, plan, (int)f, (int)d, 0, 0,
-               (int)kTileRows, 64) != cudaSuccess)
+               pair ? kPlanPair : kPlanSingle) != cudaSuccess)
         return MOE_ERR_CUDA;
     GemmOperands o{};
     o.xp = reinterpret_cast<const bf16*>(xp);
@@ -481,7 +591,7 @@ int moe_grouped_gemm(const moe_bf16* xp, const int32_t* counts, const int32_t* o
     o.f = (int)f;
     o.fs = 0;
     o.E = (int)E;
-    return run_gemms(o, plan, /*plan_ready=*/false, at<uint32_t>(ws, L.err), dev->sm_count, st);
+    return run_gemms(o, plan, /*plan_ready=*/false, at<uint32_t>(ws, L.err), dev, pair, st);
 }
 
 int moe_combine(const moe_bf16* y_p, const int32_t* inv_perm, const moe_bf16* shared_out, int64_t T, int64_t k,
@@ -546,12 +656,13 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
         return rc;
     const TopkSource src = topk_source(rs, logits, partials, bias, iT, iE);
     const int64_t P = T * k;
+    const bool pair = gemm_pair((int)P, (int)f, dev);
     if ((rc = run_topk(src, iT, iE, ik, idx, w, err, st))) return rc;
     phase_mark(prof, 1, st);
     if (P <= kSmallPairs) {
         // one CTA: histogram, scan, stable ranks and the tile plan
         if (launch(permute_small_kernel, dim3(1), dim3(1024), 0, st, (const int32_t*)idx, (int)P, iE, counts, offsets,
-                   perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared, (int)kTileRows, 64, err) !=
+                   perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared, pair ? kPlanPair : kPlanSingle, err) !=
             cudaSuccess)
             return MOE_ERR_CUDA;
         inv_perm_launch = t_launches;
@@ -562,7 +673,7 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     } else {
         if ((rc = run_permute(idx, xb, iT, id, iE, ik, counts, offsets, perm, inv_perm, xp, err,
                               at<int32_t>(ws, L.block_counts), plan, (int)f, shared_rows, (int)f_shared,
-                              dev->sm_count, st, kTileRows, 64, &inv_perm_launch)))
+                              dev->sm_count, st, pair ? kPlanPair : kPlanSingle, &inv_perm_launch)))
             return rc;
     }
     GemmOperands o{};
@@ -588,7 +699,7 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     o.E = iE;
     phase_mark(prof, 2, st);
     // the plan was written two or more launches before the gate/up GEMM (the gather is in between)
-    if ((rc = run_gemms(o, plan, /*plan_ready=*/true, err, dev->sm_count, st, prof))) return rc;
+    if ((rc = run_gemms(o, plan, /*plan_ready=*/true, err, dev, pair, st, prof))) return rc;
     phase_mark(prof, 4, st);
     rc = run_combine(y_p, inv_perm, ys, iT, ik, id, reinterpret_cast<bf16*>(out), st, inv_perm_launch);
     phase_mark(prof, 5, st);
@@ -611,6 +722,16 @@ int moe_record_phase_events(void* const* events, int n)
 }
 
 int64_t moe_launch_counter(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int moe_set_policy(int what, int value)
+{
+    if (value < -1 || value > 1) return MOE_ERR_ARG;
+    switch (what) {
+    case MOE_POLICY_ONE_LAUNCH: g_policy_fused.store(value); return MOE_OK;
+    case MOE_POLICY_CTA_PAIRS: g_policy_pair.store(value); return MOE_OK;
+    default: return MOE_ERR_ARG;
+    }
+}
 
 int moe_workspace_tensor(void* ws, int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, int64_t f_shared, int which,
                          void** ptr)
@@ -878,13 +999,13 @@ int moe_layer_forward_fp8(const moe_bf16* x, const moe_bf16* Wg, const float* bi
     phase_mark(prof, 1, st);
     if (P <= kSmallPairs) {
         if (launch(permute_small_kernel, dim3(1), dim3(1024), 0, st, (const int32_t*)idx, (int)P, iE, counts, offsets,
-                   perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared, kFp8TileRows, 128, err) !=
+                   perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared, kPlanFp8, err) !=
             cudaSuccess)
             return MOE_ERR_CUDA;
         inv_perm_launch = t_launches;
     } else if ((rc = run_permute(idx, xb, iT, id, iE, ik, counts, offsets, perm, inv_perm, nullptr, err,
                                  at<int32_t>(ws, L.ctrl.block_counts), plan, (int)f, shared_rows, (int)f_shared,
-                                 dev->sm_count, st, kFp8TileRows, 128, &inv_perm_launch))) {
+                                 dev->sm_count, st, kPlanFp8, &inv_perm_launch))) {
         return rc;
     }
     const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)dev->sm_count * 16));
@@ -996,5 +1117,5 @@ extern "C" int moe_permute_noalloc(const int32_t* topk_idx, const moe_bf16* x, i
     if (cudaMemsetAsync(err, 0, sizeof(uint32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
     return run_permute(topk_idx, reinterpret_cast<const bf16*>(x), (int)T, (int)d, (int)E, (int)k, counts, offsets,
                        perm, inv_perm, reinterpret_cast<bf16*>(xp), err, scratch, nullptr, 0, 0, 0, dev->sm_count,
-                       st);
+                       st, kPlanSingle);
 }

@@ -79,17 +79,17 @@ __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b -
 // thread tid < E holds counts[tid] in `c` and offsets[tid] in `off`):
 //   * one block per expert with tokens, plus the shared expert (T rows) when
 //     `shared_rows` > 0;
-//   * a block of n rows is cut into units = ceil(n / unit_rows) chunks of
-//     chunk = roundup16(ceil(n / units)) rows (unit_rows = 256 for bf16, 64
-//     for the FP8 path) -- the tile width follows the live count, so a
-//     3-token expert gets a 16-wide tile and a hot expert the widest ones;
+//   * a block of n rows is cut into units = ceil(n / ps.unit_rows) chunks of
+//     chunk = ceil(n / units) rounded up to ps.align rows -- the tile width
+//     follows the live count, so a 3-token expert gets a 16-wide tile and a
+//     hot expert the widest ones;
 //   * blocks sorted by n descending (ties: lower expert id), so the heaviest
 //     tiles are dealt first;
-//   * tile prefixes for both GEMMs: units * ceil(M / m1_rows) gate/up tiles
-//     (m1_rows = 64 for bf16, 128 for FP8) and units * ceil(d / 128) down tiles.
+//   * tile prefixes for both GEMMs: units * ceil(M / ps.m1_rows) gate/up tiles
+//     and units * ceil(d / ps.m2_rows) down tiles; the header records whether
+//     the tiles are cut for CTA pairs.
 __device__ __forceinline__ void build_plan(int c, int off, int E, int pairs, int32_t* __restrict__ plan, int f, int d,
-                                           int shared_rows, int f_shared, int* warp_sums, int unit_rows = kTileRows,
-                                           int m1_rows = 64)
+                                           int shared_rows, int f_shared, int* warp_sums, PlanShape ps)
 {
     __shared__ int s_n[kMaxGroups];
     __shared__ int s_order[kMaxGroups];
@@ -122,8 +122,8 @@ __device__ __forceinline__ void build_plan(int c, int off, int E, int pairs, int
     if (tid < nact) {
         const int g = s_order[tid];
         const int n = s_n[g];
-        const int units = ceil_div(n, unit_rows);
-        const int chunk = ceil_div(ceil_div(n, units), 16) * 16;
+        const int units = ceil_div(n, ps.unit_rows);
+        const int chunk = ceil_div(ceil_div(n, units), ps.align) * ps.align;
         const int M1 = g < E ? f : f_shared;
         pa.group[tid] = g;
         pa.row0[tid] = g < E ? s_off[g] : 0;
@@ -131,8 +131,8 @@ __device__ __forceinline__ void build_plan(int c, int off, int E, int pairs, int
         pa.chunk[tid] = chunk;
         pa.units[tid] = units;
         pa.dep[tid] = 0;
-        my_t1 = units * ceil_div(M1, m1_rows);
-        my_t2 = units * ceil_div(d, 128);
+        my_t1 = units * ceil_div(M1, ps.m1_rows);
+        my_t2 = units * ceil_div(d, ps.m2_rows);
         my_chunk = chunk;
     }
     const int p1 = block_inclusive_scan(my_t1, warp_sums);
@@ -153,6 +153,7 @@ __device__ __forceinline__ void build_plan(int c, int off, int E, int pairs, int
         h->n_blocks = nact;
         h->n_max = m;
         h->pairs = pairs;
+        h->pair = ps.pair;
         pa.tb1[0] = 0;
         pa.tb2[0] = 0;
         h->tiles1 = nact > 0 ? pa.tb1[nact] : 0;   // written above, visible after the barrier
@@ -168,7 +169,7 @@ __device__ __forceinline__ void build_plan(int c, int off, int E, int pairs, int
 __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ block_counts, int nblk_hist, int E,
                                                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                                     int32_t* __restrict__ plan, int f, int d, int shared_rows,
-                                                    int f_shared, int unit_rows, int m1_rows)
+                                                    int f_shared, PlanShape ps)
 {
     __shared__ int warp_sums[32];
     __shared__ int s_pairs;
@@ -195,14 +196,14 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ block_
         s_pairs = incl;
     }
     __syncthreads();
-    if (plan) build_plan(c, off, E, s_pairs, plan, f, d, shared_rows, f_shared, warp_sums, unit_rows, m1_rows);
+    if (plan) build_plan(c, off, E, s_pairs, plan, f, d, shared_rows, f_shared, warp_sums, ps);
 }
 
 // Single CTA of 1024 threads: the tile plan from counts/offsets already on the device.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ counts,
                                                     const int32_t* __restrict__ offsets, int E,
                                                     int32_t* __restrict__ plan, int f, int d, int shared_rows,
-                                                    int f_shared, int unit_rows, int m1_rows)
+                                                    int f_shared, PlanShape ps)
 {
     __shared__ int warp_sums[32];
     ptx::grid_dep_wait();
@@ -210,7 +211,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
     const int tid = threadIdx.x;
     const int c = tid < E ? counts[tid] : 0;
     const int off = tid < E ? offsets[tid] : 0;
-    build_plan(c, off, E, offsets[E], plan, f, d, shared_rows, f_shared, warp_sums, unit_rows, m1_rows);
+    build_plan(c, off, E, offsets[E], plan, f, d, shared_rows, f_shared, warp_sums, ps);
 }
 
 // ---------------------------------------------------------------- small-T permutation
@@ -226,8 +227,8 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t* __re
                                                              int32_t* __restrict__ perm,
                                                              int32_t* __restrict__ inv_perm,
                                                              int32_t* __restrict__ plan, int f, int d,
-                                                             int shared_rows, int f_shared, int unit_rows,
-                                                             int m1_rows, uint32_t* __restrict__ err)
+                                                             int shared_rows, int f_shared, PlanShape ps,
+                                                             uint32_t* __restrict__ err)
 {
     // s_wcnt[w][e]: pairs of warp w (pairs 32w..32w+31) routed to expert e (<= 32)
     __shared__ __align__(16) uint8_t s_wcnt[32][kMaxExperts];
@@ -273,7 +274,7 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t* __re
     __shared__ int s_pairs;
     if (tid == E - 1) s_pairs = incl;
     __syncthreads();
-    if (plan) build_plan(c, off, E, s_pairs, plan, f, d, shared_rows, f_shared, warp_sums, unit_rows, m1_rows);
+    if (plan) build_plan(c, off, E, s_pairs, plan, f, d, shared_rows, f_shared, warp_sums, ps);
 }
 
 // ---------------------------------------------------------------- scatter

@@ -28,7 +28,7 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_topk", 
            "moe_permute_noalloc", "moe_grouped_gemm", "moe_combine", "moe_layer_forward", "moe_workspace_tensor",
            "moe_record_phase_events", "moe_launch_counter", "moe_get_device_error", "moe_clear_device_error",
            "moe_selftest_wait_timeout",
-           "moe_status_string", "moe_quantize_fp8_rows", "moe_quantize_fp8_blocks", "moe_workspace_size_fp8",
+           "moe_status_string", "moe_set_policy", "moe_quantize_fp8_rows", "moe_quantize_fp8_blocks", "moe_workspace_size_fp8",
            "moe_workspace_tensor_fp8", "moe_layer_forward_fp8")
 
 
@@ -67,6 +67,7 @@ def lib() -> C.CDLL:
             "moe_status_string": [C.c_int],
             "moe_record_phase_events": [C.POINTER(vp), C.c_int],
             "moe_launch_counter": [],
+            "moe_set_policy": [C.c_int, C.c_int],
             "moe_quantize_fp8_rows": [vp, i64, i64, vp, vp, vp],
             "moe_quantize_fp8_blocks": [vp, i64, i64, vp, vp, vp],
             "moe_workspace_size_fp8": [i64, i64, i64, i64, i64, i64, C.POINTER(sz)],
@@ -160,6 +161,14 @@ def moe_record_phase_events(events) -> None:
             e.record()
     arr = (C.c_void_p * len(events))(*[C.c_void_p(e.cuda_event) for e in events])
     _call("moe_record_phase_events", arr, len(events))
+
+
+POLICY_ONE_LAUNCH, POLICY_CTA_PAIRS = 1, 2
+
+
+def moe_set_policy(what: int, value: int) -> None:
+    """Force (0 / 1) or restore (-1) one of the library's launch-form choices for the process."""
+    _call("moe_set_policy", what, value)
 
 
 def moe_launch_counter() -> int:

@@ -231,13 +231,28 @@ MOE_API int moe_layer_forward_fp8(const moe_bf16 *x, const moe_bf16 *Wg, const f
  * used once (the call after it records nothing).  n = 0 cancels. */
 MOE_API int moe_record_phase_events(void *const *events, int n);
 
+/* Process-wide choices of how the expert GEMMs run, for comparisons and
+ * tests (the pages have no counterpart).  value -1 restores the library's
+ * rule; 0 / 1 force the choice for every later call in the process.  Results
+ * do not depend on these choices beyond fp32 summation order inside a tile.
+ *   MOE_POLICY_ONE_LAUNCH  1: gate/up and down tiles in one persistent launch,
+ *                          0: two launches (rule: one when T*k <= 256 and f <= 4096)
+ *   MOE_POLICY_CTA_PAIRS   1: tiles of 2 x 128 weight rows on CTA pairs
+ *                          (cta_group::2), 0: single-CTA tiles of 128 rows
+ *                          (rule: pairs whenever two launches run)
+ * Returns MOE_ERR_ARG for an unknown switch or value. */
+#define MOE_POLICY_ONE_LAUNCH 1
+#define MOE_POLICY_CTA_PAIRS 2
+MOE_API int moe_set_policy(int what, int value);
+
 /* Number of kernels this library has launched in this process so far. */
 MOE_API int64_t moe_launch_counter(void);
 
 /* Device pointers of the layer intermediates inside a layer workspace
  * (which: 0 logits, 1 topk_idx, 2 topk_w, 3 counts, 4 offsets, 5 perm,
  * 6 inv_perm, 7 xp, 8 h, 9 y_p, 10 hs, 11 ys, 12 the tile plan).  The tile plan is
- * MOE_PLAN_INTS int32: a header {n_blocks, tiles1, tiles2, n_max, pairs, 3 x 0},
+ * MOE_PLAN_INTS int32: a header {n_blocks, tiles1, tiles2, n_max, pairs,
+ * pair (1: tiles cut for CTA pairs), 2 x 0},
  * then arrays of 513 entries group, row0, rows, chunk, units, two tile
  * prefixes of 514 entries (gate/up, down) and 513 per-block counters of
  * finished gate/up tiles (see the tile plan in the grouped-GEMM comment).

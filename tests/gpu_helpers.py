@@ -100,9 +100,9 @@ def decode_plan(plan) -> dict:
     """The tile plan a layer leaves in its workspace (int32 [MOE_PLAN_INTS]) as host arrays."""
     p = plan.cpu().numpy() if hasattr(plan, "cpu") else np.asarray(plan)
     G = PLAN_GROUPS
-    nb, tiles1, tiles2, n_max, pairs = (int(v) for v in p[:5])
+    nb, tiles1, tiles2, n_max, pairs, pair = (int(v) for v in p[:6])
     o = 8
-    out = {"n_blocks": nb, "tiles1": tiles1, "tiles2": tiles2, "n_max": n_max, "pairs": pairs}
+    out = {"n_blocks": nb, "tiles1": tiles1, "tiles2": tiles2, "n_max": n_max, "pairs": pairs, "pair": pair}
     for name in ("group", "row0", "rows", "chunk", "units"):
         out[name] = p[o:o + nb].astype(np.int64)
         o += G
@@ -115,12 +115,12 @@ def decode_plan(plan) -> dict:
 
 
 def check_plan(plan: dict, counts: np.ndarray, offsets: np.ndarray, T: int, f: int, d: int, f_shared: int,
-               unit_max: int, m1_rows: int, what: str = "") -> None:
+               unit_max: int, m1_rows: int, what: str = "", m2_rows: int = 128, align: int = 16) -> None:
     """The invariants of a tile plan built from the live histogram:
     * one block per expert with tokens (+ the shared expert over all T tokens),
       heaviest first (ties: lower group id);
     * each block's rows [row0, row0 + rows) are cut into `units` chunks of
-      `chunk` rows, a multiple of 16 and at most unit_max, every chunk non-empty,
+      `chunk` rows, a multiple of `align` and at most unit_max, every chunk non-empty,
       so the tiles of a block cover its rows exactly once;
     * the routed blocks' rows tile [0, offsets[E]) exactly once;
     * the tile prefixes count units x M-tiles of each GEMM, and n_max is the
@@ -138,7 +138,7 @@ def check_plan(plan: dict, counts: np.ndarray, offsets: np.ndarray, T: int, f: i
             assert rows[i] == T and r0[i] == 0, (what, i)
     key = [(-int(rows[i]), int(g[i])) for i in range(n_blocks)]
     assert key == sorted(key), f"{what}: blocks not heaviest first"
-    assert np.all(ch % 16 == 0) and np.all(ch >= 16) and np.all(ch <= unit_max), what
+    assert np.all(ch % align == 0) and np.all(ch >= align) and np.all(ch <= unit_max), what
     assert np.all(ch * un >= rows) and np.all(ch * (un - 1) < rows), f"{what}: an empty or missing unit"
     cover = np.zeros(int(offsets[-1]), dtype=np.int64)
     for i in range(n_blocks):
@@ -150,7 +150,7 @@ def check_plan(plan: dict, counts: np.ndarray, offsets: np.ndarray, T: int, f: i
             cover[a:b] += 1
     assert np.all(cover == 1), f"{what}: routed rows not covered exactly once"
     m1 = np.array([-(-(f if gi < E else f_shared) // m1_rows) for gi in g], dtype=np.int64)
-    m2 = -(-d // 128)
+    m2 = -(-d // m2_rows)
     assert np.array_equal(plan["tb1"], np.concatenate([[0], np.cumsum(un * m1)])), what
     assert np.array_equal(plan["tb2"], np.concatenate([[0], np.cumsum(un * m2)])), what
     assert plan["tiles1"] == plan["tb1"][-1] and plan["tiles2"] == plan["tb2"][-1], what
@@ -158,9 +158,44 @@ def check_plan(plan: dict, counts: np.ndarray, offsets: np.ndarray, T: int, f: i
     assert plan["pairs"] == int(offsets[-1]), what
 
 
+# The launch-form switches the tests have set through moe_set_policy (-1: the library's rule).
+POLICY = {"one_launch": -1, "pairs": -1}
+
+
+class policy:
+    """Context manager: force the library's launch-form switches, restore them after."""
+
+    def __init__(self, one_launch: int = -1, pairs: int = -1):
+        self.want = {"one_launch": one_launch, "pairs": pairs}
+
+    def __enter__(self):
+        from grouped_gemm_02_b200 import moe
+        self.prev = dict(POLICY)
+        moe.moe_set_policy(moe.POLICY_ONE_LAUNCH, self.want["one_launch"])
+        moe.moe_set_policy(moe.POLICY_CTA_PAIRS, self.want["pairs"])
+        POLICY.update(self.want)
+        return self
+
+    def __exit__(self, *exc):
+        from grouped_gemm_02_b200 import moe
+        moe.moe_set_policy(moe.POLICY_ONE_LAUNCH, self.prev["one_launch"])
+        moe.moe_set_policy(moe.POLICY_CTA_PAIRS, self.prev["pairs"])
+        POLICY.update(self.prev)
+        return False
+
+
 def fused_gemms(P: int, f: int) -> bool:
-    """The library's rule: both expert GEMMs in one launch for P <= 256 pairs and f <= 4096."""
+    """One launch for both expert GEMMs: the library's rule (P <= 256 pairs and f <= 4096) or the forced switch."""
+    if POLICY["one_launch"] >= 0:
+        return POLICY["one_launch"] == 1
     return P <= 256 and f <= 4096
+
+
+def pair_gemms(P: int, f: int) -> bool:
+    """CTA-pair tiles (bf16 path): whenever two launches run, unless forced."""
+    if POLICY["pairs"] >= 0:
+        return POLICY["pairs"] == 1
+    return not fused_gemms(P, f)
 
 
 def check_routing(views, s: wl.LayerShape, what: str):
@@ -180,10 +215,21 @@ def check_routing(views, s: wl.LayerShape, what: str):
     return g_L, o_idx, o_w, rc, ro
 
 
-def check_layer_plan(views, s: wl.LayerShape, counts, offsets, unit_max, m1_rows, what):
+def check_layer_plan(views, s: wl.LayerShape, counts, offsets, what, fp8: bool = False):
+    """The plan the layer left in its workspace: invariants for the tile shape its
+    launch form uses, and (single launch) every gate/up tile's epilogue warps
+    published their h rows: 4 per tile and CTA."""
     plan = decode_plan(views["plan"])
-    check_plan(plan, counts, offsets, s.T, s.f, s.d, s.f_shared, unit_max, m1_rows, what)
-    # the single launch counts its finished gate/up tiles per block (4 epilogue warps per tile)
+    pair = (not fp8) and pair_gemms(s.P, s.f)
+    assert plan["pair"] == int(pair), f"{what}: plan cut for pair={plan['pair']}, expected {pair}"
+    if fp8:
+        unit_max, m1_rows, m2_rows, align = 112, 128, 128, 16
+    elif pair:
+        unit_max, m1_rows, m2_rows, align = 256, 128, 256, 32
+    else:
+        unit_max, m1_rows, m2_rows, align = 256, 64, 128, 16
+    check_plan(plan, counts, offsets, s.T, s.f, s.d, s.f_shared, unit_max, m1_rows, what, m2_rows, align)
     m1 = np.array([-(-(s.f if g < s.E else s.f_shared) // m1_rows) for g in plan["group"]], dtype=np.int64)
-    need = 4 * plan["units"] * m1 if fused_gemms(s.P, s.f) else np.zeros_like(m1)
+    warps = 8 if pair else 4
+    need = warps * plan["units"] * m1 if fused_gemms(s.P, s.f) else np.zeros_like(m1)
     assert np.array_equal(plan["dep"], need), f"{what}: gate/up tiles published {plan['dep']} != {need}"

@@ -117,7 +117,7 @@ def _fp8_layer_check(s: wl.LayerShape, seed: int, n_sample=None, device_inputs=F
     what = f"fp8 layer {s}"
     # routing (the bf16 router, as in the bf16 layer): bit-exact on identical fp32 logits
     g_L, o_idx, o_w, counts, offsets = H.check_routing(views, s, what)
-    H.check_layer_plan(views, s, counts, offsets, 112, 128, what)
+    H.check_layer_plan(views, s, counts, offsets, what, fp8=True)
     x_h = inp["x"].cpu()
     tokens = np.arange(s.T) if n_sample is None else H.sample_tokens(o_idx, s.E, n_sample, seed)
     L64 = oracle.router_logits(H.bits(x_h[tokens]), H.bits(inp["Wg"].cpu()), inp["bias"].cpu().numpy())

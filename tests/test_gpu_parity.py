@@ -163,7 +163,7 @@ def _layer_check(s: wl.LayerShape, seed: int, n_sample=None, device_inputs=False
     views = moe.workspace_views(ws, s.T, s.d, s.f, s.E, s.k, s.f_shared)
     what = f"layer {s}"
     g_L, o_idx, o_w, counts, offsets = H.check_routing(views, s, what)
-    H.check_layer_plan(views, s, counts, offsets, 256, 64, what)
+    H.check_layer_plan(views, s, counts, offsets, what)
     out_h = out.float().cpu().numpy()
 
     x_h = dev_inp["x"].cpu()
@@ -257,3 +257,34 @@ def test_empty_and_single_token():
     x0 = inp["x"][:0]
     out0 = moe.moe_layer_forward(x0, inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], s.k, ws)
     assert out0.shape == (0, s.d)
+
+
+FORMS = [(1, 0), (0, 0), (1, 1), (0, 1)]     # (one launch, CTA pairs)
+
+
+@pytest.mark.parametrize("one_launch,pairs", FORMS)
+@pytest.mark.parametrize("name,kw", [
+    ("decode64", dict(alpha=0.1)),
+    ("deepseek_v3", dict(T=64, alpha=0.05)),     # shared expert
+    ("kimi_k2", dict(T=256)),                    # hot experts with units of up to 256 tokens
+])
+def test_layer_every_launch_form(name, kw, one_launch, pairs):
+    """Both expert-GEMM launch forms on single CTAs and on CTA pairs, each checked
+    against the oracle (routing bit-exact, plan invariants, outputs in tolerance)."""
+    s = wl.shape(name, **kw)
+    with H.policy(one_launch=one_launch, pairs=pairs):
+        _layer_check(s, seed=3, n_sample=12, device_inputs=s.d * s.f * s.E > 2**31)
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("one_launch,pairs", FORMS)
+@pytest.mark.parametrize("T,d,f,E,k,alpha", [
+    (300, 256, 192, 4, 2, 1.0),     # f % 128 == 64: a pair's second CTA is past f on the last tile
+    (600, 320, 256, 8, 4, 0.1),     # d % 256 == 64: the same for the down tiles
+    (45, 128, 128, 3, 2, 1.0),      # widths of 16..48 rounded to 32 for pairs
+])
+def test_grouped_gemm_every_launch_form(T, d, f, E, k, alpha, one_launch, pairs):
+    s = wl.LayerShape("g", T=T, d=d, f=f, E=E, k=k, alpha=alpha, x_std=1.0)
+    with H.policy(one_launch=one_launch, pairs=pairs):
+        out, ref = _gemm_case(s, seed=T + d + f, alpha=alpha)
+    H.assert_close(out, ref, f"grouped GEMM T={T} d={d} f={f} E={E} k={k} one={one_launch} pairs={pairs}")

@@ -46,9 +46,16 @@ def test_plan_from_live_histogram(T, E, k, alpha, fs):
     views = moe.workspace_views(ws, s.T, s.d, s.f, s.E, s.k, s.f_shared)
     what = f"plan T={T} E={E} k={k} alpha={alpha} fs={fs}"
     g_L, o_idx, o_w, counts, offsets = H.check_routing(views, s, what)
-    H.check_layer_plan(views, s, counts, offsets, 256, 64, what)
+    H.check_layer_plan(views, s, counts, offsets, what)
     tokens = H.sample_tokens(o_idx, s.E, 24, seed=T)
     sh = {n: H.bits(inp[n]) for n in ("Ws1", "Ws3", "Ws2")} if fs else None
     ref = oracle.moe_ffn(H.bits(inp["x"][tokens]), H.bits(inp["W1"]), H.bits(inp["W3"]), H.bits(inp["W2"]),
                          o_idx[tokens], o_w[tokens], shared=sh)
     H.assert_close(out.float().cpu().numpy()[tokens], ref, what)
+
+
+@pytest.mark.parametrize("pairs", [0, 1])
+@pytest.mark.parametrize("T,E,k,alpha,fs", [(1000, 8, 2, 0.1, 64), (300, 256, 8, 0.5, 128), (17, 300, 8, 0.05, 192)])
+def test_plan_for_single_ctas_and_pairs(T, E, k, alpha, fs, pairs):
+    with H.policy(pairs=pairs):
+        test_plan_from_live_histogram(T, E, k, alpha, fs)
