@@ -37,15 +37,32 @@ struct PlanHeader {
     int32_t n_max;      // widest tile (tokens) in this launch
     int32_t pairs;      // routed pairs with a valid expert id (== offsets[E])
     int32_t pair;       // 1: tiles cut for CTA pairs (2 x 128 weight rows, widths a multiple of 32)
-    int32_t pad[2];
+    int32_t cls;        // histogram class the tile cap was looked up for, or kPlanClassCap / kPlanClassBucket
+    int32_t cap;        // most tokens per tile in this plan's cut
 };
 
-// How the plan cuts blocks into tiles: at most unit_rows tokens per tile, tile
-// widths a multiple of `align`; m1_rows f rows per gate/up tile and m2_rows d
-// rows per down tile.  Single CTAs: (256, 64, 128, 16, 0) for bf16 and
-// (112, 128, 128, 16, 0) for FP8; CTA pairs: (256, 128, 256, 32, 1).
+// How the plan cuts an expert's tokens into tiles (the tile policy):
+//   kTilesMatched  the live histogram's class picks the largest tile width
+//                  (cap) from the tuned table; each expert's width then follows
+//                  its own count: ceil(n / ceil(n / cap)), rounded up to align;
+//   kTilesBucket   one fixed width (unit_rows, chosen from T alone) for every
+//                  expert, the last tile of an expert padded -- the static
+//                  token-bucket selection the histogram-matched one is
+//                  measured against;
+//   kTilesCap      the per-expert widths under a given cap (unit_rows).
+constexpr int kPlanClassCap = -1;      // PlanHeader::cls of a plan cut under a given cap
+constexpr int kPlanClassBucket = -2;   // ... and of a token-bucket plan (every tile padded to `cap`)
+constexpr int kTilesMatched = 0;
+constexpr int kTilesBucket = 1;
+constexpr int kTilesCap = 2;
+
+// The tile shape of a launch form and the tile policy: at most unit_rows
+// tokens per tile, widths a multiple of `align`; m1_rows f rows per gate/up
+// tile and m2_rows d rows per down tile.  Single CTAs: (256, 64, 128, 16, 0)
+// for bf16 and (112, 128, 128, 16, 0) for FP8; CTA pairs: (256, 128, 256, 32, 1).
 struct PlanShape {
     int unit_rows, m1_rows, m2_rows, align, pair;
+    int policy;
 };
 
 struct PlanArrays {

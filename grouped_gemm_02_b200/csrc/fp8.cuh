@@ -46,7 +46,7 @@ constexpr uint32_t kFp8AccCols = 256;            // accumulator set b at column 
 constexpr uint32_t kSfColA0 = 480;               // scale factors: W1 (or W2) at 480, W3 at 484, tokens at 488
 constexpr uint32_t kSfColA1 = 484;
 constexpr uint32_t kSfColB = 488;
-constexpr int kFp8RingBytes = kRingBytes - 4096;
+constexpr int kFp8RingBytes = 204 * 1024;
 constexpr uint32_t kSfStageBytes = 2048;         // per stage: 128 token scales (fp32, by TMA) + 3 scale atoms
 
 // Smallest power-of-two exponent e with amax <= 448 * 2^e (amax > 0), from the
@@ -283,7 +283,7 @@ __device__ __forceinline__ Fp8Tile fp8_decode(int nb, int t, const Fp8Args& a, c
     const int start = u * b.w;
     tl.rows = min(b.w, b.z - start);
     tl.row0 = b.y + start;
-    tl.n_mma = (tl.rows + 15) & ~15;
+    tl.n_mma = sp->fixed_n ? sp->fixed_n : (tl.rows + 15) & ~15;
     tl.nkb = (tl.shared ? ta.K_shared : ta.K) / kFp8BlockK;
     return tl;
 }
@@ -418,7 +418,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     {
         const PlanArrays pa = plan_arrays(const_cast<int32_t*>(args.plan));
         const int32_t* tbg = KIND == FP8_DOWN ? pa.tb2 : pa.tb1;
-        if (threadIdx.x == 0) splan->tiles1 = hdr->tiles1;
+        if (threadIdx.x == 0) {
+            splan->tiles1 = hdr->tiles1;
+            splan->fixed_n = hdr->cls == kPlanClassBucket ? hdr->cap : 0;
+        }
         for (int i = threadIdx.x; i <= nb; i += blockDim.x) {
             splan->tb[i] = tbg[i];
             if (KIND == FP8_FUSED) splan->tb2[i] = pa.tb2[i];

@@ -30,10 +30,11 @@
 // the N slot (16..256, chosen per expert from its live count by the plan), so
 // a decode expert with 3 tokens costs one 16-wide MMA column block while a hot
 // expert gets 256-wide tiles.  For the gate/up GEMM one A tile holds 64 rows
-// of W1 and the same 64 rows of W3, interleaved 16 rows at a time (rows
-// 32q..32q+15 = W1, 32q+16..32q+31 = W3 for f rows 16q..16q+15), so that in
-// TMEM lane quadrant q the lanes 0-15 hold the gate and lanes 16-31 the up
-// projection of the same f rows; one shuffle pairs them in the epilogue.
+// of W1 (rows 0-63) and the same 64 rows of W3 (rows 64-127), each brought by
+// one TMA box, so TMEM lanes 0-63 hold the gate and lanes 64-127 the up
+// projection of the same f rows.  The epilogue warps of lane quadrants q and
+// q + 2 pair up and hand each other half of every 16-column chunk through
+// shared memory, so each finishes h = silu(g) u for 8 columns of 32 rows.
 //
 // Warp roles (192 threads, one CTA per SM, persistent over the tile list):
 //   warp 0     TMA producer (one elected lane) -> ring of smem stages
@@ -72,7 +73,7 @@ constexpr int kBlockK = 64;                          // bf16 elements per 128-by
 constexpr int kATileBytes = 128 * kBlockK * 2;       // 16 KB: 128 weight rows
 constexpr int kBRowBytes = kBlockK * 2;              // 128 B per token row
 constexpr int kMaxStages = 12;
-constexpr int kRingBytes = 208 * 1024;
+constexpr int kRingBytes = 200 * 1024;
 constexpr int kBarBytes = 512;
 constexpr uint32_t kTmemCols = 512;                  // 2 accumulators x 256 columns
 constexpr uint64_t kWaitTimeoutNs = 1000000000ull;   // 1 s
@@ -119,8 +120,12 @@ struct SmemPlan {
     int4 blk[kMaxGroups];       // group, row0, rows, chunk
     int units[kMaxGroups];
     int tiles1;                 // MODE_FUSED: gate/up tiles come first
+    int fixed_n;                // token-bucket plans: every tile's MMA width (padded); 0 otherwise
 };
-constexpr int kGemmSmemBytes = 1024 + kRingBytes + kBarBytes + (int)sizeof(SmemPlan);
+// gate/up epilogue: each pair of warps hands the other half of a 16-column chunk
+// through shared memory: [2 row quarters][2 buffers][2 directions][8 columns][32 lanes] fp32
+constexpr int kExchBytes = 2 * 2 * 2 * 8 * 32 * 4;
+constexpr int kGemmSmemBytes = 1024 + kRingBytes + kBarBytes + (int)sizeof(SmemPlan) + kExchBytes;
 static_assert(kGemmSmemBytes <= 227 * 1024, "shared memory budget");
 
 template <int MODE>
@@ -188,7 +193,7 @@ __device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a, co
     tl.rows = min(chunk, b.z - start);
     tl.row0 = b.y + start;
     // MMA width: a multiple of 16, of 32 for a pair (each CTA loads N/2 rows in 16-row boxes)
-    tl.n_mma = PAIR ? (tl.rows + 31) & ~31 : (tl.rows + 15) & ~15;
+    tl.n_mma = sp->fixed_n ? sp->fixed_n : PAIR ? (tl.rows + 31) & ~31 : (tl.rows + 15) & ~15;
     tl.K = tl.shared ? a.K_shared : a.K;
     if (MODE == MODE_FUSED && !gated) tl.K = tl.shared ? a2.K_shared : a2.K;
     tl.kb0 = 0;
@@ -328,11 +333,8 @@ __device__ __forceinline__ void issue_a(const KIter& it, uint32_t a_dst, uint32_
         const CUtensorMap* w1 = tl.shared ? mA0s : mA0;
         const CUtensorMap* w3 = tl.shared ? mA1s : mA1;
         const int a_row = (tl.shared ? 0 : tl.group * a.M) + tl.ma * 64;
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-            tma_load<PAIR>(a_dst + (32 * q) * 128, w1, full, kc, a_row + 16 * q, pol);
-            tma_load<PAIR>(a_dst + (32 * q + 16) * 128, w3, full, kc, a_row + 16 * q, pol);
-        }
+        tma_load<PAIR>(a_dst, w1, full, kc, a_row, pol);              // rows 0-63: gate
+        tma_load<PAIR>(a_dst + 64 * 128, w3, full, kc, a_row, pol);   // rows 64-127: up
     } else if (MODE == MODE_FUSED) {
         const int a_row = (tl.shared ? 0 : tl.group * a2.M) + tl.ma * 128;
         tma_load<PAIR>(a_dst, tl.shared ? mA2s : mA2, full, kc, a_row, pol);
@@ -343,13 +345,18 @@ __device__ __forceinline__ void issue_a(const KIter& it, uint32_t a_dst, uint32_
     }
 }
 
+// The token rows of a stage: 64-row boxes, then 16-row boxes for the rest
+// (fewer, larger TMA requests keep the ring full at large widths).
 template <bool PAIR>
-__device__ __forceinline__ void issue_b(const Tile& tl, int kb, uint32_t b_dst, uint32_t full, const CUtensorMap* b,
-                                        uint64_t pol)
+__device__ __forceinline__ void issue_b(const Tile& tl, int kb, uint32_t b_dst, uint32_t full, const CUtensorMap* b16,
+                                        const CUtensorMap* b64, uint64_t pol)
 {
     const int kc = kb * kBlockK;
-    for (int i = 0; i < tl.b_n / 16; i++)
-        tma_load<PAIR>(b_dst + i * 16 * kBRowBytes, b, full, kc, tl.b_row0 + 16 * i, pol);
+    const int n64 = tl.b_n >> 6;
+    for (int i = 0; i < n64; i++)
+        tma_load<PAIR>(b_dst + i * 64 * kBRowBytes, b64, full, kc, tl.b_row0 + 64 * i, pol);
+    for (int r = n64 * 64; r < tl.b_n; r += 16)
+        tma_load<PAIR>(b_dst + r * kBRowBytes, b16, full, kc, tl.b_row0 + r, pol);
 }
 
 template <int MODE, bool PAIR = false>
@@ -359,10 +366,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const __grid_constant__ CUtensorMap mA1s, const __grid_constant__ CUtensorMap mBs,
                         const __grid_constant__ CUtensorMap mA2, const __grid_constant__ CUtensorMap mB2,
                         const __grid_constant__ CUtensorMap mA2s, const __grid_constant__ CUtensorMap mB2s,
+                        const __grid_constant__ CUtensorMap mB64, const __grid_constant__ CUtensorMap mBs64,
+                        const __grid_constant__ CUtensorMap mB264, const __grid_constant__ CUtensorMap mB2s64,
                         const GemmArgs args, const GemmArgs args2)
 {
     // MODE_FUSED: args describe the gate/up tiles (W1/W3 = mA0/mA1, xp = mB),
     // args2 the down tiles (W2 = mA2, h = mB2); other modes ignore args2 and mA2..mB2s.
+    // mB64..mB2s64 are mB..mB2s with 64-row boxes.
     // PAIR: launched in clusters of two CTAs; a tile is 2 x 128 weight rows and
     // the leader (rank 0) issues its MMAs for both CTAs (cta_group::2).
     static_assert(!(PAIR && MODE == MODE_ROUTER), "the router runs on single CTAs");
@@ -395,10 +405,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int stages = min(kMaxStages, (int)(kRingBytes / stage_bytes));
 
     SmemPlan* splan = reinterpret_cast<SmemPlan*>(smem + kRingBytes + kBarBytes);
+    float* exch = reinterpret_cast<float*>(smem + kRingBytes + kBarBytes + sizeof(SmemPlan));
     if (MODE != MODE_ROUTER) {
         const PlanArrays pa = plan_arrays(const_cast<int32_t*>(args.plan));
         const int32_t* tbg = MODE == MODE_DOWN ? pa.tb2 : pa.tb1;
-        if (threadIdx.x == 0) splan->tiles1 = hdr->tiles1;
+        if (threadIdx.x == 0) {
+            splan->tiles1 = hdr->tiles1;
+            splan->fixed_n = hdr->cls == kPlanClassBucket ? hdr->cap : 0;
+        }
         for (int i = threadIdx.x; i <= nb; i += blockDim.x) {
             splan->tb[i] = tbg[i];
             if (MODE == MODE_FUSED) splan->tb2[i] = pa.tb2[i];
@@ -499,15 +513,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             while (more) {
                 const uint32_t a_dst = ring + (uint32_t)s * stage_bytes;
                 const uint32_t full = leader_bar(&ctl->full[s]);
-                const CUtensorMap* b = it.tl.gated || MODE != MODE_FUSED ? (it.tl.shared ? &mBs : &mB)
-                                                                          : (it.tl.shared ? &mB2s : &mB2);
+                const bool first = it.tl.gated || MODE != MODE_FUSED;
+                const CUtensorMap* b = first ? (it.tl.shared ? &mBs : &mB) : (it.tl.shared ? &mB2s : &mB2);
+                const CUtensorMap* b64 = first ? (it.tl.shared ? &mBs64 : &mB64) : (it.tl.shared ? &mB2s64 : &mB264);
                 // a down tile of the fused launch reads h only after its block's gate/up tiles stored it
                 if (MODE == MODE_FUSED && !it.tl.gated && it.kb == 0 && !wait_block_ready(it.tl)) {
                     ok = false;
                     break;
                 }
                 if (n < pre) {
-                    issue_b<PAIR>(it.tl, it.kb, a_dst + kATileBytes, full, b, pol);
+                    issue_b<PAIR>(it.tl, it.kb, a_dst + kATileBytes, full, b, b64, pol);
                 } else {
                     if (!bounded_wait(ptx::smem_u32(&ctl->empty[s]), ph ^ 1u, ctl, args.err)) {
                         ok = false;
@@ -519,7 +534,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
                     }
                     issue_a<MODE, PAIR>(it, a_dst, full, &mA0, &mA1, &mA0s, &mA1s, &mA2, &mA2s, args, args2, pol);
-                    issue_b<PAIR>(it.tl, it.kb, a_dst + kATileBytes, full, b, pol);
+                    issue_b<PAIR>(it.tl, it.kb, a_dst + kATileBytes, full, b, b64, pol);
                 }
                 ++n;
                 if (++s == stages) {
@@ -606,6 +621,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int quad = warp & 3;            // TMEM lane quadrant this warp may access
         int acc = 0;
         uint32_t aph = 0;
+        // gate/up chunks exchanged so far: the buffer alternates across tiles too, so
+        // a chunk's writes always follow the partner's reads of the chunk before last
+        uint32_t xchunk = 0;
         for (int i = 0, t; (t = cta_tile<MODE, PAIR>(i, total, splan->tiles1, args.comp)) >= 0; i++) {
             const Tile tl = decode_tile<MODE, PAIR>(nb, t, args, args2, splan, rank);
             if (tl.kb0 >= tl.kb1) continue;
@@ -634,16 +652,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 ptx::tmem_ld16(taddr + (uint32_t)c0, v);
                 ptx::tmem_ld_wait();
                 if (MODE != MODE_ROUTER && tl.gated) {
-                    // lanes 0-15: gate of f row 16*quad + lane; lanes 16-31: up of the same row
-                    const int half = lane >> 4;
-                    const int frow = tl.ma * 64 + quad * 16 + (lane & 15);
+                    // quadrants 0/1 hold the gate, 2/3 the up projection of f rows
+                    // 32 (quad & 1) + lane; the gate warp finishes columns 0-7 of the
+                    // chunk and sends its g of columns 8-15, the up warp the reverse
+                    const int role = quad >> 1, rq = quad & 1;
+                    const int frow = tl.ma * 64 + rq * 32 + lane;
+                    float* xb = exch + (rq * 2 + (xchunk++ & 1u)) * 512;
+                    float* mine = xb + role * 256;
+                    const float* theirs = xb + (role ^ 1) * 256;
 #pragma unroll
-                    for (int p = 0; p < 8; p++) {
-                        const float send = __uint_as_float(half ? v[2 * p] : v[2 * p + 1]);
-                        const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-                        const float g = half ? recv : __uint_as_float(v[2 * p]);
-                        const float u = half ? __uint_as_float(v[2 * p + 1]) : recv;
-                        const int col = c0 + 2 * p + half;
+                    for (int j = 0; j < 8; j++) mine[j * 32 + lane] = __uint_as_float(v[role ? j : 8 + j]);
+                    ptx::named_barrier(1 + rq, 64);
+#pragma unroll
+                    for (int j = 0; j < 8; j++) {
+                        const float other = theirs[j * 32 + lane];
+                        const float g = role ? other : __uint_as_float(v[j]);
+                        const float u = role ? __uint_as_float(v[8 + j]) : other;
+                        const int col = c0 + (role ? 8 : 0) + j;
                         if (col < tl.rows && frow < Mrows)
                             out[(size_t)(tl.row0 + col) * ld + frow] = __float2bfloat16_rn(silu_f(g) * u);
                     }

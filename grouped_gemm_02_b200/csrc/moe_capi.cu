@@ -25,6 +25,8 @@
 #include "permute.cuh"
 #include "ptx.cuh"
 #include "route.cuh"
+#include "schedule.h"
+#include "tile_table.h"
 
 using namespace moe;
 
@@ -249,8 +251,9 @@ int run_router_gemm(const bf16* x, const bf16* Wg, const float* bias, int T, int
 {
     const RouterSplit rs = router_split(T, d, E);
     *out = rs;
-    CUtensorMap a, b;
-    if (!make_map(&a, Wg, d, E, 128) || !make_map(&b, x, d, T, 16)) return MOE_ERR_CUDA;
+    CUtensorMap a, b, b64;
+    if (!make_map(&a, Wg, d, E, 128) || !make_map(&b, x, d, T, 16) || !make_map(&b64, x, d, T, 64))
+        return MOE_ERR_CUDA;
     GemmArgs g{};
     g.E = E;
     g.M = E;
@@ -268,7 +271,7 @@ int run_router_gemm(const bf16* x, const bf16* Wg, const float* bias, int T, int
     g.err = err;
     const int grid = std::min(sms, rs.tiles);
     return status_of(launch(grouped_gemm_kernel<MODE_ROUTER>, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, st,
-                            a, a, b, a, a, b, a, b, a, b, g, g));
+                            a, a, b, a, a, b, a, b, a, b, b64, b64, b64, b64, g, g));
 }
 
 // Top-k over the router's output: the logits themselves, or the split-K
@@ -336,6 +339,8 @@ struct GemmOperands {
 // launch, 1: two) and MOE_GEMM_PAIR (0/1) when those are set.
 std::atomic<int> g_policy_fused{-2};
 std::atomic<int> g_policy_pair{-2};
+std::atomic<int> g_policy_tiles{-1};   // 1: token buckets; otherwise the histogram-matched table
+std::atomic<int> g_policy_cap{-1};     // > 0: every plan cut under this cap (tuning)
 
 int env_switch(const char* name)
 {
@@ -382,8 +387,29 @@ bool gemm_pair(int P, int f, const DeviceState* dev)
     return !gemm_fused(P, f);
 }
 
-constexpr PlanShape kPlanSingle{kTileRows, 64, 128, 16, 0};
-constexpr PlanShape kPlanPair{kTileRows, 128, 256, 32, 1};
+constexpr PlanShape kPlanSingle{kTileRows, 64, 128, 16, 0, kTilesMatched};
+constexpr PlanShape kPlanPair{kTileRows, 128, 256, 32, 1, kTilesMatched};
+constexpr int kTokenBucketWidth[kTokenBuckets] = MOE_TOKEN_BUCKET_WIDTH;
+
+// The plan shape of a launch form under the current tile policy: the
+// histogram-matched table (the default; the device picks the cap), the
+// token-bucket widths chosen from T alone, or a forced cap.
+PlanShape plan_shape(PlanShape ps, int64_t T)
+{
+    const int cap = g_policy_cap.load(std::memory_order_relaxed);
+    if (g_policy_tiles.load(std::memory_order_relaxed) == 1) {
+        // token buckets: the width of T's bucket, or the forced cap as the one width
+        ps.policy = kTilesBucket;
+        ps.unit_rows = std::min(cap > 0 ? cap : kTokenBucketWidth[token_bucket(T)], ps.unit_rows);
+    } else if (cap > 0) {
+        ps.policy = kTilesCap;
+        ps.unit_rows = std::min(cap, ps.unit_rows);
+    } else {
+        ps.policy = kTilesMatched;
+    }
+    ps.unit_rows = std::max(ps.align, ps.unit_rows / ps.align * ps.align);
+    return ps;
+}
 
 // plan_ready: the plan was written two or more launches before the gate/up GEMM.
 // pair: the plan was cut for CTA pairs (kPlanPair) and the pair kernels run.
@@ -391,25 +417,31 @@ int run_gemms(const GemmOperands& o, const int32_t* plan, bool plan_ready, uint3
               bool pair, cudaStream_t st, bool prof = false)
 {
     const int sms = dev->sm_count;
-    CUtensorMap a0, a1, b, a0s, a1s, bs, a2, b2, a2s, b2s;
+    CUtensorMap a0, a1, b, a0s, a1s, bs, a2, b2, a2s, b2s, b64, bs64, b264, b2s64;
     const uint64_t E = (uint64_t)o.E;
-    // gate/up: A = W1/W3 rows (16-row boxes), B = xp rows; shared: Ws1/Ws3 and x
-    if (!make_map(&a0, o.W1, o.d, E * o.f, 16) || !make_map(&a1, o.W3, o.d, E * o.f, 16) ||
-        !make_map(&b, o.xp, o.d, (uint64_t)o.P, 16))
+    // gate/up: A = 64 rows of W1 and the same 64 rows of W3 (64-row boxes), B = xp rows
+    // (64- and 16-row boxes); shared: Ws1/Ws3 and x
+    if (!make_map(&a0, o.W1, o.d, E * o.f, 64) || !make_map(&a1, o.W3, o.d, E * o.f, 64) ||
+        !make_map(&b, o.xp, o.d, (uint64_t)o.P, 16) || !make_map(&b64, o.xp, o.d, (uint64_t)o.P, 64))
         return MOE_ERR_CUDA;
     // down: A = W2 rows (128-row boxes), B = h rows; shared: Ws2 and hs
-    if (!make_map(&a2, o.W2, o.f, E * o.d, 128) || !make_map(&b2, o.h, o.f, (uint64_t)o.P, 16)) return MOE_ERR_CUDA;
+    if (!make_map(&a2, o.W2, o.f, E * o.d, 128) || !make_map(&b2, o.h, o.f, (uint64_t)o.P, 16) ||
+        !make_map(&b264, o.h, o.f, (uint64_t)o.P, 64))
+        return MOE_ERR_CUDA;
     if (o.fs > 0) {
-        if (!make_map(&a0s, o.Ws1, o.d, o.fs, 16) || !make_map(&a1s, o.Ws3, o.d, o.fs, 16) ||
-            !make_map(&bs, o.x, o.d, (uint64_t)o.T, 16) || !make_map(&a2s, o.Ws2, o.fs, o.d, 128) ||
-            !make_map(&b2s, o.hs, o.fs, (uint64_t)o.T, 16))
+        if (!make_map(&a0s, o.Ws1, o.d, o.fs, 64) || !make_map(&a1s, o.Ws3, o.d, o.fs, 64) ||
+            !make_map(&bs, o.x, o.d, (uint64_t)o.T, 16) || !make_map(&bs64, o.x, o.d, (uint64_t)o.T, 64) ||
+            !make_map(&a2s, o.Ws2, o.fs, o.d, 128) || !make_map(&b2s, o.hs, o.fs, (uint64_t)o.T, 16) ||
+            !make_map(&b2s64, o.hs, o.fs, (uint64_t)o.T, 64))
             return MOE_ERR_CUDA;
     } else {
         a0s = a0;
         a1s = a1;
         bs = b;
+        bs64 = b64;
         a2s = a2;
         b2s = b2;
+        b2s64 = b264;
     }
     GemmArgs g1{};
     g1.plan = plan;
@@ -442,24 +474,24 @@ int run_gemms(const GemmOperands& o, const int32_t* plan, bool plan_ready, uint3
         g1.comp = std::max(1, (kb1 + kb2 / 2) / kb2);
         const cudaError_t e =
             pair ? launch_pair(grouped_gemm_kernel<MODE_FUSED, true>, grid, block, kGemmSmemBytes, st, a0, a1, b, a0s,
-                               a1s, bs, a2, b2, a2s, b2s, g1, g2)
+                               a1s, bs, a2, b2, a2s, b2s, b64, bs64, b264, b2s64, g1, g2)
                  : launch(grouped_gemm_kernel<MODE_FUSED>, grid, block, kGemmSmemBytes, st, a0, a1, b, a0s, a1s, bs,
-                          a2, b2, a2s, b2s, g1, g2);
+                          a2, b2, a2s, b2s, b64, bs64, b264, b2s64, g1, g2);
         phase_mark(prof, 3, st);   // the fused launch has no boundary: the down phase reads as zero
         return status_of(e);
     }
     const cudaError_t e1 =
         pair ? launch_pair(grouped_gemm_kernel<MODE_GATED, true>, grid, block, kGemmSmemBytes, st, a0, a1, b, a0s,
-                           a1s, bs, a0, b, a0, b, g1, g1)
+                           a1s, bs, a0, b, a0, b, b64, bs64, b64, bs64, g1, g1)
              : launch(grouped_gemm_kernel<MODE_GATED>, grid, block, kGemmSmemBytes, st, a0, a1, b, a0s, a1s, bs, a0,
-                      b, a0, b, g1, g1);
+                      b, a0, b, b64, bs64, b64, bs64, g1, g1);
     if (e1 != cudaSuccess) return MOE_ERR_CUDA;
     phase_mark(prof, 3, st);
     g2.plan_ready = 1;   // written before the gate/up GEMM
     return status_of(pair ? launch_pair(grouped_gemm_kernel<MODE_DOWN, true>, grid, block, kGemmSmemBytes, st, a2, a2,
-                                        b2, a2s, a2s, b2s, a2, b2, a2s, b2s, g2, g2)
+                                        b2, a2s, a2s, b2s, a2, b2, a2s, b2s, b264, b2s64, b264, b2s64, g2, g2)
                           : launch(grouped_gemm_kernel<MODE_DOWN>, grid, block, kGemmSmemBytes, st, a2, a2, b2, a2s,
-                                   a2s, b2s, a2, b2, a2s, b2s, g2, g2));
+                                   a2s, b2s, a2, b2, a2s, b2s, b264, b2s64, b264, b2s64, g2, g2));
 }
 
 // inv_perm_launch: this thread's launch count right after the kernel that wrote
@@ -573,7 +605,7 @@ int moe_grouped_gemm(const moe_bf16* xp, const int32_t* counts, const int32_t* o
     int32_t* plan = at<int32_t>(ws, L.plan);
     const bool pair = gemm_pair((int)(T * k), (int)f, dev);
     if (launch(plan_kernel, dim3(1), dim3(1024), 0, st, counts, offsets, (int)E, plan, (int)f, (int)d, 0, 0,
-               pair ? kPlanPair : kPlanSingle) != cudaSuccess)
+               plan_shape(pair ? kPlanPair : kPlanSingle, T)) != cudaSuccess)
         return MOE_ERR_CUDA;
     GemmOperands o{};
     o.xp = reinterpret_cast<const bf16*>(xp);
@@ -662,7 +694,8 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     if (P <= kSmallPairs) {
         // one CTA: histogram, scan, stable ranks and the tile plan
         if (launch(permute_small_kernel, dim3(1), dim3(1024), 0, st, (const int32_t*)idx, (int)P, iE, counts, offsets,
-                   perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared, pair ? kPlanPair : kPlanSingle, err) !=
+                   perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared,
+                   plan_shape(pair ? kPlanPair : kPlanSingle, T), err) !=
             cudaSuccess)
             return MOE_ERR_CUDA;
         inv_perm_launch = t_launches;
@@ -673,7 +706,7 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     } else {
         if ((rc = run_permute(idx, xb, iT, id, iE, ik, counts, offsets, perm, inv_perm, xp, err,
                               at<int32_t>(ws, L.block_counts), plan, (int)f, shared_rows, (int)f_shared,
-                              dev->sm_count, st, pair ? kPlanPair : kPlanSingle, &inv_perm_launch)))
+                              dev->sm_count, st, plan_shape(pair ? kPlanPair : kPlanSingle, T), &inv_perm_launch)))
             return rc;
     }
     GemmOperands o{};
@@ -725,10 +758,19 @@ int64_t moe_launch_counter(void) { return g_launches.load(std::memory_order_rela
 
 int moe_set_policy(int what, int value)
 {
-    if (value < -1 || value > 1) return MOE_ERR_ARG;
     switch (what) {
-    case MOE_POLICY_ONE_LAUNCH: g_policy_fused.store(value); return MOE_OK;
-    case MOE_POLICY_CTA_PAIRS: g_policy_pair.store(value); return MOE_OK;
+    case MOE_POLICY_ONE_LAUNCH:
+    case MOE_POLICY_CTA_PAIRS:
+    case MOE_POLICY_TILES:
+        if (value < -1 || value > 1) return MOE_ERR_ARG;
+        (what == MOE_POLICY_ONE_LAUNCH ? g_policy_fused : what == MOE_POLICY_CTA_PAIRS ? g_policy_pair
+                                                                                        : g_policy_tiles)
+            .store(value);
+        return MOE_OK;
+    case MOE_POLICY_TILE_CAP:
+        if (value != -1 && (value < 16 || value > kTileRows || value % 16 != 0)) return MOE_ERR_ARG;
+        g_policy_cap.store(value);
+        return MOE_OK;
     default: return MOE_ERR_ARG;
     }
 }
@@ -999,13 +1041,13 @@ int moe_layer_forward_fp8(const moe_bf16* x, const moe_bf16* Wg, const float* bi
     phase_mark(prof, 1, st);
     if (P <= kSmallPairs) {
         if (launch(permute_small_kernel, dim3(1), dim3(1024), 0, st, (const int32_t*)idx, (int)P, iE, counts, offsets,
-                   perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared, kPlanFp8, err) !=
+                   perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared, plan_shape(kPlanFp8, T), err) !=
             cudaSuccess)
             return MOE_ERR_CUDA;
         inv_perm_launch = t_launches;
     } else if ((rc = run_permute(idx, xb, iT, id, iE, ik, counts, offsets, perm, inv_perm, nullptr, err,
                                  at<int32_t>(ws, L.ctrl.block_counts), plan, (int)f, shared_rows, (int)f_shared,
-                                 dev->sm_count, st, kPlanFp8, &inv_perm_launch))) {
+                                 dev->sm_count, st, plan_shape(kPlanFp8, T), &inv_perm_launch))) {
         return rc;
     }
     const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)dev->sm_count * 16));

@@ -17,8 +17,13 @@
 #include "common.cuh"
 #include "ptx.cuh"
 #include "route.cuh"
+#include "schedule.h"
+#include "tile_table.h"
 
 namespace moe {
+
+// The tuned tile cap of each histogram class (tile_table.h).
+__constant__ int c_tile_cap[kTileClasses] = MOE_TILE_CAP_TABLE;
 
 // ---------------------------------------------------------------- histogram
 // grid hist_blocks(P), block 512: CTA b counts pairs [b*kHistChunk, ...) into
@@ -116,14 +121,52 @@ __device__ __forceinline__ void build_plan(int c, int off, int E, int pairs, int
     // offsets of group g: read from the thread that owns it
     __shared__ int s_off[kMaxGroups];
     if (tid < E) s_off[tid] = off;
+    // the histogram class of the routed experts: sum of c ln c and the largest count
+    __shared__ float s_ent[32];
+    __shared__ int s_cmax[32];
+    __shared__ int s_cap, s_cls;
+    {
+        float ent = (tid < E && c > 0) ? (float)c * __logf((float)c) : 0.f;
+        int cm = tid < E ? c : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            ent += __shfl_xor_sync(0xffffffffu, ent, o);
+            cm = max(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+        }
+        if ((tid & 31) == 0) {
+            s_ent[tid >> 5] = ent;
+            s_cmax[tid >> 5] = cm;
+        }
+    }
     __syncthreads();
+    if (tid == 0) {
+        float ent = 0.f;
+        int cm = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); w++) {
+            ent += s_ent[w];
+            cm = max(cm, s_cmax[w]);
+        }
+        int cap = ps.unit_rows, cls = ps.policy == kTilesBucket ? kPlanClassBucket : kPlanClassCap;
+        if (ps.policy == kTilesMatched && pairs > 0) {
+            // effective experts = exp(entropy) = exp(ln P - sum(c ln c) / P)
+            const float P = (float)pairs;
+            const float eff = __expf(__logf(P) - ent / P);
+            cls = tile_class(P, eff, (float)cm);
+            cap = min(cap, c_tile_cap[cls]);
+        }
+        s_cap = max(ps.align, cap / ps.align * ps.align);
+        s_cls = cls;
+    }
+    __syncthreads();
+    const int cap = s_cap;
     PlanArrays pa = plan_arrays(plan);
     int my_t1 = 0, my_t2 = 0, my_chunk = 0;
     if (tid < nact) {
         const int g = s_order[tid];
         const int n = s_n[g];
-        const int units = ceil_div(n, ps.unit_rows);
-        const int chunk = ceil_div(ceil_div(n, units), ps.align) * ps.align;
+        const int units = ceil_div(n, cap);
+        // token buckets: every tile of the fixed width; otherwise the width follows the count
+        const int chunk = ps.policy == kTilesBucket ? cap : ceil_div(ceil_div(n, units), ps.align) * ps.align;
         const int M1 = g < E ? f : f_shared;
         pa.group[tid] = g;
         pa.row0[tid] = g < E ? s_off[g] : 0;
@@ -154,6 +197,8 @@ __device__ __forceinline__ void build_plan(int c, int off, int E, int pairs, int
         h->n_max = m;
         h->pairs = pairs;
         h->pair = ps.pair;
+        h->cls = s_cls;
+        h->cap = cap;
         pa.tb1[0] = 0;
         pa.tb2[0] = 0;
         h->tiles1 = nact > 0 ? pa.tb1[nact] : 0;   // written above, visible after the barrier

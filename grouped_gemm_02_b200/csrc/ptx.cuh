@@ -328,6 +328,12 @@ __device__ __forceinline__ void fence_proxy_async_global()
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// Barrier `id` (1..15) over `threads` threads of the CTA (whole warps).
+__device__ __forceinline__ void named_barrier(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // ---------------------------------------------------------------- grid dependency (PDL)
 __device__ __forceinline__ void grid_dep_wait()
 {

@@ -52,3 +52,36 @@ MOE_HD int deal_tile(int b, int grid, int i, int total, int G, int comp, bool ba
 }
 
 }  // namespace moe
+
+namespace moe {
+
+// Histogram class of a live routing, the key of the tuned tile table
+// (Decoding the Skew, abstract: the kernel is chosen by matching the live
+// routing histogram, and its skew is measured in Effective Experts).  With P
+// routed pairs, eff = exp(entropy of counts / P) the effective number of
+// experts and c_max the largest count:
+//   tokens per effective expert m = P / eff in 5 buckets (<8, <32, <128, <512, more),
+//   the hottest expert against that mean, c_max / m, in 3 buckets (<1.5, <4, more);
+// class = 3 * bucket(m) + bucket(c_max / m).
+constexpr int kTileClasses = 15;
+
+MOE_HD int tile_class(float pairs, float eff, float c_max)
+{
+    if (!(pairs > 0.f) || !(eff > 0.f)) return 0;
+    const float m = pairs / eff;
+    const int b1 = m < 8.f ? 0 : m < 32.f ? 1 : m < 128.f ? 2 : m < 512.f ? 3 : 4;
+    const float r = c_max / m;
+    const int b2 = r < 1.5f ? 0 : r < 4.f ? 1 : 2;
+    return 3 * b1 + b2;
+}
+
+// The token buckets of the static policy the histogram-matched one is measured
+// against: T <= 16, 64, 256, 1024, 4096, more.
+constexpr int kTokenBuckets = 6;
+
+MOE_HD int token_bucket(long long T)
+{
+    return T <= 16 ? 0 : T <= 64 ? 1 : T <= 256 ? 2 : T <= 1024 ? 3 : T <= 4096 ? 4 : 5;
+}
+
+}  // namespace moe

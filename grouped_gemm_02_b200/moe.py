@@ -163,11 +163,11 @@ def moe_record_phase_events(events) -> None:
     _call("moe_record_phase_events", arr, len(events))
 
 
-POLICY_ONE_LAUNCH, POLICY_CTA_PAIRS = 1, 2
+POLICY_ONE_LAUNCH, POLICY_CTA_PAIRS, POLICY_TILES, POLICY_TILE_CAP = 1, 2, 3, 4
 
 
 def moe_set_policy(what: int, value: int) -> None:
-    """Force (0 / 1) or restore (-1) one of the library's launch-form choices for the process."""
+    """Force or restore (-1) one of the library's launch-form or tile-policy choices for the process."""
     _call("moe_set_policy", what, value)
 
 

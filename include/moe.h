@@ -231,18 +231,35 @@ MOE_API int moe_layer_forward_fp8(const moe_bf16 *x, const moe_bf16 *Wg, const f
  * used once (the call after it records nothing).  n = 0 cancels. */
 MOE_API int moe_record_phase_events(void *const *events, int n);
 
-/* Process-wide choices of how the expert GEMMs run, for comparisons and
- * tests (the pages have no counterpart).  value -1 restores the library's
- * rule; 0 / 1 force the choice for every later call in the process.  Results
- * do not depend on these choices beyond fp32 summation order inside a tile.
+/* Process-wide choices of how the expert GEMMs run, for comparisons, tuning
+ * and tests.  value -1 restores the library's rule; other values force the
+ * choice for every later call in the process.  Results do not depend on these
+ * choices beyond fp32 summation order.
  *   MOE_POLICY_ONE_LAUNCH  1: gate/up and down tiles in one persistent launch,
  *                          0: two launches (rule: one when T*k <= 256 and f <= 4096)
  *   MOE_POLICY_CTA_PAIRS   1: tiles of 2 x 128 weight rows on CTA pairs
  *                          (cta_group::2), 0: single-CTA tiles of 128 rows
  *                          (rule: pairs whenever two launches run)
- * Returns MOE_ERR_ARG for an unknown switch or value. */
+ *   MOE_POLICY_TILES       0 (rule): histogram-matched tiles -- the plan step
+ *                          classifies the live histogram on the device (tokens
+ *                          per effective expert, hottest expert against that
+ *                          mean) and takes the tile cap the tuned table holds
+ *                          for the class, every expert's width following its
+ *                          own count (Decoding the Skew, abstract: kernel
+ *                          selection by matching the live routing histogram);
+ *                          1: static token buckets -- one tile width chosen
+ *                          from T alone, every expert's tiles padded to it, the
+ *                          selection that paper measures against
+ *   MOE_POLICY_TILE_CAP    16..256 (multiple of 16): every plan under this cap,
+ *                          widths following the counts, or with MOE_POLICY_TILES
+ *                          = 1 every tile of exactly this width (table
+ *                          tuning); -1: off
+ * Returns MOE_ERR_ARG for an unknown switch or value.  The pages have no
+ * counterpart to the first two switches. */
 #define MOE_POLICY_ONE_LAUNCH 1
 #define MOE_POLICY_CTA_PAIRS 2
+#define MOE_POLICY_TILES 3
+#define MOE_POLICY_TILE_CAP 4
 MOE_API int moe_set_policy(int what, int value);
 
 /* Number of kernels this library has launched in this process so far. */
@@ -252,7 +269,9 @@ MOE_API int64_t moe_launch_counter(void);
  * (which: 0 logits, 1 topk_idx, 2 topk_w, 3 counts, 4 offsets, 5 perm,
  * 6 inv_perm, 7 xp, 8 h, 9 y_p, 10 hs, 11 ys, 12 the tile plan).  The tile plan is
  * MOE_PLAN_INTS int32: a header {n_blocks, tiles1, tiles2, n_max, pairs,
- * pair (1: tiles cut for CTA pairs), 2 x 0},
+ * pair (1: tiles cut for CTA pairs), cls (the histogram class whose tuned
+ * cap was taken; -1: a forced cap, -2: token buckets), cap (most tokens per
+ * tile)},
  * then arrays of 513 entries group, row0, rows, chunk, units, two tile
  * prefixes of 514 entries (gate/up, down) and 513 per-block counters of
  * finished gate/up tiles (see the tile plan in the grouped-GEMM comment).

@@ -26,3 +26,6 @@ int deal_all(int grid, int total, int G, int comp, int balanced, int max_per, in
 }
 
 }
+
+extern "C" int tile_class_of(float pairs, float eff, float c_max) { return moe::tile_class(pairs, eff, c_max); }
+extern "C" int token_bucket_of(long long T) { return moe::token_bucket(T); }

@@ -100,9 +100,10 @@ def decode_plan(plan) -> dict:
     """The tile plan a layer leaves in its workspace (int32 [MOE_PLAN_INTS]) as host arrays."""
     p = plan.cpu().numpy() if hasattr(plan, "cpu") else np.asarray(plan)
     G = PLAN_GROUPS
-    nb, tiles1, tiles2, n_max, pairs, pair = (int(v) for v in p[:6])
+    nb, tiles1, tiles2, n_max, pairs, pair, cls, cap = (int(v) for v in p[:8])
     o = 8
-    out = {"n_blocks": nb, "tiles1": tiles1, "tiles2": tiles2, "n_max": n_max, "pairs": pairs, "pair": pair}
+    out = {"n_blocks": nb, "tiles1": tiles1, "tiles2": tiles2, "n_max": n_max, "pairs": pairs, "pair": pair,
+           "cls": cls, "cap": cap}
     for name in ("group", "row0", "rows", "chunk", "units"):
         out[name] = p[o:o + nb].astype(np.int64)
         o += G
@@ -139,6 +140,9 @@ def check_plan(plan: dict, counts: np.ndarray, offsets: np.ndarray, T: int, f: i
     key = [(-int(rows[i]), int(g[i])) for i in range(n_blocks)]
     assert key == sorted(key), f"{what}: blocks not heaviest first"
     assert np.all(ch % align == 0) and np.all(ch >= align) and np.all(ch <= unit_max), what
+    assert np.all(ch <= plan["cap"]), f"{what}: a tile wider than the plan's cap"
+    if plan["cls"] == -2:                       # token buckets: one width for every expert
+        assert np.all(ch == plan["cap"]), f"{what}: token-bucket plan with widths {np.unique(ch)}"
     assert np.all(ch * un >= rows) and np.all(ch * (un - 1) < rows), f"{what}: an empty or missing unit"
     cover = np.zeros(int(offsets[-1]), dtype=np.int64)
     for i in range(n_blocks):
@@ -159,29 +163,65 @@ def check_plan(plan: dict, counts: np.ndarray, offsets: np.ndarray, T: int, f: i
 
 
 # The launch-form switches the tests have set through moe_set_policy (-1: the library's rule).
-POLICY = {"one_launch": -1, "pairs": -1}
+POLICY = {"one_launch": -1, "pairs": -1, "tiles": -1, "cap": -1}
+
+
+def _apply(pol):
+    from grouped_gemm_02_b200 import moe
+    moe.moe_set_policy(moe.POLICY_ONE_LAUNCH, pol["one_launch"])
+    moe.moe_set_policy(moe.POLICY_CTA_PAIRS, pol["pairs"])
+    moe.moe_set_policy(moe.POLICY_TILES, pol["tiles"])
+    moe.moe_set_policy(moe.POLICY_TILE_CAP, pol["cap"])
 
 
 class policy:
-    """Context manager: force the library's launch-form switches, restore them after."""
+    """Context manager: force the library's launch-form and tile-policy switches, restore them after."""
 
-    def __init__(self, one_launch: int = -1, pairs: int = -1):
-        self.want = {"one_launch": one_launch, "pairs": pairs}
+    def __init__(self, one_launch: int = -1, pairs: int = -1, tiles: int = -1, cap: int = -1):
+        self.want = {"one_launch": one_launch, "pairs": pairs, "tiles": tiles, "cap": cap}
 
     def __enter__(self):
-        from grouped_gemm_02_b200 import moe
         self.prev = dict(POLICY)
-        moe.moe_set_policy(moe.POLICY_ONE_LAUNCH, self.want["one_launch"])
-        moe.moe_set_policy(moe.POLICY_CTA_PAIRS, self.want["pairs"])
+        _apply(self.want)
         POLICY.update(self.want)
         return self
 
     def __exit__(self, *exc):
-        from grouped_gemm_02_b200 import moe
-        moe.moe_set_policy(moe.POLICY_ONE_LAUNCH, self.prev["one_launch"])
-        moe.moe_set_policy(moe.POLICY_CTA_PAIRS, self.prev["pairs"])
+        _apply(self.prev)
         POLICY.update(self.prev)
         return False
+
+
+def tile_tables():
+    """(cap per histogram class, fixed width per token bucket) as the library was built with."""
+    import os
+    import re
+    src = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "grouped_gemm_02_b200",
+                            "csrc", "tile_table.h")).read()
+    cap = [int(v) for v in re.search(r"#define MOE_TILE_CAP_TABLE \{([^}]*)\}", src).group(1).split(",")]
+    width = [int(v) for v in re.search(r"#define MOE_TOKEN_BUCKET_WIDTH \{([^}]*)\}", src).group(1).split(",")]
+    return cap, width
+
+
+def token_bucket(T: int) -> int:
+    return 0 if T <= 16 else 1 if T <= 64 else 2 if T <= 256 else 3 if T <= 1024 else 4 if T <= 4096 else 5
+
+
+def histogram_class(counts: np.ndarray):
+    """(class, distance of its features from the nearest bucket edge, relative) of a routing,
+    as the plan step defines it: tokens per effective expert, and the hottest expert against it."""
+    c = counts[counts > 0].astype(np.float64)
+    P = c.sum()
+    if P <= 0:
+        return 0, 1.0
+    eff = np.exp(np.log(P) - (c * np.log(c)).sum() / P)
+    m = P / eff
+    r = c.max() / m
+    e1, e2 = [8, 32, 128, 512], [1.5, 4.0]
+    b1 = sum(m >= e for e in e1)
+    b2 = sum(r >= e for e in e2)
+    margin = min([abs(m / e - 1) for e in e1] + [abs(r / e - 1) for e in e2])
+    return 3 * b1 + b2, margin
 
 
 def fused_gemms(P: int, f: int) -> bool:
@@ -229,6 +269,19 @@ def check_layer_plan(views, s: wl.LayerShape, counts, offsets, what, fp8: bool =
     else:
         unit_max, m1_rows, m2_rows, align = 256, 64, 128, 16
     check_plan(plan, counts, offsets, s.T, s.f, s.d, s.f_shared, unit_max, m1_rows, what, m2_rows, align)
+    # the tile policy: a forced cap, token buckets, or the table's cap for the histogram class
+    rnd = lambda v: max(align, min(v, unit_max) // align * align)
+    caps, widths = tile_tables()
+    if POLICY["tiles"] == 1:
+        w = POLICY["cap"] if POLICY["cap"] > 0 else widths[token_bucket(s.T)]
+        assert (plan["cls"], plan["cap"]) == (-2, rnd(w)), what
+    elif POLICY["cap"] > 0:
+        assert (plan["cls"], plan["cap"]) == (-1, rnd(POLICY["cap"])), what
+    else:
+        cls, margin = histogram_class(counts)
+        if margin > 1e-3:     # features on a bucket edge may round either way in fp32
+            assert plan["cls"] == cls, f"{what}: histogram class {plan['cls']}, expected {cls}"
+        assert 0 <= plan["cls"] < len(caps) and plan["cap"] == rnd(caps[plan["cls"]]), what
     m1 = np.array([-(-(s.f if g < s.E else s.f_shared) // m1_rows) for g in plan["group"]], dtype=np.int64)
     warps = 8 if pair else 4
     need = warps * plan["units"] * m1 if fused_gemms(s.P, s.f) else np.zeros_like(m1)

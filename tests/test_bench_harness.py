@@ -171,3 +171,26 @@ def test_reference_sample_on_a_small_layer():
     assert pool.size >= 1
     assert orc.batch(4) == 4
     assert all(orc.W1[e] is not None for e in experts)
+
+
+def test_tile_table_writer(tmp_path):
+    """tune_tiles.py write: the best cap per measured class and width per token bucket."""
+    from grouped_gemm_02_b200 import tune_tiles
+    rows = [
+        {"workload": "a", "T": 8, "bucket": 0, "cls": 2, "cap_us": {"64": 5.0, "128": 4.0, "256": 4.5},
+         "width_us": {"16": 9.0, "32": 8.0, "64": 8.5, "128": 9.5, "256": 9.9}},
+        {"workload": "b", "T": 10, "bucket": 0, "cls": 2, "cap_us": {"64": 5.0, "128": 4.2, "256": 4.1},
+         "width_us": {"16": 9.0, "32": 8.0, "64": 8.5, "128": 9.5, "256": 9.9}},
+        {"workload": "c", "T": 5000, "bucket": 5, "cls": 13, "cap_us": {"64": 9.0, "128": 8.0, "256": 7.0},
+         "width_us": {"16": 20.0, "32": 15.0, "64": 12.0, "128": 11.0, "256": 10.0}},
+    ]
+    sweep = tmp_path / "s.json"
+    sweep.write_text(json.dumps({"device": "test", "rows": rows}))
+    table = tmp_path / "t.h"
+    tune_tiles.main(["write", "--sweep", str(sweep), "--table", str(table)])
+    import re
+    src = table.read_text()
+    caps = [int(v) for v in re.search(r"MOE_TILE_CAP_TABLE \{([^}]*)\}", src).group(1).split(",")]
+    widths = [int(v) for v in re.search(r"MOE_TOKEN_BUCKET_WIDTH \{([^}]*)\}", src).group(1).split(",")]
+    assert caps[2] == 128 and caps[13] == 256 and caps[0] == 256 and len(caps) == 15
+    assert widths[0] == 32 and widths[5] == 256 and widths[3] == 128 and len(widths) == 6

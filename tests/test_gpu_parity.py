@@ -288,3 +288,20 @@ def test_grouped_gemm_every_launch_form(T, d, f, E, k, alpha, one_launch, pairs)
     with H.policy(one_launch=one_launch, pairs=pairs):
         out, ref = _gemm_case(s, seed=T + d + f, alpha=alpha)
     H.assert_close(out, ref, f"grouped GEMM T={T} d={d} f={f} E={E} k={k} one={one_launch} pairs={pairs}")
+
+
+@pytest.mark.parametrize("tiles,cap", [(1, -1), (-1, 64), (-1, 128), (0, -1)])
+@pytest.mark.parametrize("name,kw", [
+    ("decode64", dict(alpha=0.1)),
+    ("deepseek_v3", dict(T=64, alpha=0.05)),
+    ("kimi_k2", dict(T=256)),
+    ("mixtral", dict(T=16)),
+])
+def test_layer_tile_policies(name, kw, tiles, cap):
+    """Token-bucket tiles (one width from T, padded), forced caps and the histogram-matched
+    table all compute the same layer: routing bit-exact, plan of the policy's shape, outputs
+    in tolerance."""
+    s = wl.shape(name, **kw)
+    with H.policy(tiles=tiles, cap=cap):
+        _layer_check(s, seed=5, n_sample=12, device_inputs=s.d * s.f * s.E > 2**31)
+    torch.cuda.empty_cache()

@@ -20,11 +20,16 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 
 
 @pytest.fixture(scope="module")
-def deal(tmp_path_factory):
+def harness(tmp_path_factory):
     out = str(tmp_path_factory.mktemp("deal") / "libdeal.so")
     subprocess.run(["g++", "-O2", "-std=c++17", "-shared", "-fPIC", "-o", out,
                     os.path.join(HERE, "deal_harness.cpp")], check=True)
-    L = C.CDLL(out)
+    return C.CDLL(out)
+
+
+@pytest.fixture(scope="module")
+def deal(harness):
+    L = harness
     L.deal_all.argtypes = [C.c_int] * 6 + [C.POINTER(C.c_int)]
     L.deal_all.restype = C.c_int
 
@@ -85,3 +90,27 @@ def test_balanced_deal_compensates_short_ctas(deal):
             rr = deal(grid, G + D, G, comp, False)
             loads_rr = [np.count_nonzero(t[t >= 0] < G) * comp + np.count_nonzero(t[t >= 0] >= G) for t in rr]
             assert max(loads) <= max(loads_rr), (G, D, grid, comp)
+
+
+def test_tile_class_and_token_buckets(harness):
+    """The histogram class and token bucket (schedule.h, compiled here) against their definition."""
+    lib = harness
+    lib.tile_class_of.argtypes = [C.c_float, C.c_float, C.c_float]
+    lib.token_bucket_of.argtypes = [C.c_longlong]
+    from tests import gpu_helpers as H
+    rng = np.random.default_rng(0)
+    for _ in range(400):
+        E = int(rng.integers(1, 512))
+        counts = rng.multinomial(int(rng.integers(1, 20000)), rng.dirichlet(np.full(E, 10 ** rng.uniform(-2, 1))))
+        cls, margin = H.histogram_class(counts)
+        c = counts[counts > 0].astype(np.float64)
+        P = c.sum()
+        eff = np.exp(np.log(P) - (c * np.log(c)).sum() / P)
+        if margin > 1e-4:
+            assert lib.tile_class_of(P, eff, c.max()) == cls
+    assert lib.tile_class_of(0, 1, 0) == 0
+    for T, b in [(1, 0), (16, 0), (17, 1), (64, 1), (65, 2), (256, 2), (1024, 3), (4096, 4), (4097, 5), (10**6, 5)]:
+        assert lib.token_bucket_of(T) == b == H.token_bucket(T)
+    caps, widths = H.tile_tables()
+    assert len(caps) == 15 and len(widths) == 6
+    assert all(16 <= v <= 256 and v % 16 == 0 for v in caps + widths)
