@@ -387,8 +387,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             const __grid_constant__ CUtensorMap mA2, const __grid_constant__ CUtensorMap mB2,
                             const __grid_constant__ CUtensorMap mA2s, const __grid_constant__ CUtensorMap mB2s,
                             const __grid_constant__ CUtensorMap mSB2, const __grid_constant__ CUtensorMap mSB2s,
+                            const __grid_constant__ CUtensorMap mB64, const __grid_constant__ CUtensorMap mBs64,
+                            const __grid_constant__ CUtensorMap mB264, const __grid_constant__ CUtensorMap mB2s64,
                             const Fp8Args args, const Fp8Args args2)
 {
+    // mB64..mB2s64: the token-row maps mB, mBs, mB2, mB2s with 64-row boxes
     // FP8_FUSED: args and mA0..mSBs describe the gate/up tiles (W1/W3, xp8, its
     // scales), args2 and mA2..mSB2s the down tiles (W2, h8, its scales).  The
     // other kinds use args and mA0..mSBs only.
@@ -490,9 +493,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int kc = kb * kFp8BlockK;
                 const uint32_t b_dst = stage + kABytes;
                 const CUtensorMap* bm = down2(tl) ? (tl.shared ? &mB2s : &mB2) : (tl.shared ? &mBs : &mB);
+                const CUtensorMap* bm64 = down2(tl) ? (tl.shared ? &mB2s64 : &mB264) : (tl.shared ? &mBs64 : &mB64);
                 const CUtensorMap* sm = down2(tl) ? (tl.shared ? &mSB2s : &mSB2) : (tl.shared ? &mSBs : &mSB);
-                for (int i = 0; i < tl.n_mma / 16; i++)
-                    ptx::tma_load_2d(b_dst + i * 16 * kFp8BlockK, bm, full, kc, tl.row0 + 16 * i, pol);
+                // token rows in 64-row boxes, then 16-row boxes (fewer TMA requests)
+                const int n64 = tl.n_mma >> 6;
+                for (int i = 0; i < n64; i++)
+                    ptx::tma_load_2d(b_dst + i * 64 * kFp8BlockK, bm64, full, kc, tl.row0 + 64 * i, pol);
+                for (int r = 64 * n64; r < tl.n_mma; r += 16)
+                    ptx::tma_load_2d(b_dst + r * kFp8BlockK, bm, full, kc, tl.row0 + r, pol);
                 // the tokens' scales of this K block: 128 fp32 from row0 rounded down to 4
                 ptx::tma_load_2d(b_dst + b_bytes, sm, full, tl.row0 & ~3, kb, pol);
             };

@@ -271,7 +271,7 @@ int run_router_gemm(const bf16* x, const bf16* Wg, const float* bias, int T, int
     g.err = err;
     const int grid = std::min(sms, rs.tiles);
     return status_of(launch(grouped_gemm_kernel<MODE_ROUTER>, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, st,
-                            a, a, b, a, a, b, a, b, a, b, b64, b64, b64, b64, g, g));
+                            a, a, b, a, a, b, a, b, a, b, b64, b64, b64, b64, b, g, g));
 }
 
 // Top-k over the router's output: the logits themselves, or the split-K
@@ -331,7 +331,8 @@ struct GemmOperands {
     const int32_t* perm;
     const float* gate_w;
     bf16 *h, *y_p, *hs, *ys;
-    int T, P, d, f, fs, E;
+    int T, P, d, f, fs, E, k;
+    bool gather;   // gate/up token rows straight from x through perm (no xp)
 };
 
 // Process-wide choices of the expert-GEMM launch form (moe_set_policy; -1 =
@@ -341,6 +342,7 @@ std::atomic<int> g_policy_fused{-2};
 std::atomic<int> g_policy_pair{-2};
 std::atomic<int> g_policy_tiles{-1};   // 1: token buckets; otherwise the histogram-matched table
 std::atomic<int> g_policy_cap{-1};     // > 0: every plan cut under this cap (tuning)
+std::atomic<int> g_policy_gather{-1};  // 1: the gate/up GEMM gathers token rows from x (no gather launch)
 
 int env_switch(const char* name)
 {
@@ -417,8 +419,10 @@ int run_gemms(const GemmOperands& o, const int32_t* plan, bool plan_ready, uint3
               bool pair, cudaStream_t st, bool prof = false)
 {
     const int sms = dev->sm_count;
-    CUtensorMap a0, a1, b, a0s, a1s, bs, a2, b2, a2s, b2s, b64, bs64, b264, b2s64;
+    CUtensorMap a0, a1, b, a0s, a1s, bs, a2, b2, a2s, b2s, b64, bs64, b264, b2s64, bx;
     const uint64_t E = (uint64_t)o.E;
+    // the row gather of the gate/up tokens: x with one-row boxes
+    if (!make_map(&bx, o.x, o.d, (uint64_t)o.T, 1)) return MOE_ERR_CUDA;
     // gate/up: A = 64 rows of W1 and the same 64 rows of W3 (64-row boxes), B = xp rows
     // (64- and 16-row boxes); shared: Ws1/Ws3 and x
     if (!make_map(&a0, o.W1, o.d, E * o.f, 64) || !make_map(&a1, o.W3, o.d, E * o.f, 64) ||
@@ -458,7 +462,10 @@ int run_gemms(const GemmOperands& o, const int32_t* plan, bool plan_ready, uint3
     g1.perm = o.perm;
     g1.gate_w = o.gate_w;
     g1.err = err;
+    g1.gather_perm = o.gather ? o.perm : nullptr;
+    g1.gather_k = o.k;
     GemmArgs g2 = g1;
+    g2.gather_perm = nullptr;
     g2.M = o.d;
     g2.M_shared = o.d;
     g2.K = o.f;
@@ -474,24 +481,24 @@ int run_gemms(const GemmOperands& o, const int32_t* plan, bool plan_ready, uint3
         g1.comp = std::max(1, (kb1 + kb2 / 2) / kb2);
         const cudaError_t e =
             pair ? launch_pair(grouped_gemm_kernel<MODE_FUSED, true>, grid, block, kGemmSmemBytes, st, a0, a1, b, a0s,
-                               a1s, bs, a2, b2, a2s, b2s, b64, bs64, b264, b2s64, g1, g2)
+                               a1s, bs, a2, b2, a2s, b2s, b64, bs64, b264, b2s64, bx, g1, g2)
                  : launch(grouped_gemm_kernel<MODE_FUSED>, grid, block, kGemmSmemBytes, st, a0, a1, b, a0s, a1s, bs,
-                          a2, b2, a2s, b2s, b64, bs64, b264, b2s64, g1, g2);
+                          a2, b2, a2s, b2s, b64, bs64, b264, b2s64, bx, g1, g2);
         phase_mark(prof, 3, st);   // the fused launch has no boundary: the down phase reads as zero
         return status_of(e);
     }
     const cudaError_t e1 =
         pair ? launch_pair(grouped_gemm_kernel<MODE_GATED, true>, grid, block, kGemmSmemBytes, st, a0, a1, b, a0s,
-                           a1s, bs, a0, b, a0, b, b64, bs64, b64, bs64, g1, g1)
+                           a1s, bs, a0, b, a0, b, b64, bs64, b64, bs64, bx, g1, g1)
              : launch(grouped_gemm_kernel<MODE_GATED>, grid, block, kGemmSmemBytes, st, a0, a1, b, a0s, a1s, bs, a0,
-                      b, a0, b, b64, bs64, b64, bs64, g1, g1);
+                      b, a0, b, b64, bs64, b64, bs64, bx, g1, g1);
     if (e1 != cudaSuccess) return MOE_ERR_CUDA;
     phase_mark(prof, 3, st);
     g2.plan_ready = 1;   // written before the gate/up GEMM
     return status_of(pair ? launch_pair(grouped_gemm_kernel<MODE_DOWN, true>, grid, block, kGemmSmemBytes, st, a2, a2,
-                                        b2, a2s, a2s, b2s, a2, b2, a2s, b2s, b264, b2s64, b264, b2s64, g2, g2)
+                                        b2, a2s, a2s, b2s, a2, b2, a2s, b2s, b264, b2s64, b264, b2s64, bx, g2, g2)
                           : launch(grouped_gemm_kernel<MODE_DOWN>, grid, block, kGemmSmemBytes, st, a2, a2, b2, a2s,
-                                   a2s, b2s, a2, b2, a2s, b2s, b264, b2s64, b264, b2s64, g2, g2));
+                                   a2s, b2s, a2, b2, a2s, b2s, b264, b2s64, b264, b2s64, bx, g2, g2));
 }
 
 // inv_perm_launch: this thread's launch count right after the kernel that wrote
@@ -623,6 +630,8 @@ int moe_grouped_gemm(const moe_bf16* xp, const int32_t* counts, const int32_t* o
     o.f = (int)f;
     o.fs = 0;
     o.E = (int)E;
+    o.k = (int)k;
+    o.gather = false;
     return run_gemms(o, plan, /*plan_ready=*/false, at<uint32_t>(ws, L.err), dev, pair, st);
 }
 
@@ -689,6 +698,10 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     const TopkSource src = topk_source(rs, logits, partials, bias, iT, iE);
     const int64_t P = T * k;
     const bool pair = gemm_pair((int)P, (int)f, dev);
+    // token rows for the gate/up GEMM: a gather pass into xp (the default), or TMA
+    // row gathers from x inside the GEMM (tile::gather4, 4 rows per instruction),
+    // which measured slower on B200 at every size: more, smaller TMA requests
+    const bool gather_in_gemm = g_policy_gather.load(std::memory_order_relaxed) == 1;
     if ((rc = run_topk(src, iT, iE, ik, idx, w, err, st))) return rc;
     phase_mark(prof, 1, st);
     if (P <= kSmallPairs) {
@@ -699,12 +712,14 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
             cudaSuccess)
             return MOE_ERR_CUDA;
         inv_perm_launch = t_launches;
-        const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)dev->sm_count * 16));
-        if (launch(gather_rows_kernel, dim3(blocks), dim3(256), 0, st, xb, (const int32_t*)perm,
-                   (const int32_t*)offsets, iE, ik, id, xp) != cudaSuccess)
-            return MOE_ERR_CUDA;
+        if (!gather_in_gemm) {
+            const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)dev->sm_count * 16));
+            if (launch(gather_rows_kernel, dim3(blocks), dim3(256), 0, st, xb, (const int32_t*)perm,
+                       (const int32_t*)offsets, iE, ik, id, xp) != cudaSuccess)
+                return MOE_ERR_CUDA;
+        }
     } else {
-        if ((rc = run_permute(idx, xb, iT, id, iE, ik, counts, offsets, perm, inv_perm, xp, err,
+        if ((rc = run_permute(idx, xb, iT, id, iE, ik, counts, offsets, perm, inv_perm, gather_in_gemm ? nullptr : xp, err,
                               at<int32_t>(ws, L.block_counts), plan, (int)f, shared_rows, (int)f_shared,
                               dev->sm_count, st, plan_shape(pair ? kPlanPair : kPlanSingle, T), &inv_perm_launch)))
             return rc;
@@ -730,9 +745,13 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     o.f = (int)f;
     o.fs = (int)f_shared;
     o.E = iE;
+    o.k = ik;
+    o.gather = gather_in_gemm;
     phase_mark(prof, 2, st);
-    // the plan was written two or more launches before the gate/up GEMM (the gather is in between)
-    if ((rc = run_gemms(o, plan, /*plan_ready=*/true, err, dev, pair, st, prof))) return rc;
+    // the plan is written two or more launches before the GEMM, except when the
+    // one-CTA permutation is directly followed by a gathering GEMM
+    const bool plan_ready = !gather_in_gemm || P > kSmallPairs;
+    if ((rc = run_gemms(o, plan, plan_ready, err, dev, pair, st, prof))) return rc;
     phase_mark(prof, 4, st);
     rc = run_combine(y_p, inv_perm, ys, iT, ik, id, reinterpret_cast<bf16*>(out), st, inv_perm_launch);
     phase_mark(prof, 5, st);
@@ -766,6 +785,10 @@ int moe_set_policy(int what, int value)
         (what == MOE_POLICY_ONE_LAUNCH ? g_policy_fused : what == MOE_POLICY_CTA_PAIRS ? g_policy_pair
                                                                                         : g_policy_tiles)
             .store(value);
+        return MOE_OK;
+    case MOE_POLICY_GATHER:
+        if (value < -1 || value > 1) return MOE_ERR_ARG;
+        g_policy_gather.store(value);
         return MOE_OK;
     case MOE_POLICY_TILE_CAP:
         if (value != -1 && (value < 16 || value > kTileRows || value % 16 != 0)) return MOE_ERR_ARG;
@@ -861,16 +884,20 @@ int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int 
     CUtensorMap a0, a1, b, a0s, a1s, bs, sb, sbs;
     // down operands: W2, h8 and its scales (shared: Ws2, hs8, shs)
     CUtensorMap a2, b2, a2s, b2s, sb2, sb2s;
+    // the same token-row maps with 64-row boxes
+    CUtensorMap b64, bs64, b264, b2s64;
     const uint64_t E = (uint64_t)o.E;
     const uint64_t lp = (uint64_t)o.ld_pairs, lt = (uint64_t)o.ld_tokens;
     if (!make_map_u8(&a0, o.W1q, o.d, E * o.f, 128) || !make_map_u8(&a1, o.W3q, o.d, E * o.f, 128) ||
         !make_map_u8(&b, o.xp8, o.d, (uint64_t)o.P, 16) || !make_map_f32(&sb, o.sxp, lp, o.d / 128) ||
+        !make_map_u8(&b64, o.xp8, o.d, (uint64_t)o.P, 64) || !make_map_u8(&b264, o.h8, o.f, (uint64_t)o.P, 64) ||
         !make_map_u8(&a2, o.W2q, o.f, E * o.d, 128) || !make_map_u8(&b2, o.h8, o.f, (uint64_t)o.P, 16) ||
         !make_map_f32(&sb2, o.sh, lp, o.f / 128))
         return MOE_ERR_CUDA;
     if (o.fs > 0) {
         if (!make_map_u8(&a0s, o.Ws1q, o.d, o.fs, 128) || !make_map_u8(&a1s, o.Ws3q, o.d, o.fs, 128) ||
             !make_map_u8(&bs, o.x8, o.d, (uint64_t)o.T, 16) || !make_map_f32(&sbs, o.sxT, lt, o.d / 128) ||
+            !make_map_u8(&bs64, o.x8, o.d, (uint64_t)o.T, 64) || !make_map_u8(&b2s64, o.hs8, o.fs, (uint64_t)o.T, 64) ||
             !make_map_u8(&a2s, o.Ws2q, o.fs, o.d, 128) || !make_map_u8(&b2s, o.hs8, o.fs, (uint64_t)o.T, 16) ||
             !make_map_f32(&sb2s, o.shs, lt, o.fs / 128))
             return MOE_ERR_CUDA;
@@ -882,6 +909,8 @@ int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int 
         a2s = a2;
         b2s = b2;
         sb2s = sb2;
+        bs64 = b64;
+        b2s64 = b264;
     }
     Fp8Args g1{};
     g1.plan = plan;
@@ -920,16 +949,18 @@ int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int 
         const int kb1 = o.d / 128, kb2 = o.f / 128;
         g1.comp = std::max(1, (kb1 + kb2 / 2) / kb2);
         const cudaError_t e = launch(grouped_gemm_fp8_kernel<FP8_FUSED>, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes,
-                                     st, a0, a1, b, a0s, a1s, bs, sb, sbs, a2, b2, a2s, b2s, sb2, sb2s, g1, g2);
+                                     st, a0, a1, b, a0s, a1s, bs, sb, sbs, a2, b2, a2s, b2s, sb2, sb2s, b64, bs64, b264,
+                                     b2s64, g1, g2);
         phase_mark(prof, 3, st);   // the single launch has no boundary: the down phase reads as zero
         return status_of(e);
     }
     if (launch(grouped_gemm_fp8_kernel<FP8_GATED>, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a0, a1, b, a0s,
-               a1s, bs, sb, sbs, a2, b2, a2s, b2s, sb2, sb2s, g1, g1) != cudaSuccess)
+               a1s, bs, sb, sbs, a2, b2, a2s, b2s, sb2, sb2s, b64, bs64, b264, b2s64, g1, g1) != cudaSuccess)
         return MOE_ERR_CUDA;
     phase_mark(prof, 3, st);
     return status_of(launch(grouped_gemm_fp8_kernel<FP8_DOWN>, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a2,
-                            a2, b2, a2s, a2s, b2s, sb2, sb2s, a2, b2, a2s, b2s, sb2, sb2s, g2, g2));
+                            a2, b2, a2s, a2s, b2s, sb2, sb2s, a2, b2, a2s, b2s, sb2, sb2s, b264, b2s64, b264, b2s64,
+                            g2, g2));
 }
 
 }  // namespace

@@ -163,7 +163,7 @@ def moe_record_phase_events(events) -> None:
     _call("moe_record_phase_events", arr, len(events))
 
 
-POLICY_ONE_LAUNCH, POLICY_CTA_PAIRS, POLICY_TILES, POLICY_TILE_CAP = 1, 2, 3, 4
+POLICY_ONE_LAUNCH, POLICY_CTA_PAIRS, POLICY_TILES, POLICY_TILE_CAP, POLICY_GATHER = 1, 2, 3, 4, 5
 
 
 def moe_set_policy(what: int, value: int) -> None:

@@ -163,7 +163,8 @@ MOE_API int moe_combine(const moe_bf16 *y_p, const int32_t *inv_perm, const moe_
  * Ws1/Ws3 [f_shared,d], Ws2 [d,f_shared] (all NULL and f_shared = 0 for none)
  * added with gate 1.  out [T,d].  Every intermediate lives in `ws`
  * (moe_workspace_size bytes).  Bit-identical to calling the steps one by one
- * on the same inputs. */
+ * on the same inputs (also under MOE_POLICY_GATHER = 1, which leaves xp
+ * untouched). */
 MOE_API int moe_layer_forward(const moe_bf16 *x, const moe_bf16 *Wg, const float *bias, const moe_bf16 *W1,
                       const moe_bf16 *W3, const moe_bf16 *W2, const moe_bf16 *Ws1, const moe_bf16 *Ws3,
                       const moe_bf16 *Ws2, int64_t f_shared, int64_t T, int64_t d, int64_t f, int64_t E, int64_t k,
@@ -254,12 +255,17 @@ MOE_API int moe_record_phase_events(void *const *events, int n);
  *                          widths following the counts, or with MOE_POLICY_TILES
  *                          = 1 every tile of exactly this width (table
  *                          tuning); -1: off
+ *   MOE_POLICY_GATHER      1: moe_layer_forward's gate/up GEMM gathers its token
+ *                          rows straight from x (TMA tile::gather4, four rows per
+ *                          request) instead of a gather pass into xp; 0 (rule):
+ *                          the gather pass, measured faster on B200 at every size
  * Returns MOE_ERR_ARG for an unknown switch or value.  The pages have no
  * counterpart to the first two switches. */
 #define MOE_POLICY_ONE_LAUNCH 1
 #define MOE_POLICY_CTA_PAIRS 2
 #define MOE_POLICY_TILES 3
 #define MOE_POLICY_TILE_CAP 4
+#define MOE_POLICY_GATHER 5
 MOE_API int moe_set_policy(int what, int value);
 
 /* Number of kernels this library has launched in this process so far. */

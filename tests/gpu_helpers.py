@@ -163,7 +163,7 @@ def check_plan(plan: dict, counts: np.ndarray, offsets: np.ndarray, T: int, f: i
 
 
 # The launch-form switches the tests have set through moe_set_policy (-1: the library's rule).
-POLICY = {"one_launch": -1, "pairs": -1, "tiles": -1, "cap": -1}
+POLICY = {"one_launch": -1, "pairs": -1, "tiles": -1, "cap": -1, "gather": -1}
 
 
 def _apply(pol):
@@ -172,13 +172,14 @@ def _apply(pol):
     moe.moe_set_policy(moe.POLICY_CTA_PAIRS, pol["pairs"])
     moe.moe_set_policy(moe.POLICY_TILES, pol["tiles"])
     moe.moe_set_policy(moe.POLICY_TILE_CAP, pol["cap"])
+    moe.moe_set_policy(moe.POLICY_GATHER, pol["gather"])
 
 
 class policy:
     """Context manager: force the library's launch-form and tile-policy switches, restore them after."""
 
-    def __init__(self, one_launch: int = -1, pairs: int = -1, tiles: int = -1, cap: int = -1):
-        self.want = {"one_launch": one_launch, "pairs": pairs, "tiles": tiles, "cap": cap}
+    def __init__(self, one_launch: int = -1, pairs: int = -1, tiles: int = -1, cap: int = -1, gather: int = -1):
+        self.want = {"one_launch": one_launch, "pairs": pairs, "tiles": tiles, "cap": cap, "gather": gather}
 
     def __enter__(self):
         self.prev = dict(POLICY)

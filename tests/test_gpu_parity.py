@@ -262,17 +262,19 @@ def test_empty_and_single_token():
 FORMS = [(1, 0), (0, 0), (1, 1), (0, 1)]     # (one launch, CTA pairs)
 
 
+@pytest.mark.parametrize("gather", [0, 1])
 @pytest.mark.parametrize("one_launch,pairs", FORMS)
 @pytest.mark.parametrize("name,kw", [
     ("decode64", dict(alpha=0.1)),
     ("deepseek_v3", dict(T=64, alpha=0.05)),     # shared expert
     ("kimi_k2", dict(T=256)),                    # hot experts with units of up to 256 tokens
 ])
-def test_layer_every_launch_form(name, kw, one_launch, pairs):
-    """Both expert-GEMM launch forms on single CTAs and on CTA pairs, each checked
-    against the oracle (routing bit-exact, plan invariants, outputs in tolerance)."""
+def test_layer_every_launch_form(name, kw, one_launch, pairs, gather):
+    """Both expert-GEMM launch forms on single CTAs and on CTA pairs, with the gather pass or
+    the TMA row gathers inside the GEMM, each checked against the oracle (routing bit-exact,
+    plan invariants, outputs in tolerance)."""
     s = wl.shape(name, **kw)
-    with H.policy(one_launch=one_launch, pairs=pairs):
+    with H.policy(one_launch=one_launch, pairs=pairs, gather=gather):
         _layer_check(s, seed=3, n_sample=12, device_inputs=s.d * s.f * s.E > 2**31)
     torch.cuda.empty_cache()
 
