@@ -53,6 +53,16 @@ def load(path: str) -> C.CDLL:
     L.oracle_moe_ffn_fp8.argtypes = [u8p, f64p, u8pp, f64pp, u8pp, f64pp, u8pp, f64pp, i64, i64, i64, i32p, f64p,
                                      i64, u8p, f64p, u8p, f64p, u8p, f64p, i64, C.POINTER(i64), i64, f64p, C.c_int]
     L.oracle_expert_h_fp8.argtypes = [u8p, f64p, u8p, f64p, u8p, f64p, i64, i64, u8p, f64p]
+    L.oracle_e2m1_decode.argtypes = [C.c_uint8]
+    L.oracle_e2m1_decode.restype = C.c_double
+    L.oracle_e2m1_encode.argtypes = [C.c_double]
+    L.oracle_e2m1_encode.restype = C.c_uint8
+    L.oracle_fp4_block_scale.argtypes = [C.c_double]
+    L.oracle_fp4_block_scale.restype = C.c_double
+    L.oracle_quantize_rows_fp4.argtypes = [u16p, i64, i64, u8p, f64p]
+    L.oracle_quantize_rows_fp4.restype = C.c_int
+    L.oracle_moe_ffn_fp4.argtypes = L.oracle_moe_ffn_fp8.argtypes
+    L.oracle_moe_ffn_fp4.restype = C.c_int
     for fn in ("oracle_quantize_rows_fp8", "oracle_quantize_blocks_fp8", "oracle_moe_ffn_fp8",
                "oracle_expert_h_fp8"):
         getattr(L, fn).restype = C.c_int
@@ -238,6 +248,11 @@ def moe_ffn_fp8(xq, sx, W1q, s1, W3q, s3, W2q, s2, idx, w, shared=None, tokens=N
     """fp64 y[t] = sum_j w[t,j] FFN8_e(x^_t) (+ shared) on dequantised e4m3 operands, with h
     requantised in 1 x 128 blocks before the down projection.  Per-expert lists may hold None
     for experts no listed token uses; shared = dict(W1q, s1, W3q, s3, W2q, s2)."""
+    return _moe_ffn_lowp(lib().oracle_moe_ffn_fp8, "moe_ffn_fp8", xq, sx, W1q, s1, W3q, s3, W2q, s2, idx, w, shared,
+                         tokens, nthreads)
+
+
+def _moe_ffn_lowp(fn, what, xq, sx, W1q, s1, W3q, s3, W2q, s2, idx, w, shared, tokens, nthreads):
     xq = np.ascontiguousarray(xq, dtype=np.uint8)
     sx = np.ascontiguousarray(sx, dtype=np.float64)
     T, d = xq.shape
@@ -246,7 +261,6 @@ def moe_ffn_fp8(xq, sx, W1q, s1, W3q, s3, W2q, s2, idx, w, shared=None, tokens=N
     k = idx.shape[1]
     E = len(W1q)
     f = next(a.shape[0] for a in W1q if a is not None)
-    up, dp = C.POINTER(C.c_uint8), C.POINTER(C.c_double)
     keep = []
 
     def arr(lst, ct, dt):
@@ -274,12 +288,11 @@ def moe_ffn_fp8(xq, sx, W1q, s1, W3q, s3, W2q, s2, idx, w, shared=None, tokens=N
         tok = np.ascontiguousarray(tokens, dtype=np.int64)
         ntok = tok.size
     out = np.empty((ntok, d), dtype=np.float64)
-    _check(lib().oracle_moe_ffn_fp8(_ptr(xq, C.c_uint8), _ptr(sx, C.c_double), pw1, ps1, pw3, ps3, pw2, ps2, d, f, E,
-                                    _ptr(idx, C.c_int32), _ptr(w, C.c_double), k,
-                                    _ptr(sh[0], C.c_uint8), _ptr(sh[1], C.c_double), _ptr(sh[2], C.c_uint8),
-                                    _ptr(sh[3], C.c_double), _ptr(sh[4], C.c_uint8), _ptr(sh[5], C.c_double), fs,
-                                    _ptr(tok, C.c_int64), ntok, _ptr(out, C.c_double), int(nthreads)),
-           "moe_ffn_fp8")
+    _check(fn(_ptr(xq, C.c_uint8), _ptr(sx, C.c_double), pw1, ps1, pw3, ps3, pw2, ps2, d, f, E,
+              _ptr(idx, C.c_int32), _ptr(w, C.c_double), k,
+              _ptr(sh[0], C.c_uint8), _ptr(sh[1], C.c_double), _ptr(sh[2], C.c_uint8),
+              _ptr(sh[3], C.c_double), _ptr(sh[4], C.c_uint8), _ptr(sh[5], C.c_double), fs,
+              _ptr(tok, C.c_int64), ntok, _ptr(out, C.c_double), int(nthreads)), what)
     return out
 
 
@@ -300,3 +313,39 @@ def expert_h_fp8(xq, sx, W1q, s1, W3q, s3):
                                      _ptr(s3, C.c_double), _ptr(xq, C.c_uint8), _ptr(sx, C.c_double), d, f,
                                      _ptr(hq, C.c_uint8), _ptr(sh, C.c_double)), "expert_h_fp8")
     return hq, sh
+
+
+# ---------------------------------------------------------------- FP4 weights (e2m1, 1 x 32 power-of-two scales)
+
+def e2m1_decode(code: int) -> float:
+    return float(lib().oracle_e2m1_decode(int(code)))
+
+
+def e2m1_encode(v: float) -> int:
+    """Nearest e2m1 code (ties to even), saturating to +-6."""
+    return int(lib().oracle_e2m1_encode(float(v)))
+
+
+def fp4_block_scale(amax: float) -> float:
+    """Smallest power of two s with amax / s <= 6 (1 for amax = 0)."""
+    return float(lib().oracle_fp4_block_scale(float(amax)))
+
+
+def quantize_rows_fp4(W: np.ndarray):
+    """1 x 32 blocks along rows: bf16 bits [R, C] -> (e2m1 codes [R, C], one per byte; scales [R, C/32])."""
+    W = _u16(W)
+    R, Cc = W.shape
+    q = np.empty((R, Cc), dtype=np.uint8)
+    sc = np.empty((R, Cc // 32), dtype=np.float64)
+    _check(lib().oracle_quantize_rows_fp4(_ptr(W, C.c_uint16), R, Cc, _ptr(q, C.c_uint8), _ptr(sc, C.c_double)),
+           "quantize_rows_fp4")
+    return q, sc
+
+
+def moe_ffn_fp4(xq, sx, W1q, s1, W3q, s3, W2q, s2, idx, w, shared=None, tokens=None, nthreads: int = 0):
+    """fp64 y[t] = sum_j w[t,j] FFN4_e(x^_t) (+ shared): e4m3 activations (1 x 128 scales), e2m1 weights
+    (one code per byte) with 1 x 32 scales ([f, d/32] for W1/W3, [d, f/32] for W2), h requantised to
+    e4m3 in 1 x 128 blocks before the down projection.  Per-expert lists may hold None for experts no
+    listed token uses; shared = dict(W1q, s1, W3q, s3, W2q, s2)."""
+    return _moe_ffn_lowp(lib().oracle_moe_ffn_fp4, "moe_ffn_fp4", xq, sx, W1q, s1, W3q, s3, W2q, s2, idx, w, shared,
+                         tokens, nthreads)

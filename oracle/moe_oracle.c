@@ -622,3 +622,233 @@ int oracle_moe_ffn_fp8(const uint8_t *xq, const double *sx,
     free(th);
     return status;
 }
+
+/* ------------------------------------------------------------------------
+ * FP4 expert weights (GC-MoE, abstract: an FP8/FP4 MoE operator with
+ * block-scaled MMA).  The pages name FP4 without a layout; the reading taken
+ * is the OCP microscaling FP4 element type with 32-element blocks (MXFP4):
+ *   e2m1 codes: bit 3 sign, bits 2-1 exponent (bias 1), bit 0 mantissa;
+ *   exponent 0 is subnormal (0 or 0.5); no infinities or NaNs; largest 6.
+ *   Weights are quantised per row in blocks of 32 consecutive K elements, a
+ *   block's scale the smallest power of two s with amax / s <= 6 (s = 1 for
+ *   an all-zero block), held to the UE8M0 range; codes are round to nearest,
+ *   ties to the even code, saturating at 6.
+ * Activations (x, and h before the down projection) stay e4m3 in 1 x 128
+ * blocks, as in the FP8 path.
+ * ------------------------------------------------------------------------ */
+
+double oracle_e2m1_decode(uint8_t code)
+{
+    int sign = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return sign ? -v : v;
+}
+
+/* Nearest e2m1 code to v (ties to the code with an even mantissa), saturating to 6. */
+uint8_t oracle_e2m1_encode(double v)
+{
+    uint8_t sign = (v < 0 || (v == 0 && signbit(v))) ? 8 : 0;
+    double a = fabs(v);
+    if (a >= 6.0)
+        return sign | 7;
+    uint8_t best = 0;
+    double best_err = a;
+    for (int c = 1; c <= 7; c++) {
+        double err = fabs(oracle_e2m1_decode((uint8_t)c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {
+            best = (uint8_t)c;
+            best_err = err;
+        }
+    }
+    return sign | best;
+}
+
+/* Smallest power of two s with amax / s <= 6 (amax = 0: s = 1), kept in the UE8M0 range 2^-127 .. 2^127. */
+double oracle_fp4_block_scale(double amax)
+{
+    if (!(amax > 0))
+        return 1.0;
+    int e = 0;
+    while (amax > ldexp(6.0, e) && e < 127)
+        e++;
+    while (amax <= ldexp(6.0, e - 1) && e > -127)
+        e--;
+    return ldexp(1.0, e);
+}
+
+/* 1 x 32 blocks along each row: W [R, C] bf16 -> codes [R, C] (one e2m1 code per
+ * byte, low 4 bits), scales [R, C/32].  C % 32 == 0. */
+int oracle_quantize_rows_fp4(const uint16_t *W, int64_t R, int64_t C, uint8_t *q, double *s)
+{
+    if (R < 0 || C <= 0 || C % 32 || (R > 0 && (!W || !q || !s)))
+        return ORACLE_EARG;
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t b = 0; b < C / 32; b++) {
+            double amax = 0;
+            for (int64_t c = 0; c < 32; c++)
+                amax = fmax(amax, fabs(bf16_value(W[r * C + b * 32 + c])));
+            double sc = oracle_fp4_block_scale(amax);
+            s[r * (C / 32) + b] = sc;
+            for (int64_t c = 0; c < 32; c++)
+                q[r * C + b * 32 + c] = oracle_e2m1_encode(bf16_value(W[r * C + b * 32 + c]) / sc);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* One FP4-weight SwiGLU expert on one token: as expert_ffn_fp8_add with the
+ * weights dequantised from e2m1 codes and 1 x 32 scales (W1/W3 [f,d] codes with
+ * [f, d/32] scales, W2 [d,f] codes with [d, f/32] scales). */
+static void expert_ffn_fp4_add(const uint8_t *W1q, const double *s1, const uint8_t *W3q, const double *s3,
+                               const uint8_t *W2q, const double *s2, const uint8_t *xq, const double *sx,
+                               int64_t d, int64_t f, double gate, double *h, uint8_t *hq, double *sh, double *y)
+{
+    const int64_t fb = f / 128;
+    for (int64_t r = 0; r < f; r++) {
+        double g = 0.0, u = 0.0;
+        for (int64_t c = 0; c < d; c++) {
+            double xc = e4m3_value(xq[c]) * sx[c / 128];
+            g += oracle_e2m1_decode(W1q[r * d + c]) * s1[r * (d / 32) + c / 32] * xc;
+            u += oracle_e2m1_decode(W3q[r * d + c]) * s3[r * (d / 32) + c / 32] * xc;
+        }
+        h[r] = g / (1.0 + exp(-g)) * u;
+    }
+    for (int64_t b = 0; b < fb; b++) {          /* requantise h in 1 x 128 blocks (e4m3) */
+        double amax = 0;
+        for (int64_t r = 0; r < 128; r++)
+            amax = fmax(amax, fabs(h[b * 128 + r]));
+        double sc = oracle_fp8_block_scale(amax);
+        sh[b] = sc;
+        for (int64_t r = 0; r < 128; r++)
+            hq[b * 128 + r] = oracle_e4m3_encode_fast(h[b * 128 + r] / sc);
+    }
+    for (int64_t r = 0; r < f; r++)
+        h[r] = e4m3_value(hq[r]) * sh[r / 128];
+    for (int64_t c = 0; c < d; c++) {
+        double z = 0.0;
+        for (int64_t r = 0; r < f; r++)
+            z += oracle_e2m1_decode(W2q[c * f + r]) * s2[c * (f / 32) + r / 32] * h[r];
+        y[c] += gate * z;
+    }
+}
+
+typedef struct {
+    const uint8_t *xq;
+    const double *sx;
+    const uint8_t *const *W1q, *const *W3q, *const *W2q;
+    const double *const *s1, *const *s3, *const *s2;
+    int64_t d, f, E, k;
+    const int32_t *idx;
+    const double *w;
+    const uint8_t *Ws1q, *Ws3q, *Ws2q;
+    const double *ss1, *ss3, *ss2;
+    int64_t fs;
+    const int64_t *tokens;
+    int64_t ntok;
+    double *out;
+    int nthreads, tid;
+    int status;
+} ffn4_job;
+
+static void *ffn4_worker(void *arg)
+{
+    ffn4_job *J = (ffn4_job *)arg;
+    int64_t hlen = J->f > J->fs ? J->f : J->fs;
+    if (hlen <= 0)
+        hlen = 128;
+    double *h = (double *)malloc((size_t)hlen * sizeof(double));
+    uint8_t *hq = (uint8_t *)malloc((size_t)hlen);
+    double *sh = (double *)malloc((size_t)(hlen / 128) * sizeof(double));
+    if (!h || !hq || !sh) {
+        free(h);
+        free(hq);
+        free(sh);
+        J->status = ORACLE_ENOMEM;
+        return NULL;
+    }
+    const int64_t db = J->d / 128;
+    for (int64_t i = J->tid; i < J->ntok; i += J->nthreads) {
+        int64_t t = J->tokens ? J->tokens[i] : i;
+        const uint8_t *xt = J->xq + t * J->d;
+        const double *st = J->sx + t * db;
+        double *y = J->out + i * J->d;
+        for (int64_t c = 0; c < J->d; c++)
+            y[c] = 0.0;
+        for (int64_t j = 0; j < J->k; j++) {
+            int32_t e = J->idx[t * J->k + j];
+            if (e < 0 || e >= J->E || !J->W1q[e] || !J->W3q[e] || !J->W2q[e]) {
+                J->status = ORACLE_ERANGE;
+                free(h);
+                free(hq);
+                free(sh);
+                return NULL;
+            }
+            expert_ffn_fp4_add(J->W1q[e], J->s1[e], J->W3q[e], J->s3[e], J->W2q[e], J->s2[e], xt, st, J->d,
+                               J->f, J->w[t * J->k + j], h, hq, sh, y);
+        }
+        if (J->fs > 0)
+            expert_ffn_fp4_add(J->Ws1q, J->ss1, J->Ws3q, J->ss3, J->Ws2q, J->ss2, xt, st, J->d, J->fs, 1.0, h, hq,
+                               sh, y);
+    }
+    free(h);
+    free(hq);
+    free(sh);
+    return NULL;
+}
+
+/* FP4-weight expert FFNs of the listed tokens (the FP4 counterpart of
+ * oracle_moe_ffn_fp8): xq [T,d] e4m3 with sx [T, d/128]; per expert W1q[e],
+ * W3q[e] [f,d] e2m1 codes (one per byte) with s1[e], s3[e] [f, d/32];
+ * W2q[e] [d,f] with s2[e] [d, f/32]; the shared expert likewise (fs > 0).
+ * d, f, fs multiples of 128. */
+int oracle_moe_ffn_fp4(const uint8_t *xq, const double *sx,
+                       const uint8_t *const *W1q, const double *const *s1,
+                       const uint8_t *const *W3q, const double *const *s3,
+                       const uint8_t *const *W2q, const double *const *s2,
+                       int64_t d, int64_t f, int64_t E, const int32_t *idx, const double *w, int64_t k,
+                       const uint8_t *Ws1q, const double *ss1, const uint8_t *Ws3q, const double *ss3,
+                       const uint8_t *Ws2q, const double *ss2, int64_t fs,
+                       const int64_t *tokens, int64_t ntok, double *out, int nthreads)
+{
+    if (d <= 0 || f <= 0 || E <= 0 || k < 1 || ntok < 0 || fs < 0 || d % 128 || f % 128 || fs % 128)
+        return ORACLE_EARG;
+    if (ntok == 0)
+        return ORACLE_OK;
+    if (!xq || !sx || !W1q || !W3q || !W2q || !s1 || !s3 || !s2 || !idx || !w || !out ||
+        (fs > 0 && (!Ws1q || !Ws3q || !Ws2q || !ss1 || !ss3 || !ss2)))
+        return ORACLE_EARG;
+    if (nthreads <= 0)
+        nthreads = oracle_default_threads();
+    if (nthreads > ntok)
+        nthreads = (int)ntok;
+    ffn4_job *jobs = (ffn4_job *)calloc((size_t)nthreads, sizeof(ffn4_job));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !th) {
+        free(jobs);
+        free(th);
+        return ORACLE_ENOMEM;
+    }
+    for (int i = 0; i < nthreads; i++) {
+        ffn4_job J = {xq, sx, W1q, W3q, W2q, s1, s3, s2, d, f, E, k, idx, w, Ws1q, Ws3q, Ws2q, ss1, ss3, ss2,
+                      fs, tokens, ntok, out, nthreads, i, ORACLE_OK};
+        jobs[i] = J;
+    }
+    int started = 0;
+    for (int i = 1; i < nthreads; i++) {
+        if (pthread_create(&th[i], NULL, ffn4_worker, &jobs[i]) != 0)
+            break;
+        started = i;
+    }
+    for (int i = started + 1; i < nthreads; i++)
+        ffn4_worker(&jobs[i]);
+    ffn4_worker(&jobs[0]);
+    for (int i = 1; i <= started; i++)
+        pthread_join(th[i], NULL);
+    int status = ORACLE_OK;
+    for (int i = 0; i < nthreads; i++)
+        if (jobs[i].status != ORACLE_OK)
+            status = jobs[i].status;
+    free(jobs);
+    free(th);
+    return status;
+}

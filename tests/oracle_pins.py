@@ -531,4 +531,129 @@ def pin_fp8_ffn_exact_operands_match_bf16_path():
     assert np.abs(y8 - y16).max() > 0 or np.allclose(h_bound, 0)
 
 
+def _e2m1_lib():
+    import ml_dtypes
+    return ml_dtypes.float4_e2m1fn
+
+
+def _fp4_dq(q, s):
+    """e2m1 codes [R, C] (one per byte) with 1 x 32 scales [R, C/32] through the library decode."""
+    v = q.astype(np.uint8).view(_e2m1_lib()).astype(np.float64)
+    return v * np.repeat(s, 32, axis=1)
+
+
+def pin_e2m1_codec_matches_library():
+    """e2m1 decode of all 16 codes and encode of a dense grid (every midpoint, past +-6,
+    signed zeros) against the ml_dtypes float4_e2m1fn conversions."""
+    lib = _e2m1_lib()
+    codes = np.arange(16, dtype=np.uint8)
+    ref = codes.view(lib).astype(np.float64)
+    ours = np.array([oracle.e2m1_decode(int(c)) for c in codes])
+    assert np.array_equal(ours, ref) and np.array_equal(np.signbit(ours), np.signbit(ref))
+    mags = np.unique(np.abs(ref))
+    mids = (mags[1:] + mags[:-1]) / 2
+    grid = np.concatenate([np.linspace(-9, 9, 7201), mids, -mids, [6.0001, 100.0, -100.0, -0.0, 1e-9, -1e-9]])
+    want = grid.astype(np.float32).astype(lib).view(np.uint8)
+    got = np.array([oracle.e2m1_encode(float(v)) for v in grid], dtype=np.uint8)
+    assert np.array_equal(got, want)
+
+
+def pin_fp4_block_scale():
+    """A power of two, the smallest with amax / s <= 6, 1 for an all-zero block, inside UE8M0."""
+    rng = np.random.default_rng(11)
+    for amax in np.concatenate([10.0 ** rng.uniform(-30, 30, 300), [6.0, 6.0001, 3.0, 1.5, 12.0]]):
+        sc = oracle.fp4_block_scale(float(amax))
+        m, e = math.frexp(sc)
+        assert m == 0.5
+        assert amax / sc <= 6.0 and amax / (sc / 2) > 6.0
+    assert oracle.fp4_block_scale(0.0) == 1.0
+    assert oracle.fp4_block_scale(1e-45) == 2.0 ** -127
+
+
+def pin_fp4_quantize_rows():
+    """1 x 32 blocks: each block's scale from its amax, codes the library cast of v / s."""
+    gen = torch.Generator().manual_seed(12)
+    W = (torch.randn(9, 256, generator=gen) * torch.logspace(-3, 3, 9)[:, None]).to(torch.bfloat16)
+    W[0, :32] = 0.0
+    W[1, 40] = 1e30
+    q, sc = oracle.quantize_rows_fp4(_bits(W))
+    Wf = W.to(torch.float64).numpy()
+    for r in range(W.shape[0]):
+        for b in range(W.shape[1] // 32):
+            blk = Wf[r, 32 * b:32 * (b + 1)]
+            s_ = oracle.fp4_block_scale(float(np.abs(blk).max()))
+            assert sc[r, b] == s_
+            want = (blk / s_).astype(np.float32).astype(_e2m1_lib()).view(np.uint8)
+            assert np.array_equal(q[r, 32 * b:32 * (b + 1)], want), (r, b)
+
+
+def _fp4_layer(E=3, k=2, T=5, d=256, f=256, fs=0, seed=31):
+    s = wl.LayerShape("p4", T=T, d=d, f=f, E=E, k=k, alpha=1.0, f_shared=fs)
+    inp = wl.make_inputs(s, seed=seed)
+    inp["x"] = inp["x"].clone()
+    inp["x"][:, 128:256] *= 32.0
+    xq, sx = oracle.quantize_rows_fp8(_bits(inp["x"]))
+    Q = {n: [oracle.quantize_rows_fp4(_bits(inp[n][e])) for e in range(E)] for n in ("W1", "W3", "W2")}
+    sh = None
+    if fs:
+        sh = {}
+        for n, key in (("Ws1", "1"), ("Ws3", "3"), ("Ws2", "2")):
+            q_, s_ = oracle.quantize_rows_fp4(_bits(inp[n]))
+            sh["W%sq" % key], sh["s%s" % key] = q_, s_
+    return s, inp, xq, sx, Q, sh
+
+
+def pin_fp4_ffn_expert_major():
+    """Expert-major float64 evaluation on library-decoded e2m1 weights (1 x 32 scales) and e4m3
+    activations, h requantised with the library e4m3 cast; shared expert included."""
+    s, inp, xq, sx, Q, sh = _fp4_layer(fs=128)
+    assert len(np.unique(Q["W1"][0][1][:, :4])) > 1      # distinct per-row block scales are exercised
+    idx = wl.random_routing(s.T, s.E, s.k, 1.0, 4).numpy()
+    w = wl.random_gates(s.T, s.k, 4).numpy().astype(np.float64)
+    y = oracle.moe_ffn_fp4(xq, sx, [q for q, _ in Q["W1"]], [c for _, c in Q["W1"]], [q for q, _ in Q["W3"]],
+                           [c for _, c in Q["W3"]], [q for q, _ in Q["W2"]], [c for _, c in Q["W2"]], idx, w,
+                           shared=sh)
+    xh = _dq(xq, sx, 1, 128)
+
+    def ffn(W1q, s1, W3q, s3, W2q, s2):
+        g = xh @ _fp4_dq(W1q, s1).T
+        u = xh @ _fp4_dq(W3q, s3).T
+        h = torch.nn.functional.silu(torch.from_numpy(g)).numpy() * u
+        return _requant_h(h) @ _fp4_dq(W2q, s2).T
+
+    ref = np.zeros((s.T, s.d))
+    for e in range(s.E):
+        gate = np.array([w[t][list(idx[t]).index(e)] if e in idx[t] else 0.0 for t in range(s.T)])
+        ref += gate[:, None] * ffn(*Q["W1"][e], *Q["W3"][e], *Q["W2"][e])
+    ref += ffn(sh["W1q"], sh["s1"], sh["W3q"], sh["s3"], sh["W2q"], sh["s2"])
+    assert np.allclose(y, ref, rtol=1e-10, atol=1e-12)
+
+
+def pin_fp4_exact_weights_match_fp8_path():
+    """Weights on the e2m1 grid times 2^-4 with every 32-block holding +-6 * 2^-4: the FP4 and the
+    FP8 quantisations both keep them exactly, so the FP4 FFN equals the (pinned) FP8 FFN."""
+    E, T, d, f = 2, 3, 128, 128
+    rng = np.random.default_rng(13)
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6, -0.5, -1, -1.5, -2, -3, -4, -6]) * 2.0 ** -4
+
+    def weights(rows, cols):
+        W = rng.choice(grid, size=(E, rows, cols))
+        W[:, :, ::32] = 6 * 2.0 ** -4
+        return torch.from_numpy(W).to(torch.bfloat16)
+
+    W1, W3, W2 = weights(f, d), weights(f, d), weights(d, f)
+    x = torch.from_numpy(rng.standard_normal((T, d))).to(torch.bfloat16)
+    xq, sx = oracle.quantize_rows_fp8(_bits(x))
+    idx = np.array([[0, 1], [1, 0], [0, 1]], dtype=np.int32)
+    w = np.array([[0.75, 0.25], [0.5, 0.5], [1.0, 0.0]])
+    Q4 = {n: [oracle.quantize_rows_fp4(_bits(t[e])) for e in range(E)] for n, t in (("1", W1), ("3", W3), ("2", W2))}
+    Q8 = {n: [oracle.quantize_blocks_fp8(_bits(t[e])) for e in range(E)] for n, t in (("1", W1), ("3", W3), ("2", W2))}
+    assert np.array_equal(_fp4_dq(*Q4["1"][0]), W1[0].to(torch.float64).numpy())
+    args = lambda Q: ([q for q, _ in Q["1"]], [c for _, c in Q["1"]], [q for q, _ in Q["3"]], [c for _, c in Q["3"]],
+                      [q for q, _ in Q["2"]], [c for _, c in Q["2"]])
+    y4 = oracle.moe_ffn_fp4(xq, sx, *args(Q4), idx, w)
+    y8 = oracle.moe_ffn_fp8(xq, sx, *args(Q8), idx, w)
+    assert np.array_equal(y4, y8)
+
+
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

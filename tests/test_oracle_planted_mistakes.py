@@ -60,6 +60,20 @@ MUTANTS = {
     "fp8_activation_first_block_scale": ("double xc = e4m3_value(xq[c]) * sx[c / 128];",
                                          "double xc = e4m3_value(xq[c]) * sx[0];"),
     "fp8_h_requant_block0_amax": ("amax = fmax(amax, fabs(h[b * 128 + r]));", "amax = fmax(amax, fabs(h[r]));"),
+    "fp4_exponent_bias": ("double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);",
+                          "double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 2);"),
+    "fp4_subnormal_value": ("double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);",
+                            "double v = e == 0 ? 0.25 * m : ldexp(1.0 + 0.5 * m, e - 1);"),
+    "fp4_ties_to_odd": ("if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {\n            best = (uint8_t)c;\n            best_err = err;\n        }\n    }\n    return sign | best;\n}\n\n/* Smallest power of two s with amax / s <= 6",
+                        "if (err < best_err || (err == best_err && (c & 1) == 1 && (best & 1) == 0)) {\n            best = (uint8_t)c;\n            best_err = err;\n        }\n    }\n    return sign | best;\n}\n\n/* Smallest power of two s with amax / s <= 6"),
+    "fp4_scale_not_smallest": ("while (amax <= ldexp(6.0, e - 1) && e > -127)",
+                               "while (amax <= ldexp(3.0, e - 1) && e > -127)"),
+    "fp4_block_of_64": ("g += oracle_e2m1_decode(W1q[r * d + c]) * s1[r * (d / 32) + c / 32] * xc;",
+                        "g += oracle_e2m1_decode(W1q[r * d + c]) * s1[r * (d / 32) + c / 64] * xc;"),
+    "fp4_up_scale_of_gate": ("u += oracle_e2m1_decode(W3q[r * d + c]) * s3[r * (d / 32) + c / 32] * xc;",
+                             "u += oracle_e2m1_decode(W3q[r * d + c]) * s1[r * (d / 32) + c / 32] * xc;"),
+    "fp4_down_scale_transposed": ("z += oracle_e2m1_decode(W2q[c * f + r]) * s2[c * (f / 32) + r / 32] * h[r];",
+                                  "z += oracle_e2m1_decode(W2q[c * f + r]) * s2[r * (d / 32) + c / 32] * h[r];"),
     "fp8_down_scale_transposed": ("z += e4m3_value(W2q[c * f + r]) * s2[(c / 128) * fb + r / 128] * h[r];",
                                   "z += e4m3_value(W2q[c * f + r]) * s2[(r / 128) * fb + c / 128] * h[r];"),
 }
