@@ -7,7 +7,7 @@ grouped GEMM, combine) over one batch of seeded synthetic tokens, through
 moe_layer_forward.  Prints ONE JSON line on rank 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--T ..] [--alpha ..] [--E ..] [--fp8] [--impl ours|reference]
+                    [--T ..] [--alpha ..] [--E ..] [--fp8 | --fp4] [--impl ours|reference]
 
 With no --workload the line times the largest layer of the workload table
 that fits one GPU: the DeepSeek-V3-shaped layer at T=16384 (d=7168, f=2048,
@@ -17,7 +17,9 @@ decode-shaped layer (decode64: T=32, d=2048, f=1024, E=64, top-8, alpha=1),
 the small-T, weight-streaming end of the table.
 
 ``--fp8`` times moe_layer_forward_fp8 (e4m3 expert weights with 128 x 128
-block scales, quantised once before the timed region).
+block scales, quantised once before the timed region); ``--fp4`` times
+moe_layer_forward_fp4 (e2m1 expert weights with 1 x 32 power-of-two scales,
+e4m3 activations).
 
 Multi-GPU (torchrun) runs independent replicas: the layer has no exchange
 step, so every rank times its own copy and the value is the tokens of all
@@ -55,6 +57,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # 2.25 PFLOP/s of dense bf16 (4.5 fp8).  Fractions of these are reported beside the
 # fractions of the measured peaks.
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+DTYPES = {"bf16": "bf16", "fp8": "fp8-e4m3 (fp32 accumulate)",
+          "fp4": "fp4-e2m1 weights x fp8-e4m3 activations (fp32 accumulate)"}
 HEADLINE = dict(workload="deepseek_v3", T=16384, alpha=0.5)
 DECODE_SUB = dict(workload="decode64", T=32, alpha=1.0)
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "roofline_traffic.json")
@@ -98,6 +102,7 @@ def peaks():
 
 
 def kernel_source_hash(fp8: bool = False) -> str:
+    """Hash of the dominant kernel's sources (the FP8 kernel serves FP4 weights too)."""
     h = hashlib.sha256()
     for rel in (FP8_KERNEL_SOURCES if fp8 else KERNEL_SOURCES):
         h.update(open(os.path.join(ROOT, rel), "rb").read())
@@ -117,7 +122,7 @@ def committed_traffic(workload_name: str, kernel: str = None):
     or None when absent, for another workload or kernel, or taken on older kernel
     source.  A record taken on a reduced case carries the full launch's bytes
     scaled from it (its "scaled_from" says how)."""
-    fp8 = workload_name.endswith(" fp8")
+    fp8 = workload_name.endswith((" fp8", " fp4"))
     for rec in traffic_records():
         if rec.get("workload") != workload_name:
             continue
@@ -220,18 +225,20 @@ def gemm_fused(P: int, f: int) -> bool:
     return P <= 256 and f <= 4096
 
 
-def algorithmic(s: wl.LayerShape, counts: np.ndarray, fp8: bool = False):
+def algorithmic(s: wl.LayerShape, counts: np.ndarray, fp8: bool = False, fmt: str = None):
     """Algorithmic bytes and flops of the layer and of the gate/up GEMM launch.
 
     bf16: 2 bytes per weight and activation.  FP8: 1 byte per weight and
     activation plus one fp32 scale per 128 x 128 weight block and per 1 x 128
-    activation block."""
+    activation block.  FP4 (fmt="fp4"): half a byte per weight plus one scale
+    byte per 32 weights; activations as FP8."""
+    fmt = fmt or ("fp8" if fp8 else "bf16")
     active = int((counts > 0).sum())
     P = int(counts.sum())
     fs = s.f_shared
-    wb = 1 if fp8 else 2
-    wsc = (4.0 / (128 * 128)) if fp8 else 0.0    # weight-scale bytes per weight
-    asc = (4.0 / 128) if fp8 else 0.0            # activation-scale bytes per activation
+    wb = {"bf16": 2, "fp8": 1, "fp4": 0.5}[fmt]
+    wsc = {"bf16": 0.0, "fp8": 4.0 / (128 * 128), "fp4": 1.0 / 32}[fmt]    # weight-scale bytes per weight
+    asc = 0.0 if fmt == "bf16" else 4.0 / 128                                # activation-scale bytes per activation
 
     def mat(rows, cols):
         return rows * cols * (wb + wsc)
@@ -263,7 +270,15 @@ def weight_sets(wbytes: int) -> int:
     return want
 
 
-def kernel_roofline(s, alg, phase_ms, fp8, pk, pk_kind):
+def fmt_suffix(fmt):
+    return "" if fmt in (None, "bf16") else " " + fmt
+
+
+def weight_format(args):
+    return "fp4" if getattr(args, "fp4", False) else "fp8" if args.fp8 else "bf16"
+
+
+def kernel_roofline(s, alg, phase_ms, fp8, pk, pk_kind, fmt=None):
     """The dominant kernel's roofline: the single expert-GEMM launch when the
     library fuses both GEMMs, else the gate/up launch (2/3 of the flops and the
     largest launch of the layer)."""
@@ -289,7 +304,7 @@ def kernel_roofline(s, alg, phase_ms, fp8, pk, pk_kind):
         roof = {"bound": "tensor", "achieved": nflops / t / 1e12, "peak": tc / 1e12, "unit": "TFLOP/s"}
         roof["frac_nominal"] = nflops / t / tc_nom
     roof["frac"] = roof["achieved"] / roof["peak"]
-    name = ("grouped_gemm_fp8_kernel" if fp8 else "grouped_gemm_kernel")
+    name = ("grouped_gemm_fp8_kernel" if fp8 else "grouped_gemm_kernel") + ("<e2m1 weights>" if fmt == "fp4" else "")
     roof["kernel"] = f"{name}<{'fused gate/up + down' if fused else 'gate/up + SwiGLU'}>"
     roof["kernel_role"] = role
     roof["scope"] = "one expert-GEMM launch (the layer's fraction is layer_roofline.frac)"
@@ -297,11 +312,11 @@ def kernel_roofline(s, alg, phase_ms, fp8, pk, pk_kind):
     roof["algorithmic_flops_per_launch"] = nflops
     roof["launch_us"] = t * 1e6
     if roof["bound"] == "tensor":
-        roof["peak_source"] = f"{pk_kind} ({'2 x sustained bf16 (fp8)' if fp8 else 'sustained bf16'})"
+        roof["peak_source"] = f"{pk_kind} ({'2 x sustained bf16 (the f8f6f4 MMA rate)' if fp8 else 'sustained bf16'})"
     else:
         roof["peak_source"] = f"{pk_kind} (HBM copy)"
     roof["nominal_peak"] = (tc_nom / 1e12 if roof["bound"] == "tensor" else bw_nom / 1e9)
-    roof["traffic"] = committed_traffic(workload_label(s) + (" fp8" if fp8 else ""), role)
+    roof["traffic"] = committed_traffic(workload_label(s) + fmt_suffix(fmt), role)
     return roof
 
 
@@ -415,6 +430,9 @@ def _make_step(moe, s, fp8, x, Wg, bias, sets, qsets, ws, out, R):
     def step(i, prof_events=None):
         if prof_events is not None:
             moe.moe_record_phase_events(prof_events)
+        if fp8 == "fp4":
+            moe.moe_layer_forward_fp4(x, Wg, bias, qsets[i % R], s.k, ws, out=out)
+            return
         if fp8:
             moe.moe_layer_forward_fp8(x, Wg, bias, qsets[i % R], s.k, ws, out=out)
             return
@@ -440,16 +458,28 @@ def measure_layer(s: wl.LayerShape, args, steps: int, warmup: int, world: int, d
     x, Wg, bias = base["x"], base["Wg"], base["bias"]
     out = torch.empty(s.T, s.d, dtype=torch.bfloat16, device=dev)
     qsets = None
-    if args.fp8:
-        # e4m3 weights with 128 x 128 block scales (quantised once, outside the timed region)
-        qsets = [moe.quantize_layer_fp8(w) for w in sets]
-        ws = moe.new_workspace_fp8(s.T, s.d, s.f, s.E, s.k, s.f_shared, device=dev)
-        wbytes = sum(t.numel() * t.element_size() for t in qsets[0].values())
+    fmt = weight_format(args)
+    if fmt != "bf16":
+        # e4m3 weights with 128 x 128 block scales, or e2m1 with 1 x 32 scales
+        # (quantised once, outside the timed region)
+        quant = moe.quantize_layer_fp4 if fmt == "fp4" else moe.quantize_layer_fp8
+        qsets = [quant(w) for w in sets]
         sets = None
+        wbytes = sum(t.numel() * t.element_size() for t in qsets[0].values())
+        # the quantised sets are smaller: add sets until they again exceed 3x L2
+        free, _ = torch.cuda.mem_get_info(dev)
+        want = int(max(1, min(weight_sets(wbytes), sets_override or weight_sets(wbytes),
+                              (free * 0.5) // max(wbytes, 1))))
+        for i in range(len(qsets), want):
+            w = wl.make_weights(s, seed=args.seed + 1000 * (i + 1), device=dev)
+            qsets.append(quant(w))
+            del w
+        R = len(qsets)
+        ws = moe.new_workspace_fp8(s.T, s.d, s.f, s.E, s.k, s.f_shared, device=dev)
         torch.cuda.empty_cache()
     else:
         ws = moe.new_workspace(s.T, s.d, s.f, s.E, s.k, s.f_shared, device=dev)
-    step = _make_step(moe, s, args.fp8, x, Wg, bias, sets, qsets, ws, out, R)
+    step = _make_step(moe, s, "fp4" if fmt == "fp4" else fmt == "fp8", x, Wg, bias, sets, qsets, ws, out, R)
 
     for i in range(warmup):
         step(i)
@@ -458,6 +488,17 @@ def measure_layer(s: wl.LayerShape, args, steps: int, warmup: int, world: int, d
     torch.cuda.synchronize()
     if moe.moe_get_device_error(ws) != 0:
         raise RuntimeError("device error after warm-up")
+    if phases_in_timed:
+        # events between the phases keep the next kernel from starting early (no
+        # programmatic overlap), a cost that only long layers can absorb: layers
+        # under 1 ms get their phase split from a second pass instead
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(3):
+            step(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        phases_in_timed = a.elapsed_time(b) / 3 >= 1.0
 
     # CUDA events for the per-phase split: inside the timed region itself (each
     # step records six events on the layer's stream), or in a second pass
@@ -521,29 +562,30 @@ def measure_layer(s: wl.LayerShape, args, steps: int, warmup: int, world: int, d
                "h2d_bytes_per_step": s.T * s.d * 2, "d2h_bytes_per_step": s.T * s.d * 2,
                "ms_per_step": e_ms / steps}
 
-    if args.fp8:
+    if fmt != "bf16":
         views = moe.workspace_views_fp8(ws, s.T, s.d, s.f, s.E, s.k, s.f_shared)
     else:
         views = moe.workspace_views(ws, s.T, s.d, s.f, s.E, s.k, s.f_shared)
     counts = views["counts"].cpu().numpy()
     idx = views["topk_idx"].cpu().numpy()
-    alg = algorithmic(s, counts, fp8=args.fp8)
+    alg = algorithmic(s, counts, fmt=fmt)
+    lowp = fmt != "bf16"
     pk, pk_kind = peaks()
     ms_per_step = ms_max / steps
     rec = {"ms_per_step": ms_per_step, "ms_total": ms_max, "launches": int(launches), "phase_ms": phase_ms,
            "phases_in_timed": phases_in_timed, "counts": counts, "alg": alg, "e2e": e2e, "R": R,
            "wbytes": wbytes,
-           "roofline": kernel_roofline(s, alg, phase_ms, args.fp8, pk, pk_kind),
-           "layer_roofline": layer_roofline(alg, ms_per_step, args.fp8, pk, pk_kind)}
+           "roofline": kernel_roofline(s, alg, phase_ms, lowp, pk, pk_kind, fmt),
+           "layer_roofline": layer_roofline(alg, ms_per_step, lowp, pk, pk_kind)}
     host = None
-    if not args.fp8:
+    if not lowp:
         host = {"x": x, "Wg": Wg, "bias": bias, "weights": one, "idx": idx}
     return rec, host
 
 
-def sub_record(s, rec, fp8):
+def sub_record(s, rec, fmt):
     """The compact form of a second workload measured in the same run."""
-    return {"workload": workload_label(s) + (" fp8" if fp8 else ""), "value": s.T / (rec["ms_per_step"] / 1e3),
+    return {"workload": workload_label(s) + fmt_suffix(fmt), "value": s.T / (rec["ms_per_step"] / 1e3),
             "unit": UNIT, "us_per_layer": rec["ms_per_step"] * 1e3, "steps": rec["steps"],
             "layer_roofline": rec["layer_roofline"], "roofline": rec["roofline"],
             "histogram": stats.histogram_stats(rec["counts"]),
@@ -584,9 +626,9 @@ def run_ours(args, s: wl.LayerShape):
     ms_per_step = rec["ms_per_step"]
     line = {"metric": METRIC, "value": s.T * K * world / (rec["ms_total"] / 1e3), "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3 (fp32 accumulate)" if args.fp8 else "bf16",
+            "scaling": "weak", "vs_baseline": None, "dtype": DTYPES[weight_format(args)],
             "data": "synthetic (seeded; Dirichlet routing skew; random-init weights of the layer's shape)",
-            "config": {"workload": workload_label(s) + (" fp8" if args.fp8 else ""), "T": s.T, "d": s.d, "f": s.f,
+            "config": {"workload": workload_label(s) + fmt_suffix(weight_format(args)), "T": s.T, "d": s.d, "f": s.f,
                        "E": s.E, "k": s.k,
                        "alpha": s.alpha, "f_shared": s.f_shared, "seed": args.seed,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
@@ -594,8 +636,9 @@ def run_ours(args, s: wl.LayerShape):
                              f"{rec['wbytes'] / 2**20:.0f} MiB",
                        "histogram": stats.histogram_stats(rec["counts"]),
                        "us_per_layer": ms_per_step * 1e3,
-                       "phase_note": "per-phase means from CUDA events recorded between the phases inside the "
-                                     "timed region",
+                       "phase_note": ("per-phase means from CUDA events recorded between the phases inside the "
+                                      "timed region" if rec["phases_in_timed"] else
+                                      "per-phase means from a second pass with CUDA events between phases"),
                        "phase_us": {n: float(v * 1e3) for n, v in
                                     zip(("route", "permute", "gemm_gate_up", "gemm_down", "combine"),
                                         rec["phase_ms"])}},
@@ -605,7 +648,7 @@ def run_ours(args, s: wl.LayerShape):
         ds = wl.shape(DECODE_SUB["workload"], T=DECODE_SUB["T"], alpha=DECODE_SUB["alpha"])
         drec, _ = measure_layer(ds, args, args.sub_steps, 20, world, dev, phases_in_timed=False, with_e2e=False)
         drec["steps"] = args.sub_steps
-        line["decode64"] = sub_record(ds, drec, args.fp8)
+        line["decode64"] = sub_record(ds, drec, weight_format(args))
     if rank == 0 and world == 1 and not args.no_cpu_baseline and host is not None:
         line["cpu_baseline"] = cpu_baseline(s, host, args.cpu_budget)
     if world > 1:
@@ -678,7 +721,9 @@ def build_parser():
     ap.add_argument("--E", type=int, default=None, help="override the number of routed experts (profiling cases)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--sets", type=int, default=0, help="rotating weight sets (0: enough to exceed 3x L2)")
-    ap.add_argument("--fp8", action="store_true", help="FP8 block-scaled expert GEMMs (moe_layer_forward_fp8)")
+    fmt = ap.add_mutually_exclusive_group()
+    fmt.add_argument("--fp8", action="store_true", help="FP8 block-scaled expert GEMMs (moe_layer_forward_fp8)")
+    fmt.add_argument("--fp4", action="store_true", help="FP4 expert weights, FP8 activations (moe_layer_forward_fp4)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub", action="store_true", help="skip the decode64 sub-record")

@@ -129,6 +129,70 @@ __global__ void __launch_bounds__(256) quantize_rows_fp8_kernel(const bf16* __re
     }
 }
 
+// ---------------------------------------------------------------- FP4 weights (e2m1, 1 x 32 blocks)
+// Smallest power-of-two exponent e with amax <= 6 * 2^e (amax > 0): amax = m 2^x,
+// m in [0.5, 1); held to the UE8M0 range [-127, 127].
+__device__ __forceinline__ int fp4_scale_exp(float amax)
+{
+    if (!(amax > 0.f)) return 0;
+    int x;
+    const float m = frexpf(amax, &x);
+    return max(-127, min(127, m <= 0.75f ? x - 3 : x - 2));
+}
+
+// Nearest e2m1 code of v (|v| <= 6 after scaling; larger saturates to 6), ties
+// to the even code: the magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 are codes 0..7 and
+// the thresholds are their midpoints, a midpoint going to the even code.
+__device__ __forceinline__ uint32_t e2m1_of(float v)
+{
+    const float a = fabsf(v);
+    const uint32_t c = a <= 0.25f ? 0u : a < 0.75f ? 1u : a <= 1.25f ? 2u : a < 1.75f ? 3u
+                     : a <= 2.5f ? 4u : a < 3.5f ? 5u : a <= 5.f ? 6u : 7u;
+    return c | (signbit(v) ? 8u : 0u);
+}
+
+// Byte offset of row r's scale of 32-wide K sub-block j inside the 512-byte
+// scale atom of its 128-row tile and 128-wide K block: row r0 + 32 r1 at byte
+// 16 r0 + 4 r1, sub-block j in the byte after that -- the layout the
+// block-scaled MMA reads from TMEM after a 32x128b.warpx4 copy.
+__host__ __device__ __forceinline__ int sf_atom_byte(int r, int j)
+{
+    return 16 * (r & 31) + 4 * ((r >> 5) & 3) + j;
+}
+
+// 1 x 32 blocks along rows: W [R, C] bf16 -> packed e2m1 codes q [R, C/2]
+// (element 2i in the low nibble of byte i) and UE8M0 scale bytes in atoms
+// [R/128][C/128][512].  One warp per (row, 128-column block): lane l holds
+// columns 4l..4l+3, the 8 lanes of a 32-wide block share its scale.
+// R % 128 == 0, C % 128 == 0.
+__global__ void __launch_bounds__(256) quantize_rows_fp4_kernel(const bf16* __restrict__ src, int64_t R, int C,
+                                                                uint8_t* __restrict__ q, uint8_t* __restrict__ atoms)
+{
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
+    const int nb = C / 128;
+    const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (wid >= R * nb) return;
+    const int64_t r = wid / nb;
+    const int b = (int)(wid - r * nb);
+    const uint2 raw = *reinterpret_cast<const uint2*>(src + r * C + b * 128 + lane * 4);
+    float v[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u), __uint_as_float(raw.y << 16),
+                  __uint_as_float(raw.y & 0xFFFF0000u)};
+    float a = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));   // 8 lanes of a block
+    const int e = fp4_scale_exp(a);
+    uint32_t packed = 0;
+#pragma unroll
+    for (int i = 0; i < 4; i++) packed |= e2m1_of(ldexpf(v[i], -e)) << (4 * i);
+    *reinterpret_cast<uint16_t*>(q + r * (C / 2) + b * 64 + lane * 2) = (uint16_t)packed;
+    if ((lane & 7) == 0) {
+        const int64_t tile = (r >> 7) * nb + b;
+        atoms[tile * 512 + sf_atom_byte((int)(r & 127), lane >> 3)] = (uint8_t)(e + 127);
+    }
+}
+
 // 128 x 128 blocks: one CTA of 256 threads per block; thread t covers half of row t/2.
 __global__ void __launch_bounds__(256) quantize_blocks_fp8_kernel(const bf16* __restrict__ src, int64_t R, int64_t C,
                                                                   uint8_t* __restrict__ dst,
@@ -235,6 +299,9 @@ struct Fp8Args {
     const float* gate_w;
     uint32_t* err;
     int comp;                       // FP8_FUSED: down tiles per gate/up tile, for the balanced order (cta_tile)
+    // FP4 weights (e2m1, 1 x 32 blocks): the scale atoms of A0 / A1 (and the shared
+    // expert's), [rows/128][K/128][512 bytes]; the weight-block scales above are unused
+    const uint8_t *fA0, *fA1, *fA0s, *fA1s;
 };
 
 // What one launch of the FP8 GEMM runs: the down tiles, the gate/up tiles, or
@@ -378,7 +445,13 @@ __device__ __forceinline__ float pick4f(const float (&v)[4], int i)
 // the four lane quadrants) and issues the MMAs.  tcgen05.cp and tcgen05.mma
 // from one thread execute in issue order, so one set of scale-factor columns
 // serves every K block.
-template <int KIND>
+//
+// W4: the weights are e2m1 (FP4) with 1 x 32 scales.  The TMA unpacks the
+// packed 4-bit rows into the same 128-byte shared-memory rows an e4m3 tile
+// takes (tensor-map type 16U4_ALIGN16B), the MMA reads A as e2m1, the weight
+// scale atoms come ready-made from global memory by a bulk copy, and the k-th
+// 32-wide K step of a block selects scale byte k of the atom's words.
+template <int KIND, bool W4 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mA1,
                             const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mA0s,
@@ -475,8 +548,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint64_t pol = ptx::policy_evict_normal();
             uint32_t armed = 0, armed_ph = 0;
             bool ok = true;
+            // an FP4 weight box counts its packed global bytes (4 bits an element), though
+            // it fills the 128-byte shared-memory rows of an e4m3 box
             auto tx_bytes = [&](const Fp8Tile& tl) {
-                return (tl.gated ? 2u : 1u) * 128u * kFp8BlockK + (uint32_t)tl.n_mma * kFp8BlockK + 512u;
+                return (tl.gated ? 2u : 1u) * (128u * kFp8BlockK / (W4 ? 2u : 1u) + (W4 ? 512u : 0u)) +
+                       (uint32_t)tl.n_mma * kFp8BlockK + 512u;
             };
             // the down tiles of the single launch read the second set of maps and args
             auto down2 = [&](const Fp8Tile& tl) { return KIND == FP8_FUSED && !tl.gated; };
@@ -488,6 +564,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const CUtensorMap* a0 = down2(tl) ? (tl.shared ? &mA2s : &mA2) : (tl.shared ? &mA0s : &mA0);
                 ptx::tma_load_2d(a_dst, a0, full, kc, a_row, pol);
                 if (tl.gated) ptx::tma_load_2d(a_dst + 128 * kFp8BlockK, tl.shared ? &mA1s : &mA1, full, kc, a_row, pol);
+                if (W4) {
+                    // the weight tiles' scale atoms, into the stage's A0 / A1 atom slots
+                    const int64_t atom = ((int64_t)(a_row >> 7) * tl.nkb + kb) * 512;
+                    const uint32_t sf_dst = a_dst + kABytes + b_bytes + 512;
+                    ptx::bulk_load(sf_dst, (tl.shared ? ta.fA0s : ta.fA0) + atom, 512, full);
+                    if (tl.gated) ptx::bulk_load(sf_dst + 512, (tl.shared ? ta.fA1s : ta.fA1) + atom, 512, full);
+                }
             };
             auto issue_b = [&](const Fp8Tile& tl, int kb, uint32_t stage, uint32_t full) {
                 const int kc = kb * kFp8BlockK;
@@ -580,7 +663,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // The weight-block scales of a tile (lane l: K blocks l, l + 32, l + 64, l + 96)
         // are loaded one tile ahead, so their latency hides behind the previous tile.
         auto load_scales = [&](int t, float (&wa)[4], float (&wb)[4]) {
-            if (t < 0) return;
+            if (t < 0 || W4) return;   // FP4 weights: the atoms come with the stage
             const Fp8Tile tl = fp8_decode<KIND>(nb, t, args, args2, splan);
             const Fp8Args& ta = (KIND == FP8_FUSED && !tl.gated) ? args2 : args;
             const int Mrows = tl.shared ? ta.M_shared : ta.M;
@@ -618,7 +701,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!ok) break;
             ptx::tc_fence_after();
             const uint32_t d_g = tmem_base + (uint32_t)acc * kFp8AccCols;
-            const uint32_t idesc = idesc_mxf8_ue8m0(128, (uint32_t)tl.n_mma);
+            // A as e2m1 (format 5, bits 7-9) for FP4 weights
+            const uint32_t idesc = idesc_mxf8_ue8m0(128, (uint32_t)tl.n_mma) | (W4 ? (5u << 7) : 0u);
             const int shift = tl.row0 & 3;
             for (int kb = 0; kb < tl.nkb; kb++) {
                 ok = __all_sync(0xffffffffu, bounded_wait(ptx::smem_u32(&ctl->full[s]), ph, ctl, args.err));
@@ -634,13 +718,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     w[m1] = e * 0x01010101u;
                 }
                 *reinterpret_cast<uint4*>(atoms + 1024 + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
-                const uint32_t a0 = ue8m0_of(__uint_as_float(__shfl_sync(0xffffffffu, pick4(ea, kb >> 5), kb & 31))) *
-                                    0x01010101u;
-                *reinterpret_cast<uint4*>(atoms + 16 * lane) = make_uint4(a0, a0, a0, a0);
-                if (tl.gated) {
-                    const uint32_t a1 =
-                        ue8m0_of(__uint_as_float(__shfl_sync(0xffffffffu, pick4(eb, kb >> 5), kb & 31))) * 0x01010101u;
-                    *reinterpret_cast<uint4*>(atoms + 512 + 16 * lane) = make_uint4(a1, a1, a1, a1);
+                if (!W4) {
+                    const uint32_t a0 =
+                        ue8m0_of(__uint_as_float(__shfl_sync(0xffffffffu, pick4(ea, kb >> 5), kb & 31))) * 0x01010101u;
+                    *reinterpret_cast<uint4*>(atoms + 16 * lane) = make_uint4(a0, a0, a0, a0);
+                    if (tl.gated) {
+                        const uint32_t a1 =
+                            ue8m0_of(__uint_as_float(__shfl_sync(0xffffffffu, pick4(eb, kb >> 5), kb & 31))) *
+                            0x01010101u;
+                        *reinterpret_cast<uint4*>(atoms + 512 + 16 * lane) = make_uint4(a1, a1, a1, a1);
+                    }
                 }
                 ptx::fence_proxy_async_smem();   // the atoms are read by tcgen05.cp (async proxy)
                 __syncwarp();
@@ -653,17 +740,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (tl.gated)
                         ptx::tmem_cp_32x128b_warpx4(tmem_base + kSfColA1, ptx::plain_rows16_desc(atoms_addr + 512));
                     ptx::tmem_cp_32x128b_warpx4(tmem_base + kSfColB, ptx::plain_rows16_desc(atoms_addr + 1024));
+                    // FP4 weights: the kk-th 32-wide K step reads scale byte kk of A's atom (bits 29-30)
 #pragma unroll
                     for (int kk = 0; kk < kFp8BlockK / 32; kk++)
                         mma_mxf8_ss(d_g, ptx::sw128_kmajor_desc(a_addr + kk * 32), ptx::sw128_kmajor_desc(b_addr + kk * 32),
-                                    idesc, tmem_base + kSfColA0, tmem_base + kSfColB, (kb > 0 || kk > 0) ? 1u : 0u);
+                                    idesc | (W4 ? (uint32_t)kk << 29 : 0u), tmem_base + kSfColA0, tmem_base + kSfColB,
+                                    (kb > 0 || kk > 0) ? 1u : 0u);
                     if (tl.gated) {
 #pragma unroll
                         for (int kk = 0; kk < kFp8BlockK / 32; kk++)
                             mma_mxf8_ss(d_g + (uint32_t)kFp8TileRows,
                                         ptx::sw128_kmajor_desc(a_addr + 128 * kFp8BlockK + kk * 32),
-                                        ptx::sw128_kmajor_desc(b_addr + kk * 32), idesc, tmem_base + kSfColA1,
-                                        tmem_base + kSfColB, (kb > 0 || kk > 0) ? 1u : 0u);
+                                        ptx::sw128_kmajor_desc(b_addr + kk * 32), idesc | (W4 ? (uint32_t)kk << 29 : 0u),
+                                        tmem_base + kSfColA1, tmem_base + kSfColB, (kb > 0 || kk > 0) ? 1u : 0u);
                     }
                     ptx::mma_commit(ptx::smem_u32(&ctl->empty[s]));
                 }

@@ -472,135 +472,229 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        // Lane 0 waits on the ring, arms the stages and loads the weight tiles;
-        // routed gate/up tiles of a layer whose rows are gathered (args.gather_perm)
-        // take their token rows straight from x, four rows per TMA gather and lane.
-        const bool lead = lane == 0;
-        const uint64_t pol = ptx::policy_evict_normal();
-        uint32_t armed = 0, armed_ph = 0;   // slots with a load issued (leader's count), and its phase
-        bool ok = true;
-        // MODE_FUSED: all gate/up tiles of the tile's block have stored their h rows
-        auto wait_block_ready = [&](const Tile& tl) -> bool {
-            const int32_t* dep = plan_arrays(const_cast<int32_t*>(args.plan)).dep + tl.blk;
-            const int m1 = tl.shared ? args.M_shared : args.M;
-            // 4 epilogue warps per CTA and gate/up tile (two CTAs per pair tile of 128 f rows)
-            const int need = PAIR ? 8 * splan->units[tl.blk] * ((m1 + 127) / 128)
-                                  : 4 * splan->units[tl.blk] * ((m1 + 63) / 64);
-            if (!bounded_count_wait(dep, need, ctl, args.err)) return false;
-            ptx::fence_proxy_async_global();   // the TMA reads below come after the acquire
-            return true;
-        };
-        // pass 1 (before the dependency wait): weight tiles into the free stages
-        int pre = 0;
-        if (!waited_early) {
-            if (lead) {
+        // One elected lane issues every load; only when the gate/up tokens are
+        // gathered from x does the whole warp take part (each lane gathers rows).
+        if (MODE == MODE_ROUTER || MODE == MODE_DOWN || !args.gather_perm) {
+            if (ptx::elect_one()) {
+                const uint64_t pol = ptx::policy_evict_normal();
+                uint32_t armed = 0, armed_ph = 0;   // slots with a load issued (leader's count), and its phase
+                bool ok = true;
+                // MODE_FUSED: all gate/up tiles of the tile's block have stored their h rows
+                auto wait_block_ready = [&](const Tile& tl) -> bool {
+                    const int32_t* dep = plan_arrays(const_cast<int32_t*>(args.plan)).dep + tl.blk;
+                    const int m1 = tl.shared ? args.M_shared : args.M;
+                    // 4 epilogue warps per CTA and gate/up tile (two CTAs per pair tile of 128 f rows)
+                    const int need = PAIR ? 8 * splan->units[tl.blk] * ((m1 + 127) / 128)
+                                          : 4 * splan->units[tl.blk] * ((m1 + 63) / 64);
+                    if (!bounded_count_wait(dep, need, ctl, args.err)) return false;
+                    ptx::fence_proxy_async_global();   // the TMA reads below come after the acquire
+                    return true;
+                };
+                // pass 1 (before the dependency wait): weight tiles into the free stages
+                int pre = 0;
+                if (!waited_early) {
+                    KIter it;
+                    bool more = kiter_begin<MODE, PAIR>(it, nb, total, args, args2, splan, rank);
+                    while (more && pre < stages) {
+                        const uint32_t full = leader_bar(&ctl->full[pre]);
+                        if (leader) {
+                            ptx::mbar_arrive_expect_tx(ptx::smem_u32(&ctl->full[pre]), stage_tx(it.tl));
+                            armed |= 1u << pre;
+                        }
+                        issue_a<MODE, PAIR>(it, ring + (uint32_t)pre * stage_bytes, full, &mA0, &mA1, &mA0s, &mA1s, &mA2,
+                                            &mA2s, args, args2, pol);
+                        ++pre;
+                        more = kiter_next<MODE, PAIR>(it, nb, total, args, args2, splan, rank);
+                    }
+                    ptx::grid_dep_wait();
+                }
+                // After the wait, never before it: the layer's later kernels read data
+                // written two launches back (the combine reads inv_perm before its own
+                // wait), which holds only if every kernel waits before it triggers.
+                ptx::grid_dep_launch();
+                // pass 2: the same sequence again; the first `pre` stages only need their token tiles
+                int s = 0, n = 0;
+                uint32_t ph = 0;
                 KIter it;
                 bool more = kiter_begin<MODE, PAIR>(it, nb, total, args, args2, splan, rank);
-                while (more && pre < stages) {
-                    const uint32_t full = leader_bar(&ctl->full[pre]);
-                    if (leader) {
-                        ptx::mbar_arrive_expect_tx(ptx::smem_u32(&ctl->full[pre]), stage_tx(it.tl));
-                        armed |= 1u << pre;
+                while (more) {
+                    const uint32_t a_dst = ring + (uint32_t)s * stage_bytes;
+                    const uint32_t full = leader_bar(&ctl->full[s]);
+                    const bool first = it.tl.gated || MODE != MODE_FUSED;
+                    const CUtensorMap* b = first ? (it.tl.shared ? &mBs : &mB) : (it.tl.shared ? &mB2s : &mB2);
+                    const CUtensorMap* b64 = first ? (it.tl.shared ? &mBs64 : &mB64) : (it.tl.shared ? &mB2s64 : &mB264);
+                    // a down tile of the fused launch reads h only after its block's gate/up tiles stored it
+                    if (MODE == MODE_FUSED && !it.tl.gated && it.kb == 0 && !wait_block_ready(it.tl)) {
+                        ok = false;
+                        break;
                     }
-                    issue_a<MODE, PAIR>(it, ring + (uint32_t)pre * stage_bytes, full, &mA0, &mA1, &mA0s, &mA1s, &mA2,
-                                        &mA2s, args, args2, pol);
-                    ++pre;
-                    more = kiter_next<MODE, PAIR>(it, nb, total, args, args2, splan, rank);
-                }
-            }
-            pre = __shfl_sync(0xffffffffu, pre, 0);
-            ptx::grid_dep_wait();
-        }
-        // After the wait, never before it: the layer's later kernels read data
-        // written two launches back (the combine reads inv_perm before its own
-        // wait), which holds only if every kernel waits before it triggers.
-        if (lead) ptx::grid_dep_launch();
-        // pass 2: the same sequence again; the first `pre` stages only need their token tiles
-        int s = 0, n = 0;
-        uint32_t ph = 0;
-        int tok[8];          // gathered tiles: the tokens of this lane's rows 4q..4q+3, q = lane, lane + 32
-        KIter it;
-        bool more = kiter_begin<MODE, PAIR>(it, nb, total, args, args2, splan, rank);
-        while (more) {
-            const uint32_t a_dst = ring + (uint32_t)s * stage_bytes;
-            const uint32_t full = leader_bar(&ctl->full[s]);
-            const bool first = it.tl.gated || MODE != MODE_FUSED;
-            const bool gather = MODE != MODE_ROUTER && args.gather_perm && it.tl.gated && !it.tl.shared;
-            if (gather && it.kb == it.tl.kb0) {
-                // rows past the tile's tokens (MMA padding) repeat its last token
-                const int last = it.tl.row0 + it.tl.rows - 1;
-#pragma unroll
-                for (int j = 0; j < 8; j++) {
-                    const int r = 4 * (lane + 32 * (j >> 2)) + (j & 3);
-                    const int pos = min(it.tl.b_row0 + r, last);
-                    tok[j] = r < it.tl.b_n ? __ldg(args.gather_perm + pos) / args.gather_k : 0;
-                }
-            }
-            // a down tile of the fused launch reads h only after its block's gate/up tiles stored it
-            if (MODE == MODE_FUSED && !it.tl.gated && it.kb == 0) {
-                if (lead) ok = wait_block_ready(it.tl);
-                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
-                    ok = false;
-                    break;
-                }
-            }
-            if (n >= pre) {
-                if (lead) {
-                    ok = bounded_wait(ptx::smem_u32(&ctl->empty[s]), ph ^ 1u, ctl, args.err);
-                    if (ok) {
+                    if (n < pre) {
+                        issue_b<PAIR>(it.tl, it.kb, a_dst + kATileBytes, full, b, b64, pol);
+                    } else {
+                        if (!bounded_wait(ptx::smem_u32(&ctl->empty[s]), ph ^ 1u, ctl, args.err)) {
+                            ok = false;
+                            break;
+                        }
                         if (leader) {
                             ptx::mbar_arrive_expect_tx(ptx::smem_u32(&ctl->full[s]), stage_tx(it.tl));
                             armed |= 1u << s;
                             armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
                         }
-                        issue_a<MODE, PAIR>(it, a_dst, full, &mA0, &mA1, &mA0s, &mA1s, &mA2, &mA2s, args, args2,
-                                            pol);
+                        issue_a<MODE, PAIR>(it, a_dst, full, &mA0, &mA1, &mA0s, &mA1s, &mA2, &mA2s, args, args2, pol);
+                        issue_b<PAIR>(it.tl, it.kb, a_dst + kATileBytes, full, b, b64, pol);
+                    }
+                    ++n;
+                    if (++s == stages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                    more = kiter_next<MODE, PAIR>(it, nb, total, args, args2, splan, rank);
+                }
+                if (!ok) {
+                    // drain: wait (bounded) for every stage the leader armed; a pair's
+                    // loads from both CTAs complete on the leader's barriers, and the
+                    // peer does not leave before the leader (cluster barrier below)
+                    const uint64_t t0 = ptx::globaltimer();
+                    for (int i = 0; i < stages; i++) {
+                        if (!(armed >> i & 1u)) continue;
+                        const uint32_t bar = ptx::smem_u32(&ctl->full[i]);
+                        while (!ptx::mbar_try_wait(bar, (armed_ph >> i) & 1u) &&
+                               ptx::globaltimer() - t0 < kWaitTimeoutNs) {
+                        }
                     }
                 }
-                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
-                    ok = false;
-                    break;
-                }
             }
-            if (gather) {
-                const int kc = it.kb * kBlockK;
-                const uint32_t b_dst = a_dst + kATileBytes;
-#pragma unroll
-                for (int h = 0; h < 2; h++) {
-                    const int q = lane + 32 * h;
-                    if (4 * q < it.tl.b_n) {
-                        if (PAIR)
-                            ptx::tma_gather4_pair(b_dst + 512u * q, &mBx, full, kc, tok[4 * h], tok[4 * h + 1],
-                                                  tok[4 * h + 2], tok[4 * h + 3], pol);
-                        else
-                            ptx::tma_gather4(b_dst + 512u * q, &mBx, full, kc, tok[4 * h], tok[4 * h + 1],
-                                             tok[4 * h + 2], tok[4 * h + 3], pol);
+        } else {
+            // Row gathers (args.gather_perm): lane 0 waits on the ring, arms the stages
+            // and loads the weight tiles; routed gate/up tiles take their token rows
+            // straight from x, four rows per TMA gather and lane.
+            const bool lead = lane == 0;
+            const uint64_t pol = ptx::policy_evict_normal();
+            uint32_t armed = 0, armed_ph = 0;   // slots with a load issued (leader's count), and its phase
+            bool ok = true;
+            // MODE_FUSED: all gate/up tiles of the tile's block have stored their h rows
+            auto wait_block_ready = [&](const Tile& tl) -> bool {
+                const int32_t* dep = plan_arrays(const_cast<int32_t*>(args.plan)).dep + tl.blk;
+                const int m1 = tl.shared ? args.M_shared : args.M;
+                // 4 epilogue warps per CTA and gate/up tile (two CTAs per pair tile of 128 f rows)
+                const int need = PAIR ? 8 * splan->units[tl.blk] * ((m1 + 127) / 128)
+                                      : 4 * splan->units[tl.blk] * ((m1 + 63) / 64);
+                if (!bounded_count_wait(dep, need, ctl, args.err)) return false;
+                ptx::fence_proxy_async_global();   // the TMA reads below come after the acquire
+                return true;
+            };
+            // pass 1 (before the dependency wait): weight tiles into the free stages
+            int pre = 0;
+            if (!waited_early) {
+                if (lead) {
+                    KIter it;
+                    bool more = kiter_begin<MODE, PAIR>(it, nb, total, args, args2, splan, rank);
+                    while (more && pre < stages) {
+                        const uint32_t full = leader_bar(&ctl->full[pre]);
+                        if (leader) {
+                            ptx::mbar_arrive_expect_tx(ptx::smem_u32(&ctl->full[pre]), stage_tx(it.tl));
+                            armed |= 1u << pre;
+                        }
+                        issue_a<MODE, PAIR>(it, ring + (uint32_t)pre * stage_bytes, full, &mA0, &mA1, &mA0s, &mA1s, &mA2,
+                                            &mA2s, args, args2, pol);
+                        ++pre;
+                        more = kiter_next<MODE, PAIR>(it, nb, total, args, args2, splan, rank);
                     }
                 }
-            } else if (lead) {
-                const CUtensorMap* b = first ? (it.tl.shared ? &mBs : &mB) : (it.tl.shared ? &mB2s : &mB2);
-                const CUtensorMap* b64 =
-                    first ? (it.tl.shared ? &mBs64 : &mB64) : (it.tl.shared ? &mB2s64 : &mB264);
-                issue_b<PAIR>(it.tl, it.kb, a_dst + kATileBytes, full, b, b64, pol);
+                pre = __shfl_sync(0xffffffffu, pre, 0);
+                ptx::grid_dep_wait();
             }
-            __syncwarp();
-            ++n;
-            if (++s == stages) {
-                s = 0;
-                ph ^= 1u;
+            // After the wait, never before it: the layer's later kernels read data
+            // written two launches back (the combine reads inv_perm before its own
+            // wait), which holds only if every kernel waits before it triggers.
+            if (lead) ptx::grid_dep_launch();
+            // pass 2: the same sequence again; the first `pre` stages only need their token tiles
+            int s = 0, n = 0;
+            uint32_t ph = 0;
+            int tok[8];          // gathered tiles: the tokens of this lane's rows 4q..4q+3, q = lane, lane + 32
+            KIter it;
+            bool more = kiter_begin<MODE, PAIR>(it, nb, total, args, args2, splan, rank);
+            while (more) {
+                const uint32_t a_dst = ring + (uint32_t)s * stage_bytes;
+                const uint32_t full = leader_bar(&ctl->full[s]);
+                const bool first = it.tl.gated || MODE != MODE_FUSED;
+                const bool gather = MODE != MODE_ROUTER && args.gather_perm && it.tl.gated && !it.tl.shared;
+                if (gather && it.kb == it.tl.kb0) {
+                    // rows past the tile's tokens (MMA padding) repeat its last token
+                    const int last = it.tl.row0 + it.tl.rows - 1;
+    #pragma unroll
+                    for (int j = 0; j < 8; j++) {
+                        const int r = 4 * (lane + 32 * (j >> 2)) + (j & 3);
+                        const int pos = min(it.tl.b_row0 + r, last);
+                        tok[j] = r < it.tl.b_n ? __ldg(args.gather_perm + pos) / args.gather_k : 0;
+                    }
+                }
+                // a down tile of the fused launch reads h only after its block's gate/up tiles stored it
+                if (MODE == MODE_FUSED && !it.tl.gated && it.kb == 0) {
+                    if (lead) ok = wait_block_ready(it.tl);
+                    if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (n >= pre) {
+                    if (lead) {
+                        ok = bounded_wait(ptx::smem_u32(&ctl->empty[s]), ph ^ 1u, ctl, args.err);
+                        if (ok) {
+                            if (leader) {
+                                ptx::mbar_arrive_expect_tx(ptx::smem_u32(&ctl->full[s]), stage_tx(it.tl));
+                                armed |= 1u << s;
+                                armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
+                            }
+                            issue_a<MODE, PAIR>(it, a_dst, full, &mA0, &mA1, &mA0s, &mA1s, &mA2, &mA2s, args, args2,
+                                                pol);
+                        }
+                    }
+                    if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (gather) {
+                    const int kc = it.kb * kBlockK;
+                    const uint32_t b_dst = a_dst + kATileBytes;
+    #pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        const int q = lane + 32 * h;
+                        if (4 * q < it.tl.b_n) {
+                            if (PAIR)
+                                ptx::tma_gather4_pair(b_dst + 512u * q, &mBx, full, kc, tok[4 * h], tok[4 * h + 1],
+                                                      tok[4 * h + 2], tok[4 * h + 3], pol);
+                            else
+                                ptx::tma_gather4(b_dst + 512u * q, &mBx, full, kc, tok[4 * h], tok[4 * h + 1],
+                                                 tok[4 * h + 2], tok[4 * h + 3], pol);
+                        }
+                    }
+                } else if (lead) {
+                    const CUtensorMap* b = first ? (it.tl.shared ? &mBs : &mB) : (it.tl.shared ? &mB2s : &mB2);
+                    const CUtensorMap* b64 =
+                        first ? (it.tl.shared ? &mBs64 : &mB64) : (it.tl.shared ? &mB2s64 : &mB264);
+                    issue_b<PAIR>(it.tl, it.kb, a_dst + kATileBytes, full, b, b64, pol);
+                }
+                __syncwarp();
+                ++n;
+                if (++s == stages) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+                more = kiter_next<MODE, PAIR>(it, nb, total, args, args2, splan, rank);
             }
-            more = kiter_next<MODE, PAIR>(it, nb, total, args, args2, splan, rank);
-        }
-        if (!ok && lead) {
-            // drain: wait (bounded) for every stage the leader armed; a pair's
-            // loads from both CTAs complete on the leader's barriers, and the
-            // peer does not leave before the leader (cluster barrier below)
-            const uint64_t t0 = ptx::globaltimer();
-            for (int i = 0; i < stages; i++) {
-                if (!(armed >> i & 1u)) continue;
-                const uint32_t bar = ptx::smem_u32(&ctl->full[i]);
-                while (!ptx::mbar_try_wait(bar, (armed_ph >> i) & 1u) &&
-                       ptx::globaltimer() - t0 < kWaitTimeoutNs) {
+            if (!ok && lead) {
+                // drain: wait (bounded) for every stage the leader armed; a pair's
+                // loads from both CTAs complete on the leader's barriers, and the
+                // peer does not leave before the leader (cluster barrier below)
+                const uint64_t t0 = ptx::globaltimer();
+                for (int i = 0; i < stages; i++) {
+                    if (!(armed >> i & 1u)) continue;
+                    const uint32_t bar = ptx::smem_u32(&ctl->full[i]);
+                    while (!ptx::mbar_try_wait(bar, (armed_ph >> i) & 1u) &&
+                           ptx::globaltimer() - t0 < kWaitTimeoutNs) {
+                    }
                 }
             }
         }

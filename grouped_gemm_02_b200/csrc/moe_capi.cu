@@ -150,6 +150,12 @@ int device_setup(DeviceState** out)
                                      kFp8SmemBytes) != cudaSuccess ||
                 cudaFuncSetAttribute(grouped_gemm_fp8_kernel<FP8_FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kFp8SmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(grouped_gemm_fp8_kernel<FP8_GATED, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kFp8SmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(grouped_gemm_fp8_kernel<FP8_DOWN, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kFp8SmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(grouped_gemm_fp8_kernel<FP8_FUSED, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kFp8SmemBytes) != cudaSuccess ||
                 cudaFuncSetAttribute(grouped_gemm_kernel<MODE_GATED, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) != cudaSuccess ||
                 cudaFuncSetAttribute(grouped_gemm_kernel<MODE_DOWN, true>,
@@ -218,6 +224,22 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows
     cuuint32_t box[2] = {128, box_rows};
     cuuint32_t estr[2] = {1, 1};
     return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over packed e2m1 (FP4) rows [rows, inner elements], inner / 2 bytes a
+// row; box = [128 elements, box_rows].  The TMA unpacks each 16 elements (8
+// bytes) into 16 bytes of shared memory, the row layout an e4m3 tile takes, for
+// the block-scaled MMA to read as e2m1.
+bool make_map_u4(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows)
+{
+    if (rows == 0) rows = 1;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner / 2};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -876,7 +898,16 @@ struct Fp8Operands {
     bf16 *y_p, *ys;
     int T, P, d, f, fs, E;
     int64_t ld_pairs, ld_tokens;
+    // FP4 weights: the W*q are packed e2m1 and these their 1 x 32 scale atoms
+    bool w4;
+    const uint8_t *f1, *f3, *f2, *fs1, *fs3, *fs2;
 };
+
+// An A-operand (weight) map: e4m3 bytes, or packed e2m1 unpacked by the TMA.
+bool make_map_w(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, bool w4)
+{
+    return w4 ? make_map_u4(m, base, inner, rows, 128) : make_map_u8(m, base, inner, rows, 128);
+}
 
 int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int sms, cudaStream_t st, bool prof)
 {
@@ -888,17 +919,17 @@ int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int 
     CUtensorMap b64, bs64, b264, b2s64;
     const uint64_t E = (uint64_t)o.E;
     const uint64_t lp = (uint64_t)o.ld_pairs, lt = (uint64_t)o.ld_tokens;
-    if (!make_map_u8(&a0, o.W1q, o.d, E * o.f, 128) || !make_map_u8(&a1, o.W3q, o.d, E * o.f, 128) ||
+    if (!make_map_w(&a0, o.W1q, o.d, E * o.f, o.w4) || !make_map_w(&a1, o.W3q, o.d, E * o.f, o.w4) ||
         !make_map_u8(&b, o.xp8, o.d, (uint64_t)o.P, 16) || !make_map_f32(&sb, o.sxp, lp, o.d / 128) ||
         !make_map_u8(&b64, o.xp8, o.d, (uint64_t)o.P, 64) || !make_map_u8(&b264, o.h8, o.f, (uint64_t)o.P, 64) ||
-        !make_map_u8(&a2, o.W2q, o.f, E * o.d, 128) || !make_map_u8(&b2, o.h8, o.f, (uint64_t)o.P, 16) ||
+        !make_map_w(&a2, o.W2q, o.f, E * o.d, o.w4) || !make_map_u8(&b2, o.h8, o.f, (uint64_t)o.P, 16) ||
         !make_map_f32(&sb2, o.sh, lp, o.f / 128))
         return MOE_ERR_CUDA;
     if (o.fs > 0) {
-        if (!make_map_u8(&a0s, o.Ws1q, o.d, o.fs, 128) || !make_map_u8(&a1s, o.Ws3q, o.d, o.fs, 128) ||
+        if (!make_map_w(&a0s, o.Ws1q, o.d, o.fs, o.w4) || !make_map_w(&a1s, o.Ws3q, o.d, o.fs, o.w4) ||
             !make_map_u8(&bs, o.x8, o.d, (uint64_t)o.T, 16) || !make_map_f32(&sbs, o.sxT, lt, o.d / 128) ||
             !make_map_u8(&bs64, o.x8, o.d, (uint64_t)o.T, 64) || !make_map_u8(&b2s64, o.hs8, o.fs, (uint64_t)o.T, 64) ||
-            !make_map_u8(&a2s, o.Ws2q, o.fs, o.d, 128) || !make_map_u8(&b2s, o.hs8, o.fs, (uint64_t)o.T, 16) ||
+            !make_map_w(&a2s, o.Ws2q, o.fs, o.d, o.w4) || !make_map_u8(&b2s, o.hs8, o.fs, (uint64_t)o.T, 16) ||
             !make_map_f32(&sb2s, o.shs, lt, o.fs / 128))
             return MOE_ERR_CUDA;
     } else {
@@ -933,6 +964,10 @@ int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int 
     g1.perm = o.perm;
     g1.gate_w = o.gate_w;
     g1.err = err;
+    g1.fA0 = o.f1;
+    g1.fA1 = o.f3;
+    g1.fA0s = o.fs1;
+    g1.fA1s = o.fs3;
     Fp8Args g2 = g1;
     g2.M = o.d;
     g2.M_shared = o.d;
@@ -942,25 +977,31 @@ int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int 
     g2.sA1 = nullptr;
     g2.sA0s = o.ss2;
     g2.sA1s = nullptr;
+    g2.fA0 = o.f2;
+    g2.fA1 = nullptr;
+    g2.fA0s = o.fs2;
+    g2.fA1s = nullptr;
     g2.out = o.y_p;
     g2.out_shared = o.ys;
+    // the kernel instances of the weight format
+    auto k_fused = o.w4 ? grouped_gemm_fp8_kernel<FP8_FUSED, true> : grouped_gemm_fp8_kernel<FP8_FUSED>;
+    auto k_gated = o.w4 ? grouped_gemm_fp8_kernel<FP8_GATED, true> : grouped_gemm_fp8_kernel<FP8_GATED>;
+    auto k_down = o.w4 ? grouped_gemm_fp8_kernel<FP8_DOWN, true> : grouped_gemm_fp8_kernel<FP8_DOWN>;
     if (gemm_fused(o.P, o.f)) {
         // one launch: a gate/up tile streams d/128 k-blocks, a down tile f/128
         const int kb1 = o.d / 128, kb2 = o.f / 128;
         g1.comp = std::max(1, (kb1 + kb2 / 2) / kb2);
-        const cudaError_t e = launch(grouped_gemm_fp8_kernel<FP8_FUSED>, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes,
-                                     st, a0, a1, b, a0s, a1s, bs, sb, sbs, a2, b2, a2s, b2s, sb2, sb2s, b64, bs64, b264,
-                                     b2s64, g1, g2);
+        const cudaError_t e = launch(k_fused, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a0, a1, b, a0s, a1s,
+                                     bs, sb, sbs, a2, b2, a2s, b2s, sb2, sb2s, b64, bs64, b264, b2s64, g1, g2);
         phase_mark(prof, 3, st);   // the single launch has no boundary: the down phase reads as zero
         return status_of(e);
     }
-    if (launch(grouped_gemm_fp8_kernel<FP8_GATED>, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a0, a1, b, a0s,
-               a1s, bs, sb, sbs, a2, b2, a2s, b2s, sb2, sb2s, b64, bs64, b264, b2s64, g1, g1) != cudaSuccess)
+    if (launch(k_gated, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a0, a1, b, a0s, a1s, bs, sb, sbs, a2, b2,
+               a2s, b2s, sb2, sb2s, b64, bs64, b264, b2s64, g1, g1) != cudaSuccess)
         return MOE_ERR_CUDA;
     phase_mark(prof, 3, st);
-    return status_of(launch(grouped_gemm_fp8_kernel<FP8_DOWN>, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a2,
-                            a2, b2, a2s, a2s, b2s, sb2, sb2s, a2, b2, a2s, b2s, sb2, sb2s, b264, b2s64, b264, b2s64,
-                            g2, g2));
+    return status_of(launch(k_down, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a2, a2, b2, a2s, a2s, b2s, sb2,
+                            sb2s, a2, b2, a2s, b2s, sb2, sb2s, b264, b2s64, b264, b2s64, g2, g2));
 }
 
 }  // namespace
@@ -1017,11 +1058,16 @@ int moe_workspace_tensor_fp8(void* ws, int64_t T, int64_t d, int64_t f, int64_t 
     return MOE_OK;
 }
 
-int moe_layer_forward_fp8(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const uint8_t* W1q,
-                          const float* W1s, const uint8_t* W3q, const float* W3s, const uint8_t* W2q, const float* W2s,
-                          const uint8_t* Ws1q, const float* Ws1s, const uint8_t* Ws3q, const float* Ws3s,
-                          const uint8_t* Ws2q, const float* Ws2s, int64_t f_shared, int64_t T, int64_t d, int64_t f,
-                          int64_t E, int64_t k, moe_bf16* out, void* ws, size_t ws_bytes, void* stream)
+// The FP8 layer and the FP4-weight layer share everything but the weights'
+// format: e4m3 with fp32 128 x 128 block scales (W*s), or packed e2m1 with 1 x 32
+// scale atoms (W*f, w4).
+static int layer_forward_lowp(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const uint8_t* W1q,
+                              const float* W1s, const uint8_t* W3q, const float* W3s, const uint8_t* W2q,
+                              const float* W2s, const uint8_t* Ws1q, const float* Ws1s, const uint8_t* Ws3q,
+                              const float* Ws3s, const uint8_t* Ws2q, const float* Ws2s, int64_t f_shared, int64_t T,
+                              int64_t d, int64_t f, int64_t E, int64_t k, moe_bf16* out, void* ws, size_t ws_bytes,
+                              void* stream, bool w4, const uint8_t* W1f, const uint8_t* W3f, const uint8_t* W2f,
+                              const uint8_t* Ws1f, const uint8_t* Ws3f, const uint8_t* Ws2f)
 {
     int rc = check_sizes(T, d, E, k);
     if (rc) return rc;
@@ -1029,8 +1075,12 @@ int moe_layer_forward_fp8(const moe_bf16* x, const moe_bf16* Wg, const float* bi
     if (d % 128 != 0 || f % 128 != 0 || f_shared % 128 != 0) return MOE_ERR_ALIGN;
     if (d > kFp8MaxK || f > kFp8MaxK || f_shared > kFp8MaxK) return MOE_ERR_ARG;
     if (T == 0) return MOE_OK;
-    if (!x || !Wg || !W1q || !W1s || !W3q || !W3s || !W2q || !W2s || !out || !ws) return MOE_ERR_ARG;
-    if (f_shared > 0 && (!Ws1q || !Ws1s || !Ws3q || !Ws3s || !Ws2q || !Ws2s)) return MOE_ERR_ARG;
+    const bool scales_ok = w4 ? (W1f && W3f && W2f) : (W1s && W3s && W2s);
+    const bool shared_scales_ok = w4 ? (Ws1f && Ws3f && Ws2f) : (Ws1s && Ws3s && Ws2s);
+    if (!x || !Wg || !W1q || !W3q || !W2q || !scales_ok || !out || !ws) return MOE_ERR_ARG;
+    if (f_shared > 0 && (!Ws1q || !Ws3q || !Ws2q || !shared_scales_ok)) return MOE_ERR_ARG;
+    if (w4 && !(al16(W1f) && al16(W3f) && al16(W2f) && (f_shared == 0 || (al16(Ws1f) && al16(Ws3f) && al16(Ws2f)))))
+        return MOE_ERR_ALIGN;
     if (!al16(x) || !al16(Wg) || !al16(W1q) || !al16(W3q) || !al16(W2q) || !al16(out) || !al16(ws))
         return MOE_ERR_ALIGN;
     if (f_shared > 0 && (!al16(Ws1q) || !al16(Ws3q) || !al16(Ws2q))) return MOE_ERR_ALIGN;
@@ -1104,6 +1154,13 @@ int moe_layer_forward_fp8(const moe_bf16* x, const moe_bf16* Wg, const float* bi
     o.ss1 = Ws1s;
     o.ss3 = Ws3s;
     o.ss2 = Ws2s;
+    o.w4 = w4;
+    o.f1 = W1f;
+    o.f3 = W3f;
+    o.f2 = W2f;
+    o.fs1 = Ws1f;
+    o.fs3 = Ws3f;
+    o.fs2 = Ws2f;
     o.perm = perm;
     o.gate_w = w;
     o.h8 = at<uint8_t>(ws, L.h8);
@@ -1124,6 +1181,45 @@ int moe_layer_forward_fp8(const moe_bf16* x, const moe_bf16* Wg, const float* bi
     rc = run_combine(y_p, inv_perm, o.ys, iT, ik, id, reinterpret_cast<bf16*>(out), st, inv_perm_launch);
     phase_mark(prof, 5, st);
     return rc;
+}
+
+int moe_layer_forward_fp8(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const uint8_t* W1q,
+                          const float* W1s, const uint8_t* W3q, const float* W3s, const uint8_t* W2q, const float* W2s,
+                          const uint8_t* Ws1q, const float* Ws1s, const uint8_t* Ws3q, const float* Ws3s,
+                          const uint8_t* Ws2q, const float* Ws2s, int64_t f_shared, int64_t T, int64_t d, int64_t f,
+                          int64_t E, int64_t k, moe_bf16* out, void* ws, size_t ws_bytes, void* stream)
+{
+    return layer_forward_lowp(x, Wg, bias, W1q, W1s, W3q, W3s, W2q, W2s, Ws1q, Ws1s, Ws3q, Ws3s, Ws2q, Ws2s, f_shared,
+                              T, d, f, E, k, out, ws, ws_bytes, stream, false, nullptr, nullptr, nullptr, nullptr,
+                              nullptr, nullptr);
+}
+
+int moe_layer_forward_fp4(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const uint8_t* W1q,
+                          const uint8_t* W1sf, const uint8_t* W3q, const uint8_t* W3sf, const uint8_t* W2q,
+                          const uint8_t* W2sf, const uint8_t* Ws1q, const uint8_t* Ws1sf, const uint8_t* Ws3q,
+                          const uint8_t* Ws3sf, const uint8_t* Ws2q, const uint8_t* Ws2sf, int64_t f_shared, int64_t T,
+                          int64_t d, int64_t f, int64_t E, int64_t k, moe_bf16* out, void* ws, size_t ws_bytes,
+                          void* stream)
+{
+    return layer_forward_lowp(x, Wg, bias, W1q, nullptr, W3q, nullptr, W2q, nullptr, Ws1q, nullptr, Ws3q, nullptr,
+                              Ws2q, nullptr, f_shared, T, d, f, E, k, out, ws, ws_bytes, stream, true, W1sf, W3sf, W2sf,
+                              Ws1sf, Ws3sf, Ws2sf);
+}
+
+int moe_quantize_fp4_rows(const moe_bf16* W, int64_t rows, int64_t cols, uint8_t* q, uint8_t* scale_atoms,
+                          void* stream)
+{
+    if (rows < 0 || cols <= 0 || cols > (int64_t(1) << 30)) return MOE_ERR_ARG;
+    if (rows % 128 != 0 || cols % 128 != 0) return MOE_ERR_ALIGN;
+    if (rows == 0) return MOE_OK;
+    if (!W || !q || !scale_atoms) return MOE_ERR_ARG;
+    if (!al16(W) || !al16(q) || !al16(scale_atoms)) return MOE_ERR_ALIGN;
+    DeviceState* dev;
+    int rc;
+    if ((rc = device_setup(&dev))) return rc;
+    const int64_t warps = rows * (cols / 128);
+    return status_of(launch(quantize_rows_fp4_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0,
+                            as_stream(stream), reinterpret_cast<const bf16*>(W), rows, (int)cols, q, scale_atoms));
 }
 
 }  // extern "C"

@@ -29,7 +29,7 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_topk", 
            "moe_record_phase_events", "moe_launch_counter", "moe_get_device_error", "moe_clear_device_error",
            "moe_selftest_wait_timeout",
            "moe_status_string", "moe_set_policy", "moe_quantize_fp8_rows", "moe_quantize_fp8_blocks", "moe_workspace_size_fp8",
-           "moe_workspace_tensor_fp8", "moe_layer_forward_fp8")
+           "moe_workspace_tensor_fp8", "moe_layer_forward_fp8", "moe_quantize_fp4_rows", "moe_layer_forward_fp4")
 
 
 class MoEError(RuntimeError):
@@ -73,6 +73,9 @@ def lib() -> C.CDLL:
             "moe_workspace_size_fp8": [i64, i64, i64, i64, i64, i64, C.POINTER(sz)],
             "moe_workspace_tensor_fp8": [vp, i64, i64, i64, i64, i64, i64, C.c_int, C.POINTER(vp)],
             "moe_layer_forward_fp8": [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
+                                      i64, i64, vp, vp, sz, vp],
+            "moe_quantize_fp4_rows": [vp, i64, i64, vp, vp, vp],
+            "moe_layer_forward_fp4": [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
                                       i64, i64, vp, vp, sz, vp],
         }
         for name, args in sig.items():
@@ -337,6 +340,43 @@ def moe_layer_forward_fp8(x, Wg, bias, Q: dict, k: int, ws: torch.Tensor, out=No
     g = lambda n: _p(Q.get(n))
     _call("moe_layer_forward_fp8", _p(x), _p(Wg), _p(bias), g("W1q"), g("W1s"), g("W3q"), g("W3s"), g("W2q"),
           g("W2s"), g("Ws1q"), g("Ws1s"), g("Ws3q"), g("Ws3s"), g("Ws2q"), g("Ws2s"), fs, T, d, f, E, k, _p(out),
+          _p(ws), ws.numel(), _stream(stream))
+    return out
+
+
+# ---------------------------------------------------------------- FP4 weights
+
+def moe_quantize_fp4_rows(W: torch.Tensor, stream=None):
+    """1 x 32 blocks along rows: bf16 [R, C] (or [E, R', C], taken as [E*R', C]) -> (packed e2m1
+    codes uint8 [..., C/2], UE8M0 scale atoms uint8 [R/128, C/128, 512])."""
+    W2d = W.reshape(-1, W.shape[-1])
+    _bf16(W2d)
+    R, Cc = W2d.shape
+    q = torch.empty(*W.shape[:-1], Cc // 2, dtype=torch.uint8, device=W.device)
+    atoms = torch.empty(R // 128, Cc // 128, 512, dtype=torch.uint8, device=W.device)
+    _call("moe_quantize_fp4_rows", _p(W2d), R, Cc, _p(q), _p(atoms), _stream(stream))
+    return q, atoms
+
+
+def quantize_layer_fp4(w: dict, stream=None) -> dict:
+    """The expert weights of a layer (W1, W3, W2 and optionally Ws1, Ws3, Ws2) as packed e2m1 with scale atoms."""
+    out = {}
+    for n in ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2"):
+        if w.get(n) is not None:
+            out[n + "q"], out[n + "sf"] = moe_quantize_fp4_rows(w[n], stream)
+    return out
+
+
+def moe_layer_forward_fp4(x, Wg, bias, Q: dict, k: int, ws: torch.Tensor, out=None, stream=None):
+    """FP4-weight layer; Q holds W1q/W1sf, W3q/W3sf, W2q/W2sf (and Ws1q/Ws1sf, ... for the shared expert)."""
+    T, d = x.shape
+    E, f, _ = Q["W1q"].shape
+    fs = 0 if Q.get("Ws1q") is None else Q["Ws1q"].shape[0]
+    _bf16(x), _bf16(Wg, (E, d))
+    out = torch.empty(T, d, dtype=torch.bfloat16, device=x.device) if out is None else out
+    g = lambda n: _p(Q.get(n))
+    _call("moe_layer_forward_fp4", _p(x), _p(Wg), _p(bias), g("W1q"), g("W1sf"), g("W3q"), g("W3sf"), g("W2q"),
+          g("W2sf"), g("Ws1q"), g("Ws1sf"), g("Ws3q"), g("Ws3sf"), g("Ws2q"), g("Ws2sf"), fs, T, d, f, E, k, _p(out),
           _p(ws), ws.numel(), _stream(stream))
     return out
 

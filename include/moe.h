@@ -225,6 +225,43 @@ MOE_API int moe_layer_forward_fp8(const moe_bf16 *x, const moe_bf16 *Wg, const f
                                   int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, moe_bf16 *out, void *ws,
                                   size_t ws_bytes, void *stream);
 
+/* ---------------------------------------------------------------- FP4 weights
+ * FP4 expert weights (GC-MoE, abstract: an FP8/FP4 MoE operator with
+ * block-scaled MMA).  Weights are OCP e2m1 codes (sign, 2 exponent bits with
+ * bias 1, 1 mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) in blocks of
+ * 32 consecutive elements along each row (MXFP4): a block's scale is the
+ * smallest power of two s with max|v| / s <= 6 (s = 1 for an all-zero block),
+ * held to the UE8M0 range; codes round to nearest, ties to even, saturating at
+ * 6.  Activations stay e4m3 with 1 x 128 scales, as in the FP8 path. */
+
+/* W [rows, cols] bf16 -> q [rows, cols/2] bytes of packed e2m1 codes (element
+ * 2i in the low nibble of byte i) and scale_atoms [rows/128][cols/128][512]
+ * bytes: the UE8M0 exponent byte (e + 127 for scale 2^e) of row r's 32-wide
+ * block j of each 128 x 128 tile at byte 16 (r % 32) + 4 (r / 32) + j of that
+ * tile's 512 bytes (the layout the block-scaled MMA reads).  Expert weights are
+ * quantised as one matrix: W1/W3 as [E*f, d], W2 as [E*d, f].  rows and cols
+ * multiples of 128 (MOE_ERR_ALIGN otherwise); q and scale_atoms 16-byte
+ * aligned. */
+MOE_API int moe_quantize_fp4_rows(const moe_bf16 *W, int64_t rows, int64_t cols, uint8_t *q, uint8_t *scale_atoms,
+                                  void *stream);
+
+/* The whole layer with FP4 expert weights (packed e2m1 W1q/W3q [E, f, d/2],
+ * W2q [E, d, f/2] with the scale atoms moe_quantize_fp4_rows writes, and the
+ * shared expert's likewise, or all NULL and f_shared = 0):
+ *   h   = silu(x^ W1^T) * (x^ W3^T), requantised to e4m3 in 1 x 128 blocks
+ *   y_p = gate * (h^ W2^T)   (bf16), then the combine of moe_combine,
+ * where ^ marks dequantised values and every product accumulates in fp32 (the
+ * tensor cores apply both operands' power-of-two block scales inside the MMA,
+ * kind::mxf8f6f4 with e2m1 A and e4m3 B).  Routing is the bf16 router.  The
+ * workspace is the FP8 layer's (moe_workspace_size_fp8); the same size limits
+ * and errors as moe_layer_forward_fp8. */
+MOE_API int moe_layer_forward_fp4(const moe_bf16 *x, const moe_bf16 *Wg, const float *bias, const uint8_t *W1q,
+                                  const uint8_t *W1sf, const uint8_t *W3q, const uint8_t *W3sf, const uint8_t *W2q,
+                                  const uint8_t *W2sf, const uint8_t *Ws1q, const uint8_t *Ws1sf, const uint8_t *Ws3q,
+                                  const uint8_t *Ws3sf, const uint8_t *Ws2q, const uint8_t *Ws2sf, int64_t f_shared,
+                                  int64_t T, int64_t d, int64_t f, int64_t E, int64_t k, moe_bf16 *out, void *ws,
+                                  size_t ws_bytes, void *stream);
+
 /* Per-phase timing of the next moe_layer_forward call made on this host
  * thread: `events` holds n >= 6 cudaEvent_t handles; that call records
  * events[0..5] on its stream before the router, the permutation, the gate/up
