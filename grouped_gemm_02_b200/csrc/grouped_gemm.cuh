@@ -220,7 +220,8 @@ __device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a, co
 struct SmemCtl {
     uint64_t full[kMaxStages];
     uint64_t empty[kMaxStages];
-    uint64_t tfull[4];     // accumulator buffers: 2 in the bf16 GEMM, 4 partials in the FP8 GEMM
+    uint64_t sfull[kMaxStages];   // FP8 pair, second CTA: its own token scales (and FP4 weight scales) landed
+    uint64_t tfull[4];     // accumulators 0-1; FP8 gate/up: the epilogue warps' amax exchange at 2 (and 3)
     uint64_t tempty[4];
     uint64_t drain;
     uint32_t tmem_base;
@@ -230,14 +231,18 @@ static_assert(sizeof(SmemCtl) <= kBarBytes, "control block too large");
 
 // Spin on an mbarrier phase with a deadline.  Returns false (and flags the
 // whole CTA) when the deadline passes or another role already gave up.
+// kCluster: acquire at cluster scope (a barrier the other CTA of a pair arrives on
+// after writing shared memory that this CTA then reads).
+template <bool kCluster = false>
 __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, SmemCtl* ctl, uint32_t* err)
 {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    auto test = [&]() { return kCluster ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity); };
+    if (test()) return true;
     const uint64_t t0 = ptx::globaltimer();
     while (true) {
 #pragma unroll 1
         for (int i = 0; i < 256; i++)
-            if (ptx::mbar_try_wait(bar, parity)) return true;
+            if (test()) return true;
         if (*reinterpret_cast<volatile int*>(&ctl->abort)) return false;
         if (ptx::globaltimer() - t0 > kWaitTimeoutNs) {
             *reinterpret_cast<volatile int*>(&ctl->abort) = 1;

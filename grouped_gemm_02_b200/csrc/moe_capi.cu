@@ -38,7 +38,8 @@ struct DeviceState {
     bool ready = false;
     bool supported = false;
     int sm_count = 0;
-    int pair_grid = 0;   // CTAs of a CTA-pair GEMM launch: 2 x the clusters that fit at once (0: none)
+    int pair_grid = 0;       // CTAs of a CTA-pair GEMM launch: 2 x the clusters that fit at once (0: none)
+    int fp8_pair_grid = 0;   // the same for the FP8 / FP4 GEMM
 };
 
 std::mutex g_mu;
@@ -99,11 +100,11 @@ cudaError_t launch_pair(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t 
 
 // How many clusters of two CTAs of `kernel` can be resident at once (0 on error).
 template <typename... KArgs>
-int max_pair_clusters(void (*kernel)(KArgs...), size_t smem)
+int max_pair_clusters(void (*kernel)(KArgs...), size_t smem, int threads = kGemmThreads)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2);
-    cfg.blockDim = dim3(kGemmThreads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -156,6 +157,14 @@ int device_setup(DeviceState** out)
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kFp8SmemBytes) != cudaSuccess ||
                 cudaFuncSetAttribute(grouped_gemm_fp8_kernel<FP8_FUSED, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kFp8SmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(grouped_gemm_fp8_kernel<FP8_GATED, false, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kFp8SmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(grouped_gemm_fp8_kernel<FP8_DOWN, false, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kFp8SmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(grouped_gemm_fp8_kernel<FP8_GATED, true, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kFp8SmemBytes) != cudaSuccess ||
+                cudaFuncSetAttribute(grouped_gemm_fp8_kernel<FP8_DOWN, true, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kFp8SmemBytes) != cudaSuccess ||
                 cudaFuncSetAttribute(grouped_gemm_kernel<MODE_GATED, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) != cudaSuccess ||
                 cudaFuncSetAttribute(grouped_gemm_kernel<MODE_DOWN, true>,
@@ -169,6 +178,14 @@ int device_setup(DeviceState** out)
             pc = std::min(pc, max_pair_clusters(grouped_gemm_kernel<MODE_DOWN, true>, kGemmSmemBytes));
             pc = std::min(pc, max_pair_clusters(grouped_gemm_kernel<MODE_FUSED, true>, kGemmSmemBytes));
             st.pair_grid = 2 * std::min(pc, sms / 2);
+            int pc8 = max_pair_clusters(grouped_gemm_fp8_kernel<FP8_GATED, false, true>, kFp8SmemBytes, kFp8Threads);
+            pc8 = std::min(pc8, max_pair_clusters(grouped_gemm_fp8_kernel<FP8_DOWN, false, true>, kFp8SmemBytes,
+                                                  kFp8Threads));
+            pc8 = std::min(pc8, max_pair_clusters(grouped_gemm_fp8_kernel<FP8_GATED, true, true>, kFp8SmemBytes,
+                                                  kFp8Threads));
+            pc8 = std::min(pc8, max_pair_clusters(grouped_gemm_fp8_kernel<FP8_DOWN, true, true>, kFp8SmemBytes,
+                                                  kFp8Threads));
+            st.fp8_pair_grid = 2 * std::min(pc8, sms / 2);
             if (!g_encode) {
                 cudaDriverEntryPointQueryResult q;
                 void* fn = nullptr;
@@ -903,14 +920,28 @@ struct Fp8Operands {
     const uint8_t *f1, *f3, *f2, *fs1, *fs3, *fs2;
 };
 
-// An A-operand (weight) map: e4m3 bytes, or packed e2m1 unpacked by the TMA.
-bool make_map_w(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, bool w4)
+// An A-operand (weight) map: e4m3 bytes, or packed e2m1 unpacked by the TMA;
+// boxes of 128 rows (64 for the gate/up weights of CTA-pair tiles).
+bool make_map_w(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, bool w4, uint32_t box_rows = 128)
 {
-    return w4 ? make_map_u4(m, base, inner, rows, 128) : make_map_u8(m, base, inner, rows, 128);
+    return w4 ? make_map_u4(m, base, inner, rows, box_rows) : make_map_u8(m, base, inner, rows, box_rows);
 }
 
-int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int sms, cudaStream_t st, bool prof)
+// Whether the FP8 / FP4 expert GEMMs of P pairs and width f run on CTA pairs:
+// only when the policy asks for pairs and they run as two launches (the single
+// launch has no pair form).  Single CTAs are the default: on the B200 the pair
+// form measured 2-2.8x slower (its stages wait on both CTAs' scale atoms).
+bool fp8_pair(int64_t P, int64_t f, const DeviceState* dev)
 {
+    if (dev->fp8_pair_grid < 2) return false;
+    return policy(g_policy_pair, "MOE_GEMM_PAIR", /*invert=*/false) == 1 && !gemm_fused((int)P, (int)f);
+}
+
+int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, const DeviceState* dev, cudaStream_t st,
+                  bool prof, bool pair)
+{
+    const int sms = dev->sm_count;
+    const uint32_t gbox = pair ? 64 : 128;   // rows of a W1 / W3 box
     // gate/up operands: W1/W3, xp8 and its scales (shared: Ws1/Ws3, x8, sxT)
     CUtensorMap a0, a1, b, a0s, a1s, bs, sb, sbs;
     // down operands: W2, h8 and its scales (shared: Ws2, hs8, shs)
@@ -919,14 +950,14 @@ int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int 
     CUtensorMap b64, bs64, b264, b2s64;
     const uint64_t E = (uint64_t)o.E;
     const uint64_t lp = (uint64_t)o.ld_pairs, lt = (uint64_t)o.ld_tokens;
-    if (!make_map_w(&a0, o.W1q, o.d, E * o.f, o.w4) || !make_map_w(&a1, o.W3q, o.d, E * o.f, o.w4) ||
+    if (!make_map_w(&a0, o.W1q, o.d, E * o.f, o.w4, gbox) || !make_map_w(&a1, o.W3q, o.d, E * o.f, o.w4, gbox) ||
         !make_map_u8(&b, o.xp8, o.d, (uint64_t)o.P, 16) || !make_map_f32(&sb, o.sxp, lp, o.d / 128) ||
         !make_map_u8(&b64, o.xp8, o.d, (uint64_t)o.P, 64) || !make_map_u8(&b264, o.h8, o.f, (uint64_t)o.P, 64) ||
         !make_map_w(&a2, o.W2q, o.f, E * o.d, o.w4) || !make_map_u8(&b2, o.h8, o.f, (uint64_t)o.P, 16) ||
         !make_map_f32(&sb2, o.sh, lp, o.f / 128))
         return MOE_ERR_CUDA;
     if (o.fs > 0) {
-        if (!make_map_w(&a0s, o.Ws1q, o.d, o.fs, o.w4) || !make_map_w(&a1s, o.Ws3q, o.d, o.fs, o.w4) ||
+        if (!make_map_w(&a0s, o.Ws1q, o.d, o.fs, o.w4, gbox) || !make_map_w(&a1s, o.Ws3q, o.d, o.fs, o.w4, gbox) ||
             !make_map_u8(&bs, o.x8, o.d, (uint64_t)o.T, 16) || !make_map_f32(&sbs, o.sxT, lt, o.d / 128) ||
             !make_map_u8(&bs64, o.x8, o.d, (uint64_t)o.T, 64) || !make_map_u8(&b2s64, o.hs8, o.fs, (uint64_t)o.T, 64) ||
             !make_map_w(&a2s, o.Ws2q, o.fs, o.d, o.w4) || !make_map_u8(&b2s, o.hs8, o.fs, (uint64_t)o.T, 16) ||
@@ -991,16 +1022,30 @@ int run_gemms_fp8(const Fp8Operands& o, const int32_t* plan, uint32_t* err, int 
         // one launch: a gate/up tile streams d/128 k-blocks, a down tile f/128
         const int kb1 = o.d / 128, kb2 = o.f / 128;
         g1.comp = std::max(1, (kb1 + kb2 / 2) / kb2);
-        const cudaError_t e = launch(k_fused, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a0, a1, b, a0s, a1s,
+        const cudaError_t e = launch(k_fused, dim3(sms), dim3(kFp8Threads), kFp8SmemBytes, st, a0, a1, b, a0s, a1s,
                                      bs, sb, sbs, a2, b2, a2s, b2s, sb2, sb2s, b64, bs64, b264, b2s64, g1, g2);
         phase_mark(prof, 3, st);   // the single launch has no boundary: the down phase reads as zero
         return status_of(e);
     }
-    if (launch(k_gated, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a0, a1, b, a0s, a1s, bs, sb, sbs, a2, b2,
+    if (pair) {
+        // CTA pairs (M = 256): the grid holds exactly the clusters that fit at once
+        auto p_gated = o.w4 ? grouped_gemm_fp8_kernel<FP8_GATED, true, true>
+                            : grouped_gemm_fp8_kernel<FP8_GATED, false, true>;
+        auto p_down = o.w4 ? grouped_gemm_fp8_kernel<FP8_DOWN, true, true>
+                           : grouped_gemm_fp8_kernel<FP8_DOWN, false, true>;
+        const dim3 grid(dev->fp8_pair_grid);
+        if (launch_pair(p_gated, grid, dim3(kFp8Threads), kFp8SmemBytes, st, a0, a1, b, a0s, a1s, bs, sb, sbs, a2, b2,
+                        a2s, b2s, sb2, sb2s, b64, bs64, b264, b2s64, g1, g1) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        phase_mark(prof, 3, st);
+        return status_of(launch_pair(p_down, grid, dim3(kFp8Threads), kFp8SmemBytes, st, a2, a2, b2, a2s, a2s, b2s,
+                                     sb2, sb2s, a2, b2, a2s, b2s, sb2, sb2s, b264, b2s64, b264, b2s64, g2, g2));
+    }
+    if (launch(k_gated, dim3(sms), dim3(kFp8Threads), kFp8SmemBytes, st, a0, a1, b, a0s, a1s, bs, sb, sbs, a2, b2,
                a2s, b2s, sb2, sb2s, b64, bs64, b264, b2s64, g1, g1) != cudaSuccess)
         return MOE_ERR_CUDA;
     phase_mark(prof, 3, st);
-    return status_of(launch(k_down, dim3(sms), dim3(kGemmThreads), kFp8SmemBytes, st, a2, a2, b2, a2s, a2s, b2s, sb2,
+    return status_of(launch(k_down, dim3(sms), dim3(kFp8Threads), kFp8SmemBytes, st, a2, a2, b2, a2s, a2s, b2s, sb2,
                             sb2s, a2, b2, a2s, b2s, sb2, sb2s, b264, b2s64, b264, b2s64, g2, g2));
 }
 
@@ -1107,6 +1152,9 @@ static int layer_forward_lowp(const moe_bf16* x, const moe_bf16* Wg, const float
     const bf16* xb = reinterpret_cast<const bf16*>(x);
     const int iT = (int)T, id = (int)d, iE = (int)E, ik = (int)k, shared_rows = f_shared > 0 ? (int)T : 0;
     const int64_t P = T * k;
+    // the plan is cut for the tile shape the expert GEMMs will run
+    const bool pair = fp8_pair(P, f, dev);
+    const PlanShape ps = plan_shape(pair ? kPlanFp8Pair : kPlanFp8, T);
 
     const bool prof = t_phase_armed;
     t_phase_armed = false;
@@ -1122,13 +1170,13 @@ static int layer_forward_lowp(const moe_bf16* x, const moe_bf16* Wg, const float
     phase_mark(prof, 1, st);
     if (P <= kSmallPairs) {
         if (launch(permute_small_kernel, dim3(1), dim3(1024), 0, st, (const int32_t*)idx, (int)P, iE, counts, offsets,
-                   perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared, plan_shape(kPlanFp8, T), err) !=
+                   perm, inv_perm, plan, (int)f, id, shared_rows, (int)f_shared, ps, err) !=
             cudaSuccess)
             return MOE_ERR_CUDA;
         inv_perm_launch = t_launches;
     } else if ((rc = run_permute(idx, xb, iT, id, iE, ik, counts, offsets, perm, inv_perm, nullptr, err,
                                  at<int32_t>(ws, L.ctrl.block_counts), plan, (int)f, shared_rows, (int)f_shared,
-                                 dev->sm_count, st, plan_shape(kPlanFp8, T), &inv_perm_launch))) {
+                                 dev->sm_count, st, ps, &inv_perm_launch))) {
         return rc;
     }
     const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)dev->sm_count * 16));
@@ -1176,7 +1224,7 @@ static int layer_forward_lowp(const moe_bf16* x, const moe_bf16* Wg, const float
     o.fs = (int)f_shared;
     o.E = iE;
     phase_mark(prof, 2, st);
-    if ((rc = run_gemms_fp8(o, plan, err, dev->sm_count, st, prof))) return rc;
+    if ((rc = run_gemms_fp8(o, plan, err, dev, st, prof, pair))) return rc;
     phase_mark(prof, 4, st);
     rc = run_combine(y_p, inv_perm, o.ys, iT, ik, id, reinterpret_cast<bf16*>(out), st, inv_perm_launch);
     phase_mark(prof, 5, st);

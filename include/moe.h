@@ -277,7 +277,9 @@ MOE_API int moe_record_phase_events(void *const *events, int n);
  *                          0: two launches (rule: one when T*k <= 256 and f <= 4096)
  *   MOE_POLICY_CTA_PAIRS   1: tiles of 2 x 128 weight rows on CTA pairs
  *                          (cta_group::2), 0: single-CTA tiles of 128 rows
- *                          (rule: pairs whenever two launches run)
+ *                          (rule: the bf16 GEMMs take pairs whenever two
+ *                          launches run; the FP8 / FP4 GEMMs take them only
+ *                          when this is 1 and two launches run)
  *   MOE_POLICY_TILES       0 (rule): histogram-matched tiles -- the plan step
  *                          classifies the live histogram on the device (tokens
  *                          per effective expert, hottest expert against that

@@ -239,6 +239,12 @@ def pair_gemms(P: int, f: int) -> bool:
     return not fused_gemms(P, f)
 
 
+def pair_gemms_lowp(P: int, f: int) -> bool:
+    """CTA-pair tiles (FP8 / FP4 path): only when forced on and two launches run
+    (the single launch has no pair form)."""
+    return not fused_gemms(P, f) and POLICY["pairs"] == 1
+
+
 def check_routing(views, s: wl.LayerShape, what: str):
     """Routing on identical fp32 logits: the oracle's top-k of the GPU's own logits
     equals the GPU's indices for every token (gates within 1e-6), and counts,
@@ -261,9 +267,11 @@ def check_layer_plan(views, s: wl.LayerShape, counts, offsets, what, fp8: bool =
     launch form uses, and (single launch) every gate/up tile's epilogue warps
     published their h rows: 4 per tile and CTA."""
     plan = decode_plan(views["plan"])
-    pair = (not fp8) and pair_gemms(s.P, s.f)
+    pair = pair_gemms_lowp(s.P, s.f) if fp8 else pair_gemms(s.P, s.f)
     assert plan["pair"] == int(pair), f"{what}: plan cut for pair={plan['pair']}, expected {pair}"
-    if fp8:
+    if fp8 and pair:
+        unit_max, m1_rows, m2_rows, align = 224, 128, 256, 32
+    elif fp8:
         unit_max, m1_rows, m2_rows, align = 112, 128, 128, 16
     elif pair:
         unit_max, m1_rows, m2_rows, align = 256, 128, 256, 32

@@ -141,6 +141,17 @@ def test_fp4_layer_small(name, kw):
     _fp4_layer_check(s, seed=0, n_sample=sample, device_inputs=s.d * s.f * s.E > 2**31)
 
 
+@pytest.mark.parametrize("pairs", [0, 1])
+@pytest.mark.parametrize("name", ["odd", "skew"])
+def test_fp4_layer_tile_shapes(name, pairs):
+    """FP4 weights on both tile shapes of the two-launch form (the small layers of the
+    FP8 tests: "odd" has d = 384, so the last down pair tile's second CTA lies past d
+    and its atom is held to the last tile)."""
+    from tests.test_gpu_fp8 import TILE_SHAPES
+    with H.policy(pairs=pairs):
+        _fp4_layer_check(TILE_SHAPES[name], seed=1)
+
+
 @pytest.mark.parametrize("name,kw", [("deepseek_v3", dict(T=1024, alpha=0.5)), ("mixtral", dict(T=256))])
 def test_fp4_layer_full_size_sampled(name, kw):
     s = wl.shape(name, **kw)

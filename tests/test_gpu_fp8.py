@@ -174,6 +174,36 @@ def test_fp8_layer_full_size_sampled(name, kw):
     torch.cuda.empty_cache()
 
 
+# Small layers for the two tile shapes of the two-launch form:
+#   odd:    d = 384 is not a multiple of 256, so the second CTA of the last down
+#           pair tile lies past d (its rows are dropped, its weight scales held to
+#           the last tile); with a shared expert;
+#   skew:   Dirichlet alpha = 0.02 over 16 experts, so a few experts take most of
+#           the 2048 pairs and get the widest tiles (224 tokens on pairs);
+#   shared: f = 384 (three gate/up pair tiles) with a shared expert of 256.
+TILE_SHAPES = {
+    "odd": wl.LayerShape("odd", T=300, d=384, f=256, E=8, k=2, alpha=1.0, f_shared=128),
+    "skew": wl.LayerShape("skew", T=512, d=1024, f=512, E=16, k=4, alpha=0.02, f_shared=0),
+    "shared": wl.LayerShape("shared", T=200, d=512, f=384, E=8, k=2, alpha=1.0, f_shared=256),
+}
+
+
+@pytest.mark.parametrize("pairs", [0, 1])
+@pytest.mark.parametrize("name", sorted(TILE_SHAPES))
+def test_fp8_layer_tile_shapes(name, pairs):
+    """Both tile shapes of the two-launch form (CTA pairs of up to 224 tokens, single
+    CTAs of up to 112) against the oracle on every token."""
+    with H.policy(pairs=pairs):
+        _fp8_layer_check(TILE_SHAPES[name], seed=1)
+
+
+@pytest.mark.parametrize("tiles,cap", [(1, -1), (1, 64), (-1, 96)])
+def test_fp8_pair_tile_policies(tiles, cap):
+    """The pair tiles under the token-bucket policy and a forced cap (widths rounded to 32)."""
+    with H.policy(tiles=tiles, cap=cap):
+        _fp8_layer_check(TILE_SHAPES["skew"], seed=2)
+
+
 def test_fp8_deterministic():
     s = wl.DECODE64.with_(alpha=0.1)
     d = {n: v.to(DEV) for n, v in wl.make_inputs(s, seed=5).items()}
