@@ -36,7 +36,8 @@ struct PlanHeader {
     int32_t tiles2;     // tiles of the down GEMM (M-tile = 128 rows of W2)
     int32_t n_max;      // widest tile (tokens) in this launch
     int32_t pairs;      // routed pairs with a valid expert id (== offsets[E])
-    int32_t pair;       // 1: tiles cut for CTA pairs (2 x 128 weight rows, widths a multiple of 32)
+    int32_t pair;       // bit 0: tiles cut for CTA pairs (2 x 128 weight rows, widths a multiple of 32);
+                        // bit 1: a down tile spans two units (FP8 / FP4 GEMMs of the two-launch form)
     int32_t cls;        // histogram class the tile cap was looked up for, or kPlanClassCap / kPlanClassBucket
     int32_t cap;        // most tokens per tile in this plan's cut
 };
@@ -63,6 +64,7 @@ constexpr int kTilesCap = 2;
 struct PlanShape {
     int unit_rows, m1_rows, m2_rows, align, pair;
     int policy;
+    int merge = 1;   // units one down tile spans (2: the FP8 down GEMM of the two-launch form)
 };
 
 struct PlanArrays {

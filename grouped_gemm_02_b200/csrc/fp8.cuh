@@ -39,6 +39,8 @@ namespace moe {
 
 constexpr int kFp8TileRows = 112;                // most tokens one FP8 tile carries
 constexpr PlanShape kPlanFp8{kFp8TileRows, 128, 128, 16, 0};
+// the two-launch form: a down tile (one accumulator) spans two units, up to 224 tokens
+constexpr PlanShape kPlanFp8Wide{kFp8TileRows, 128, 128, 16, 0, 0, 2};
 // CTA-pair tiles (large token counts): up to 224 tokens, 128 f rows (gate/up) or
 // 256 d rows (down) per pair; two accumulators of 224 columns and the scale
 // factors (8 columns for two token atoms) fit the 512 TMEM columns.
@@ -355,8 +357,11 @@ __device__ __forceinline__ Fp8Tile fp8_decode(int nb, int t, const Fp8Args& a, c
         else hi = mid - 1;
     }
     const int local = t - tb[lo];
-    const int units = sp->units[lo];
     const int4 b = sp->blk[lo];
+    // a down tile of the two-launch form may span `merge` units of the block
+    const int merge = (KIND == FP8_DOWN && !PAIR) ? sp->merge : 1;
+    const int units = (sp->units[lo] + merge - 1) / merge;
+    const int width = merge * b.w;
     const Fp8Args& ta = (KIND == FP8_FUSED && !gated) ? a2 : a;
     Fp8Tile tl;
     tl.blk = lo;
@@ -365,11 +370,11 @@ __device__ __forceinline__ Fp8Tile fp8_decode(int nb, int t, const Fp8Args& a, c
     tl.shared = tl.group == ta.E;
     tl.m = local / units;
     const int u = local - tl.m * units;
-    const int start = u * b.w;
-    tl.rows = min(b.w, b.z - start);
+    const int start = u * width;
+    tl.rows = min(width, b.z - start);
     tl.row0 = b.y + start;
     // a multiple of 16, of 32 for a pair (each CTA loads n/2 rows in 16-row boxes)
-    tl.n_mma = sp->fixed_n ? sp->fixed_n : PAIR ? (tl.rows + 31) & ~31 : (tl.rows + 15) & ~15;
+    tl.n_mma = sp->fixed_n ? merge * sp->fixed_n : PAIR ? (tl.rows + 31) & ~31 : (tl.rows + 15) & ~15;
     tl.nkb = (tl.shared ? ta.K_shared : ta.K) / kFp8BlockK;
     tl.b_n = PAIR ? tl.n_mma >> 1 : tl.n_mma;
     tl.b_row0 = tl.row0 + rank * tl.b_n;
@@ -556,13 +561,15 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
     constexpr int kRows = PAIR ? kFp8PairTileRows : kFp8TileRows;
     // A region of a stage: W1 and W3 tiles of 128 rows (single-CTA gate/up), or 128 weight rows
     constexpr uint32_t kABytes = (KIND != FP8_DOWN && !PAIR) ? 2 * 128 * kFp8BlockK : 128 * kFp8BlockK;
-    constexpr uint32_t kSfBytes = PAIR ? kSfStageBytesPair : kSfStageBytes;
+    // tiles of up to 224 tokens: a pair's, and the down GEMM's of the two-launch form
+    constexpr bool kWide = PAIR || KIND == FP8_DOWN;
+    constexpr uint32_t kSfBytes = kWide ? kSfStageBytesPair : kSfStageBytes;
     constexpr int kRing = PAIR ? kFp8PairRingBytes : kFp8RingBytes;
     // scale-factor region of a stage: token scales (fp32), then the atoms
-    constexpr uint32_t kSfScales = PAIR ? 1024 : 512;       // bytes of staged token scales
+    constexpr uint32_t kSfScales = kWide ? 1024 : 512;      // bytes of staged token scales
     constexpr uint32_t kAtomA0 = kSfScales;                 // this CTA's weight rows
     constexpr uint32_t kAtomA1 = kAtomA0 + 512;             // single-CTA gate/up: W3
-    constexpr uint32_t kAtomB = PAIR ? kAtomA0 + 512 : kAtomA1 + 512;   // tokens (two atoms for a pair)
+    constexpr uint32_t kAtomB = kWide ? kAtomA0 + 512 : kAtomA1 + 512;   // tokens (two atoms when wide)
     constexpr uint32_t kRawW = kAtomB + 1024;               // PAIR W4 gate/up: the W1 and W3 atoms as stored
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -584,14 +591,15 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
     const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(args.plan);
     // a plan made for wider tiles or the other tile shape: refuse, touch nothing
     // (every CTA sees the same header and leaves before any barrier)
-    if (hdr->n_max > kRows || hdr->pair != (PAIR ? 1 : 0)) {
+    if (hdr->n_max > kRows || (hdr->pair & 1) != (PAIR ? 1 : 0) || (KIND == FP8_FUSED && hdr->pair != 0)) {
         if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(args.err, DEVERR_PLAN);
         return;
     }
     const int nb = hdr->n_blocks;
     const int total = KIND == FP8_FUSED ? hdr->tiles1 + hdr->tiles2 : KIND == FP8_GATED ? hdr->tiles1 : hdr->tiles2;
+    const int merge = (KIND == FP8_DOWN && !PAIR && (hdr->pair & 2)) ? 2 : 1;
     const int n_max = max(PAIR ? 32 : 16, hdr->n_max);
-    const uint32_t b_bytes = (uint32_t)(PAIR ? n_max / 2 : n_max) * kFp8BlockK;   // B region of a stage
+    const uint32_t b_bytes = (uint32_t)(PAIR ? n_max / 2 : merge * n_max) * kFp8BlockK;   // B region of a stage
     const uint32_t stage_bytes = kABytes + b_bytes + kSfBytes;
     const int stages = min(kMaxStages, (int)(kRing / stage_bytes));
     {
@@ -600,6 +608,7 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
         if (threadIdx.x == 0) {
             splan->tiles1 = hdr->tiles1;
             splan->fixed_n = hdr->cls == kPlanClassBucket ? hdr->cap : 0;
+            splan->merge = merge;
         }
         for (int i = threadIdx.x; i <= nb; i += blockDim.x) {
             splan->tb[i] = tbg[i];
@@ -758,7 +767,7 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
                 // token of the tile) from row0 rounded down to 4, into this CTA
                 const uint32_t sf = b_dst + b_bytes;
                 ptx::tma_load_2d(sf, sm, own_bar(s), tl.row0 & ~3, kb, pol);
-                if (PAIR) ptx::tma_load_2d(sf + 512, sm, own_bar(s), (tl.row0 & ~3) + 128, kb, pol);
+                if (kWide) ptx::tma_load_2d(sf + 512, sm, own_bar(s), (tl.row0 & ~3) + 128, kb, pol);
             };
             // FP8_FUSED: a down tile reads h8 and its scales only after every gate/up
             // tile of its block has published them (4 epilogue warps per tile)
@@ -881,6 +890,8 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
                         if (tl.gated)
                             ptx::tmem_cp_32x128b_warpx4(tmem_base + kSfColA1, ptx::plain_rows16_desc(atoms + kAtomA1));
                         ptx::tmem_cp_32x128b_warpx4(tmem_base + kSfColB, ptx::plain_rows16_desc(atoms + kAtomB));
+                        if (kWide && tl.n_mma > 128)
+                            ptx::tmem_cp_32x128b_warpx4(tmem_base + kSfColB + 4, ptx::plain_rows16_desc(atoms + kAtomB + 512));
 #pragma unroll
                         for (int kk = 0; kk < kFp8BlockK / 32; kk++)
                             mma_mxf8_ss(d_g, ptx::sw128_kmajor_desc(a_addr + kk * 32),
@@ -970,7 +981,7 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
                 const float* staged = reinterpret_cast<const float*>(sfp);
                 // the tokens' atoms: token c = 128 q + lane + 32 m1 at byte 16 lane + 4 m1 of atom q
 #pragma unroll
-                for (int q = 0; q < (PAIR ? 2 : 1); q++) {
+                for (int q = 0; q < (kWide ? 2 : 1); q++) {
                     uint32_t w[4];
 #pragma unroll
                     for (int m1 = 0; m1 < 4; m1++) {
@@ -1029,7 +1040,7 @@ __global__ void __launch_bounds__(kFp8Threads, 1)
             float gates[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
             if (!tl.gated && !tl.shared) {
 #pragma unroll
-                for (int i = 0; i < (PAIR ? 8 : 4); i++) {
+                for (int i = 0; i < (kWide ? 8 : 4); i++) {
                     const int col = 32 * i + lane;
                     if (col < tl.rows) gates[i] = __ldg(ea.gate_w + __ldg(ea.perm + tl.row0 + col));
                 }

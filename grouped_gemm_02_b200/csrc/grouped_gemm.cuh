@@ -125,6 +125,7 @@ struct SmemPlan {
     int units[kMaxGroups];
     int tiles1;                 // MODE_FUSED: gate/up tiles come first
     int fixed_n;                // token-bucket plans: every tile's MMA width (padded); 0 otherwise
+    int merge;                  // FP8 down GEMM: units one tile spans (1 or 2)
 };
 // gate/up epilogue: each pair of warps hands the other half of a 16-column chunk
 // through shared memory: [2 row quarters][2 buffers][2 directions][8 columns][32 lanes] fp32

@@ -1154,7 +1154,7 @@ static int layer_forward_lowp(const moe_bf16* x, const moe_bf16* Wg, const float
     const int64_t P = T * k;
     // the plan is cut for the tile shape the expert GEMMs will run
     const bool pair = fp8_pair(P, f, dev);
-    const PlanShape ps = plan_shape(pair ? kPlanFp8Pair : kPlanFp8, T);
+    const PlanShape ps = plan_shape(pair ? kPlanFp8Pair : gemm_fused((int)P, (int)f) ? kPlanFp8 : kPlanFp8Wide, T);
 
     const bool prof = t_phase_armed;
     t_phase_armed = false;

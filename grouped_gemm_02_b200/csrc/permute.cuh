@@ -91,8 +91,9 @@ __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b -
 //   * blocks sorted by n descending (ties: lower expert id), so the heaviest
 //     tiles are dealt first;
 //   * tile prefixes for both GEMMs: units * ceil(M / ps.m1_rows) gate/up tiles
-//     and units * ceil(d / ps.m2_rows) down tiles; the header records whether
-//     the tiles are cut for CTA pairs.
+//     and ceil(units / ps.merge) * ceil(d / ps.m2_rows) down tiles (a down tile
+//     may span ps.merge units); the header records whether the tiles are cut
+//     for CTA pairs and whether down tiles span two units.
 __device__ __forceinline__ void build_plan(int c, int off, int E, int pairs, int32_t* __restrict__ plan, int f, int d,
                                            int shared_rows, int f_shared, int* warp_sums, PlanShape ps)
 {
@@ -175,7 +176,7 @@ __device__ __forceinline__ void build_plan(int c, int off, int E, int pairs, int
         pa.units[tid] = units;
         pa.dep[tid] = 0;
         my_t1 = units * ceil_div(M1, ps.m1_rows);
-        my_t2 = units * ceil_div(d, ps.m2_rows);
+        my_t2 = ceil_div(units, ps.merge) * ceil_div(d, ps.m2_rows);
         my_chunk = chunk;
     }
     const int p1 = block_inclusive_scan(my_t1, warp_sums);
@@ -196,7 +197,7 @@ __device__ __forceinline__ void build_plan(int c, int off, int E, int pairs, int
         h->n_blocks = nact;
         h->n_max = m;
         h->pairs = pairs;
-        h->pair = ps.pair;
+        h->pair = ps.pair | (ps.merge == 2 ? 2 : 0);
         h->cls = s_cls;
         h->cap = cap;
         pa.tb1[0] = 0;

@@ -314,7 +314,8 @@ MOE_API int64_t moe_launch_counter(void);
  * (which: 0 logits, 1 topk_idx, 2 topk_w, 3 counts, 4 offsets, 5 perm,
  * 6 inv_perm, 7 xp, 8 h, 9 y_p, 10 hs, 11 ys, 12 the tile plan).  The tile plan is
  * MOE_PLAN_INTS int32: a header {n_blocks, tiles1, tiles2, n_max, pairs,
- * pair (1: tiles cut for CTA pairs), cls (the histogram class whose tuned
+ * pair (bit 0: tiles cut for CTA pairs; bit 1: a down tile spans two units,
+ * the FP8 / FP4 layer's two-launch form), cls (the histogram class whose tuned
  * cap was taken; -1: a forced cap, -2: token buckets), cap (most tokens per
  * tile)},
  * then arrays of 513 entries group, row0, rows, chunk, units, two tile

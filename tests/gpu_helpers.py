@@ -116,7 +116,8 @@ def decode_plan(plan) -> dict:
 
 
 def check_plan(plan: dict, counts: np.ndarray, offsets: np.ndarray, T: int, f: int, d: int, f_shared: int,
-               unit_max: int, m1_rows: int, what: str = "", m2_rows: int = 128, align: int = 16) -> None:
+               unit_max: int, m1_rows: int, what: str = "", m2_rows: int = 128, align: int = 16,
+               merge: int = 1) -> None:
     """The invariants of a tile plan built from the live histogram:
     * one block per expert with tokens (+ the shared expert over all T tokens),
       heaviest first (ties: lower group id);
@@ -124,8 +125,9 @@ def check_plan(plan: dict, counts: np.ndarray, offsets: np.ndarray, T: int, f: i
       `chunk` rows, a multiple of `align` and at most unit_max, every chunk non-empty,
       so the tiles of a block cover its rows exactly once;
     * the routed blocks' rows tile [0, offsets[E]) exactly once;
-    * the tile prefixes count units x M-tiles of each GEMM, and n_max is the
-      widest chunk."""
+    * the tile prefixes count units x M-tiles of the gate/up GEMM and
+      ceil(units / merge) x M-tiles of the down GEMM (a down tile spanning
+      `merge` units), and n_max is the widest chunk."""
     E = counts.size
     active = np.nonzero(counts > 0)[0]
     n_blocks = active.size + (1 if f_shared else 0)
@@ -156,7 +158,7 @@ def check_plan(plan: dict, counts: np.ndarray, offsets: np.ndarray, T: int, f: i
     m1 = np.array([-(-(f if gi < E else f_shared) // m1_rows) for gi in g], dtype=np.int64)
     m2 = -(-d // m2_rows)
     assert np.array_equal(plan["tb1"], np.concatenate([[0], np.cumsum(un * m1)])), what
-    assert np.array_equal(plan["tb2"], np.concatenate([[0], np.cumsum(un * m2)])), what
+    assert np.array_equal(plan["tb2"], np.concatenate([[0], np.cumsum(-(-un // merge) * m2)])), what
     assert plan["tiles1"] == plan["tb1"][-1] and plan["tiles2"] == plan["tb2"][-1], what
     assert plan["n_max"] == (int(ch.max()) if n_blocks else 0), what
     assert plan["pairs"] == int(offsets[-1]), what
@@ -268,7 +270,10 @@ def check_layer_plan(views, s: wl.LayerShape, counts, offsets, what, fp8: bool =
     published their h rows: 4 per tile and CTA."""
     plan = decode_plan(views["plan"])
     pair = pair_gemms_lowp(s.P, s.f) if fp8 else pair_gemms(s.P, s.f)
-    assert plan["pair"] == int(pair), f"{what}: plan cut for pair={plan['pair']}, expected {pair}"
+    # FP8 / FP4 on single CTAs in two launches: a down tile spans two units (header bit 1)
+    merge = 2 if fp8 and not pair and not fused_gemms(s.P, s.f) else 1
+    want = int(pair) | (2 if merge == 2 else 0)
+    assert plan["pair"] == want, f"{what}: plan header pair={plan['pair']}, expected {want}"
     if fp8 and pair:
         unit_max, m1_rows, m2_rows, align = 224, 128, 256, 32
     elif fp8:
@@ -277,7 +282,7 @@ def check_layer_plan(views, s: wl.LayerShape, counts, offsets, what, fp8: bool =
         unit_max, m1_rows, m2_rows, align = 256, 128, 256, 32
     else:
         unit_max, m1_rows, m2_rows, align = 256, 64, 128, 16
-    check_plan(plan, counts, offsets, s.T, s.f, s.d, s.f_shared, unit_max, m1_rows, what, m2_rows, align)
+    check_plan(plan, counts, offsets, s.T, s.f, s.d, s.f_shared, unit_max, m1_rows, what, m2_rows, align, merge)
     # the tile policy: a forced cap, token buckets, or the table's cap for the histogram class
     rnd = lambda v: max(align, min(v, unit_max) // align * align)
     caps, widths = tile_tables()
