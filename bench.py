@@ -591,7 +591,9 @@ def sub_record(s, rec, fmt):
             "histogram": stats.histogram_stats(rec["counts"]),
             "phase_us": {n: float(v * 1e3) for n, v in
                          zip(("route", "permute", "gemm_gate_up", "gemm_down", "combine"), rec["phase_ms"])},
-            "phase_note": "per-phase means from a second pass with CUDA events between phases"}
+            "phase_note": ("per-phase means from CUDA events recorded between the phases inside the timed region"
+                           if rec.get("phases_in_timed") else
+                           "per-phase means from a second pass with CUDA events between phases")}
 
 
 def cpu_baseline(s, host, budget_s):
@@ -644,6 +646,17 @@ def run_ours(args, s: wl.LayerShape):
                                         rec["phase_ms"])}},
             "roofline": rec["roofline"], "layer_roofline": rec["layer_roofline"], "e2e": rec["e2e"],
             "gpu_launches": rec["launches"], "clocks": clocks}
+    if not args.no_sub and weight_format(args) == "bf16" and args.lowp_steps > 0:
+        # the same layer with FP8 and with FP4 expert weights (quantised outside the timed region)
+        import copy
+        for fmt in ("fp8", "fp4"):
+            a2 = copy.copy(args)
+            a2.fp8, a2.fp4 = fmt == "fp8", fmt == "fp4"
+            lrec, _ = measure_layer(s, a2, args.lowp_steps, max(3, args.warmup), world, dev, phases_in_timed=True,
+                                    with_e2e=False)
+            lrec["steps"] = args.lowp_steps
+            line[fmt] = sub_record(s, lrec, fmt)
+            torch.cuda.empty_cache()
     if not args.no_sub and s.name != DECODE_SUB["workload"]:
         ds = wl.shape(DECODE_SUB["workload"], T=DECODE_SUB["T"], alpha=DECODE_SUB["alpha"])
         drec, _ = measure_layer(ds, args, args.sub_steps, 20, world, dev, phases_in_timed=False, with_e2e=False)
@@ -728,6 +741,8 @@ def build_parser():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub", action="store_true", help="skip the decode64 sub-record")
     ap.add_argument("--sub-steps", type=int, default=2000, help="timed steps of the decode64 sub-record")
+    ap.add_argument("--lowp-steps", type=int, default=20,
+                    help="timed steps of the FP8 and FP4 sub-records of a bf16 run (0: none)")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     return ap
 
