@@ -368,8 +368,18 @@ __device__ __forceinline__ Fp8Tile fp8_decode(int nb, int t, const Fp8Args& a, c
     tl.gated = gated;
     tl.group = b.x;
     tl.shared = tl.group == ta.E;
-    tl.m = local / units;
-    const int u = local - tl.m * units;
+    // tile order inside the block: M-tile-major, or unit-major when the block has
+    // more token rows than weight rows (as in the bf16 GEMM's decode_tile)
+    const int wrows = (gated ? 2 : 1) * (tl.shared ? ta.M_shared : ta.M);
+    const int mtiles = (tb[lo + 1] - tb[lo]) / units;
+    int u;
+    if (b.z > wrows) {
+        u = local / mtiles;
+        tl.m = local - u * mtiles;
+    } else {
+        tl.m = local / units;
+        u = local - tl.m * units;
+    }
     const int start = u * width;
     tl.rows = min(width, b.z - start);
     tl.row0 = b.y + start;

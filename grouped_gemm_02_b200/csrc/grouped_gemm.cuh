@@ -192,8 +192,21 @@ __device__ __forceinline__ Tile decode_tile(int nb, int t, const GemmArgs& a, co
     tl.gated = gated;
     tl.group = b.x;
     tl.shared = tl.group == a.E;
-    tl.m = local / units;
-    const int u = local - tl.m * units;
+    // Order of a block's tiles: M-tile-major (the units of one weight M-tile run
+    // together and share its fetch in L2, while the block's token rows stay in L2
+    // across M-tiles), unless the block has more token rows than weight rows: then
+    // unit-major (the block's weights stay in L2 and each unit's rows stream once).
+    const GemmArgs& wa = (MODE == MODE_FUSED && !gated) ? a2 : a;
+    const int wrows = (gated ? 2 : 1) * (tl.shared ? wa.M_shared : wa.M);
+    const int mtiles = (tb[lo + 1] - tb[lo]) / units;
+    int u;
+    if (b.z > wrows) {
+        u = local / mtiles;
+        tl.m = local - u * mtiles;
+    } else {
+        tl.m = local / units;
+        u = local - tl.m * units;
+    }
     const int start = u * chunk;
     tl.rows = min(chunk, b.z - start);
     tl.row0 = b.y + start;

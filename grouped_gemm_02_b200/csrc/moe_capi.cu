@@ -739,8 +739,12 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
     const bool pair = gemm_pair((int)P, (int)f, dev);
     // token rows for the gate/up GEMM: a gather pass into xp (the default), or TMA
     // row gathers from x inside the GEMM (tile::gather4, 4 rows per instruction),
-    // which measured slower on B200 at every size: more, smaller TMA requests
-    const bool gather_in_gemm = g_policy_gather.load(std::memory_order_relaxed) == 1;
+    // which measured slower on B200 at every size: more, smaller TMA requests.
+    // The row gathers run only in the two-launch form: in the single launch they
+    // gave wrong rows on a layer with several token units per expert and a shared
+    // expert (T=2048, E=4, f=128, f_shared=128), a fault not yet traced.
+    const bool gather_in_gemm =
+        g_policy_gather.load(std::memory_order_relaxed) == 1 && !gemm_fused((int)(T * k), (int)f);
     if ((rc = run_topk(src, iT, iE, ik, idx, w, err, st))) return rc;
     phase_mark(prof, 1, st);
     if (P <= kSmallPairs) {

@@ -296,8 +296,10 @@ MOE_API int moe_record_phase_events(void *const *events, int n);
  *                          tuning); -1: off
  *   MOE_POLICY_GATHER      1: moe_layer_forward's gate/up GEMM gathers its token
  *                          rows straight from x (TMA tile::gather4, four rows per
- *                          request) instead of a gather pass into xp; 0 (rule):
- *                          the gather pass, measured faster on B200 at every size
+ *                          request) instead of a gather pass into xp, when the
+ *                          expert GEMMs run as two launches (the single launch
+ *                          keeps the gather pass); 0 (rule): the gather pass,
+ *                          measured faster on B200 at every size
  * Returns MOE_ERR_ARG for an unknown switch or value.  The pages have no
  * counterpart to the first two switches. */
 #define MOE_POLICY_ONE_LAUNCH 1

@@ -180,11 +180,14 @@ def test_fp8_layer_full_size_sampled(name, kw):
 #           the last tile); with a shared expert;
 #   skew:   Dirichlet alpha = 0.02 over 16 experts, so a few experts take most of
 #           the 2048 pairs and get the widest tiles (224 tokens on pairs);
-#   shared: f = 384 (three gate/up pair tiles) with a shared expert of 256.
+#   shared: f = 384 (three gate/up pair tiles) with a shared expert of 256;
+#   tall:   more token rows per expert than weight rows (tiles taken unit-major).
 TILE_SHAPES = {
     "odd": wl.LayerShape("odd", T=300, d=384, f=256, E=8, k=2, alpha=1.0, f_shared=128),
     "skew": wl.LayerShape("skew", T=512, d=1024, f=512, E=16, k=4, alpha=0.02, f_shared=0),
     "shared": wl.LayerShape("shared", T=200, d=512, f=384, E=8, k=2, alpha=1.0, f_shared=256),
+    # more token rows per expert than weight rows: tiles taken unit-major
+    "tall": wl.LayerShape("tall", T=2048, d=256, f=128, E=4, k=2, alpha=1.0, f_shared=128),
 }
 
 

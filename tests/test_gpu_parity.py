@@ -260,6 +260,9 @@ def test_empty_and_single_token():
 
 
 FORMS = [(1, 0), (0, 0), (1, 1), (0, 1)]     # (one launch, CTA pairs)
+# more token rows per expert (and in the shared expert) than weight rows: the GEMMs
+# take such a block's tiles unit-major
+TALL = wl.LayerShape("tall", T=2048, d=256, f=128, E=4, k=2, alpha=1.0, f_shared=128)
 
 
 @pytest.mark.parametrize("gather", [0, 1])
@@ -268,14 +271,15 @@ FORMS = [(1, 0), (0, 0), (1, 1), (0, 1)]     # (one launch, CTA pairs)
     ("decode64", dict(alpha=0.1)),
     ("deepseek_v3", dict(T=64, alpha=0.05)),     # shared expert
     ("kimi_k2", dict(T=256)),                    # hot experts with units of up to 256 tokens
+    ("tall", dict()),                            # unit-major tile order
 ])
 def test_layer_every_launch_form(name, kw, one_launch, pairs, gather):
     """Both expert-GEMM launch forms on single CTAs and on CTA pairs, with the gather pass or
     the TMA row gathers inside the GEMM, each checked against the oracle (routing bit-exact,
     plan invariants, outputs in tolerance)."""
-    s = wl.shape(name, **kw)
+    s = TALL if name == "tall" else wl.shape(name, **kw)
     with H.policy(one_launch=one_launch, pairs=pairs, gather=gather):
-        _layer_check(s, seed=3, n_sample=12, device_inputs=s.d * s.f * s.E > 2**31)
+        _layer_check(s, seed=3, n_sample=None if name == "tall" else 12, device_inputs=s.d * s.f * s.E > 2**31)
     torch.cuda.empty_cache()
 
 
