@@ -257,35 +257,38 @@ __global__ void __launch_bounds__(256) quantize_blocks_fp8_kernel(const bf16* __
     if (threadIdx.x == 0) scale[br * nbc + bc] = ldexpf(1.f, e);
 }
 
-// xp8[pos, :] = x8[perm[pos] / k, :], and the row's scales K-block-major:
-// sxpT[b * ld + pos] = sx[perm[pos] / k, b]; one warp per row.
+// xp8[inv_perm[t k + j], :] = x8[t, :] and the row's scales K-block-major,
+// sxpT[b * ld + pos] = sx[t, b], for every pair with a valid position: x8[pos] of
+// perm[pos] / k, taken in token order so that each x8 row is read once for its k
+// copies.  One warp per (token, 512-byte chunk of the row); the chunk-0 warp also
+// writes the scales.  Requires d % 128 == 0, k <= 32.
 __global__ void __launch_bounds__(256) gather_rows_fp8_kernel(const uint8_t* __restrict__ x8,
                                                               const float* __restrict__ sx,
-                                                              const int32_t* __restrict__ perm,
-                                                              const int32_t* __restrict__ offsets, int E, int k, int d,
+                                                              const int32_t* __restrict__ inv_perm, int T, int k, int d,
                                                               uint8_t* __restrict__ xp8, float* __restrict__ sxpT,
                                                               int64_t ld)
 {
     ptx::grid_dep_wait();
     ptx::grid_dep_launch();
-    const int pairs = offsets[E];
     const int nvec = d / 16, nsb = d / 128;
+    const int nch = (nvec + 31) / 32;
     const int lane = threadIdx.x & 31;
-    for (int64_t r = (int64_t)(blockIdx.x * blockDim.x + threadIdx.x) / 32; r < pairs;
-         r += (int64_t)gridDim.x * blockDim.x / 32) {
-        const int t = perm[r] / k;
-        const uint4* src = reinterpret_cast<const uint4*>(x8 + (size_t)t * d);
-        uint4* dst = reinterpret_cast<uint4*>(xp8 + (size_t)r * d);
-        for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
-            uint4 buf[4];
-#pragma unroll
-            for (int u = 0; u < 4; u++)
-                if (v0 + 32 * u < nvec) buf[u] = __ldg(src + v0 + 32 * u);
-#pragma unroll
-            for (int u = 0; u < 4; u++)
-                if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = buf[u];
+    const int64_t items = (int64_t)T * nch;
+    for (int64_t w = (int64_t)(blockIdx.x * blockDim.x + threadIdx.x) / 32; w < items;
+         w += (int64_t)gridDim.x * blockDim.x / 32) {
+        const int64_t t = w / nch;
+        const int c = (int)(w - t * nch);
+        const int v = c * 32 + lane;
+        const int mine = lane < k ? inv_perm[t * k + lane] : -1;
+        uint4 buf = make_uint4(0u, 0u, 0u, 0u);
+        if (v < nvec) buf = __ldg(reinterpret_cast<const uint4*>(x8 + (size_t)t * d) + v);
+        for (int j = 0; j < k; j++) {
+            const int pos = __shfl_sync(0xffffffffu, mine, j);
+            if (pos < 0) continue;
+            if (v < nvec) reinterpret_cast<uint4*>(xp8 + (size_t)pos * d)[v] = buf;
+            if (c == 0)
+                for (int b = lane; b < nsb; b += 32) sxpT[(size_t)b * ld + pos] = sx[(size_t)t * nsb + b];
         }
-        for (int b = lane; b < nsb; b += 32) sxpT[(size_t)b * ld + r] = sx[(size_t)t * nsb + b];
     }
 }
 

@@ -341,6 +341,15 @@ int run_topk(const TopkSource& s, int T, int E, int k, int32_t* idx, float* w, u
                             s.bias, T, E, k, s.logits_out, idx, w, err));
 }
 
+// Blocks of 8 warps for a token-order row gather over T tokens of `nvec`
+// 16-byte vectors a row: one warp per (token, 32-vector chunk), at most 16
+// blocks per SM (the kernel strides over the rest).
+int gather_blocks(int64_t T, int nvec, int sms)
+{
+    const int64_t warps = T * ((nvec + 31) / 32);
+    return (int)std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, (int64_t)sms * 16));
+}
+
 // The general (multi-CTA) histogram / scan / scatter (/ gather of bf16 rows
 // into xp when xp is given).  `ps` shapes the tile plan.
 int run_permute(const int32_t* idx, const bf16* x, int T, int d, int E, int k, int32_t* counts, int32_t* offsets,
@@ -360,9 +369,8 @@ int run_permute(const int32_t* idx, const bf16* x, int T, int d, int E, int k, i
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     if (inv_perm_launch) *inv_perm_launch = t_launches;
     if (!xp) return MOE_OK;
-    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)sms * 16));
-    return status_of(launch(gather_rows_kernel, dim3(blocks), dim3(256), 0, st, x, (const int32_t*)perm,
-                            (const int32_t*)offsets, E, k, d, xp));
+    return status_of(launch(gather_rows_kernel, dim3(gather_blocks(T, d / 8, sms)), dim3(256), 0, st, x,
+                            (const int32_t*)inv_perm, T, k, d, xp));
 }
 
 struct GemmOperands {
@@ -756,9 +764,8 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
             return MOE_ERR_CUDA;
         inv_perm_launch = t_launches;
         if (!gather_in_gemm) {
-            const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)dev->sm_count * 16));
-            if (launch(gather_rows_kernel, dim3(blocks), dim3(256), 0, st, xb, (const int32_t*)perm,
-                       (const int32_t*)offsets, iE, ik, id, xp) != cudaSuccess)
+            if (launch(gather_rows_kernel, dim3(gather_blocks(T, d / 8, dev->sm_count)), dim3(256), 0, st, xb,
+                       (const int32_t*)inv_perm, iT, ik, id, xp) != cudaSuccess)
                 return MOE_ERR_CUDA;
         }
     } else {
@@ -1183,9 +1190,9 @@ static int layer_forward_lowp(const moe_bf16* x, const moe_bf16* Wg, const float
                                  dev->sm_count, st, ps, &inv_perm_launch))) {
         return rc;
     }
-    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((P + 7) / 8, (int64_t)dev->sm_count * 16));
-    if (launch(gather_rows_fp8_kernel, dim3(blocks), dim3(256), 0, st, (const uint8_t*)x8, (const float*)sx,
-               (const int32_t*)perm, (const int32_t*)offsets, iE, ik, id, xp8, sxp, L.ld_pairs) != cudaSuccess)
+    if (launch(gather_rows_fp8_kernel, dim3(gather_blocks(T, d / 16, dev->sm_count)), dim3(256), 0, st,
+               (const uint8_t*)x8, (const float*)sx, (const int32_t*)inv_perm, iT, ik, id, xp8, sxp,
+               L.ld_pairs) != cudaSuccess)
         return MOE_ERR_CUDA;
     Fp8Operands o{};
     o.xp8 = xp8;

@@ -368,31 +368,31 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
 }
 
 // ---------------------------------------------------------------- gather
-// xp[pos, :] = x[perm[pos] / k, :] for pos < pairs; one warp per row, 16-byte
-// vectors.  Requires d % 8 == 0.
-__global__ void __launch_bounds__(256) gather_rows_kernel(const bf16* __restrict__ x, const int32_t* __restrict__ perm,
-                                                          const int32_t* __restrict__ offsets, int E, int k, int d,
+// xp[inv_perm[t k + j], :] = x[t, :] for every pair with a valid position
+// (inv_perm >= 0): xp[pos] = x[perm[pos] / k] for pos < pairs, taken in token
+// order so that each x row is read once for its k copies (x is read T d 2
+// bytes, not T k d 2).  One warp per (token, 512-byte chunk of the row): a
+// 16-byte vector per lane, then its k stores.  Requires d % 8 == 0, k <= 32.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const bf16* __restrict__ x,
+                                                          const int32_t* __restrict__ inv_perm, int T, int k, int d,
                                                           bf16* __restrict__ xp)
 {
     ptx::grid_dep_wait();
     ptx::grid_dep_launch();
-    const int pairs = offsets[E];
     const int nvec = d / 8;
+    const int nch = (nvec + 31) / 32;
     const int lane = threadIdx.x & 31;
-    constexpr int kUnroll = 8;
-    for (int64_t r = (int64_t)(blockIdx.x * blockDim.x + threadIdx.x) / 32; r < pairs;
-         r += (int64_t)gridDim.x * blockDim.x / 32) {
-        const int t = perm[r] / k;
-        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
-        uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * d);
-        for (int v0 = lane; v0 < nvec; v0 += 32 * kUnroll) {
-            uint4 buf[kUnroll];
-#pragma unroll
-            for (int u = 0; u < kUnroll; u++)
-                if (v0 + 32 * u < nvec) buf[u] = __ldg(src + v0 + 32 * u);
-#pragma unroll
-            for (int u = 0; u < kUnroll; u++)
-                if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = buf[u];
+    const int64_t items = (int64_t)T * nch;
+    for (int64_t w = (int64_t)(blockIdx.x * blockDim.x + threadIdx.x) / 32; w < items;
+         w += (int64_t)gridDim.x * blockDim.x / 32) {
+        const int64_t t = w / nch;
+        const int v = (int)(w - t * nch) * 32 + lane;
+        const int mine = lane < k ? inv_perm[t * k + lane] : -1;
+        uint4 buf = make_uint4(0u, 0u, 0u, 0u);
+        if (v < nvec) buf = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d) + v);
+        for (int j = 0; j < k; j++) {
+            const int pos = __shfl_sync(0xffffffffu, mine, j);
+            if (pos >= 0 && v < nvec) reinterpret_cast<uint4*>(xp + (size_t)pos * d)[v] = buf;
         }
     }
 }
