@@ -194,3 +194,35 @@ def test_tile_table_writer(tmp_path):
     widths = [int(v) for v in re.search(r"MOE_TOKEN_BUCKET_WIDTH \{([^}]*)\}", src).group(1).split(",")]
     assert caps[2] == 128 and caps[13] == 256 and caps[0] == 256 and len(caps) == 15
     assert widths[0] == 32 and widths[5] == 256 and widths[3] == 128 and len(widths) == 6
+
+
+def test_algorithmic_bytes_per_weight_format():
+    """Weight bytes per element: bf16 2, FP8 1 + a 4-byte scale per 128 x 128 block, FP4 half a byte + a scale
+    byte per 32; the flops do not depend on the format."""
+    s = wl.LayerShape("a", T=4, d=128, f=128, E=3, k=2, alpha=1.0)
+    counts = np.array([5, 3, 0])
+    per = {"bf16": 2.0, "fp8": 1.0 + 4.0 / (128 * 128), "fp4": 0.5 + 1.0 / 32}
+    flops = None
+    for fmt, b in per.items():
+        a = bench.algorithmic(s, counts, fmt=fmt)
+        assert a["active"] == 2 and a["pairs"] == 8
+        assert a["w_act"] == pytest.approx(2 * 3 * 128 * 128 * b)
+        flops = flops or a["flops"]
+        assert a["flops"] == flops == 6.0 * 8 * 128 * 128
+    assert bench.algorithmic(s, counts, fp8=True) == bench.algorithmic(s, counts, fmt="fp8")
+
+
+def test_weight_format_and_traffic_key(tmp_path, monkeypatch):
+    """--fp4 selects the FP4 weights; an FP4 workload's traffic record is keyed to the FP8 kernel's source."""
+    args = bench.build_parser().parse_args(["--fp4"])
+    assert bench.weight_format(args) == "fp4" and bench.fmt_suffix("fp4") == " fp4"
+    assert bench.weight_format(bench.build_parser().parse_args([])) == "bf16"
+    with pytest.raises(SystemExit):
+        bench.build_parser().parse_args(["--fp4", "--fp8"])
+    rec = [{"workload": "w fp4", "kernel_role": "gate_up", "source_sha": bench.kernel_source_hash(True),
+            "dram_bytes_per_launch": 7}]
+    p = tmp_path / "t.json"
+    p.write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(p))
+    assert bench.committed_traffic("w fp4", "gate_up") == 7
+    assert bench.committed_traffic("w fp4", "down") is None

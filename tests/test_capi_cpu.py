@@ -117,6 +117,38 @@ def test_fp8_host_argument_checks(L):
     assert L.moe_quantize_fp8_blocks(FAKE, 128, 128, FAKE, None, None) == -1
 
 
+def _layer_fp4(L, **kw):
+    a = dict(x=FAKE, Wg=FAKE, bias=None, W1q=FAKE, W1sf=FAKE, W3q=FAKE, W3sf=FAKE, W2q=FAKE, W2sf=FAKE, Ws1q=None,
+             Ws1sf=None, Ws3q=None, Ws3sf=None, Ws2q=None, Ws2sf=None, fs=0, T=4, d=256, f=256, E=4, k=2, out=FAKE,
+             ws=FAKE, ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    return L.moe_layer_forward_fp4(a["x"], a["Wg"], a["bias"], a["W1q"], a["W1sf"], a["W3q"], a["W3sf"], a["W2q"],
+                                   a["W2sf"], a["Ws1q"], a["Ws1sf"], a["Ws3q"], a["Ws3sf"], a["Ws2q"], a["Ws2sf"],
+                                   a["fs"], a["T"], a["d"], a["f"], a["E"], a["k"], a["out"], a["ws"], a["ws_bytes"],
+                                   a["stream"])
+
+
+def test_fp4_host_argument_checks(L):
+    """The FP4-weight layer and row quantiser refuse bad arguments on the host, before any device work."""
+    assert _layer_fp4(L, d=192) == -2          # a multiple of 64 but not of 128
+    assert _layer_fp4(L, f=64) == -2
+    assert _layer_fp4(L, fs=64) == -2
+    assert _layer_fp4(L, d=16512) == -1
+    assert _layer_fp4(L, W2sf=None) == -1      # a weight's scale atoms missing
+    assert _layer_fp4(L, fs=128) == -1         # shared expert without weights
+    assert _layer_fp4(L, fs=128, Ws1q=FAKE, Ws3q=FAKE, Ws2q=FAKE, Ws1sf=FAKE, Ws3sf=FAKE, Ws2sf=None) == -1
+    assert _layer_fp4(L, W1sf=C.c_void_p(0x10008)) == -2   # scale atoms not 16-byte aligned
+    assert _layer_fp4(L, x=C.c_void_p(0x10008)) == -2
+    assert _layer_fp4(L, ws_bytes=1024) == -3
+    assert _layer_fp4(L, T=0) == 0
+    assert L.moe_quantize_fp4_rows(FAKE, 100, 128, FAKE, FAKE, None) == -2    # rows not a multiple of 128
+    assert L.moe_quantize_fp4_rows(FAKE, 128, 96, FAKE, FAKE, None) == -2     # cols not a multiple of 128
+    assert L.moe_quantize_fp4_rows(FAKE, -128, 128, FAKE, FAKE, None) == -1
+    assert L.moe_quantize_fp4_rows(FAKE, 128, 128, None, FAKE, None) == -1
+    assert L.moe_quantize_fp4_rows(FAKE, 128, 128, FAKE, C.c_void_p(0x10008), None) == -2
+    assert L.moe_quantize_fp4_rows(FAKE, 0, 128, FAKE, FAKE, None) == 0
+
+
 def test_product_path_refuses_missing_library(monkeypatch, tmp_path):
     monkeypatch.setattr(moe, "_lib", None)
     monkeypatch.setattr(moe, "library_path", lambda: str(tmp_path / "absent.so"))
